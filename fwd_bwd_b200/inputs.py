@@ -1,0 +1,161 @@
+"""Seeded synthetic inputs for SageBwd attention (no method arithmetic lives here).
+
+Both the CUDA path (through the tests and ``bench.py``) and the CPU oracle are fed from the
+arrays this module returns, so it is the one piece of code they share.  It only draws random
+numbers and stores them as 16-bit floats; it performs none of the quantization, normalization
+or attention arithmetic.
+
+Recipe (the same for every workload):
+
+* ``numpy.random.Generator(PCG64(seed + offset))`` with offsets Q:0, K:1, V:2, dO:3, mu:4;
+* ``standard_normal`` in float64, multiplied by the tensor's sigma, rounded to float32;
+* float32 rounded to the 16-bit storage type with round-half-to-even (bf16 by bit
+  manipulation, fp16 by numpy's own RNE cast).
+
+Arrays are returned as ``uint16`` bit patterns in ``[B, H, N, d]`` order (``d`` innermost),
+plus an exact float32 view for CPU consumers.
+
+The workloads are the attention shapes of the SageBwd page ("SageBwd: trainable low-bit
+attention", aitrends.kr): the 325M-Llama attention layer it pretrains, a K-outlier stress case
+for the K-smoothing ablation, a long-sequence case for the small-dS regime and the
+tokens-per-step sweep.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Optional
+
+import numpy as np
+
+OFFSET_Q, OFFSET_K, OFFSET_V, OFFSET_DO, OFFSET_MU = 0, 1, 2, 3, 4
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """Shape, dtype and value distribution of one synthetic attention problem."""
+
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    dtype: str  # "bf16" or "fp16"
+    q_block: int = 128
+    k_block: int = 64
+    qknorm: bool = True
+    ksmooth: bool = True
+    sigma_qkv: float = 1.0
+    sigma_do: float = 1.0
+    k_outlier: bool = False  # per-channel offsets mu_c ~ N(0, 4^2), 4 channels +20
+    seed: int = 0
+
+    @property
+    def tokens(self) -> int:
+        return self.B * self.N
+
+    def ops(self, part: str = "fwdbwd") -> float:
+        """Tensor-core op count (FlashAttention convention, masked half not credited)."""
+        per_gemm = 2.0 * self.N * self.N * self.d * (0.5 if self.causal else 1.0)
+        n = {"fwd": 2, "bwd": 5, "fwdbwd": 7}[part]
+        return self.B * self.H * n * per_gemm
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS: Dict[str, Workload] = {
+    # tiny correctness case (oracle finishes instantly)
+    "tiny": Workload("tiny", 1, 2, 128, 64, False, "fp16", q_block=64, k_block=64,
+                     sigma_do=1e-2),
+    # 325M-Llama-like attention layer
+    "llama325m": Workload("llama325m", 8, 16, 2048, 64, True, "bf16", sigma_do=1e-3),
+    # K-outlier stress (run with the qknorm / ksmooth flags on and off)
+    "koutlier": Workload("koutlier", 4, 16, 4096, 128, True, "bf16", k_outlier=True),
+    # long sequence, small-dS regime
+    "long16k": Workload("long16k", 1, 32, 16384, 128, True, "bf16", sigma_do=1e-4),
+}
+# tokens-per-step sweep: B*N = 262144 tokens, H=16, d=128, causal
+for _n in (1024, 2048, 4096, 8192):
+    WORKLOADS[f"sweep{_n}"] = Workload(f"sweep{_n}", 262144 // _n, 16, _n, 128, True, "bf16")
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16 (round-half-to-even) and return the uint16 bit pattern."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def bits_to_f32(bits: np.ndarray, dtype: str) -> np.ndarray:
+    """Exact float32 value of 16-bit storage given as uint16 bit patterns."""
+    if dtype == "bf16":
+        return (bits.astype(np.uint32) << 16).view(np.float32)
+    if dtype == "fp16":
+        return bits.view(np.float16).astype(np.float32)
+    raise ValueError(dtype)
+
+
+def f32_to_bits(x: np.ndarray, dtype: str) -> np.ndarray:
+    if dtype == "bf16":
+        return f32_to_bf16_bits(x)
+    if dtype == "fp16":
+        return np.ascontiguousarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
+    raise ValueError(dtype)
+
+
+def _normal(seed: int, shape, sigma: float) -> np.ndarray:
+    g = np.random.Generator(np.random.PCG64(seed))
+    return (g.standard_normal(shape) * sigma).astype(np.float32)
+
+
+def make_inputs(w: Workload, heads: Optional[slice] = None) -> Dict[str, np.ndarray]:
+    """Return {'q','k','v','do'} as uint16 bit arrays [B,H,N,d] (and '<name>_f32' views).
+
+    ``heads`` restricts the result to a slice of the flattened (b, h) index; the values of the
+    kept heads are identical to those of the full draw (the full array is drawn, then sliced),
+    so a sampled head can be checked against the same head of a full-size GPU run.
+    """
+    shape = (w.B, w.H, w.N, w.d)
+    out: Dict[str, np.ndarray] = {}
+    q = _normal(w.seed + OFFSET_Q, shape, w.sigma_qkv)
+    k = _normal(w.seed + OFFSET_K, shape, w.sigma_qkv)
+    v = _normal(w.seed + OFFSET_V, shape, w.sigma_qkv)
+    do = _normal(w.seed + OFFSET_DO, shape, w.sigma_do)
+    if w.k_outlier:
+        g = np.random.Generator(np.random.PCG64(w.seed + OFFSET_MU))
+        mu = (g.standard_normal((w.B, w.H, 1, w.d)) * 4.0).astype(np.float32)
+        chans = g.choice(w.d, size=4, replace=False)
+        mu[..., chans] += np.float32(20.0)
+        k = (k + mu).astype(np.float32)
+    for name, arr in (("q", q), ("k", k), ("v", v), ("do", do)):
+        if heads is not None:
+            arr = arr.reshape(w.B * w.H, w.N, w.d)[heads]
+        bits = f32_to_bits(arr, w.dtype)
+        out[name] = bits
+        out[name + "_f32"] = bits_to_f32(bits, w.dtype)
+    return out
+
+
+def make_inputs_fast(w: Workload, device: str = "cpu"):
+    """Large-workload inputs drawn with torch's generator (used only for timing runs).
+
+    Same distributions as :func:`make_inputs` but a different (torch Philox) stream, so values
+    are not comparable with ``make_inputs``; parity checks always use ``make_inputs``.
+    """
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+    shape = (w.B, w.H, w.N, w.d)
+    res = {}
+    for name, sig in (("q", w.sigma_qkv), ("k", w.sigma_qkv), ("v", w.sigma_qkv),
+                      ("do", w.sigma_do)):
+        res[name] = (torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+                     * sig).to(tdt)
+    if w.k_outlier:
+        mu = torch.randn((w.B, w.H, 1, w.d), generator=g, device=device) * 4.0
+        mu[..., :4] += 20.0
+        res["k"] = (res["k"].float() + mu).to(tdt)
+    return res
