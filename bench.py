@@ -1,0 +1,320 @@
+#!/usr/bin/env python
+"""Benchmark: SageBwd INT8 attention forward + backward on B200.
+
+One step = the whole hot path on one batch: the quantization prologue (QK-norm, K-smoothing,
+INT8 codes), the forward kernel and the three backward stages, on synthetic bf16 inputs that
+are resident in HBM (each input tensor is 1 GiB, far larger than the 126 MB L2, so no flush is
+needed between steps).  Metric: effective tensor-core TOPS over the step, counting the seven
+attention GEMMs (FlashAttention convention, causal half not credited).
+
+Multi-GPU (torchrun): every (batch, head) is independent and the operator has no weights, so
+each rank runs its own full-size batch with no collective on the data path (weak scaling); the
+harness takes the maximum elapsed time over ranks.
+
+``--impl reference`` times the CPU oracle (the plain restatement of the method the tests
+check the kernels against) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd+bwd effective TOPS at 1 B200 and % of INT8/FP16 TC roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="sage", choices=["sage", "reference"])
+    ap.add_argument("--workload", default="sweep8192")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    """Roofline denominators: measured bf16 peaks; INT8 = 2x bf16 (nominal dense ratio)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        m = json.load(open(path))
+        return {"bf16_burst": m["bf16_tflops"], "bf16_sustained": m["bf16_tflops_sustained"],
+                "hbm_gbs": m["hbm_gbs"], "basis": "measured"}
+    return {"bf16_burst": 1590.0, "bf16_sustained": 1400.0, "hbm_gbs": 6650.0,
+            "basis": "fallback"}
+
+
+def weighted_peak(p_bf16: float, n_i8: int, n_f16: int) -> float:
+    """Peak of a mix of equal-size INT8 and 16-bit GEMMs (INT8 at twice the bf16 rate)."""
+    p_i8 = 2.0 * p_bf16
+    n = n_i8 + n_f16
+    return 1.0 / (n_i8 / n / p_i8 + n_f16 / n / p_bf16)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", uuid], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit()
+                else None, "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_baseline(w, n_heads: int):
+    """Time the oracle (as it stands) on the first n_heads heads of the workload."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    import oracle.sage_oracle as O
+    from fwd_bwd_b200.inputs import make_inputs
+
+    x = make_inputs(w, heads=range(n_heads))
+    args = [x[n + "_f32"] for n in ("q", "k", "v", "do")]
+    t0 = time.perf_counter()
+    O.sage_attention(*args, causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth,
+                     q_block=w.q_block, k_block=w.k_block, dtype=w.dtype)
+    dt = time.perf_counter() - t0
+    ops = w.ops() / (w.B * w.H) * n_heads
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    del np
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+            "seconds": dt,
+            "sample": f"{n_heads} of {w.B * w.H} heads (flattened b*H+h = 0..{n_heads - 1}) of "
+                      f"the workload, prologue+fwd+bwd, numpy oracle"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    times = []
+    res = None
+    for s in range(args.warmup + args.steps):
+        res = cpu_baseline(w, 1)
+        if s >= args.warmup:
+            times.append(res["seconds"])
+    sec = statistics.mean(times)
+    ops = w.ops() / (w.B * w.H)
+    val = ops / sec / 1e12
+    cb = dict(res, value=val)
+    cb.pop("seconds", None)
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TOPS",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8+f64", "data": "synthetic",
+            "config": config_of(w), "cpu_baseline": cb,
+            "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "io_dtype": w.dtype, "q_block": w.q_block, "k_block": w.k_block,
+            "qknorm": w.qknorm, "ksmooth": w.ksmooth,
+            "l2": "no flush: every input tensor (1 GiB at the default workload) exceeds L2"}
+
+
+def main():
+    args = parse()
+    from fwd_bwd_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from fwd_bwd_b200 import ops
+    from fwd_bwd_b200.inputs import make_inputs_fast
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    cfg = ops.Config(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth, q_block=w.q_block,
+                     k_block=w.k_block)
+    x = make_inputs_fast(w.replace(seed=w.seed + rank), device=str(dev))
+    q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+    prm = cfg.params(q)
+    qb = ops.QuantBufs.empty(tuple(q.shape), cfg, dev)
+    ws_pro = torch.empty(max(ops.workspace_bytes(prm, 0), 16), dtype=torch.uint8, device=dev)
+    ws_bwd = torch.empty(ops.workspace_bytes(prm, 2), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = (3 if w.ksmooth else 1) + 1 + 3
+
+    def step(ev=None):
+        ops.quant_prologue(q, k, v, cfg, out=qb, workspace=ws_pro)
+        if ev is not None:
+            ev[0].record(stream)
+        ops.attn_fwd(qb, q, cfg, o=o, lse=lse)
+        if ev is not None:
+            ev[1].record(stream)
+        ops.attn_bwd(q, k, v, qb, o, lse, do, cfg, dq, dk, dv, workspace=ws_bwd, stage=0)
+        if ev is not None:
+            ev[2].record(stream)
+        ops.attn_bwd(q, k, v, qb, o, lse, do, cfg, dq, dk, dv, workspace=ws_bwd, stage=1)
+        if ev is not None:
+            ev[3].record(stream)
+        ops.attn_bwd(q, k, v, qb, o, lse, do, cfg, dq, dk, dv, workspace=ws_bwd, stage=2)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ops.device_status(dev) != 0:
+        raise RuntimeError("device status reports a kernel timeout during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    time.sleep(0.3)
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    elapsed = t_start.elapsed_time(t_end)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+    if ops.device_status(dev) != 0:
+        raise RuntimeError("device status reports a kernel timeout in the timed region")
+    ms = elapsed / args.steps
+    total_ops = w.ops() * world
+    value = total_ops / (ms * 1e-3) / 1e12
+
+    # end to end through the same API with pinned host buffers: H2D inputs, D2H results
+    e2e = None
+    if not args.no_e2e:
+        hin = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, dq, dk, dv)]
+        for _ in range(1):
+            for h, dst in zip(hin, (q, k, v, do)):
+                dst.copy_(h, non_blocking=True)
+            step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            for h, dst in zip(hin, (q, k, v, do)):
+                dst.copy_(h, non_blocking=True)
+            step()
+            for src, h in zip((o, dq, dk, dv), hout):
+                h.copy_(src, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": total_ops / (e_ms / args.steps * 1e-3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hin),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout)}
+
+    pk = peaks()
+    basis = pk["basis"]
+    p_bwd = weighted_peak(pk["bf16_sustained"], 4, 1)
+    p_fwd = weighted_peak(pk["bf16_sustained"], 2, 0)
+    p_all = weighted_peak(pk["bf16_sustained"], 6, 1)
+    bwd_ops = w.ops("bwd")
+    fwd_ops = w.ops("fwd")
+    kernels = {
+        "attn_bwd_kernel": {"ms": bwd_main_ms, "achieved": bwd_ops / (bwd_main_ms * 1e-3) / 1e12,
+                            "peak": p_bwd},
+        "attn_fwd_kernel": {"ms": fwd_ms, "achieved": fwd_ops / (fwd_ms * 1e-3) / 1e12,
+                            "peak": p_fwd},
+    }
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+    kd = kernels[dom]
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": kd["achieved"],
+                "peak": kd["peak"], "unit": "TFLOP/s", "frac": kd["achieved"] / kd["peak"],
+                "traffic": None,
+                "peak_note": f"{basis} sustained bf16 x (INT8 = 2x bf16), weighted by the "
+                             f"kernel's INT8:16-bit GEMM mix"}
+
+    line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8+bf16", "data": "synthetic", "config": config_of(w),
+            "frac_of_weighted_peak": value / world / p_all,
+            "weighted_peak_tops": p_all,
+            "kernels": {n: {"ms": round(v_["ms"], 4), "tops": round(v_["achieved"], 2),
+                            "frac": round(v_["achieved"] / v_["peak"], 4)}
+                        for n, v_ in kernels.items()},
+            "roofline": roofline, "clocks": clocks, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, 4)
+        line["cpu_baseline"].pop("seconds", None)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

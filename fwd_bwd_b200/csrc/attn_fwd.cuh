@@ -1,0 +1,333 @@
+// attn_fwd.cuh -- SageBwd forward attention on sm_100a (quantization-strategy paragraph of
+// "SageBwd: trainable low-bit attention": S = Q K^T and O = P V in INT8).
+//
+// Per CTA: two tiles of 128 query rows of one (batch, head), walking 64-key blocks.
+//   warp 8      TMA producer: the Q code tiles once, then K and V code blocks through a
+//               4-stage ring (K and V blocks are shared by both query tiles).
+//   warp 9      MMA issuer (one thread): S_j = Qc Kc_j^T (kind::i8, M=128, N=64, into TMEM,
+//               double-buffered per tile) and PV_j = Pc_j Vc_j (kind::i8, M=128, N=d).
+//   warps 0-7   softmax, one query row per thread (warps 0-3 tile 0, 4-7 tile 1):
+//               z = A * (sQ sK tau), causal mask, block max, p~ = exp(z - max_block),
+//               P codes = rne(127 p~) written to shared memory in the tensor core's swizzled
+//               K-major layout, running max / sum, and the dequantizing fold
+//               O <- alpha O + PV * beta with beta = exp(max_block - max_running) sV / 127.
+// TMEM (512 columns): tile g uses columns [256g, 256g+256): S buffers at +0 and +64, PV at
+// +128 (d columns, INT32).  O (float32) lives in registers.
+//
+// P quantization: one scale per (query row, 64-key block).  The codes rne(127 p / max p) do
+// not depend on which running maximum p was taken against, so computing them against the
+// block's own maximum (as here) equals any other evaluation order in exact arithmetic.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+#include "rowops.cuh"
+
+namespace sage {
+namespace fwd {
+
+constexpr int BM = 128;   // query rows per tile (MMA M)
+constexpr int BKV = 64;   // keys per block (= k_block)
+constexpr int NT = 2;     // query tiles per CTA
+constexpr int NST = 4;    // K/V pipeline stages
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+
+template <int D>
+struct Smem {
+  int8_t q[NT][BM * D];
+  int8_t k[NST][BKV * D];
+  int8_t v[NST][BKV * D];
+  int8_t p[NT][2][BM * BKV];
+  uint64_t q_full;
+  uint64_t k_full[NST], v_full[NST], kv_empty[NST];
+  uint64_t s_full[NT][2], p_full[NT][2], pv_full[NT], pv_free[NT];
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D>
+constexpr size_t smem_bytes() {
+  return sizeof(Smem<D>) + 1024;  // + alignment slack (tiles need 1024-byte alignment)
+}
+
+struct Args {
+  const float* q_scale;
+  const float* k_scale;
+  const float* v_scale;
+  void* o;
+  float* lse;
+  int BH, N, q_block, causal;
+  float scale_log2;  // softmax_scale * log2(e)
+  int nsup;          // CTAs per head: ceil(N / 256)
+};
+
+template <int D>
+__device__ __forceinline__ Smem<D>& smem_ref(uint8_t* raw) {
+  const uint32_t a = smem_u32(raw);
+  return *reinterpret_cast<Smem<D>*>(raw + ((1024u - (a & 1023u)) & 1023u));
+}
+
+// Issue S = Qc Kc^T for one tile / block: d/32 MMAs of K = 32 bytes.
+template <int D>
+__device__ __forceinline__ void issue_scores(uint32_t d_tmem, const int8_t* qs,
+                                             const int8_t* ks, int n_keys) {
+  constexpr uint32_t kSw = (D == 128) ? kSwizzle128B : kSwizzle64B;
+  constexpr uint32_t kSbo = 8 * D;  // 8 rows of D bytes
+  const uint32_t idesc = instr_desc(2, 1, 1, false, false, BM, n_keys);
+  const uint32_t qa = smem_u32(qs), ka = smem_u32(ks);
+#pragma unroll
+  for (int kk = 0; kk < D / 32; ++kk) {
+    mma_i8(d_tmem, smem_desc(qa + kk * 32, 16, kSbo, kSw), smem_desc(ka + kk * 32, 16, kSbo, kSw),
+           idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, Args args) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem<D>& sm = smem_ref<D>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = args.N;
+  const int cta = blockIdx.x;
+  const int sup = args.causal ? (args.nsup - 1 - cta / args.BH) : (cta / args.BH);
+  const int bh = cta % args.BH;
+  int q0[NT], nb[NT];
+  bool active[NT];
+  int nb_max = 0;
+#pragma unroll
+  for (int g = 0; g < NT; ++g) {
+    q0[g] = sup * (NT * BM) + g * BM;
+    active[g] = q0[g] < N;
+    nb[g] = active[g] ? (args.causal ? (q0[g] + BM) / BKV : N / BKV) : 0;
+    nb_max = max(nb_max, nb[g]);
+  }
+
+  if (threadIdx.x == 0) {
+    sm.abort = device_aborted() ? 1 : 0;
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int g = 0; g < NT; ++g) {
+      mbar_init(&sm.s_full[g][0], 1);
+      mbar_init(&sm.s_full[g][1], 1);
+      mbar_init(&sm.p_full[g][0], BM);
+      mbar_init(&sm.p_full[g][1], BM);
+      mbar_init(&sm.pv_full[g], 1);
+      mbar_init(&sm.pv_free[g], BM);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (sm.abort) return;
+  if (warp == kMmaWarp) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const int row_base = bh * N;
+      int nact = 0;
+      for (int g = 0; g < NT; ++g) nact += active[g] ? 1 : 0;
+      mbar_arrive_expect_tx(&sm.q_full, nact * BM * D);
+      for (int g = 0; g < NT; ++g)
+        if (active[g]) tma_load_2d(sm.q[g], &tm_q, 0, row_base + q0[g], &sm.q_full);
+      for (int j = 0; j < nb_max; ++j) {
+        const int st = j % NST;
+        if (j >= NST) mbar_wait(&sm.kv_empty[st], ((j / NST) - 1) & 1, 100);
+        mbar_arrive_expect_tx(&sm.k_full[st], BKV * D);
+        tma_load_2d(sm.k[st], &tm_k, 0, row_base + j * BKV, &sm.k_full[st]);
+        mbar_arrive_expect_tx(&sm.v_full[st], BKV * D);
+        tma_load_2d(sm.v[st], &tm_v, 0, row_base + j * BKV, &sm.v_full[st]);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t kSw = (D == 128) ? kSwizzle128B : kSwizzle64B;
+      constexpr uint32_t kSbo = 8 * D;
+      const uint32_t idesc_pv = instr_desc(2, 1, 1, false, true, BM, D);
+      mbar_wait(&sm.q_full, 0, 101);
+      tc_fence_after();
+      mbar_wait(&sm.k_full[0], 0, 102);
+      tc_fence_after();
+      for (int g = 0; g < NT; ++g)
+        if (nb[g] > 0) {
+          issue_scores<D>(tmem + g * 256, sm.q[g], sm.k[0], BKV);
+          mma_commit(&sm.s_full[g][0]);
+        }
+      for (int j = 0; j < nb_max; ++j) {
+        const int st = j % NST;
+        if (j + 1 < nb_max) {
+          const int st1 = (j + 1) % NST;
+          mbar_wait(&sm.k_full[st1], ((j + 1) / NST) & 1, 103);
+          tc_fence_after();
+          for (int g = 0; g < NT; ++g)
+            if (j + 1 < nb[g]) {
+              issue_scores<D>(tmem + g * 256 + ((j + 1) & 1) * 64, sm.q[g], sm.k[st1], BKV);
+              mma_commit(&sm.s_full[g][(j + 1) & 1]);
+            }
+        }
+        mbar_wait(&sm.v_full[st], (j / NST) & 1, 104);
+        for (int g = 0; g < NT; ++g) {
+          if (j >= nb[g]) continue;
+          mbar_wait(&sm.p_full[g][j & 1], (j >> 1) & 1, 105);
+          if (j > 0) mbar_wait(&sm.pv_free[g], (j - 1) & 1, 106);
+          tc_fence_after();
+          const uint32_t pa = smem_u32(sm.p[g][j & 1]);
+          const uint32_t va = smem_u32(sm.v[st]);
+#pragma unroll
+          for (int kk = 0; kk < BKV / 32; ++kk) {
+            mma_i8(tmem + g * 256 + 128, smem_desc(pa + kk * 32, 16, 8 * BKV, kSwizzle64B),
+                   smem_desc(va + kk * 32 * D, BKV * D, kSbo, kSw), idesc_pv, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&sm.pv_full[g]);
+        }
+        mma_commit(&sm.kv_empty[st]);
+      }
+    }
+  } else {
+    // ---------------- softmax warps ----------------
+    const int g = warp >> 2, quarter = warp & 3;
+    if (active[g]) {
+      const int r = quarter * 32 + lane;
+      const int i = q0[g] + r;
+      const int nqb = N / args.q_block, nkb = N / BKV;
+      const float cq = args.q_scale[bh * nqb + i / args.q_block] * args.scale_log2;
+      const float* ksc = args.k_scale + static_cast<size_t>(bh) * nkb;
+      const float* vsc = args.v_scale + static_cast<size_t>(bh) * nkb;
+      const uint32_t lane_base = tmem + ((quarter * 32u) << 16) + g * 256;
+      float O[D];
+#pragma unroll
+      for (int c = 0; c < D; ++c) O[c] = 0.0f;
+      float m2 = -INFINITY, l = 0.0f, alpha_prev = 1.0f, beta_prev = 0.0f;
+      int8_t* pbase = sm.p[g][0];
+
+      auto fold_pv = [&](int jj) {
+        mbar_wait(&sm.pv_full[g], jj & 1, 110);
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t a0[16], a1[16];
+          tmem_ld16(lane_base + 128 + c0, a0);
+          tmem_ld16(lane_base + 128 + c0 + 16, a1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            O[c0 + c] = fmaf(i2f_exact(a0[c]), beta_prev, O[c0 + c] * alpha_prev);
+            O[c0 + 16 + c] = fmaf(i2f_exact(a1[c]), beta_prev, O[c0 + 16 + c] * alpha_prev);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sm.pv_free[g]);
+      };
+
+      for (int j = 0; j < nb[g]; ++j) {
+        const float c = cq * ksc[j];
+        const bool diag = args.causal && (j * BKV + BKV - 1 > q0[g]);
+        const int key0 = j * BKV;
+        mbar_wait(&sm.s_full[g][j & 1], (j >> 1) & 1, 111);
+        tc_fence_after();
+        const uint32_t sa = lane_base + (j & 1) * 64;
+        // pass 1: block maximum of the (masked) integer scores
+        int amax = INT_MIN;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t a0[16], a1[16];
+          tmem_ld16(sa + h * 32, a0);
+          tmem_ld16(sa + h * 32 + 16, a1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc) {
+            const int k0 = key0 + h * 32 + cc, k1 = k0 + 16;
+            if (!diag || k0 <= i) amax = max(amax, static_cast<int>(a0[cc]));
+            if (!diag || k1 <= i) amax = max(amax, static_cast<int>(a1[cc]));
+          }
+        }
+        const bool has = amax != INT_MIN;
+        const float mblk = has ? c * i2f_exact(static_cast<uint32_t>(amax)) : -INFINITY;
+        // pass 2: p~ = exp2(z - mblk), codes rne(127 p~), row sum
+        float rs = 0.0f;
+        int8_t* prow = pbase + (j & 1) * (BM * BKV);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t a0[16], a1[16];
+          tmem_ld16(sa + h * 32, a0);
+          tmem_ld16(sa + h * 32 + 16, a1);
+          tmem_ld_wait();
+          uint32_t pk[8];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t b[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int cc = q4 * 4 + e;
+                const uint32_t av = half ? a1[cc] : a0[cc];
+                const int kidx = key0 + h * 32 + half * 16 + cc;
+                float p = ex2_approx(fmaf(i2f_exact(av), c, -mblk));
+                if (diag && kidx > i) p = 0.0f;
+                rs += p;
+                b[e] = rne_byte(p * 127.0f);
+              }
+              pk[half * 4 + q4] = pack4(b[0], b[1], b[2], b[3]);
+            }
+          }
+          // keys h*32 .. h*32+31 are 16-byte chunks 2h and 2h+1 of this row
+          *reinterpret_cast<uint4*>(prow + swz_offset(r, 2 * h, 64)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(prow + swz_offset(r, 2 * h + 1, 64)) =
+              make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+        const float m2n = fmaxf(m2, mblk);
+        const float alpha = ex2_approx(m2 - m2n);
+        const float eblk = has ? ex2_approx(mblk - m2n) : 0.0f;
+        l = fmaf(l, alpha, eblk * rs);
+        const float beta = eblk * vsc[j] * (1.0f / 127.0f);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sm.p_full[g][j & 1]);
+        if (j > 0) fold_pv(j - 1);
+        alpha_prev = alpha;
+        beta_prev = beta;
+        m2 = m2n;
+      }
+      fold_pv(nb[g] - 1);
+      // epilogue: O / l in the output type, LSE = (m2 + log2 l) ln 2
+      const float inv_l = 1.0f / l;
+      T* orow = reinterpret_cast<T*>(args.o) + (static_cast<size_t>(bh) * N + i) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 8) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = O[c0 + e] * inv_l;
+        *reinterpret_cast<uint4*>(orow + c0) = pack8<T>(f);
+      }
+      args.lse[static_cast<size_t>(bh) * N + i] = (m2 + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace fwd
+}  // namespace sage

@@ -1,0 +1,338 @@
+// rowops.cuh -- HBM-bound row kernels of the SageBwd path:
+//   * the prologue (QK-norm paragraph: per-token RMSNorm of q and k; K-smoothing paragraph:
+//     per-channel mean of k over tokens subtracted before quantization; Triton-kernel
+//     paragraph: per-block INT8 quantization of q, k, v),
+//   * the backward preprocess (D = rowsum(dO o O), dO quantized per q_block tokens, dQ
+//     accumulator cleared),
+//   * the dQ finalize (float32 dQ accumulator -> RMSNorm backward -> 16-bit dq).
+//
+// Row mapping: a row of d 16-bit values is read by d/8 consecutive lanes with one 128-bit load
+// each (lane l owns channels 8l .. 8l+7); a warp therefore covers 32/(d/8) rows per step.
+// Reductions inside a row are xor-butterflies over those lanes.
+//
+// The prologue's float32 operation order is part of its definition (its codes, scales,
+// inverse RMS values and K means are reproducible bit for bit):
+//   RMSNorm: per lane, p = 0; p = p + x_c * x_c over its 8 channels in ascending order; then
+//            p_l = p_l + p_(l xor o) for o = d/16, ..., 1; ss = p; inv = 1 / sqrt(ss/d + eps);
+//            xhat = x * inv;
+//   K mean:  per 64-token block, each channel summed over the block's tokens in ascending order
+//            from 0; block sums added in ascending block order from 0; m = S / N;
+//   quantize: s = absmax / 127, code = rint(x / s) (round half to even), s = 0 -> codes 0.
+// All operations use the _rn intrinsics, which the compiler never contracts into FMAs.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace sage {
+
+constexpr int kRowThreads = 256;  // 8 warps; a CTA handles 128 rows (16 per warp)
+constexpr int kRowsPerCta = 128;
+
+template <typename T>
+struct Cvt;
+
+template <>
+struct Cvt<__nv_bfloat16> {
+  static __device__ __forceinline__ void load8(const uint4& u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+  static __device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+};
+
+template <>
+struct Cvt<__half> {
+  static __device__ __forceinline__ void load8(const uint4& u, float (&f)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+      float2 t = __half22float2(h);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+  static __device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+};
+
+template <typename T>
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  return make_uint4(Cvt<T>::pack2(f[0], f[1]), Cvt<T>::pack2(f[2], f[3]),
+                    Cvt<T>::pack2(f[4], f[5]), Cvt<T>::pack2(f[6], f[7]));
+}
+
+// Butterfly sum across the LPR lanes that hold one row (mask = those lanes).
+template <int LPR>
+__device__ __forceinline__ float row_sum(float p, uint32_t mask) {
+#pragma unroll
+  for (int o = LPR / 2; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(mask, p, o));
+  return p;
+}
+
+// RMSNorm of the 8 values a lane holds (the row is spread over LPR lanes).  Returns inv.
+template <int D>
+__device__ __forceinline__ float rms_norm8(float (&x)[8], float eps, uint32_t mask) {
+  float p = 0.0f;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) p = __fadd_rn(p, __fmul_rn(x[c], x[c]));
+  const float ss = row_sum<D / 8>(p, mask);
+  const float ms = __fdiv_rn(ss, static_cast<float>(D));
+  const float r = __fsqrt_rn(__fadd_rn(ms, eps));
+  const float inv = __fdiv_rn(1.0f, r);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) x[c] = __fmul_rn(x[c], inv);
+  return inv;
+}
+
+// code = clamp(rint(x / s), -127, 127) as a byte (two's complement), 0 when s == 0.
+__device__ __forceinline__ uint32_t quant_code(float x, float s) {
+  if (!(s > 0.0f)) return 0u;
+  int c = __float2int_rn(__fdiv_rn(x, s));
+  c = max(-127, min(127, c));
+  return static_cast<uint32_t>(c) & 0xFFu;
+}
+
+__device__ __forceinline__ uint2 quant8(const float (&x)[8], float s) {
+  return make_uint2(pack4(quant_code(x[0], s), quant_code(x[1], s), quant_code(x[2], s),
+                          quant_code(x[3], s)),
+                    pack4(quant_code(x[4], s), quant_code(x[5], s), quant_code(x[6], s),
+                          quant_code(x[7], s)));
+}
+
+// ---------------------------------------------------------------------------------------------
+// Prologue pass 1 (only with K-smoothing): per 64-token block of k, the column sums of khat.
+// One group of D/8 lanes walks one block's 64 tokens in order.  partials: [BH * N/64, D].
+// ---------------------------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kRowThreads) prologue_kstats_kernel(
+    const T* __restrict__ k, float* __restrict__ partials, int total_blocks, int qknorm,
+    float eps) {
+  constexpr int LPR = D / 8, GPW = 32 / LPR;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = lane / LPR, sub = lane % LPR;
+  const int blk = (blockIdx.x * (kRowThreads / 32) + warp) * GPW + grp;
+  if (blk >= total_blocks) return;  // whole lane groups leave together
+  const uint32_t mask = ((LPR == 32) ? 0xFFFFFFFFu : ((1u << LPR) - 1u)) << (grp * LPR);
+  const T* src = k + static_cast<size_t>(blk) * 64 * D + sub * 8;
+  float c[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) c[i] = 0.0f;
+#pragma unroll 4
+  for (int t = 0; t < 64; ++t) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * D));
+    float x[8];
+    Cvt<T>::load8(u, x);
+    if (qknorm) rms_norm8<D>(x, eps, mask);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = __fadd_rn(c[i], x[i]);
+  }
+  float4* dst = reinterpret_cast<float4*>(partials + static_cast<size_t>(blk) * D + sub * 8);
+  dst[0] = make_float4(c[0], c[1], c[2], c[3]);
+  dst[1] = make_float4(c[4], c[5], c[6], c[7]);
+}
+
+// Prologue pass 2 (only with K-smoothing): m[bh][c] = (sum over blocks in order) / N.
+template <int D>
+__global__ void prologue_kmean_kernel(const float* __restrict__ partials,
+                                      float* __restrict__ k_mean, int nkb, int N) {
+  const int bh = blockIdx.x, c = threadIdx.x;
+  const float* src = partials + static_cast<size_t>(bh) * nkb * D + c;
+  float s = 0.0f;
+  for (int t = 0; t < nkb; ++t) s = __fadd_rn(s, src[static_cast<size_t>(t) * D]);
+  k_mean[static_cast<size_t>(bh) * D + c] = __fdiv_rn(s, static_cast<float>(N));
+}
+
+// Block absmax over the CTA's 128 rows: rows 0-63 are warps 0-3, rows 64-127 warps 4-7.
+// Returns the absmax of the block this thread's row belongs to (blocks of `blk` rows).
+__device__ __forceinline__ float block_absmax(float local, int blk, float* red) {
+  const int warp = threadIdx.x >> 5;
+  const float wm = warp_max(local);
+  if ((threadIdx.x & 31) == 0) red[warp] = wm;
+  __syncthreads();
+  float a = 0.0f;
+  if (blk == 128) {
+#pragma unroll
+    for (int w = 0; w < 8; ++w) a = fmaxf(a, red[w]);
+  } else {
+    const int w0 = (warp >> 2) << 2;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) a = fmaxf(a, red[w0 + w]);
+  }
+  return a;
+}
+
+struct PrologueArgs {
+  const void* src[3];      // q, k, v
+  int8_t* codes[3];        // q, k, v codes
+  float* scale[3];         // q, k, v scales
+  float* inv_rms[2];       // q, k
+  const float* k_mean;     // [BH, D] (ksmooth)
+  int BH, N, q_block, qknorm, ksmooth;
+  float eps;
+};
+
+// Prologue pass 3: one CTA per 128-token chunk of q, k or v (grid = 3 * BH * N/128):
+// RMSNorm (q, k), mean subtraction (k), block absmax and quantization.
+template <typename T, int D>
+__global__ void __launch_bounds__(kRowThreads) prologue_quant_kernel(PrologueArgs a) {
+  constexpr int LPR = D / 8, GPW = 32 / LPR, STEPS = 16 / GPW;
+  __shared__ float red[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = lane / LPR, sub = lane % LPR;
+  const uint32_t mask = ((LPR == 32) ? 0xFFFFFFFFu : ((1u << LPR) - 1u)) << (grp * LPR);
+  const int nchunk = a.N / kRowsPerCta;
+  const int per = a.BH * nchunk;
+  const int which = blockIdx.x / per;
+  const int rem = blockIdx.x % per;
+  const int bh = rem / nchunk, ch = rem % nchunk;
+  const size_t row0 = static_cast<size_t>(bh) * a.N + static_cast<size_t>(ch) * kRowsPerCta;
+  const T* src = reinterpret_cast<const T*>(a.src[which]);
+
+  float x[STEPS][8];
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int r = warp * 16 + s * GPW + grp;
+    const uint4 u =
+        __ldg(reinterpret_cast<const uint4*>(src + (row0 + r) * D + sub * 8));
+    Cvt<T>::load8(u, x[s]);
+  }
+  if (which < 2 && a.qknorm) {
+#pragma unroll
+    for (int s = 0; s < STEPS; ++s) {
+      const float inv = rms_norm8<D>(x[s], a.eps, mask);
+      const int r = warp * 16 + s * GPW + grp;
+      if (sub == 0) a.inv_rms[which][row0 + r] = inv;
+    }
+  }
+  if (which == 1 && a.ksmooth) {
+    const float4* mp =
+        reinterpret_cast<const float4*>(a.k_mean + static_cast<size_t>(bh) * D + sub * 8);
+    const float4 m0 = mp[0], m1 = mp[1];
+    const float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+    for (int s = 0; s < STEPS; ++s)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) x[s][c] = __fsub_rn(x[s][c], m[c]);
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) amax = fmaxf(amax, fabsf(x[s][c]));
+  const int blk = (which == 0) ? a.q_block : 64;
+  const float am = block_absmax(amax, blk, red);
+  const float sc = __fdiv_rn(am, 127.0f);
+  if (threadIdx.x == 0 || (blk == 64 && threadIdx.x == 128)) {
+    const int sub_blk = (blk == 64) ? (threadIdx.x >> 7) : 0;
+    const size_t idx = static_cast<size_t>(bh) * (a.N / blk) +
+                       static_cast<size_t>(ch) * (kRowsPerCta / blk) + sub_blk;
+    a.scale[which][idx] = sc;
+  }
+  int8_t* dst = a.codes[which];
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int r = warp * 16 + s * GPW + grp;
+    *reinterpret_cast<uint2*>(dst + (row0 + r) * D + sub * 8) = quant8(x[s], sc);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Backward preprocess: D_i = sum_c dO_ic O_ic (float32), dO codes per q_block tokens, and the
+// float32 dQ accumulator rows cleared.  One CTA per 128 rows.
+// ---------------------------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kRowThreads) bwd_preprocess_kernel(
+    const T* __restrict__ o, const T* __restrict__ dout, float* __restrict__ Dvec,
+    int8_t* __restrict__ do_codes, float* __restrict__ do_scale, float* __restrict__ dq_acc,
+    int N, int q_block) {
+  constexpr int LPR = D / 8, GPW = 32 / LPR, STEPS = 16 / GPW;
+  __shared__ float red[8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = lane / LPR, sub = lane % LPR;
+  const uint32_t mask = ((LPR == 32) ? 0xFFFFFFFFu : ((1u << LPR) - 1u)) << (grp * LPR);
+  const size_t row0 = static_cast<size_t>(blockIdx.x) * kRowsPerCta;
+  float x[STEPS][8];
+  float amax = 0.0f;
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int r = warp * 16 + s * GPW + grp;
+    const size_t off = (row0 + r) * D + sub * 8;
+    float y[8];
+    Cvt<T>::load8(__ldg(reinterpret_cast<const uint4*>(dout + off)), x[s]);
+    Cvt<T>::load8(__ldg(reinterpret_cast<const uint4*>(o + off)), y);
+    float p = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      p = fmaf(x[s][c], y[c], p);
+      amax = fmaxf(amax, fabsf(x[s][c]));
+    }
+    p = row_sum<LPR>(p, mask);
+    if (sub == 0) Dvec[row0 + r] = p;
+    float4* z = reinterpret_cast<float4*>(dq_acc + off);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const float am = block_absmax(amax, q_block, red);
+  const float sc = __fdiv_rn(am, 127.0f);
+  if (threadIdx.x == 0 || (q_block == 64 && threadIdx.x == 128))
+    do_scale[(row0 + (threadIdx.x >> 7) * 64) / q_block] = sc;
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int r = warp * 16 + s * GPW + grp;
+    *reinterpret_cast<uint2*>(do_codes + (row0 + r) * D + sub * 8) = quant8(x[s], sc);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// dQ finalize: dq = inv * (dqhat - qhat * (sum_c dqhat_c qhat_c) / d) when qknorm (RMSNorm
+// backward, qhat = q * inv recomputed in float32), else dq = dqhat; rounded to T.
+// ---------------------------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(kRowThreads) dq_finalize_kernel(
+    const float* __restrict__ dq_acc, const T* __restrict__ q, const float* __restrict__ inv_rms,
+    T* __restrict__ dq, int qknorm) {
+  constexpr int LPR = D / 8, GPW = 32 / LPR, STEPS = 16 / GPW;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = lane / LPR, sub = lane % LPR;
+  const uint32_t mask = ((LPR == 32) ? 0xFFFFFFFFu : ((1u << LPR) - 1u)) << (grp * LPR);
+  const size_t row0 = static_cast<size_t>(blockIdx.x) * kRowsPerCta;
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int r = warp * 16 + s * GPW + grp;
+    const size_t off = (row0 + r) * D + sub * 8;
+    const float4 g0 = *reinterpret_cast<const float4*>(dq_acc + off);
+    const float4 g1 = *reinterpret_cast<const float4*>(dq_acc + off + 4);
+    float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    if (qknorm) {
+      const float inv = inv_rms[row0 + r];
+      float xh[8];
+      Cvt<T>::load8(__ldg(reinterpret_cast<const uint4*>(q + off)), xh);
+      float p = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        xh[c] = __fmul_rn(xh[c], inv);
+        p = fmaf(g[c], xh[c], p);
+      }
+      const float dot = row_sum<LPR>(p, mask) * (1.0f / D);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) g[c] = inv * fmaf(-xh[c], dot, g[c]);
+    }
+    *reinterpret_cast<uint4*>(dq + off) = pack8<T>(g);
+  }
+}
+
+}  // namespace sage

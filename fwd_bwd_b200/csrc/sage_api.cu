@@ -1,0 +1,416 @@
+// sage_api.cu -- the C ABI of libsage (declared in include/sage.h): argument validation,
+// workspace layout, TMA tensor-map construction and kernel launches.  The whole library is one
+// translation unit so that every kernel shares the device status word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "sage.h"
+#include "attn_bwd.cuh"
+#include "attn_fwd.cuh"
+#include "debug_kernels.cuh"
+#include "ptx.cuh"
+#include "rowops.cuh"
+
+namespace {
+
+using sage::kRowThreads;
+using sage::kRowsPerCta;
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_params(const sage_params* p) {
+  if (!p) return SAGE_ERR_INVALID_ARG;
+  if (p->B <= 0 || p->H <= 0 || p->N <= 0 || p->d <= 0) return SAGE_ERR_INVALID_ARG;
+  if (p->dtype != SAGE_FP16 && p->dtype != SAGE_BF16) return SAGE_ERR_INVALID_ARG;
+  if (p->rms_eps < 0.0f || !std::isfinite(p->rms_eps)) return SAGE_ERR_INVALID_ARG;
+  if (!std::isfinite(p->softmax_scale)) return SAGE_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return SAGE_ERR_UNSUPPORTED;
+  if (p->k_block != 64) return SAGE_ERR_UNSUPPORTED;
+  if (p->q_block != 64 && p->q_block != 128) return SAGE_ERR_UNSUPPORTED;
+  if (p->N % 128 != 0) return SAGE_ERR_UNSUPPORTED;
+  // row indices of [B*H*N, d] tensors are passed to TMA as int32
+  if (static_cast<long long>(p->B) * p->H * p->N >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+float tau_of(const sage_params* p) {
+  return p->softmax_scale > 0.0f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(p->d));
+}
+
+int check_qbufs(const sage_params* p, const sage_qbufs* qb) {
+  if (!qb || !qb->q_codes || !qb->k_codes || !qb->v_codes || !qb->q_scale || !qb->k_scale ||
+      !qb->v_scale)
+    return SAGE_ERR_INVALID_ARG;
+  if (p->qknorm && (!qb->q_inv_rms || !qb->k_inv_rms)) return SAGE_ERR_INVALID_ARG;
+  if (p->ksmooth && !qb->k_mean) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(qb->q_codes) || !aligned16(qb->k_codes) || !aligned16(qb->v_codes))
+    return SAGE_ERR_ALIGNMENT;
+  if (qb->k_mean && !aligned16(qb->k_mean)) return SAGE_ERR_ALIGNMENT;
+  return SAGE_OK;
+}
+
+// ---- workspace layouts ------------------------------------------------------------------
+struct BwdWs {
+  size_t dvec, doc, dos, dq, total;
+};
+BwdWs bwd_ws(const sage_params* p) {
+  const size_t BH = static_cast<size_t>(p->B) * p->H, N = p->N, d = p->d;
+  BwdWs w;
+  w.dvec = 0;
+  w.doc = align_up(w.dvec + BH * N * 4);
+  w.dos = align_up(w.doc + BH * N * d);
+  w.dq = align_up(w.dos + BH * (N / p->q_block) * 4);
+  w.total = align_up(w.dq + BH * N * d * 4);
+  return w;
+}
+size_t prologue_ws(const sage_params* p) {
+  if (!p->ksmooth) return 0;
+  return align_up(static_cast<size_t>(p->B) * p->H * (p->N / 64) * p->d * 4);
+}
+
+// ---- TMA tensor maps --------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major [rows][inner] array of 1- or 2-byte elements.
+bool make_map(CUtensorMap* m, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
+              uint32_t box_inner, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const uint32_t row_bytes_box = box_inner * elem_bytes;
+  CUtensorMapSwizzle sw = row_bytes_box == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : row_bytes_box == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_32B;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * elem_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                  2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
+
+template <typename K>
+int set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(bytes)) == cudaSuccess
+             ? SAGE_OK
+             : SAGE_ERR_CUDA;
+}
+
+// ---- prologue ---------------------------------------------------------------------------
+template <typename T, int D>
+int run_prologue(const sage_params* p, const void* q, const void* k, const void* v,
+                 const sage_qbufs* out, void* ws, cudaStream_t st) {
+  const int BH = p->B * p->H, N = p->N;
+  if (p->ksmooth) {
+    float* partials = reinterpret_cast<float*>(ws);
+    const int total = BH * (N / 64);
+    const int per_cta = (kRowThreads / 32) * (32 / (D / 8));
+    sage::prologue_kstats_kernel<T, D><<<(total + per_cta - 1) / per_cta, kRowThreads, 0, st>>>(
+        reinterpret_cast<const T*>(k), partials, total, p->qknorm, p->rms_eps);
+    sage::prologue_kmean_kernel<D><<<BH, D, 0, st>>>(partials, out->k_mean, N / 64, N);
+  }
+  sage::PrologueArgs a;
+  a.src[0] = q;
+  a.src[1] = k;
+  a.src[2] = v;
+  a.codes[0] = out->q_codes;
+  a.codes[1] = out->k_codes;
+  a.codes[2] = out->v_codes;
+  a.scale[0] = out->q_scale;
+  a.scale[1] = out->k_scale;
+  a.scale[2] = out->v_scale;
+  a.inv_rms[0] = out->q_inv_rms;
+  a.inv_rms[1] = out->k_inv_rms;
+  a.k_mean = out->k_mean;
+  a.BH = BH;
+  a.N = N;
+  a.q_block = p->q_block;
+  a.qknorm = p->qknorm;
+  a.ksmooth = p->ksmooth;
+  a.eps = p->rms_eps;
+  sage::prologue_quant_kernel<T, D><<<3 * BH * (N / kRowsPerCta), kRowThreads, 0, st>>>(a);
+  return launch_status();
+}
+
+// ---- forward ----------------------------------------------------------------------------
+template <typename T, int D>
+int run_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse, cudaStream_t st) {
+  const int BH = p->B * p->H, N = p->N;
+  const uint64_t rows = static_cast<uint64_t>(BH) * N;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, qb->q_codes, 1, D, rows, D, sage::fwd::BM) ||
+      !make_map(&tk, qb->k_codes, 1, D, rows, D, sage::fwd::BKV) ||
+      !make_map(&tv, qb->v_codes, 1, D, rows, D, sage::fwd::BKV))
+    return SAGE_ERR_CUDA;
+  sage::fwd::Args a;
+  a.q_scale = qb->q_scale;
+  a.k_scale = qb->k_scale;
+  a.v_scale = qb->v_scale;
+  a.o = o;
+  a.lse = lse;
+  a.BH = BH;
+  a.N = N;
+  a.q_block = p->q_block;
+  a.causal = p->causal;
+  a.scale_log2 = tau_of(p) * 1.4426950408889634f;
+  a.nsup = (N + sage::fwd::NT * sage::fwd::BM - 1) / (sage::fwd::NT * sage::fwd::BM);
+  const size_t smem = sage::fwd::smem_bytes<D>();
+  auto kern = sage::fwd::attn_fwd_kernel<T, D>;
+  if (set_smem(kern, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+  kern<<<BH * a.nsup, sage::fwd::kThreads, smem, st>>>(tq, tk, tv, a);
+  return launch_status();
+}
+
+// ---- backward ---------------------------------------------------------------------------
+// stage 0: preprocess (D, dO codes, dQ accumulator cleared); 1: main tensor-core kernel;
+// 2: dq finalize.
+template <typename T, int D>
+int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const void* v,
+            const sage_qbufs* qb, const void* o, const float* lse, const void* dout, void* dq,
+            void* dk, void* dv, void* ws, cudaStream_t st) {
+  const int BH = p->B * p->H, N = p->N;
+  const uint64_t rows = static_cast<uint64_t>(BH) * N;
+  const BwdWs w = bwd_ws(p);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+  float* dvec = reinterpret_cast<float*>(wsb + w.dvec);
+  int8_t* doc = reinterpret_cast<int8_t*>(wsb + w.doc);
+  float* dos = reinterpret_cast<float*>(wsb + w.dos);
+  float* dqacc = reinterpret_cast<float*>(wsb + w.dq);
+  if (stage == 0) {
+    sage::bwd_preprocess_kernel<T, D>
+        <<<static_cast<int>(rows / kRowsPerCta), kRowThreads, 0, st>>>(
+            reinterpret_cast<const T*>(o), reinterpret_cast<const T*>(dout), dvec, doc, dos,
+            dqacc, N, p->q_block);
+    return launch_status();
+  }
+  if (stage == 2) {
+    sage::dq_finalize_kernel<T, D><<<static_cast<int>(rows / kRowsPerCta), kRowThreads, 0, st>>>(
+        dqacc, reinterpret_cast<const T*>(q), qb->q_inv_rms, reinterpret_cast<T*>(dq),
+        p->qknorm);
+    return launch_status();
+  }
+  CUtensorMap tqc, tkc, tdoc, tdo, tv;
+  if (!make_map(&tqc, qb->q_codes, 1, D, rows, D, sage::bwd::BQ) ||
+      !make_map(&tkc, qb->k_codes, 1, D, rows, D, sage::bwd::BKT) ||
+      !make_map(&tdoc, doc, 1, D, rows, D, sage::bwd::BQ) ||
+      !make_map(&tdo, dout, 2, D, rows, 64, sage::bwd::BQ) ||
+      !make_map(&tv, v, 2, D, rows, 64, sage::bwd::BKT))
+    return SAGE_ERR_CUDA;
+  sage::bwd::Args a;
+  a.q_scale = qb->q_scale;
+  a.k_scale = qb->k_scale;
+  a.do_scale = dos;
+  a.lse = lse;
+  a.dvec = dvec;
+  a.k_raw = k;
+  a.k_inv_rms = qb->k_inv_rms;
+  a.dq_acc = dqacc;
+  a.dk = dk;
+  a.dv = dv;
+  a.BH = BH;
+  a.N = N;
+  a.q_block = p->q_block;
+  a.causal = p->causal;
+  a.qknorm = p->qknorm;
+  a.tau = tau_of(p);
+  a.scale_log2 = a.tau * 1.4426950408889634f;
+  const size_t smem = sage::bwd::smem_bytes<D>();
+  auto kern = sage::bwd::attn_bwd_kernel<T, D>;
+  if (set_smem(kern, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+  kern<<<BH * (N / sage::bwd::BKT), sage::bwd::kThreads, smem, st>>>(tqc, tkc, tdoc, tdo, tv, a);
+  return launch_status();
+}
+
+int bwd_stage(int stage, const sage_params* p, const void* q, const void* k, const void* v,
+              const sage_qbufs* qb, const void* o, const float* lse, const void* dout, void* dq,
+              void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream) {
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if (stage < 0 || stage > 2) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_qbufs(p, qb)) != SAGE_OK) return s;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return SAGE_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return SAGE_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < bwd_ws(p).total) return SAGE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_bwd<__nv_bfloat16, 128>(stage, p, q, k, v, qb, o, lse, dout, dq, dk, dv,
+                                             workspace, st)
+              : run_bwd<__half, 128>(stage, p, q, k, v, qb, o, lse, dout, dq, dk, dv, workspace,
+                                     st);
+  return bf ? run_bwd<__nv_bfloat16, 64>(stage, p, q, k, v, qb, o, lse, dout, dq, dk, dv,
+                                          workspace, st)
+            : run_bwd<__half, 64>(stage, p, q, k, v, qb, o, lse, dout, dq, dk, dv, workspace, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sage_workspace_bytes(const sage_params* p, int which) {
+  if (check_params(p) != SAGE_OK) return 0;
+  if (which == 0) return prologue_ws(p);
+  if (which == 1) return 0;
+  if (which == 2) return bwd_ws(p).total;
+  return 0;
+}
+
+int sage_quant_prologue(const sage_params* p, const void* q, const void* k, const void* v,
+                        const sage_qbufs* out, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if (!q || !k || !v) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_qbufs(p, out)) != SAGE_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SAGE_ERR_ALIGNMENT;
+  const size_t need = prologue_ws(p);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return SAGE_ERR_WORKSPACE;
+  if (workspace && !aligned16(workspace)) return SAGE_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_prologue<__nv_bfloat16, 128>(p, q, k, v, out, workspace, st)
+              : run_prologue<__half, 128>(p, q, k, v, out, workspace, st);
+  return bf ? run_prologue<__nv_bfloat16, 64>(p, q, k, v, out, workspace, st)
+            : run_prologue<__half, 64>(p, q, k, v, out, workspace, st);
+}
+
+int sage_attn_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if ((s = check_qbufs(p, qb)) != SAGE_OK) return s;
+  if (!o || !lse) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(lse)) return SAGE_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_fwd<__nv_bfloat16, 128>(p, qb, o, lse, st)
+              : run_fwd<__half, 128>(p, qb, o, lse, st);
+  return bf ? run_fwd<__nv_bfloat16, 64>(p, qb, o, lse, st)
+            : run_fwd<__half, 64>(p, qb, o, lse, st);
+}
+
+int sage_attn_bwd(const sage_params* p, const void* q, const void* k, const void* v,
+                  const sage_qbufs* qb, const void* o, const float* lse, const void* dout,
+                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  for (int stage = 0; stage < 3; ++stage) {
+    const int s = bwd_stage(stage, p, q, k, v, qb, o, lse, dout, dq, dk, dv, workspace,
+                            workspace_bytes, stream);
+    if (s != SAGE_OK) return s;
+  }
+  return SAGE_OK;
+}
+
+int sage_attn_bwd_stage(int stage, const sage_params* p, const void* q, const void* k,
+                        const void* v, const sage_qbufs* qb, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  return bwd_stage(stage, p, q, k, v, qb, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
+                   stream);
+}
+
+int sage_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, sage::g_status, sizeof(int)) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(sage::g_status, &zero, sizeof(int)) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  return v;
+}
+
+const char* sage_status_string(int status) {
+  switch (status) {
+    case SAGE_OK: return "SAGE_OK";
+    case SAGE_ERR_INVALID_ARG: return "SAGE_ERR_INVALID_ARG";
+    case SAGE_ERR_UNSUPPORTED: return "SAGE_ERR_UNSUPPORTED";
+    case SAGE_ERR_ALIGNMENT: return "SAGE_ERR_ALIGNMENT";
+    case SAGE_ERR_WORKSPACE: return "SAGE_ERR_WORKSPACE";
+    case SAGE_ERR_CUDA: return "SAGE_ERR_CUDA";
+    case SAGE_ERR_TIMEOUT: return "SAGE_ERR_TIMEOUT";
+    default: return "SAGE_ERR_UNKNOWN";
+  }
+}
+
+int sage_debug_qk_int32(const sage_params* p, const sage_qbufs* qb, int bh, int q_tile,
+                        int32_t* s_out, void* stream) {
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if ((s = check_qbufs(p, qb)) != SAGE_OK) return s;
+  if (!s_out) return SAGE_ERR_INVALID_ARG;
+  if (bh < 0 || bh >= p->B * p->H || q_tile < 0 || q_tile >= p->N / 128)
+    return SAGE_ERR_INVALID_ARG;
+  const uint64_t rows = static_cast<uint64_t>(p->B) * p->H * p->N;
+  CUtensorMap tq, tk;
+  if (!make_map(&tq, qb->q_codes, 1, p->d, rows, p->d, 128) ||
+      !make_map(&tk, qb->k_codes, 1, p->d, rows, p->d, 64))
+    return SAGE_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (p->d == 128) {
+    const size_t smem = sizeof(sage::dbg::QkSmem<128>) + 1024;
+    if (set_smem(sage::dbg::debug_qk_kernel<128>, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+    sage::dbg::debug_qk_kernel<128><<<1, 128, smem, st>>>(tq, tk, bh, q_tile, p->N, s_out);
+  } else {
+    const size_t smem = sizeof(sage::dbg::QkSmem<64>) + 1024;
+    if (set_smem(sage::dbg::debug_qk_kernel<64>, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+    sage::dbg::debug_qk_kernel<64><<<1, 128, smem, st>>>(tq, tk, bh, q_tile, p->N, s_out);
+  }
+  return launch_status();
+}
+
+int sage_debug_umma_gemm(int kind, int a_mn_major, int b_mn_major, int N, int K, const void* A,
+                         const void* B, void* C, void* stream) {
+  if (kind < 0 || kind > 2 || !A || !B || !C) return SAGE_ERR_INVALID_ARG;
+  if ((N != 64 && N != 128) || (K != 64 && K != 128)) return SAGE_ERR_UNSUPPORTED;
+  if (kind != 0 && (a_mn_major || b_mn_major)) return SAGE_ERR_UNSUPPORTED;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return SAGE_ERR_ALIGNMENT;
+  const int M = 128;
+  CUtensorMap ta, tb;
+  bool ok;
+  if (kind == 0) {
+    ok = (a_mn_major ? make_map(&ta, A, 1, M, K, M, K) : make_map(&ta, A, 1, K, M, K, M)) &&
+         (b_mn_major ? make_map(&tb, B, 1, N, K, N, K) : make_map(&tb, B, 1, K, N, K, N));
+  } else {
+    ok = make_map(&ta, A, 2, K, M, 64, M) && make_map(&tb, B, 2, K, N, 64, N);
+  }
+  if (!ok) return SAGE_ERR_CUDA;
+  const size_t smem = sizeof(sage::dbg::GemmSmem) + 1024;
+  if (set_smem(sage::dbg::debug_gemm_kernel, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+  sage::dbg::debug_gemm_kernel<<<1, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+      ta, tb, kind, a_mn_major, b_mn_major, N, K, C);
+  return launch_status();
+}
+
+}  // extern "C"

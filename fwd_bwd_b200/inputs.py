@@ -7,7 +7,8 @@ or attention arithmetic.
 
 Recipe (the same for every workload):
 
-* ``numpy.random.Generator(PCG64(seed + offset))`` with offsets Q:0, K:1, V:2, dO:3, mu:4;
+* per flattened head ``bh``, ``numpy.random.Generator(PCG64(SeedSequence([seed, offset,
+  bh])))`` with offsets Q:0, K:1, V:2, dO:3, mu:4 (the K-outlier channel offsets);
 * ``standard_normal`` in float64, multiplied by the tensor's sigma, rounded to float32;
 * float32 rounded to the 16-bit storage type with round-half-to-even (bf16 by bit
   manipulation, fp16 by numpy's own RNE cast).
@@ -23,7 +24,7 @@ tokens-per-step sweep.
 from __future__ import annotations
 
 import dataclasses
-from typing import Dict, Optional
+from typing import Dict, Optional, Sequence
 
 import numpy as np
 
@@ -104,33 +105,40 @@ def f32_to_bits(x: np.ndarray, dtype: str) -> np.ndarray:
     raise ValueError(dtype)
 
 
-def _normal(seed: int, shape, sigma: float) -> np.ndarray:
-    g = np.random.Generator(np.random.PCG64(seed))
-    return (g.standard_normal(shape) * sigma).astype(np.float32)
+def _rng(w: Workload, offset: int, bh: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seed, offset, bh])))
 
 
-def make_inputs(w: Workload, heads: Optional[slice] = None) -> Dict[str, np.ndarray]:
-    """Return {'q','k','v','do'} as uint16 bit arrays [B,H,N,d] (and '<name>_f32' views).
-
-    ``heads`` restricts the result to a slice of the flattened (b, h) index; the values of the
-    kept heads are identical to those of the full draw (the full array is drawn, then sliced),
-    so a sampled head can be checked against the same head of a full-size GPU run.
-    """
-    shape = (w.B, w.H, w.N, w.d)
-    out: Dict[str, np.ndarray] = {}
-    q = _normal(w.seed + OFFSET_Q, shape, w.sigma_qkv)
-    k = _normal(w.seed + OFFSET_K, shape, w.sigma_qkv)
-    v = _normal(w.seed + OFFSET_V, shape, w.sigma_qkv)
-    do = _normal(w.seed + OFFSET_DO, shape, w.sigma_do)
+def make_head(w: Workload, bh: int) -> Dict[str, np.ndarray]:
+    """float32 values (before 16-bit rounding) of q, k, v, dO for flattened head ``bh``."""
+    shape = (w.N, w.d)
+    out = {}
+    for name, off, sig in (("q", OFFSET_Q, w.sigma_qkv), ("k", OFFSET_K, w.sigma_qkv),
+                           ("v", OFFSET_V, w.sigma_qkv), ("do", OFFSET_DO, w.sigma_do)):
+        out[name] = (_rng(w, off, bh).standard_normal(shape) * sig).astype(np.float32)
     if w.k_outlier:
-        g = np.random.Generator(np.random.PCG64(w.seed + OFFSET_MU))
-        mu = (g.standard_normal((w.B, w.H, 1, w.d)) * 4.0).astype(np.float32)
+        g = _rng(w, OFFSET_MU, bh)
+        mu = (g.standard_normal(w.d) * 4.0).astype(np.float32)
         chans = g.choice(w.d, size=4, replace=False)
-        mu[..., chans] += np.float32(20.0)
-        k = (k + mu).astype(np.float32)
-    for name, arr in (("q", q), ("k", k), ("v", v), ("do", do)):
-        if heads is not None:
-            arr = arr.reshape(w.B * w.H, w.N, w.d)[heads]
+        mu[chans] += np.float32(20.0)
+        out["k"] = (out["k"] + mu[None, :]).astype(np.float32)
+    return out
+
+
+def make_inputs(w: Workload, heads: Optional[Sequence[int]] = None) -> Dict[str, np.ndarray]:
+    """Return {'q','k','v','do'} as uint16 bit arrays and '<name>_f32' exact float32 views.
+
+    Each (batch, head) pair -- flattened index ``bh = b * H + h`` -- is drawn from its own
+    stream, so any subset of heads can be regenerated alone.  Without ``heads`` the arrays
+    are ``[B, H, N, d]``; with ``heads`` they are ``[len(heads), N, d]``.
+    """
+    idx = list(range(w.B * w.H)) if heads is None else list(heads)
+    parts = [make_head(w, bh) for bh in idx]
+    out: Dict[str, np.ndarray] = {}
+    for name in ("q", "k", "v", "do"):
+        arr = np.stack([p[name] for p in parts])
+        if heads is None:
+            arr = arr.reshape(w.B, w.H, w.N, w.d)
         bits = f32_to_bits(arr, w.dtype)
         out[name] = bits
         out[name + "_f32"] = bits_to_f32(bits, w.dtype)

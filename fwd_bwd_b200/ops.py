@@ -1,0 +1,212 @@
+"""PyTorch-facing binding of libsage: argument marshalling only.
+
+Every step of the computation runs in the CUDA kernels behind the C ABI; PyTorch provides the
+device memory (tensors) and the stream.  Names follow the C ABI: ``quant_prologue``,
+``attn_fwd``, ``attn_bwd``; ``sage_attention`` wraps the three in an autograd function.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import SageParams, SageQBufs, check, lib
+
+_DTYPES = {torch.float16: _lib.SAGE_FP16, torch.bfloat16: _lib.SAGE_BF16}
+
+
+@dataclasses.dataclass
+class Config:
+    """Problem flags shared by the three calls (see include/sage.h, ``sage_params``)."""
+
+    causal: bool = True
+    qknorm: bool = True
+    ksmooth: bool = True
+    q_block: int = 128
+    k_block: int = 64
+    softmax_scale: float = 0.0  # <= 0: 1/sqrt(d)
+    rms_eps: float = 1e-6
+
+    def params(self, x: torch.Tensor) -> SageParams:
+        B, H, N, d = x.shape
+        return SageParams(B, H, N, d, _DTYPES[x.dtype], int(self.causal), int(self.qknorm),
+                          int(self.ksmooth), self.q_block, self.k_block,
+                          float(self.softmax_scale), float(self.rms_eps))
+
+
+@dataclasses.dataclass
+class QuantBufs:
+    """Quantized views of Q, K, V (INT8 codes + per-block scales), reused by fwd and bwd."""
+
+    q_codes: torch.Tensor
+    k_codes: torch.Tensor
+    v_codes: torch.Tensor
+    q_scale: torch.Tensor
+    k_scale: torch.Tensor
+    v_scale: torch.Tensor
+    q_inv_rms: Optional[torch.Tensor]
+    k_inv_rms: Optional[torch.Tensor]
+    k_mean: Optional[torch.Tensor]
+
+    @staticmethod
+    def empty(shape, cfg: Config, device) -> "QuantBufs":
+        B, H, N, d = shape
+        f32 = dict(dtype=torch.float32, device=device)
+        i8 = dict(dtype=torch.int8, device=device)
+        return QuantBufs(
+            torch.empty(shape, **i8), torch.empty(shape, **i8), torch.empty(shape, **i8),
+            torch.empty((B, H, N // cfg.q_block), **f32),
+            torch.empty((B, H, N // cfg.k_block), **f32),
+            torch.empty((B, H, N // cfg.k_block), **f32),
+            torch.empty((B, H, N), **f32) if cfg.qknorm else None,
+            torch.empty((B, H, N), **f32) if cfg.qknorm else None,
+            torch.empty((B, H, d), **f32) if cfg.ksmooth else None)
+
+    def c_struct(self) -> SageQBufs:
+        p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        return SageQBufs(p(self.q_codes), p(self.k_codes), p(self.v_codes), p(self.q_scale),
+                         p(self.k_scale), p(self.v_scale), p(self.q_inv_rms),
+                         p(self.k_inv_rms), p(self.k_mean))
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_inputs(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("libsage works on CUDA tensors only")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, H, N, d]")
+
+
+def workspace_bytes(params: SageParams, which: int) -> int:
+    return int(lib().sage_workspace_bytes(ctypes.byref(params), which))
+
+
+def _workspace(params: SageParams, which: int, device) -> Tuple[Optional[torch.Tensor], int]:
+    n = workspace_bytes(params, which)
+    if n == 0:
+        return None, 0
+    return torch.empty(n, dtype=torch.uint8, device=device), n
+
+
+def quant_prologue(q, k, v, cfg: Config, out: Optional[QuantBufs] = None,
+                   workspace: Optional[torch.Tensor] = None) -> QuantBufs:
+    """QK-norm, K-smoothing and per-block INT8 quantization of q, k, v (sage_quant_prologue)."""
+    _check_inputs(q, k, v)
+    prm = cfg.params(q)
+    qb = out if out is not None else QuantBufs.empty(tuple(q.shape), cfg, q.device)
+    if workspace is None:
+        workspace, n = _workspace(prm, 0, q.device)
+    else:
+        n = workspace.numel()
+    st = qb.c_struct()
+    check("sage_quant_prologue", lib().sage_quant_prologue(
+        ctypes.byref(prm), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(st),
+        None if workspace is None else workspace.data_ptr(), n, _stream(q.device)))
+    return qb
+
+
+def attn_fwd(qb: QuantBufs, like: torch.Tensor, cfg: Config, o=None, lse=None):
+    """INT8 forward attention (sage_attn_fwd): returns (o, lse)."""
+    prm = cfg.params(like)
+    B, H, N, d = like.shape
+    if o is None:
+        o = torch.empty_like(like)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=like.device)
+    st = qb.c_struct()
+    check("sage_attn_fwd", lib().sage_attn_fwd(ctypes.byref(prm), ctypes.byref(st),
+                                               o.data_ptr(), lse.data_ptr(), None, 0,
+                                               _stream(like.device)))
+    return o, lse
+
+
+def attn_bwd(q, k, v, qb: QuantBufs, o, lse, dout, cfg: Config, dq=None, dk=None, dv=None,
+             workspace: Optional[torch.Tensor] = None, stage: Optional[int] = None):
+    """INT8 backward attention (sage_attn_bwd): returns (dq, dk, dv).
+
+    ``stage`` in {0, 1, 2} runs only that stage (sage_attn_bwd_stage); the caller then owns
+    ``workspace`` across the three calls.
+    """
+    _check_inputs(q, k, v, o, dout)
+    prm = cfg.params(q)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace, n = _workspace(prm, 2, q.device)
+    else:
+        n = workspace.numel()
+    st = qb.c_struct()
+    args = (ctypes.byref(prm), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(st),
+            o.data_ptr(), lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+            dv.data_ptr(), workspace.data_ptr(), n, _stream(q.device))
+    if stage is None:
+        check("sage_attn_bwd", lib().sage_attn_bwd(*args))
+    else:
+        check("sage_attn_bwd_stage", lib().sage_attn_bwd_stage(stage, *args))
+    return dq, dk, dv
+
+
+def device_status(device=None) -> int:
+    """Synchronize the current stream and read (and clear) the device status word."""
+    return int(lib().sage_last_device_status(_stream(device)))
+
+
+class _SageAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, cfg: Config):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        qb = quant_prologue(q, k, v, cfg)
+        o, lse = attn_fwd(qb, q, cfg)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.qb, ctx.cfg = qb, cfg
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = attn_bwd(q, k, v, ctx.qb, o, lse, do.contiguous(), ctx.cfg)
+        return dq, dk, dv, None
+
+
+def sage_attention(q, k, v, causal: bool = True, qknorm: bool = True, ksmooth: bool = True,
+                   q_block: int = 128, k_block: int = 64, softmax_scale: float = 0.0,
+                   rms_eps: float = 1e-6):
+    """SageBwd attention with autograd: q, k, v are CUDA [B, H, N, d] fp16/bf16 tensors."""
+    cfg = Config(causal, qknorm, ksmooth, q_block, k_block, softmax_scale, rms_eps)
+    return _SageAttention.apply(q, k, v, cfg)
+
+
+def umma_gemm_debug(kind: int, a: torch.Tensor, b: torch.Tensor, a_mn: bool, b_mn: bool,
+                    N: int, K: int) -> torch.Tensor:
+    """Run the tensor-core path on one 128 x N x K product (sage_debug_umma_gemm)."""
+    c = torch.empty((128, N), dtype=torch.int32 if kind == 0 else torch.float32,
+                    device=a.device)
+    check("sage_debug_umma_gemm", lib().sage_debug_umma_gemm(
+        kind, int(a_mn), int(b_mn), N, K, a.data_ptr(), b.data_ptr(), c.data_ptr(),
+        _stream(a.device)))
+    return c
+
+
+def qk_int32_debug(qb: QuantBufs, like: torch.Tensor, cfg: Config, bh: int,
+                   q_tile: int) -> torch.Tensor:
+    """INT8 score tile Qc Kc^T of the forward kernel's MMA path (sage_debug_qk_int32)."""
+    prm = cfg.params(like)
+    N = like.shape[2]
+    s = torch.empty((128, N), dtype=torch.int32, device=like.device)
+    st = qb.c_struct()
+    check("sage_debug_qk_int32", lib().sage_debug_qk_int32(
+        ctypes.byref(prm), ctypes.byref(st), bh, q_tile, s.data_ptr(), _stream(like.device)))
+    return s
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,143 @@
+/*
+ * sage.h -- C ABI of libsage: SageBwd quantized attention training on NVIDIA B200 (sm_100a).
+ *
+ * The operation ("SageBwd: trainable low-bit attention", aitrends.kr):
+ *   - QK-norm paragraph: every token vector of Q and K is RMS-normalized over the head dim;
+ *   - K-smoothing paragraph: a mean over tokens is subtracted from each channel of K right
+ *     before quantization;
+ *   - Triton-kernel paragraph: Q, K, V (and P, dS, dO) are quantized to INT8 per block;
+ *   - quantization-strategy paragraph: six of the seven attention matmuls run in INT8
+ *     (S = Q K^T forward and recomputed, O = P V, dV = P^T dO, dQ = dS K, dK = dS^T Q); only
+ *     dP = dO V^T runs in 16-bit float, being the most error-sensitive;
+ *   - error-propagation paragraph: dQ = dS K and dK = dS^T Q carry the quantization error of dS.
+ *
+ * Conventions shared by every entry point
+ *   Layout     All tensors are contiguous [B, H, N, d] with d innermost; per-block scales are
+ *              [B, H, N / block]; per-token vectors [B, H, N]; K means [B, H, d].
+ *   Pointers   Every pointer is a DEVICE pointer, allocated and owned by the caller; the
+ *              library never allocates, frees or retains memory.  Tensor pointers must be
+ *              16-byte aligned.  Work is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *              legacy default stream); buffers must stay valid until the stream reaches it.
+ *   Shapes     d in {64, 128}; k_block == 64; q_block in {64, 128}; N a multiple of 128.
+ *   Errors     Argument errors return a negative sage_status synchronously and launch nothing.
+ *              A failed launch returns SAGE_ERR_CUDA.  Kernels never trap: a device-side wait
+ *              that exceeds its time limit records SAGE_ERR_TIMEOUT in a status word that
+ *              sage_last_device_status() reads.  No C++ exception crosses this boundary.
+ *   Threads    Calls are thread-safe as far as the CUDA runtime is; calls that share output
+ *              or workspace buffers must be ordered by the caller.
+ */
+#ifndef SAGE_H_
+#define SAGE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, inconsistent parameters   */
+  SAGE_ERR_UNSUPPORTED = -2, /* valid but unimplemented shape (d, block sizes, N)          */
+  SAGE_ERR_ALIGNMENT = -3,   /* a tensor pointer is not 16-byte aligned                    */
+  SAGE_ERR_WORKSPACE = -4,   /* workspace missing or smaller than sage_workspace_bytes()   */
+  SAGE_ERR_CUDA = -5,        /* a CUDA runtime / driver call failed                        */
+  SAGE_ERR_TIMEOUT = -6      /* a kernel gave up waiting on a barrier (device status only) */
+} sage_status;
+
+typedef enum { SAGE_FP16 = 0, SAGE_BF16 = 1 } sage_dtype;
+
+/* Problem description.  softmax_scale <= 0 selects 1/sqrt(d); rms_eps is the RMSNorm epsilon
+ * (the page gives none; 1e-6 is the library's default in its bindings). */
+typedef struct {
+  int B, H, N, d;
+  int dtype;   /* sage_dtype of q, k, v, o, dout, dq, dk, dv                          */
+  int causal;  /* 1: key j visible to query i iff j <= i (square, top-left aligned)   */
+  int qknorm;  /* 1: per-token RMSNorm of q and k before quantization                 */
+  int ksmooth; /* 1: subtract the per-channel mean over tokens from k before quant.   */
+  int q_block; /* tokens per Q (and dO) quantization block: 64 or 128                 */
+  int k_block; /* tokens per K and V quantization block: 64                           */
+  float softmax_scale;
+  float rms_eps;
+} sage_params;
+
+/* Quantized views of Q, K, V produced once by the prologue and read by both the forward and
+ * the backward pass.  Codes are int8 in [-127, 127]; scale = absmax / 127 of the block. */
+typedef struct {
+  int8_t *q_codes, *k_codes, *v_codes; /* [B,H,N,d]                                        */
+  float *q_scale;                      /* [B,H,N/q_block]                                  */
+  float *k_scale, *v_scale;            /* [B,H,N/k_block]                                  */
+  float *q_inv_rms, *k_inv_rms;        /* [B,H,N]; written when qknorm (else unused, may be
+                                          NULL)                                            */
+  float *k_mean;                       /* [B,H,d]; written when ksmooth (else may be NULL) */
+} sage_qbufs;
+
+/* Bytes of scratch each call needs: which = 0 prologue, 1 forward, 2 backward.  Returns 0 for
+ * invalid parameters.  The scratch is caller-owned device memory, 256-byte aligned. */
+size_t sage_workspace_bytes(const sage_params* p, int which);
+
+/* Prologue (QK-norm, K-smoothing and quantization paragraphs).  In float32:
+ *   qknorm:  inv = 1/sqrt(sum(x^2)/d + eps), xhat = x * inv for every token of q and k;
+ *   ksmooth: m_c = (sum over all N tokens of khat_c) / N, ktilde = khat - m;
+ *   quantize: per block of q_block (q) or k_block (k, v) tokens spanning all d channels,
+ *            s = absmax/127, code = round-half-even(x / s); s = 0 and codes 0 if absmax = 0.
+ * The float32 operation order is fixed, so codes, scales, inv_rms and k_mean are
+ * reproducible bit for bit.  q, k, v: 16-bit inputs [B,H,N,d].  out: all buffers written. */
+int sage_quant_prologue(const sage_params* p, const void* q, const void* k, const void* v,
+                        const sage_qbufs* out, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Forward attention with INT8 S = Qc Kc^T and O = Pc Vc (quantization-strategy paragraph).
+ * z = A * sQ * sK * softmax_scale; P is quantized with one scale per (query row, K block);
+ * o: [B,H,N,d] in dtype; lse: [B,H,N] float32, natural log-sum-exp of the scaled scores. */
+int sage_attn_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward attention (quantization-strategy and error-propagation paragraphs): recomputes the
+ * INT8 scores from the same codes, dP = dO V^T in 16-bit float with float32 accumulation,
+ * dS = P (dP - rowsum(dO o O)), P and dS quantized per q_block x k_block tile, dO per q_block
+ * tokens; dV = P^T dO, dK = dS^T Q, dQ = dS K in INT8.  q, k, v are the raw 16-bit inputs
+ * (needed for dP and the RMSNorm backward); o, lse the forward's outputs; dout = dL/do.
+ * dq, dk, dv: [B,H,N,d] in dtype, gradients with respect to the raw q, k, v. */
+int sage_attn_bwd(const sage_params* p, const void* q, const void* k, const void* v,
+                  const sage_qbufs* qb, const void* o, const float* lse, const void* dout,
+                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/* The three stages sage_attn_bwd runs, for callers that schedule or time them separately;
+ * same arguments as sage_attn_bwd, and they must run in order on the same workspace:
+ *   stage 0  preprocess: D_i = sum_c dO_ic O_ic, dO quantized per q_block tokens, the float32
+ *            dQ accumulator (in the workspace) cleared;
+ *   stage 1  the tensor-core kernel: dk and dv written, dQ accumulated in the workspace;
+ *   stage 2  dq from the accumulator (with the RMSNorm backward when qknorm).
+ * Returns SAGE_ERR_INVALID_ARG for any other stage. */
+int sage_attn_bwd_stage(int stage, const sage_params* p, const void* q, const void* k,
+                        const void* v, const sage_qbufs* qb, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* Synchronizes `stream`, returns the device status word of the current device (SAGE_OK or
+ * SAGE_ERR_TIMEOUT) and clears it.  Returns SAGE_ERR_CUDA if the synchronization fails. */
+int sage_last_device_status(void* stream);
+
+/* Human-readable name of a sage_status value (static storage). */
+const char* sage_status_string(int status);
+
+/* ---- test support: run single pieces of the kernels' tensor-core path ---------------------
+ * sage_debug_qk_int32: the forward kernel's INT8 score product for one head `bh` and one tile
+ *   of 128 queries `q_tile`, against all N keys: s_out[128][N] int32 = Qc Kc^T, computed by
+ *   the same shared-memory staging and tcgen05 MMA code as the forward kernel.
+ * sage_debug_umma_gemm: C[M][N] = A B with M = 128, N and K in {64, 128}.
+ *   kind 0: int8 x int8 -> int32; kind 1: fp16 -> fp32; kind 2: bf16 -> fp32 (K-major only).
+ *   a_mn_major = 0: A stored [M][K]; 1: A stored [K][M].  b_mn_major = 0: B stored [N][K];
+ *   1: B stored [K][N].  All pointers are device pointers; C is row-major [M][N]. */
+int sage_debug_qk_int32(const sage_params* p, const sage_qbufs* qb, int bh, int q_tile,
+                        int32_t* s_out, void* stream);
+int sage_debug_umma_gemm(int kind, int a_mn_major, int b_mn_major, int N, int K, const void* A,
+                         const void* B, void* C, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SAGE_H_ */

@@ -1,0 +1,100 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol the
+header declares, sizes workspaces, names status codes and rejects bad arguments before any
+CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fwd_bwd_b200 import _lib
+from fwd_bwd_b200._lib import SageParams, SageQBufs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    import fwd_bwd_b200.build as b
+
+    b.build()
+    return _lib.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "sage.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sage_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) == 9
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def _params(**kw):
+    p = dict(B=2, H=4, N=1024, d=128, dtype=1, causal=1, qknorm=1, ksmooth=1, q_block=128,
+             k_block=64, softmax_scale=0.0, rms_eps=1e-6)
+    p.update(kw)
+    return SageParams(**p)
+
+
+def test_workspace_sizes(L):
+    p = _params()
+    BH, N, d = 8, 1024, 128
+    assert L.sage_workspace_bytes(ctypes.byref(p), 0) == BH * (N // 64) * d * 4
+    assert L.sage_workspace_bytes(ctypes.byref(p), 1) == 0
+    bwd = L.sage_workspace_bytes(ctypes.byref(p), 2)
+    assert bwd >= BH * N * (4 + d + 4 * d)
+    p0 = _params(ksmooth=0)
+    assert L.sage_workspace_bytes(ctypes.byref(p0), 0) == 0
+    assert L.sage_workspace_bytes(ctypes.byref(_params(d=96)), 2) == 0
+
+
+def test_status_strings(L):
+    for code, name in ((0, "SAGE_OK"), (-1, "SAGE_ERR_INVALID_ARG"), (-6, "SAGE_ERR_TIMEOUT")):
+        assert _lib.status_string(code) == name
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), _lib.SAGE_ERR_UNSUPPORTED),
+    (dict(N=200), _lib.SAGE_ERR_UNSUPPORTED),
+    (dict(k_block=128), _lib.SAGE_ERR_UNSUPPORTED),
+    (dict(q_block=32), _lib.SAGE_ERR_UNSUPPORTED),
+    (dict(B=0), _lib.SAGE_ERR_INVALID_ARG),
+    (dict(dtype=7), _lib.SAGE_ERR_INVALID_ARG),
+    (dict(rms_eps=-1.0), _lib.SAGE_ERR_INVALID_ARG),
+])
+def test_bad_params_rejected_without_launch(L, kw, code):
+    p = _params(**kw)
+    qb = SageQBufs(*([16] * 9))
+    assert L.sage_quant_prologue(ctypes.byref(p), 16, 16, 16, ctypes.byref(qb), 16, 1 << 40,
+                                 None) == code
+    assert L.sage_attn_fwd(ctypes.byref(p), ctypes.byref(qb), 16, 16, None, 0, None) == code
+
+
+def test_null_and_misaligned_pointers_rejected(L):
+    p = _params()
+    qb = SageQBufs(*([16] * 9))
+    assert L.sage_quant_prologue(ctypes.byref(p), None, 16, 16, ctypes.byref(qb), 16, 1 << 40,
+                                 None) == _lib.SAGE_ERR_INVALID_ARG
+    assert L.sage_quant_prologue(ctypes.byref(p), 18, 16, 16, ctypes.byref(qb), 16, 1 << 40,
+                                 None) == _lib.SAGE_ERR_ALIGNMENT
+    bad = SageQBufs(*([16] * 6 + [None, 16, 16]))  # qknorm needs q_inv_rms
+    assert L.sage_attn_fwd(ctypes.byref(p), ctypes.byref(bad), 16, 16, None, 0,
+                           None) == _lib.SAGE_ERR_INVALID_ARG
+    assert L.sage_quant_prologue(ctypes.byref(p), 16, 16, 16, ctypes.byref(qb), 16, 100,
+                                 None) == _lib.SAGE_ERR_WORKSPACE
+    assert L.sage_attn_bwd(ctypes.byref(p), 16, 16, 16, ctypes.byref(qb), 16, 16, 16, 16, 16,
+                           16, 16, 1, None) == _lib.SAGE_ERR_WORKSPACE
+
+
+def test_debug_entry_validation(L):
+    assert L.sage_debug_umma_gemm(0, 0, 0, 96, 64, 16, 16, 16, None) == \
+        _lib.SAGE_ERR_UNSUPPORTED
+    assert L.sage_debug_umma_gemm(1, 1, 0, 64, 64, 16, 16, 16, None) == \
+        _lib.SAGE_ERR_UNSUPPORTED
+    assert L.sage_debug_umma_gemm(0, 0, 0, 64, 64, None, 16, 16, None) == \
+        _lib.SAGE_ERR_INVALID_ARG
