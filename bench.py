@@ -37,6 +37,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="sage", choices=["sage", "reference"])
     ap.add_argument("--workload", default="sweep8192")
+    ap.add_argument("--B", type=int, default=0, help="override the batch (small profiling runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -158,6 +159,8 @@ def main():
     from fwd_bwd_b200.inputs import WORKLOADS
 
     w = WORKLOADS[args.workload]
+    if args.B > 0:
+        w = w.replace(B=args.B)
     if args.impl == "reference":
         run_reference(args, w)
         return

@@ -72,8 +72,29 @@ def test_backward_matches_oracle(case, results):
 
 @pytest.mark.parametrize("case", sorted(CASES))
 def test_cosine_vs_full_precision(case, results):
-    w, g, _, x = _run(case, results)
+    """cosine >= 0.995 vs float64 attention for the recipe as specified (K-smoothing on).
+
+    The K-smoothing ablation on K-outlier inputs (smoothing off) is where the page reports the
+    recipe degrading; there the GPU must reproduce the oracle's own (lower) cosine.
+    """
+    w, g, o, x = _run(case, results)
     BH = w.B * w.H
     for n in ("o", "dq", "dk", "dv"):
         c = cosine(g[n].reshape(BH, w.N, w.d), x[n])
-        assert c >= TOL_COS, (n, c)
+        if w.ksmooth or not w.k_outlier:
+            assert c >= TOL_COS, (n, c)
+        else:
+            assert abs(c - cosine(o[n], x[n])) <= 1e-3, (n, c)
+
+
+def test_k_smoothing_ablation_trend(results):
+    """With channel outliers in K, turning K-smoothing off lowers the dQ cosine vs float64
+    (K-smoothing paragraph and ablation of the SageBwd page), on the GPU as in the oracle."""
+    for norm in ("on", "off"):
+        on_case = "koutlier_on_on" if norm == "on" else "koutlier_norm_off"
+        off_case = "koutlier_smooth_off" if norm == "on" else "koutlier_off_off"
+        cs = {}
+        for case in (on_case, off_case):
+            w, g, _, x = _run(case, results)
+            cs[case] = cosine(g["dq"].reshape(w.B * w.H, w.N, w.d), x["dq"])
+        assert cs[on_case] > cs[off_case] + 0.01, cs

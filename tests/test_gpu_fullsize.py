@@ -1,0 +1,67 @@
+"""Parity at the full BASELINE sizes, in the launch configuration bench.py times.
+
+The whole batch runs on the GPU; a few sampled (batch, head) pairs carry inputs from the seeded
+per-head numpy streams (the rest are filled on the device) and are checked against the oracle
+one head at a time -- every head is an independent problem, so a head's outputs depend on that
+head's inputs only.  Gates as in test_gpu_attention: prologue bit-exact, rel-L2 <= 2e-3 on O,
+dQ, dK, dV, |dLSE| <= 1e-3, cosine >= 0.995 vs float64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.sage_oracle as O
+from fwd_bwd_b200 import ops
+from fwd_bwd_b200.inputs import WORKLOADS, make_inputs
+
+from gpu_helpers import TORCH_DT, cfg_of, cosine, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "sweep8192": [0, 511],      # the bench workload: B32 H16 N8192 d128 causal
+    "llama325m": [0, 127],      # B8 H16 N2048 d64 causal
+    "long16k": [31],            # B1 H32 N16384 d128 causal, dO sigma 1e-4
+    "koutlier": [5],            # B4 H16 N4096 d128 causal, K outliers
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_full_size_sampled_heads(name):
+    w = WORKLOADS[name]
+    heads = CASES[name]
+    dev = torch.device("cuda")
+    dt = TORCH_DT[w.dtype]
+    g = torch.Generator(device=dev).manual_seed(1)
+    shape = (w.B * w.H, w.N, w.d)
+    t = {n: (torch.randn(shape, generator=g, device=dev) *
+             (w.sigma_do if n == "do" else w.sigma_qkv)).to(dt) for n in ("q", "k", "v", "do")}
+    x = make_inputs(w, heads=heads)
+    for n in ("q", "k", "v", "do"):
+        for i, bh in enumerate(heads):
+            t[n][bh] = torch.from_numpy(x[n][i].view(np.int16)).view(dt).to(dev)
+    q, k, v, do = (t[n].view(w.B, w.H, w.N, w.d) for n in ("q", "k", "v", "do"))
+    cfg = cfg_of(w)
+    qb = ops.quant_prologue(q, k, v, cfg)
+    o, lse = ops.attn_fwd(qb, q, cfg)
+    dq, dk, dv = ops.attn_bwd(q, k, v, qb, o, lse, do, cfg)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    args = [x[n + "_f32"] for n in ("q", "k", "v", "do")]
+    kw = dict(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth, q_block=w.q_block,
+              k_block=w.k_block, dtype=w.dtype)
+    ref = O.sage_attention(*args, **kw)
+    full = O.sage_attention(*args, quant=False, round_outputs=False, **kw)
+    flat = lambda a: a.reshape(w.B * w.H, *a.shape[2:])  # noqa: E731
+    for i, bh in enumerate(heads):
+        for n in ("q_codes", "k_codes", "v_codes"):
+            assert torch.equal(flat(getattr(qb, n))[bh].cpu(), torch.from_numpy(ref[n][i])), n
+        for n in ("q_scale", "k_scale", "v_scale"):
+            assert np.array_equal(flat(getattr(qb, n))[bh].cpu().numpy().view(np.uint32),
+                                  ref[n][i].view(np.uint32)), n
+        got = {"o": o, "dq": dq, "dk": dk, "dv": dv}
+        for n, tt in got.items():
+            a = flat(tt)[bh].float().cpu().numpy()
+            assert rel_l2(a, ref[n][i]) <= 2e-3, (n, bh, rel_l2(a, ref[n][i]))
+            assert cosine(a, full[n][i]) >= 0.995, (n, bh)
+        assert np.abs(flat(lse)[bh].cpu().numpy() - ref["lse"][i]).max() <= 1e-3
