@@ -54,6 +54,22 @@ def peaks():
             "basis": "fallback"}
 
 
+def traffic_per_launch(kernel: str, src: str):
+    """DRAM bytes per full launch from profiles/traffic.txt, if the kernel source still matches
+    the one the counters were taken on (else None)."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:16]
+    for line in open(path):
+        f = line.split()
+        if len(f) >= 3 and f[0] == kernel and f[1] == sha:
+            return float(f[2]) * 1e9
+    return None
+
+
 def weighted_peak(p_bf16: float, n_i8: int, n_f16: int) -> float:
     """Peak of a mix of equal-size INT8 and 16-bit GEMMs (INT8 at twice the bf16 rate)."""
     p_i8 = 2.0 * p_bf16
@@ -293,9 +309,12 @@ def main():
     }
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
     kd = kernels[dom]
+    src = {"attn_bwd_kernel": "fwd_bwd_b200/csrc/attn_bwd.cuh",
+           "attn_fwd_kernel": "fwd_bwd_b200/csrc/attn_fwd.cuh"}[dom]
+    traffic = traffic_per_launch(dom, src) if w.name == "sweep8192" and w.B == 32 else None
     roofline = {"bound": "tensor", "kernel": dom, "achieved": kd["achieved"],
                 "peak": kd["peak"], "unit": "TFLOP/s", "frac": kd["achieved"] / kd["peak"],
-                "traffic": None,
+                "traffic": traffic,
                 "peak_note": f"{basis} sustained bf16 x (INT8 = 2x bf16), weighted by the "
                              f"kernel's INT8:16-bit GEMM mix"}
 
