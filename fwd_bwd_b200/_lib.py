@@ -58,6 +58,8 @@ def lib() -> ctypes.CDLL:
         L.sage_workspace_bytes.restype = sz
         L.sage_quant_prologue.argtypes = [P(SageParams), vp, vp, vp, P(SageQBufs), vp, sz, vp]
         L.sage_quant_prologue.restype = i
+        L.sage_quant_prologue_noalloc.argtypes = [P(SageParams), vp, vp, vp, P(SageQBufs), vp]
+        L.sage_quant_prologue_noalloc.restype = i
         L.sage_attn_fwd.argtypes = [P(SageParams), P(SageQBufs), vp, vp, vp, sz, vp]
         L.sage_attn_fwd.restype = i
         L.sage_attn_bwd.argtypes = [P(SageParams), vp, vp, vp, P(SageQBufs), vp, vp, vp, vp,

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "sage.h"
 #include "attn_bwd.cuh"
@@ -271,6 +272,33 @@ int bwd_stage(int stage, const sage_params* p, const void* q, const void* k, con
             : run_bwd<__half, 64>(stage, p, q, k, v, qb, o, lse, dout, dq, dk, dv, workspace, st);
 }
 
+// ---- prologue scratch for callers that cannot allocate -------------------------------------
+// A fixed device array that sage_quant_prologue_noalloc uses instead of a caller workspace for
+// the K-smoothing column sums.  Every device that loads the library holds it until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device.  In
+// host code the array's name is only a host-side stand-in, so kernels must be given this
+// address instead.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SAGE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return SAGE_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SAGE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -301,6 +329,26 @@ int sage_quant_prologue(const sage_params* p, const void* q, const void* k, cons
               : run_prologue<__half, 128>(p, q, k, v, out, workspace, st);
   return bf ? run_prologue<__nv_bfloat16, 64>(p, q, k, v, out, workspace, st)
             : run_prologue<__half, 64>(p, q, k, v, out, workspace, st);
+}
+
+int sage_quant_prologue_noalloc(const sage_params* p, const void* q, const void* k,
+                                const void* v, const sage_qbufs* out, void* stream) {
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if (!q || !k || !v) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_qbufs(p, out)) != SAGE_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SAGE_ERR_ALIGNMENT;
+  const size_t need = prologue_ws(p);
+  if (need > kNoAllocScratchBytes) return SAGE_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (need > 0 && (s = noalloc_scratch(&ws)) != SAGE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_prologue<__nv_bfloat16, 128>(p, q, k, v, out, ws, st)
+              : run_prologue<__half, 128>(p, q, k, v, out, ws, st);
+  return bf ? run_prologue<__nv_bfloat16, 64>(p, q, k, v, out, ws, st)
+            : run_prologue<__half, 64>(p, q, k, v, out, ws, st);
 }
 
 int sage_attn_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse,

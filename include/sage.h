@@ -88,6 +88,25 @@ int sage_quant_prologue(const sage_params* p, const void* q, const void* k, cons
                         const sage_qbufs* out, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/* sage_quant_prologue for callers that cannot allocate device memory.  (The SageBwd page has
+ * no counterpart: this is a deployment variant of the prologue, not part of the method.)
+ * Some callers cannot call cudaMalloc: code embedded in a host runtime that owns every device
+ * allocation through its own memory pool, code running under a fixed device-memory budget set
+ * at start-up, and latency-critical host threads that must not risk the device-wide
+ * synchronization cudaMalloc / cudaFree can cause.  This entry point takes no workspace: the
+ * K-smoothing column sums go to a fixed 32 MiB array in the library's own device memory (every
+ * GPU that loads the library holds it until exit), so it supports shapes with
+ * B * H * (N / 64) * d * 4 <= 32 MiB (e.g. B*H*N*d up to 2^29 elements) and returns
+ * SAGE_ERR_WORKSPACE beyond that, before launching anything.  Everything else -- arguments,
+ * outputs, results (bit for bit) -- is as for sage_quant_prologue.  It allocates nothing.
+ * The first call on each device looks up the array's device address (with that device
+ * current); make that first call before any stream capture.  All calls share the one array,
+ * which keeps the last call's contents; every value a call reads from it is written by that
+ * same call first, so nothing needs clearing, but calls whose kernels overlap on the GPU (on
+ * different streams) race on it and must be ordered by the caller. */
+int sage_quant_prologue_noalloc(const sage_params* p, const void* q, const void* k,
+                                const void* v, const sage_qbufs* out, void* stream);
+
 /* Forward attention with INT8 S = Qc Kc^T and O = Pc Vc (quantization-strategy paragraph).
  * z = A * sQ * sK * softmax_scale; P is quantized with one scale per (query row, K block);
  * o: [B,H,N,d] in dtype; lse: [B,H,N] float32, natural log-sum-exp of the scaled scores. */
