@@ -11,13 +11,18 @@
 //      128-byte swizzled layout, which the tensor core reads K-major (for dQ) and MN-major
 //      (for dV, dK);
 //   3. dV_t = Pc^T dOc and dK_t = dSc^T Qc (kind::i8, M = 128 keys, one per q_block group),
-//      dequantized by the tile scales and added to float32 accumulators held in TMEM;
+//      dequantized by the tile scales and added to float32 accumulators in registers;
 //   4. dQ_t = dSc Kc per 64-key block (kind::i8), dequantized, summed and added to a float32
 //      dQ accumulator in global memory with vector atomics.
-// Warps 0-7 compute (warpgroup h owns keys 64h .. 64h+63 in steps 2 and d columns
-// h*d/2 .. in steps 3-4), warp 8 is the TMA producer, warp 9 the MMA issuer.
-// TMEM (512 columns): [0,128) S -> P -> dV_t -> dQ_t(block 0); [128,256) dP -> dS -> dK_t ->
-// dQ_t(block 1); [256, 256+d) dV accumulator; [256+d, 256+2d) dK accumulator.
+// S and dP are double-buffered in TMEM, so the tensor core computes them for query tile i+1
+// while the compute warps turn tile i into codes.
+//
+// Warps 0-7 compute (warpgroup h owns keys 64h .. 64h+63 in step 2 and d columns h*d/2 ..
+// in steps 3-4), warp 8 is the TMA producer, warp 9 the MMA issuer, warps 10-11 idle.  The
+// producer warpgroup gives registers to the compute warpgroups (setmaxnreg): at launch every
+// thread holds 168, afterwards 256 x 232 + 128 x 40 = 64512 = 384 x 168.
+// TMEM (512 columns): buffer b in {0,1} at [256b, 256b+256): [0,128) S -> P -> dV_t ->
+// dQ_t(block 0); [128,256) dP -> dS -> dK_t -> dQ_t(block 1).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -32,8 +37,13 @@ namespace bwd {
 
 constexpr int BQ = 128;   // query rows per tile
 constexpr int BKT = 128;  // keys per CTA
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kLaunchRegs = 168;   // registers per thread the kernel must be launched with
+constexpr int kComputeRegs = 232;  // compute warpgroups after setmaxnreg.inc
+constexpr int kOtherRegs = 40;     // producer / MMA warpgroup after setmaxnreg.dec
+static_assert(2 * 128 * kComputeRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 
 template <typename T>
 struct IsBf16 {
@@ -59,10 +69,10 @@ struct Smem {
   int8_t pc[BQ * BKT];     // P codes  [128 q][128 keys], 128-byte swizzle
   int8_t dsc[BQ * BKT];    // dS codes [128 q][128 keys], 128-byte swizzle
   float red_p[8], red_ds[8];
-  float sp[2][2], sds[2][2];  // tile scales [q group][key half]
-  float dot[BKT];             // RMSNorm-backward row dot products (warpgroup 1 -> 0)
+  float sp[2][2][2], sds[2][2][2];  // tile scales [tile parity][q group][key half]
+  float dot[BKT];                   // RMSNorm-backward row dot products (warpgroup 1 -> 0)
   uint64_t kv_full, q_full[2], q_empty[2];
-  uint64_t sdp_full, pds_ready, dvdk_full, dvdk_free, dq_full, dq_free;
+  uint64_t sdp_full[2], pds_ready, dvdk_full, dvdk_free, dq_full, dq_free;
   uint32_t tmem_base;
   int abort;
 };
@@ -94,6 +104,13 @@ __device__ __forceinline__ Smem<D>& smem_ref(uint8_t* raw) {
   return *reinterpret_cast<Smem<D>*>(raw + ((1024u - (a & 1023u)) & 1023u));
 }
 
+// Four codes (each the low byte of a float x + 1.5*2^23) packed into one word, byte 0 first.
+__device__ __forceinline__ uint32_t pack_magic4(float a, float b, float c, float d) {
+  const uint32_t lo = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);
+  const uint32_t hi = __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_qc,
@@ -108,8 +125,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem<D>& sm = smem_ref<D>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = args.N;
-  const int t = blockIdx.x / args.BH;  // key tile; causal tile 0 has the most work: first
-  const int bh = blockIdx.x % args.BH;
+  const int nkt = N / BKT;
+  // head-major order: the key tiles of one head run together and share its query-side tiles
+  // and dQ accumulator in L2; within a head the tile with the most work (t = 0) comes first
+  const int bh = blockIdx.x / nkt;
+  const int t = blockIdx.x % nkt;
   const int i_first = args.causal ? t : 0;
   const int nq = N / BQ - i_first;
   const int G = BQ / args.q_block;  // q_block groups per query tile (1 or 2)
@@ -120,8 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.q_full[s], 1);
       mbar_init(&sm.q_empty[s], 1);
+      mbar_init(&sm.sdp_full[s], 1);
     }
-    mbar_init(&sm.sdp_full, 1);
     mbar_init(&sm.pds_ready, 256);
     mbar_init(&sm.dvdk_full, 1);
     mbar_init(&sm.dvdk_free, 256);
@@ -141,8 +161,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const int row_base = bh * N;
 
-  if (warp == kProducerWarp) {
-    if (lane == 0) {
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
+    if (warp == kProducerWarp && lane == 0) {
       tma_prefetch_desc(&tm_qc);
       tma_prefetch_desc(&tm_kc);
       tma_prefetch_desc(&tm_doc);
@@ -162,9 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int a = 0; a < D / 64; ++a)
           tma_load_2d(sm.st[s].dor + a * BQ * 128, &tm_do, a * 64, row, &sm.q_full[s]);
       }
-    }
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
       const uint32_t id_s = instr_desc(2, 1, 1, false, false, BQ, BKT);
       const uint32_t ab = IsBf16<T>::value ? 1u : 0u;
       const uint32_t id_dp = instr_desc(1, ab, ab, false, false, BQ, BKT);
@@ -172,37 +191,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t id_dq = instr_desc(2, 1, 1, false, true, BQ, D);   // dQ_t
       const uint32_t kca = smem_u32(sm.kc), va = smem_u32(sm.v);
       const uint32_t pca = smem_u32(sm.pc), dsa = smem_u32(sm.dsc);
-      mbar_wait(&sm.kv_full, 0, 201);
-      int dvdk_cnt = 0;
-      for (int it = 0; it < nq; ++it) {
+      // S and dP of query tile `it` into TMEM buffer it & 1
+      auto issue_sdp = [&](int it) {
         const int s = it & 1;
-        const uint32_t qca = smem_u32(sm.st[s].qc), doca = smem_u32(sm.st[s].doc);
-        const uint32_t dora = smem_u32(sm.st[s].dor);
+        const uint32_t dst = tmem + s * 256;
+        const uint32_t qca = smem_u32(sm.st[s].qc), dora = smem_u32(sm.st[s].dor);
         mbar_wait(&sm.q_full[s], (it >> 1) & 1, 202);
-        if (it > 0) mbar_wait(&sm.dq_free, (it - 1) & 1, 203);
         tc_fence_after();
-        // S = Qc Kc^T
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
-          mma_i8(tmem, smem_desc(qca + kk * 32, 16, kSboC, kSwC),
+          mma_i8(dst, smem_desc(qca + kk * 32, 16, kSboC, kSwC),
                  smem_desc(kca + kk * 32, 16, kSboC, kSwC), id_s, kk > 0 ? 1u : 0u);
-        // dP = dO V^T (16-bit operands, float32 accumulation)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk * 16 / 64) * (BQ * 128) + (kk * 16 % 64) * 2;
-          mma_f16(tmem + 128, smem_desc(dora + off, 16, 1024, kSwizzle128B),
+          mma_f16(dst + 128, smem_desc(dora + off, 16, 1024, kSwizzle128B),
                   smem_desc(va + off, 16, 1024, kSwizzle128B), id_dp, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sm.sdp_full);
+        mma_commit(&sm.sdp_full[s]);
+      };
+      mbar_wait(&sm.kv_full, 0, 201);
+      issue_sdp(0);
+      int dvdk_cnt = 0;
+      for (int it = 0; it < nq; ++it) {
+        const int s = it & 1;
+        const uint32_t buf = tmem + s * 256;
+        if (it + 1 < nq) {
+          // buffer (it+1)&1 last held tile it-1: free once its dQ has been read out
+          if (it >= 1) mbar_wait(&sm.dq_free, (it - 1) & 1, 203);
+          issue_sdp(it + 1);
+        }
+        const uint32_t qca = smem_u32(sm.st[s].qc), doca = smem_u32(sm.st[s].doc);
         mbar_wait(&sm.pds_ready, it & 1, 204);
         tc_fence_after();
         for (int g = 0; g < G; ++g) {
           const int q0 = g * args.q_block;
           for (int kk = 0; kk < args.q_block / 32; ++kk) {
             const int qr = q0 + kk * 32;
-            mma_i8(tmem, smem_desc(pca + qr * 128, BQ * BKT, 1024, kSwizzle128B),
+            mma_i8(buf, smem_desc(pca + qr * 128, BQ * BKT, 1024, kSwizzle128B),
                    smem_desc(doca + qr * D, BQ * D, kSboC, kSwC), id_mn, kk > 0 ? 1u : 0u);
-            mma_i8(tmem + 128, smem_desc(dsa + qr * 128, BQ * BKT, 1024, kSwizzle128B),
+            mma_i8(buf + 128, smem_desc(dsa + qr * 128, BQ * BKT, 1024, kSwizzle128B),
                    smem_desc(qca + qr * D, BQ * D, kSboC, kSwC), id_mn, kk > 0 ? 1u : 0u);
           }
           mma_commit(&sm.dvdk_full);
@@ -215,25 +243,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
-            mma_i8(tmem + hh * 128, smem_desc(dsa + hh * 64 + kk * 32, 16, 1024, kSwizzle128B),
+            mma_i8(buf + hh * 128, smem_desc(dsa + hh * 64 + kk * 32, 16, 1024, kSwizzle128B),
                    smem_desc(kca + (hh * 64 + kk * 32) * D, BKT * D, kSboC, kSwC), id_dq,
                    kk > 0 ? 1u : 0u);
         mma_commit(&sm.dq_full);
         mma_commit(&sm.q_empty[s]);
       }
     }
+    // teardown: every MMA has completed once the compute warps pass this barrier
+    __syncwarp();
+    tc_fence_before();
+    named_barrier_sync(15, kThreads);
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kComputeRegs));
     // ---------------- compute warps ----------------
     const int h = warp >> 2, quarter = warp & 3;
     const int r = quarter * 32 + lane;  // TMEM lane = query row (steps 1-2, 4) / key row (3)
-    const uint32_t lane_base = tmem + ((quarter * 32u) << 16);
+    const uint32_t lane_off = (quarter * 32u) << 16;
     const int nqb = N / args.q_block, nkb = N / 64;
     const float* ksc = args.k_scale + static_cast<size_t>(bh) * nkb;
     const float sk_h = ksc[2 * t + h];
     const float sk0 = ksc[2 * t], sk1 = ksc[2 * t + 1];
     const int key_base = t * BKT;
+    const int wpg = args.q_block / 32;  // warps per q_block group
+    float accv[kHalfD], acck[kHalfD];
+#pragma unroll
+    for (int c = 0; c < kHalfD; ++c) accv[c] = acck[c] = 0.0f;
     int dvdk_cnt = 0;
     for (int it = 0; it < nq; ++it) {
+      const int b = it & 1;
+      const uint32_t lane_base = tmem + lane_off + b * 256;
       const int qt = i_first + it;
       const int qrow = qt * BQ + r;  // query index of this thread's row
       const size_t grow = static_cast<size_t>(row_base) + qrow;
@@ -243,27 +284,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float lse2 = args.lse[grow] * 1.4426950408889634f;
       const float dv_row = args.dvec[grow];
       const bool diag = args.causal && (qt == t);
-      mbar_wait(&sm.sdp_full, it & 1, 210);
+      mbar_wait(&sm.sdp_full[b], (it >> 1) & 1, 210);
       tc_fence_after();
       // pass A: P and dS in float32, back into TMEM; row maxima
       float pmax = 0.0f, dsmax = 0.0f;
-#pragma unroll
+#pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         const int col = h * 64 + ch * 16;
         uint32_t sa[16], pa[16];
         tmem_ld16(lane_base + col, sa);
         tmem_ld16(lane_base + 128 + col, pa);
         tmem_ld_wait();
+        if (diag) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int key = key_base + col + e;
-          float p = ex2_approx(fmaf(i2f_exact(sa[e]), c, -lse2));
-          if (diag && key > qrow) p = 0.0f;
-          const float ds = p * (__uint_as_float(pa[e]) - dv_row);
-          pmax = fmaxf(pmax, p);
-          dsmax = fmaxf(dsmax, fabsf(ds));
-          sa[e] = __float_as_uint(p);
-          pa[e] = __float_as_uint(ds);
+          for (int e = 0; e < 16; ++e) {
+            const int key = key_base + col + e;
+            float p = ex2_approx(fmaf(i2f_exact(sa[e]), c, -lse2));
+            p = key > qrow ? 0.0f : p;
+            const float ds = p * (__uint_as_float(pa[e]) - dv_row);
+            pmax = fmaxf(pmax, p);
+            dsmax = fmaxf(dsmax, fabsf(ds));
+            sa[e] = __float_as_uint(p);
+            pa[e] = __float_as_uint(ds);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p = ex2_approx(fmaf(i2f_exact(sa[e]), c, -lse2));
+            const float ds = p * (__uint_as_float(pa[e]) - dv_row);
+            pmax = fmaxf(pmax, p);
+            dsmax = fmaxf(dsmax, fabsf(ds));
+            sa[e] = __float_as_uint(p);
+            pa[e] = __float_as_uint(ds);
+          }
         }
         tmem_st16(lane_base + col, sa);
         tmem_st16(lane_base + 128 + col, pa);
@@ -279,16 +332,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_barrier_sync(1 + h, 128);
       float tp = 0.0f, tds = 0.0f;
       {
-        const int wpg = args.q_block / 32;  // warps per q_block group
         const int w0 = (quarter / wpg) * wpg;
         for (int w = w0; w < w0 + wpg; ++w) {
           tp = fmaxf(tp, sm.red_p[h * 4 + w]);
           tds = fmaxf(tds, sm.red_ds[h * 4 + w]);
         }
       }
-      if (lane == 0 && (quarter % (args.q_block / 32)) == 0) {
-        sm.sp[g_row][h] = __fdiv_rn(tp, 127.0f);
-        sm.sds[g_row][h] = __fdiv_rn(tds, 127.0f);
+      if (lane == 0 && (quarter % wpg) == 0) {
+        sm.sp[b][g_row][h] = __fdiv_rn(tp, 127.0f);
+        sm.sds[b][g_row][h] = __fdiv_rn(tds, 127.0f);
       }
       const float ip = tp > 0.0f ? __fdiv_rn(127.0f, tp) : 0.0f;
       const float ids = tds > 0.0f ? __fdiv_rn(127.0f, tds) : 0.0f;
@@ -296,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       named_barrier_sync(3, 256);  // all tile scales written; reads of sm.red_* done
       tc_fence_after();
       // pass B: INT8 codes into shared memory
-#pragma unroll
+#pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         const int col = h * 64 + ch * 16;
         uint32_t sa[16], pa[16];
@@ -306,14 +358,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t cp[4], cd[4];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          cp[q4] = pack4(rne_byte(__uint_as_float(sa[q4 * 4 + 0]) * ip),
-                         rne_byte(__uint_as_float(sa[q4 * 4 + 1]) * ip),
-                         rne_byte(__uint_as_float(sa[q4 * 4 + 2]) * ip),
-                         rne_byte(__uint_as_float(sa[q4 * 4 + 3]) * ip));
-          cd[q4] = pack4(rne_byte(__uint_as_float(pa[q4 * 4 + 0]) * ids),
-                         rne_byte(__uint_as_float(pa[q4 * 4 + 1]) * ids),
-                         rne_byte(__uint_as_float(pa[q4 * 4 + 2]) * ids),
-                         rne_byte(__uint_as_float(pa[q4 * 4 + 3]) * ids));
+          float fp[4], fd[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            fp[e] = __fmaf_rn(__uint_as_float(sa[q4 * 4 + e]), ip, 12582912.0f);
+            fd[e] = __fmaf_rn(__uint_as_float(pa[q4 * 4 + e]), ids, 12582912.0f);
+          }
+          cp[q4] = pack_magic4(fp[0], fp[1], fp[2], fp[3]);
+          cd[q4] = pack_magic4(fd[0], fd[1], fd[2], fd[3]);
         }
         const uint32_t off = swz_offset(r, h * 4 + ch, 128);
         *reinterpret_cast<uint4*>(sm.pc + off) = make_uint4(cp[0], cp[1], cp[2], cp[3]);
@@ -322,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sm.pds_ready);
-      // step 3: dV_t, dK_t (thread = key row r, d columns of warpgroup h)
+      // step 3: dV_t, dK_t (thread = key row r, d columns of warpgroup h) into registers
       for (int g = 0; g < G; ++g) {
         const size_t qb = static_cast<size_t>(bh) * nqb + (qt * BQ + g * args.q_block) /
                                                               args.q_block;
@@ -331,31 +383,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kh = r >> 6;
         mbar_wait(&sm.dvdk_full, dvdk_cnt & 1, 211);
         tc_fence_after();
-        const float s_v = sm.sp[g][kh] * sdo;
-        const float s_k = sm.sds[g][kh] * sqg * args.tau;
-        const bool first = (it == 0 && g == 0);
+        const float s_v = sm.sp[b][g][kh] * sdo;
+        const float s_k = sm.sds[b][g][kh] * sqg * args.tau;
 #pragma unroll
         for (int c0 = 0; c0 < kHalfD; c0 += 16) {
           const int col = h * kHalfD + c0;
-          uint32_t tv[16], tk[16], av[16], ak[16];
+          uint32_t tv[16], tk[16];
           tmem_ld16(lane_base + col, tv);
           tmem_ld16(lane_base + 128 + col, tk);
-          if (!first) {
-            tmem_ld16(lane_base + 256 + col, av);
-            tmem_ld16(lane_base + 256 + D + col, ak);
-          }
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float bv = first ? 0.0f : __uint_as_float(av[e]);
-            const float bk = first ? 0.0f : __uint_as_float(ak[e]);
-            av[e] = __float_as_uint(fmaf(i2f_exact(tv[e]), s_v, bv));
-            ak[e] = __float_as_uint(fmaf(i2f_exact(tk[e]), s_k, bk));
+            accv[c0 + e] = fmaf(i2f_exact(tv[e]), s_v, accv[c0 + e]);
+            acck[c0 + e] = fmaf(i2f_exact(tk[e]), s_k, acck[c0 + e]);
           }
-          tmem_st16(lane_base + 256 + col, av);
-          tmem_st16(lane_base + 256 + D + col, ak);
         }
-        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sm.dvdk_free);
         ++dvdk_cnt;
@@ -364,10 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&sm.dq_full, it & 1, 212);
       tc_fence_after();
       {
-        const float s0 = sm.sds[g_row][0] * sk0 * args.tau;
-        const float s1 = sm.sds[g_row][1] * sk1 * args.tau;
+        const float s0 = sm.sds[b][g_row][0] * sk0 * args.tau;
+        const float s1 = sm.sds[b][g_row][1] * sk1 * args.tau;
         float* dst = args.dq_acc + grow * D + h * kHalfD;
-#pragma unroll
+#pragma unroll 1
         for (int c0 = 0; c0 < kHalfD; c0 += 16) {
           uint32_t a0[16], a1[16];
           tmem_ld16(lane_base + h * kHalfD + c0, a0);
@@ -387,76 +429,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&sm.dq_free);
     }
-    // epilogue: dv, dk (thread = key row r, d columns of warpgroup h)
+    // epilogue: dv, dk from the register accumulators (thread = key row r, d half h)
     {
       const size_t krow = static_cast<size_t>(row_base) + key_base + r;
       T* dvp = reinterpret_cast<T*>(args.dv) + krow * D + h * kHalfD;
       T* dkp = reinterpret_cast<T*>(args.dk) + krow * D + h * kHalfD;
-      float inv = 0.0f, part = 0.0f;
       if (args.qknorm) {
-        inv = args.k_inv_rms[krow];
+        // RMSNorm backward: dk = inv * (dkhat - khat * (sum_c dkhat_c khat_c) / d), with
+        // khat = k * inv recomputed from the raw row (bitwise the prologue's value)
+        const float inv = args.k_inv_rms[krow];
         const T* kp = reinterpret_cast<const T*>(args.k_raw) + krow * D + h * kHalfD;
+        float part = 0.0f;
 #pragma unroll
-        for (int c0 = 0; c0 < kHalfD; c0 += 16) {
-          uint32_t ak[16];
-          tmem_ld16(lane_base + 256 + D + h * kHalfD + c0, ak);
-          tmem_ld_wait();
+        for (int c0 = 0; c0 < kHalfD; c0 += 8) {
+          float x[8];
+          Cvt<T>::load8(__ldg(reinterpret_cast<const uint4*>(kp + c0)), x);
 #pragma unroll
-          for (int e8 = 0; e8 < 16; e8 += 8) {
-            float x[8];
-            Cvt<T>::load8(__ldg(reinterpret_cast<const uint4*>(kp + c0 + e8)), x);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) part = fmaf(__uint_as_float(ak[e8 + e]),
-                                                    __fmul_rn(x[e], inv), part);
-          }
+          for (int e = 0; e < 8; ++e) part = fmaf(acck[c0 + e], __fmul_rn(x[e], inv), part);
         }
         if (h == 1) sm.dot[r] = part;
         named_barrier_sync(3, 256);
         if (h == 0) sm.dot[r] += part;
         named_barrier_sync(3, 256);
+        const float dotd = sm.dot[r] * (1.0f / D);
+#pragma unroll
+        for (int c0 = 0; c0 < kHalfD; c0 += 8) {
+          float x[8];
+          Cvt<T>::load8(__ldg(reinterpret_cast<const uint4*>(kp + c0)), x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            acck[c0 + e] = inv * fmaf(-__fmul_rn(x[e], inv), dotd, acck[c0 + e]);
+        }
       }
-      const float dotd = args.qknorm ? sm.dot[r] * (1.0f / D) : 0.0f;
 #pragma unroll
-      for (int c0 = 0; c0 < kHalfD; c0 += 16) {
-        uint32_t av[16], ak[16];
-        tmem_ld16(lane_base + 256 + h * kHalfD + c0, av);
-        tmem_ld16(lane_base + 256 + D + h * kHalfD + c0, ak);
-        tmem_ld_wait();
-        float fk[16];
-        if (args.qknorm) {
-          const T* kp = reinterpret_cast<const T*>(args.k_raw) + krow * D + h * kHalfD;
+      for (int c0 = 0; c0 < kHalfD; c0 += 8) {
+        float fv[8], fk[8];
 #pragma unroll
-          for (int e8 = 0; e8 < 16; e8 += 8) {
-            float x[8];
-            Cvt<T>::load8(__ldg(reinterpret_cast<const uint4*>(kp + c0 + e8)), x);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float xh = __fmul_rn(x[e], inv);
-              fk[e8 + e] = inv * fmaf(-xh, dotd, __uint_as_float(ak[e8 + e]));
-            }
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) fk[e] = __uint_as_float(ak[e]);
+        for (int e = 0; e < 8; ++e) {
+          fv[e] = accv[c0 + e];
+          fk[e] = acck[c0 + e];
         }
-#pragma unroll
-        for (int e8 = 0; e8 < 16; e8 += 8) {
-          float fv[8], fkk[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            fv[e] = __uint_as_float(av[e8 + e]);
-            fkk[e] = fk[e8 + e];
-          }
-          *reinterpret_cast<uint4*>(dvp + c0 + e8) = pack8<T>(fv);
-          *reinterpret_cast<uint4*>(dkp + c0 + e8) = pack8<T>(fkk);
-        }
+        *reinterpret_cast<uint4*>(dvp + c0) = pack8<T>(fv);
+        *reinterpret_cast<uint4*>(dkp + c0) = pack8<T>(fk);
       }
     }
+    tc_fence_before();
+    named_barrier_sync(15, kThreads);
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace bwd

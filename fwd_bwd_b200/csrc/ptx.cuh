@@ -73,7 +73,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int site) {
+// Waits until the phase with the given parity has completed.  Returns false on timeout.
+// Fully inlined: kernels that move registers between warpgroups (setmaxnreg) must not make
+// calls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   const uint64_t limit = device_aborted() ? 1000000ull : 2000000000ull;  // 1 ms / 2 s
   while (true) {
@@ -85,12 +89,6 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int 
       return false;
     }
   }
-}
-
-// Waits until the phase with the given parity has completed.  Returns false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site) {
-  if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, site);
 }
 
 // Named barrier among `nthreads` threads (a multiple of 32) of the CTA.

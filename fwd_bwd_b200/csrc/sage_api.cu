@@ -123,6 +123,13 @@ int set_smem(K kernel, size_t bytes) {
              : SAGE_ERR_CUDA;
 }
 
+template <typename K>
+int launch_regs(K kernel) {
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return -1;
+  return fa.numRegs;
+}
+
 // ---- prologue ---------------------------------------------------------------------------
 template <typename T, int D>
 int run_prologue(const sage_params* p, const void* q, const void* k, const void* v,
@@ -244,6 +251,10 @@ int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const
   const size_t smem = sage::bwd::smem_bytes<D>();
   auto kern = sage::bwd::attn_bwd_kernel<T, D>;
   if (set_smem(kern, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+  // The kernel moves registers between warpgroups (setmaxnreg); the split is sized for a launch
+  // allocation of exactly kLaunchRegs per thread.  Any other allocation could leave the
+  // increasing warpgroups waiting, so refuse to launch.
+  if (launch_regs(kern) != sage::bwd::kLaunchRegs) return SAGE_ERR_UNSUPPORTED;
   kern<<<BH * (N / sage::bwd::BKT), sage::bwd::kThreads, smem, st>>>(tqc, tkc, tdoc, tdo, tv, a);
   return launch_status();
 }
