@@ -12,6 +12,8 @@
 //      (for dV, dK);
 //   3. dV_t = Pc^T dOc and dK_t = dSc^T Qc (kind::i8, M = 128 keys, one per q_block group),
 //      dequantized by the tile scales and added to float32 accumulators in registers;
+//      every INT32 accumulator region is preloaded with the bits of 1.5 * 2^23 so the results
+//      read back as floats that one exact FMA dequantizes (see kMagicBits);
 //   4. dQ_t = dSc Kc per 64-key block (kind::i8), dequantized, summed and added to a float32
 //      dQ accumulator in global memory with vector atomics.
 // S and dP are double-buffered in TMEM, so the tensor core computes them for query tile i+1
@@ -69,7 +71,7 @@ struct Smem {
   int8_t pc[BQ * BKT];     // P codes  [128 q][128 keys], 128-byte swizzle
   int8_t dsc[BQ * BKT];    // dS codes [128 q][128 keys], 128-byte swizzle
   float red_p[8], red_ds[8];
-  float sp[2][2][2], sds[2][2][2];  // tile scales [tile parity][q group][key half]
+  float sp[3][2][2], sds[3][2][2];  // tile scales [tile % 3][q group][key half]
   float dot[BKT];                   // RMSNorm-backward row dot products (warpgroup 1 -> 0)
   uint64_t kv_full, q_full[2], q_empty[2];
   uint64_t sdp_full[2], pds_ready, dvdk_full, dvdk_free, dq_full, dq_free;
@@ -102,13 +104,6 @@ template <int D>
 __device__ __forceinline__ Smem<D>& smem_ref(uint8_t* raw) {
   const uint32_t a = smem_u32(raw);
   return *reinterpret_cast<Smem<D>*>(raw + ((1024u - (a & 1023u)) & 1023u));
-}
-
-// Four codes (each the low byte of a float x + 1.5*2^23) packed into one word, byte 0 first.
-__device__ __forceinline__ uint32_t pack_magic4(float a, float b, float c, float d) {
-  const uint32_t lo = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);
-  const uint32_t hi = __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040);
-  return __byte_perm(lo, hi, 0x5410);
 }
 
 template <typename T, int D>
@@ -160,6 +155,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const int row_base = bh * N;
+  if (warp < 8) {
+    // INT32 accumulators are preloaded with the bits of 1.5 * 2^23 (see kMagicBits): the S
+    // regions of both TMEM buffers, this thread's lane, this warpgroup's 64-column half
+    const uint32_t lb = tmem + (((warp & 3) * 32u) << 16) + (warp >> 2) * 64;
+#pragma unroll
+    for (int c = 0; c < 64; c += 16) {
+      tmem_fill16(lb + c, kMagicBits);
+      tmem_fill16(lb + 256 + c, kMagicBits);
+    }
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
@@ -201,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
           mma_i8(dst, smem_desc(qca + kk * 32, 16, kSboC, kSwC),
-                 smem_desc(kca + kk * 32, 16, kSboC, kSwC), id_s, kk > 0 ? 1u : 0u);
+                 smem_desc(kca + kk * 32, 16, kSboC, kSwC), id_s, 1u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk * 16 / 64) * (BQ * 128) + (kk * 16 % 64) * 2;
@@ -229,9 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < args.q_block / 32; ++kk) {
             const int qr = q0 + kk * 32;
             mma_i8(buf, smem_desc(pca + qr * 128, BQ * BKT, 1024, kSwizzle128B),
-                   smem_desc(doca + qr * D, BQ * D, kSboC, kSwC), id_mn, kk > 0 ? 1u : 0u);
+                   smem_desc(doca + qr * D, BQ * D, kSboC, kSwC), id_mn, 1u);
             mma_i8(buf + 128, smem_desc(dsa + qr * 128, BQ * BKT, 1024, kSwizzle128B),
-                   smem_desc(qca + qr * D, BQ * D, kSboC, kSwC), id_mn, kk > 0 ? 1u : 0u);
+                   smem_desc(qca + qr * D, BQ * D, kSboC, kSwC), id_mn, 1u);
           }
           mma_commit(&sm.dvdk_full);
           mbar_wait(&sm.dvdk_free, dvdk_cnt & 1, 205);
@@ -244,8 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)
             mma_i8(buf + hh * 128, smem_desc(dsa + hh * 64 + kk * 32, 16, 1024, kSwizzle128B),
-                   smem_desc(kca + (hh * 64 + kk * 32) * D, BKT * D, kSboC, kSwC), id_dq,
-                   kk > 0 ? 1u : 0u);
+                   smem_desc(kca + (hh * 64 + kk * 32) * D, BKT * D, kSboC, kSwC), id_dq, 1u);
         mma_commit(&sm.dq_full);
         mma_commit(&sm.q_empty[s]);
       }
@@ -259,6 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kComputeRegs));
     // ---------------- compute warps ----------------
+    // Software-pipelined: pass A of tile it+1 (TMEM buffer (it+1)&1 only) runs between pass B
+    // of tile it and the read-outs of tile it, so the tensor core computes dV_t / dK_t / dQ_t
+    // of tile it meanwhile.
     const int h = warp >> 2, quarter = warp & 3;
     const int r = quarter * 32 + lane;  // TMEM lane = query row (steps 1-2, 4) / key row (3)
     const uint32_t lane_off = (quarter * 32u) << 16;
@@ -268,25 +279,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sk0 = ksc[2 * t], sk1 = ksc[2 * t + 1];
     const int key_base = t * BKT;
     const int wpg = args.q_block / 32;  // warps per q_block group
+    const int g_row = r / args.q_block;
     float accv[kHalfD], acck[kHalfD];
 #pragma unroll
     for (int c = 0; c < kHalfD; ++c) accv[c] = acck[c] = 0.0f;
     int dvdk_cnt = 0;
-    for (int it = 0; it < nq; ++it) {
-      const int b = it & 1;
+
+    // per-row inputs of query tile `it`: (c, lse2, D) for this thread's row
+    auto row_inputs = [&](int it, float& c, float& lse2, float& dvr) {
+      const int qrow = (i_first + it) * BQ + r;
+      const size_t grow = static_cast<size_t>(row_base) + qrow;
+      c = args.q_scale[static_cast<size_t>(bh) * nqb + qrow / args.q_block] * sk_h *
+          args.scale_log2;
+      lse2 = args.lse[grow] * 1.4426950408889634f;
+      dvr = args.dvec[grow];
+    };
+    // pass A of tile it: P, dS into TMEM buffer it&1, tile maxima -> scales in slot it%3
+    auto pass_a = [&](int it, float c, float lse2, float dvr, float& ip, float& ids) {
+      const int b = it & 1, slot = it % 3;
       const uint32_t lane_base = tmem + lane_off + b * 256;
       const int qt = i_first + it;
-      const int qrow = qt * BQ + r;  // query index of this thread's row
-      const size_t grow = static_cast<size_t>(row_base) + qrow;
-      const int g_row = r / args.q_block;
-      const float sq_row = args.q_scale[static_cast<size_t>(bh) * nqb + qrow / args.q_block];
-      const float c = sq_row * sk_h * args.scale_log2;
-      const float lse2 = args.lse[grow] * 1.4426950408889634f;
-      const float dv_row = args.dvec[grow];
+      const int qrow = qt * BQ + r;
       const bool diag = args.causal && (qt == t);
+      const float c22 = scale22(c);
+      const float nc22 = __fmul_rn(-kMagic, c22);
       mbar_wait(&sm.sdp_full[b], (it >> 1) & 1, 210);
       tc_fence_after();
-      // pass A: P and dS in float32, back into TMEM; row maxima
       float pmax = 0.0f, dsmax = 0.0f;
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
@@ -299,10 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int key = key_base + col + e;
-            float p = ex2_approx(fmaf(i2f_exact(sa[e]), c, -lse2));
+            float p = ex2_approx(deq(sa[e], c22, nc22) - lse2);
             p = key > qrow ? 0.0f : p;
-            const float ds = p * (__uint_as_float(pa[e]) - dv_row);
-            pmax = fmaxf(pmax, p);
+            const float ds = p * (__uint_as_float(pa[e]) - dvr);
             dsmax = fmaxf(dsmax, fabsf(ds));
             sa[e] = __float_as_uint(p);
             pa[e] = __float_as_uint(ds);
@@ -310,14 +327,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p = ex2_approx(fmaf(i2f_exact(sa[e]), c, -lse2));
-            const float ds = p * (__uint_as_float(pa[e]) - dv_row);
-            pmax = fmaxf(pmax, p);
+            const float p = ex2_approx(deq(sa[e], c22, nc22) - lse2);
+            const float ds = p * (__uint_as_float(pa[e]) - dvr);
             dsmax = fmaxf(dsmax, fabsf(ds));
             sa[e] = __float_as_uint(p);
             pa[e] = __float_as_uint(ds);
           }
         }
+#pragma unroll
+        for (int e = 0; e < 16; e += 2)
+          pmax = fmax3(pmax, __uint_as_float(sa[e]), __uint_as_float(sa[e + 1]));
         tmem_st16(lane_base + col, sa);
         tmem_st16(lane_base + 128 + col, pa);
       }
@@ -331,23 +350,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       named_barrier_sync(1 + h, 128);
       float tp = 0.0f, tds = 0.0f;
-      {
-        const int w0 = (quarter / wpg) * wpg;
-        for (int w = w0; w < w0 + wpg; ++w) {
-          tp = fmaxf(tp, sm.red_p[h * 4 + w]);
-          tds = fmaxf(tds, sm.red_ds[h * 4 + w]);
-        }
+      const int w0 = (quarter / wpg) * wpg;
+      for (int w = w0; w < w0 + wpg; ++w) {
+        tp = fmaxf(tp, sm.red_p[h * 4 + w]);
+        tds = fmaxf(tds, sm.red_ds[h * 4 + w]);
       }
       if (lane == 0 && (quarter % wpg) == 0) {
-        sm.sp[b][g_row][h] = __fdiv_rn(tp, 127.0f);
-        sm.sds[b][g_row][h] = __fdiv_rn(tds, 127.0f);
+        sm.sp[slot][g_row][h] = __fdiv_rn(tp, 127.0f);
+        sm.sds[slot][g_row][h] = __fdiv_rn(tds, 127.0f);
       }
-      const float ip = tp > 0.0f ? __fdiv_rn(127.0f, tp) : 0.0f;
-      const float ids = tds > 0.0f ? __fdiv_rn(127.0f, tds) : 0.0f;
+      ip = tp > 0.0f ? __fdiv_rn(127.0f, tp) : 0.0f;
+      ids = tds > 0.0f ? __fdiv_rn(127.0f, tds) : 0.0f;
       tc_fence_before();
       named_barrier_sync(3, 256);  // all tile scales written; reads of sm.red_* done
       tc_fence_after();
-      // pass B: INT8 codes into shared memory
+    };
+
+    float c_n, lse2_n, dvr_n, ip, ids;
+    row_inputs(0, c_n, lse2_n, dvr_n);
+    pass_a(0, c_n, lse2_n, dvr_n, ip, ids);
+    for (int it = 0; it < nq; ++it) {
+      const int b = it & 1, slot = it % 3;
+      const uint32_t lane_base = tmem + lane_off + b * 256;
+      const int qt = i_first + it;
+      const size_t grow = static_cast<size_t>(row_base) + qt * BQ + r;
+      if (it + 1 < nq) row_inputs(it + 1, c_n, lse2_n, dvr_n);  // loads in flight during pass B
+      // pass B: INT8 codes into shared memory; the dV_t / dK_t regions re-preloaded
 #pragma unroll 1
       for (int ch = 0; ch < 4; ++ch) {
         const int col = h * 64 + ch * 16;
@@ -361,8 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float fp[4], fd[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            fp[e] = __fmaf_rn(__uint_as_float(sa[q4 * 4 + e]), ip, 12582912.0f);
-            fd[e] = __fmaf_rn(__uint_as_float(pa[q4 * 4 + e]), ids, 12582912.0f);
+            fp[e] = __fmaf_rn(__uint_as_float(sa[q4 * 4 + e]), ip, kMagic);
+            fd[e] = __fmaf_rn(__uint_as_float(pa[q4 * 4 + e]), ids, kMagic);
           }
           cp[q4] = pack_magic4(fp[0], fp[1], fp[2], fp[3]);
           cd[q4] = pack_magic4(fd[0], fd[1], fd[2], fd[3]);
@@ -370,11 +398,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t off = swz_offset(r, h * 4 + ch, 128);
         *reinterpret_cast<uint4*>(sm.pc + off) = make_uint4(cp[0], cp[1], cp[2], cp[3]);
         *reinterpret_cast<uint4*>(sm.dsc + off) = make_uint4(cd[0], cd[1], cd[2], cd[3]);
+        if (col < D) {  // dV_t occupies columns [0, D), dK_t [128, 128 + D)
+          tmem_fill16(lane_base + col, kMagicBits);
+          tmem_fill16(lane_base + 128 + col, kMagicBits);
+        }
       }
+      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sm.pds_ready);
-      // step 3: dV_t, dK_t (thread = key row r, d columns of warpgroup h) into registers
+      // pass A of the next tile while the tensor core works on this one
+      float ip_n = 0.0f, ids_n = 0.0f;
+      if (it + 1 < nq) pass_a(it + 1, c_n, lse2_n, dvr_n, ip_n, ids_n);
+      // step 3: dV_t, dK_t (thread = key row r, d columns of warpgroup h) into registers;
+      // the read columns are re-preloaded for dQ_t
       for (int g = 0; g < G; ++g) {
         const size_t qb = static_cast<size_t>(bh) * nqb + (qt * BQ + g * args.q_block) /
                                                               args.q_block;
@@ -383,8 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kh = r >> 6;
         mbar_wait(&sm.dvdk_full, dvdk_cnt & 1, 211);
         tc_fence_after();
-        const float s_v = sm.sp[b][g][kh] * sdo;
-        const float s_k = sm.sds[b][g][kh] * sqg * args.tau;
+        const float sv22 = scale22(sm.sp[slot][g][kh] * sdo);
+        const float sk22 = scale22(sm.sds[slot][g][kh] * sqg * args.tau);
+        const float nsv = __fmul_rn(-kMagic, sv22), nsk = __fmul_rn(-kMagic, sk22);
 #pragma unroll
         for (int c0 = 0; c0 < kHalfD; c0 += 16) {
           const int col = h * kHalfD + c0;
@@ -394,20 +432,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            accv[c0 + e] = fmaf(i2f_exact(tv[e]), s_v, accv[c0 + e]);
-            acck[c0 + e] = fmaf(i2f_exact(tk[e]), s_k, acck[c0 + e]);
+            accv[c0 + e] += deq(tv[e], sv22, nsv);
+            acck[c0 + e] += deq(tk[e], sk22, nsk);
           }
+          tmem_fill16(lane_base + col, kMagicBits);
+          tmem_fill16(lane_base + 128 + col, kMagicBits);
         }
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sm.dvdk_free);
         ++dvdk_cnt;
       }
-      // step 4: dQ (thread = query row r, d columns of warpgroup h)
+      // step 4: dQ (thread = query row r, d columns of warpgroup h); afterwards the S region
+      // of this buffer is re-preloaded for tile it+2
       mbar_wait(&sm.dq_full, it & 1, 212);
       tc_fence_after();
       {
-        const float s0 = sm.sds[b][g_row][0] * sk0 * args.tau;
-        const float s1 = sm.sds[b][g_row][1] * sk1 * args.tau;
+        const float s0 = scale22(sm.sds[slot][g_row][0] * sk0 * args.tau);
+        const float s1 = scale22(sm.sds[slot][g_row][1] * sk1 * args.tau);
+        const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
         float* dst = args.dq_acc + grow * D + h * kHalfD;
 #pragma unroll 1
         for (int c0 = 0; c0 < kHalfD; c0 += 16) {
@@ -418,16 +461,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
             float4 v4;
-            v4.x = fmaf(i2f_exact(a0[e + 0]), s0, i2f_exact(a1[e + 0]) * s1);
-            v4.y = fmaf(i2f_exact(a0[e + 1]), s0, i2f_exact(a1[e + 1]) * s1);
-            v4.z = fmaf(i2f_exact(a0[e + 2]), s0, i2f_exact(a1[e + 2]) * s1);
-            v4.w = fmaf(i2f_exact(a0[e + 3]), s0, i2f_exact(a1[e + 3]) * s1);
+            v4.x = deq(a0[e + 0], s0, n0) + deq(a1[e + 0], s1, n1);
+            v4.y = deq(a0[e + 1], s0, n0) + deq(a1[e + 1], s1, n1);
+            v4.z = deq(a0[e + 2], s0, n0) + deq(a1[e + 2], s1, n1);
+            v4.w = deq(a0[e + 3], s0, n0) + deq(a1[e + 3], s1, n1);
             atomicAdd(reinterpret_cast<float4*>(dst + c0 + e), v4);
           }
         }
+        // S occupies columns [0, 128): each thread refills the dQ_t0 columns it read
+        // ([h*d/2, (h+1)*d/2)) and its warpgroup's half of [d, 128), so no thread writes a
+        // column the other warpgroup may still be reading
+#pragma unroll
+        for (int c = 0; c < kHalfD; c += 16) tmem_fill16(lane_base + h * kHalfD + c, kMagicBits);
+#pragma unroll
+        for (int c = 0; c < (128 - D) / 2; c += 16)
+          tmem_fill16(lane_base + D + h * ((128 - D) / 2) + c, kMagicBits);
+        tmem_st_wait();
       }
       tc_fence_before();
       mbar_arrive(&sm.dq_free);
+      ip = ip_n;
+      ids = ids_n;
     }
     // epilogue: dv, dk from the register accumulators (thread = key row r, d half h)
     {

@@ -11,8 +11,12 @@
 //               P codes = rne(127 p~) written to shared memory in the tensor core's swizzled
 //               K-major layout, running max / sum, and the dequantizing fold
 //               O <- alpha O + PV * beta with beta = exp(max_block - max_running) sV / 127.
+//   warps 10-11 idle (they complete the producer warpgroup, which gives its registers to the
+//               softmax warpgroups: 256 x 232 + 128 x 40 = 64512 = 384 x 168).
 // TMEM (512 columns): tile g uses columns [256g, 256g+256): S buffers at +0 and +64, PV at
-// +128 (d columns, INT32).  O (float32) lives in registers.
+// +128 (d columns, INT32).  The INT32 regions are preloaded with the bits of 1.5 * 2^23 before
+// each MMA (see kMagicBits), so results read back as floats that one FMA dequantizes.
+// O (float32) lives in registers.
 //
 // P quantization: one scale per (query row, 64-key block).  The codes rne(127 p / max p) do
 // not depend on which running maximum p was taken against, so computing them against the
@@ -33,8 +37,13 @@ constexpr int BM = 128;   // query rows per tile (MMA M)
 constexpr int BKV = 64;   // keys per block (= k_block)
 constexpr int NT = 2;     // query tiles per CTA
 constexpr int NST = 4;    // K/V pipeline stages
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 232;
+constexpr int kOtherRegs = 40;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 
 template <int D>
 struct Smem {
@@ -71,10 +80,11 @@ __device__ __forceinline__ Smem<D>& smem_ref(uint8_t* raw) {
   return *reinterpret_cast<Smem<D>*>(raw + ((1024u - (a & 1023u)) & 1023u));
 }
 
-// Issue S = Qc Kc^T for one tile / block: d/32 MMAs of K = 32 bytes.
+// Issue S (+)= Qc Kc^T for one tile / block: d/32 MMAs of K = 32 bytes.  accumulate = 1 adds
+// onto the preloaded accumulator.
 template <int D>
 __device__ __forceinline__ void issue_scores(uint32_t d_tmem, const int8_t* qs,
-                                             const int8_t* ks, int n_keys) {
+                                             const int8_t* ks, int n_keys, uint32_t accumulate) {
   constexpr uint32_t kSw = (D == 128) ? kSwizzle128B : kSwizzle64B;
   constexpr uint32_t kSbo = 8 * D;  // 8 rows of D bytes
   const uint32_t idesc = instr_desc(2, 1, 1, false, false, BM, n_keys);
@@ -82,7 +92,7 @@ __device__ __forceinline__ void issue_scores(uint32_t d_tmem, const int8_t* qs,
 #pragma unroll
   for (int kk = 0; kk < D / 32; ++kk) {
     mma_i8(d_tmem, smem_desc(qa + kk * 32, 16, kSbo, kSw), smem_desc(ka + kk * 32, 16, kSbo, kSw),
-           idesc, kk > 0 ? 1u : 0u);
+           idesc, (kk > 0 || accumulate) ? 1u : 0u);
   }
 }
 
@@ -95,9 +105,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem<D>& sm = smem_ref<D>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = args.N;
-  const int cta = blockIdx.x;
-  const int sup = args.causal ? (args.nsup - 1 - cta / args.BH) : (cta / args.BH);
-  const int bh = cta % args.BH;
+  // head-major order (a head's CTAs share its K / V codes in L2); within a head the query
+  // tiles with the most key blocks come first when causal
+  const int bh = blockIdx.x / args.nsup;
+  const int sidx = blockIdx.x % args.nsup;
+  const int sup = args.causal ? (args.nsup - 1 - sidx) : sidx;
   int q0[NT], nb[NT];
   bool active[NT];
   int nb_max = 0;
@@ -137,9 +149,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  if (warp < 8) {
+    // preload both S buffers and the PV region of this thread's lane with the magic value
+    const uint32_t lb = tmem + (((warp & 3) * 32u) << 16) + (warp >> 2) * 256;
+#pragma unroll
+    for (int c = 0; c < 128 + D; c += 16) tmem_fill16(lb + c, kMagicBits);
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
-  if (warp == kProducerWarp) {
-    if (lane == 0) {
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
+    if (warp == kProducerWarp && lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -157,19 +180,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&sm.v_full[st], BKV * D);
         tma_load_2d(sm.v[st], &tm_v, 0, row_base + j * BKV, &sm.v_full[st]);
       }
-    }
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
       constexpr uint32_t kSw = (D == 128) ? kSwizzle128B : kSwizzle64B;
       constexpr uint32_t kSbo = 8 * D;
       const uint32_t idesc_pv = instr_desc(2, 1, 1, false, true, BM, D);
       mbar_wait(&sm.q_full, 0, 101);
-      tc_fence_after();
       mbar_wait(&sm.k_full[0], 0, 102);
       tc_fence_after();
       for (int g = 0; g < NT; ++g)
         if (nb[g] > 0) {
-          issue_scores<D>(tmem + g * 256, sm.q[g], sm.k[0], BKV);
+          issue_scores<D>(tmem + g * 256, sm.q[g], sm.k[0], BKV, 1u);
           mma_commit(&sm.s_full[g][0]);
         }
       for (int j = 0; j < nb_max; ++j) {
@@ -180,7 +200,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           for (int g = 0; g < NT; ++g)
             if (j + 1 < nb[g]) {
-              issue_scores<D>(tmem + g * 256 + ((j + 1) & 1) * 64, sm.q[g], sm.k[st1], BKV);
+              // buffer (j+1)&1 held S_{j-1}: read and re-preloaded before p_full[j-1]
+              issue_scores<D>(tmem + g * 256 + ((j + 1) & 1) * 64, sm.q[g], sm.k[st1], BKV,
+                              1u);
               mma_commit(&sm.s_full[g][(j + 1) & 1]);
             }
         }
@@ -195,14 +217,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BKV / 32; ++kk) {
             mma_i8(tmem + g * 256 + 128, smem_desc(pa + kk * 32, 16, 8 * BKV, kSwizzle64B),
-                   smem_desc(va + kk * 32 * D, BKV * D, kSbo, kSw), idesc_pv, kk > 0 ? 1u : 0u);
+                   smem_desc(va + kk * 32 * D, BKV * D, kSbo, kSw), idesc_pv, 1u);
           }
           mma_commit(&sm.pv_full[g]);
         }
         mma_commit(&sm.kv_empty[st]);
       }
     }
+    __syncwarp();
+    tc_fence_before();
+    named_barrier_sync(15, kThreads);
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
     // ---------------- softmax warps ----------------
     const int g = warp >> 2, quarter = warp & 3;
     if (active[g]) {
@@ -218,8 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < D; ++c) O[c] = 0.0f;
       float m2 = -INFINITY, l = 0.0f, alpha_prev = 1.0f, beta_prev = 0.0f;
       int8_t* pbase = sm.p[g][0];
+      float sk_next = ksc[0], sv_next = vsc[0];
 
+      // O <- alpha O + PV_jj * beta (PV read back as 1.5*2^23 + PV), then re-preload PV
       auto fold_pv = [&](int jj) {
+        const float b22 = scale22(beta_prev);
+        const float nb22 = __fmul_rn(-kMagic, b22);
         mbar_wait(&sm.pv_full[g], jj & 1, 110);
         tc_fence_after();
 #pragma unroll
@@ -230,38 +262,54 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            O[c0 + c] = fmaf(i2f_exact(a0[c]), beta_prev, O[c0 + c] * alpha_prev);
-            O[c0 + 16 + c] = fmaf(i2f_exact(a1[c]), beta_prev, O[c0 + 16 + c] * alpha_prev);
+            O[c0 + c] = fmaf(O[c0 + c], alpha_prev, deq(a0[c], b22, nb22));
+            O[c0 + 16 + c] = fmaf(O[c0 + 16 + c], alpha_prev, deq(a1[c], b22, nb22));
           }
+          tmem_fill16(lane_base + 128 + c0, kMagicBits);
+          tmem_fill16(lane_base + 128 + c0 + 16, kMagicBits);
         }
+        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sm.pv_free[g]);
       };
 
       for (int j = 0; j < nb[g]; ++j) {
-        const float c = cq * ksc[j];
+        const float sk = sk_next, sv = sv_next;
+        if (j + 1 < nb[g]) {
+          sk_next = ksc[j + 1];
+          sv_next = vsc[j + 1];
+        }
+        const float c22 = scale22(cq * sk);
+        const float nc22 = __fmul_rn(-kMagic, c22);
         const bool diag = args.causal && (j * BKV + BKV - 1 > q0[g]);
         const int key0 = j * BKV;
         mbar_wait(&sm.s_full[g][j & 1], (j >> 1) & 1, 111);
         tc_fence_after();
         const uint32_t sa = lane_base + (j & 1) * 64;
-        // pass 1: block maximum of the (masked) integer scores
-        int amax = INT_MIN;
+        // pass 1: block maximum of kMagic + A (floats, ordered like A) over unmasked keys
+        float mx = -INFINITY;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t a0[16], a1[16];
           tmem_ld16(sa + h * 32, a0);
           tmem_ld16(sa + h * 32 + 16, a1);
           tmem_ld_wait();
+          if (diag) {
 #pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {
-            const int k0 = key0 + h * 32 + cc, k1 = k0 + 16;
-            if (!diag || k0 <= i) amax = max(amax, static_cast<int>(a0[cc]));
-            if (!diag || k1 <= i) amax = max(amax, static_cast<int>(a1[cc]));
+            for (int cc = 0; cc < 16; ++cc) {
+              const int k0 = key0 + h * 32 + cc;
+              const float f0 = k0 <= i ? __uint_as_float(a0[cc]) : -INFINITY;
+              const float f1 = k0 + 16 <= i ? __uint_as_float(a1[cc]) : -INFINITY;
+              mx = fmax3(mx, f0, f1);
+            }
+          } else {
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc)
+              mx = fmax3(mx, __uint_as_float(a0[cc]), __uint_as_float(a1[cc]));
           }
         }
-        const bool has = amax != INT_MIN;
-        const float mblk = has ? c * i2f_exact(static_cast<uint32_t>(amax)) : -INFINITY;
+        const bool has = mx != -INFINITY;
+        const float mblk = has ? __fmaf_rn(mx, c22, nc22) : -INFINITY;  // fl(c * A_max)
         // pass 2: p~ = exp2(z - mblk), codes rne(127 p~), row sum
         float rs = 0.0f;
         int8_t* prow = pbase + (j & 1) * (BM * BKV);
@@ -276,18 +324,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int half = 0; half < 2; ++half) {
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-              uint32_t b[4];
+              float f[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int cc = q4 * 4 + e;
                 const uint32_t av = half ? a1[cc] : a0[cc];
-                const int kidx = key0 + h * 32 + half * 16 + cc;
-                float p = ex2_approx(fmaf(i2f_exact(av), c, -mblk));
-                if (diag && kidx > i) p = 0.0f;
+                float p = ex2_approx(deq(av, c22, nc22) - mblk);
+                if (diag && key0 + h * 32 + half * 16 + cc > i) p = 0.0f;
                 rs += p;
-                b[e] = rne_byte(p * 127.0f);
+                f[e] = __fmaf_rn(p, 127.0f, kMagic);
               }
-              pk[half * 4 + q4] = pack4(b[0], b[1], b[2], b[3]);
+              pk[half * 4 + q4] = pack_magic4(f[0], f[1], f[2], f[3]);
             }
           }
           // keys h*32 .. h*32+31 are 16-byte chunks 2h and 2h+1 of this row
@@ -296,11 +343,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(prow + swz_offset(r, 2 * h + 1, 64)) =
               make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
+        // the S buffer is read: preload it for S_{j+2}
+#pragma unroll
+        for (int c = 0; c < 64; c += 16) tmem_fill16(sa + c, kMagicBits);
         const float m2n = fmaxf(m2, mblk);
         const float alpha = ex2_approx(m2 - m2n);
         const float eblk = has ? ex2_approx(mblk - m2n) : 0.0f;
         l = fmaf(l, alpha, eblk * rs);
-        const float beta = eblk * vsc[j] * (1.0f / 127.0f);
+        const float beta = eblk * sv * (1.0f / 127.0f);
+        tmem_st_wait();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sm.p_full[g][j & 1]);
@@ -322,11 +373,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       args.lse[static_cast<size_t>(bh) * N + i] = (m2 + log2f(l)) * 0.69314718055994531f;
     }
+    tc_fence_before();
+    named_barrier_sync(15, kThreads);
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace fwd

@@ -139,6 +139,13 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   for (int j = 0; j < N / 64; ++j) {
+    // the forward kernel's accumulator convention: preload 1.5 * 2^23, accumulate onto it
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 16) tmem_fill16(tmem + ((warp * 32u) << 16) + c0, kMagicBits);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
     if (threadIdx.x == 0) {
       const int bytes = (j == 0 ? 128 * D : 0) + 64 * D;
       mbar_arrive_expect_tx(&sm.full, bytes);
@@ -146,7 +153,7 @@ __global__ void __launch_bounds__(128, 1)
       tma_load_2d(sm.k, &tm_k, 0, bh * N + j * 64, &sm.full);
       mbar_wait(&sm.full, j & 1, 310);
       tc_fence_after();
-      fwd::issue_scores<D>(tmem, sm.q, sm.k, 64);
+      fwd::issue_scores<D>(tmem, sm.q, sm.k, 64, 1u);
       mma_commit(&sm.done);
     }
     __syncwarp();
@@ -158,7 +165,8 @@ __global__ void __launch_bounds__(128, 1)
       uint32_t v[16];
       tmem_ld16(tmem + ((warp * 32u) << 16) + c0, v);
       tmem_ld_wait();
-      for (int e = 0; e < 16; ++e) dst[c0 + e] = static_cast<int32_t>(v[e]);
+      for (int e = 0; e < 16; ++e)
+        dst[c0 + e] = static_cast<int32_t>(v[e]) - static_cast<int32_t>(kMagicBits);
     }
     tc_fence_before();
     __syncthreads();  // TMEM and the K tile are free for the next block

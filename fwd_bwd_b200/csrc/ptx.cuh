@@ -196,6 +196,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// Fills 16 consecutive 32-bit columns of the thread's TMEM lane with the same word.
+__device__ __forceinline__ void tmem_fill16(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+      "%1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -251,6 +260,36 @@ __device__ __forceinline__ uint32_t swz_offset(uint32_t row, uint32_t chunk,
 // ---------------------------------------------------------------------------------------------
 // Small numeric helpers
 // ---------------------------------------------------------------------------------------------
+// INT32 accumulators are preloaded with kMagicBits (the float 1.5 * 2^23) before the MMAs add
+// into them, so a result a (|a| < 2^22) reads back as the bit pattern of the float
+// 1.5 * 2^23 + a, with no integer instruction.
+constexpr uint32_t kMagicBits = 0x4B400000u;
+constexpr float kMagic = 12582912.0f;
+
+// s rounded toward zero to 22 significant bits: kMagic * scale22(s) is then exact in float32.
+__device__ __forceinline__ float scale22(float s) {
+  return __uint_as_float(__float_as_uint(s) & 0xFFFFFFFCu);
+}
+
+// Exact fl(a * s22) from the bits of the float kMagic + a, given s22 = scale22(s) and
+// neg_ms = -kMagic * s22: the fused multiply-add forms (kMagic + a) * s22 - kMagic * s22 =
+// a * s22 without intermediate rounding and rounds once.
+__device__ __forceinline__ float deq(uint32_t magic_plus_a, float s22, float neg_ms) {
+  return __fmaf_rn(__uint_as_float(magic_plus_a), s22, neg_ms);
+}
+
+// Four codes (each the low byte of a float x + 1.5*2^23) packed into one word, byte 0 first.
+__device__ __forceinline__ uint32_t pack_magic4(float a, float b, float c, float d) {
+  const uint32_t lo = __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x0040);
+  const uint32_t hi = __byte_perm(__float_as_uint(c), __float_as_uint(d), 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 // Exact int32 -> float for |v| < 2^22: the integer is placed in the mantissa of 1.5 * 2^23.
 __device__ __forceinline__ float i2f_exact(uint32_t v) {
   return __int_as_float(static_cast<int>(v) + 0x4B400000) - 12582912.0f;

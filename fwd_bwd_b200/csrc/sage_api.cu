@@ -191,6 +191,8 @@ int run_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse, cud
   const size_t smem = sage::fwd::smem_bytes<D>();
   auto kern = sage::fwd::attn_fwd_kernel<T, D>;
   if (set_smem(kern, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+  // register split between warpgroups (setmaxnreg) assumes exactly kLaunchRegs at launch
+  if (launch_regs(kern) != sage::fwd::kLaunchRegs) return SAGE_ERR_UNSUPPORTED;
   kern<<<BH * a.nsup, sage::fwd::kThreads, smem, st>>>(tq, tk, tv, a);
   return launch_status();
 }
