@@ -14,8 +14,9 @@
 //      dequantized by the tile scales and added to float32 accumulators in registers;
 //      every INT32 accumulator region is preloaded with the bits of 1.5 * 2^23 so the results
 //      read back as floats that one exact FMA dequantizes (see kMagicBits);
-//   4. dQ_t = dSc Kc per 64-key block (kind::i8), dequantized, summed and added to a float32
-//      dQ accumulator in global memory with vector atomics.
+//   4. dQ_t = dSc Kc per 64-key block (kind::i8; computed transposed for d = 128 so each
+//      warp's atomics cover contiguous channels of one row), dequantized, summed and added to a
+//      float32 dQ accumulator in global memory with atomics.
 // S and dP are double-buffered in TMEM, so the tensor core computes them for query tile i+1
 // while the compute warps turn tile i into codes.
 //
@@ -197,7 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ab = IsBf16<T>::value ? 1u : 0u;
       const uint32_t id_dp = instr_desc(1, ab, ab, false, false, BQ, BKT);
       const uint32_t id_mn = instr_desc(2, 1, 1, true, true, BKT, D);   // dV_t, dK_t
-      const uint32_t id_dq = instr_desc(2, 1, 1, false, true, BQ, D);   // dQ_t
+      const uint32_t id_dq = instr_desc(2, 1, 1, false, true, BQ, D);   // dQ_t (d = 64)
+      const uint32_t id_dqt = instr_desc(2, 1, 1, true, false, D, BQ);  // dQ_t^T (d = 128)
       const uint32_t kca = smem_u32(sm.kc), va = smem_u32(sm.v);
       const uint32_t pca = smem_u32(sm.pc), dsa = smem_u32(sm.dsc);
       // S and dP of query tile `it` into TMEM buffer it & 1
@@ -247,13 +249,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++dvdk_cnt;
           tc_fence_after();
         }
-        // dQ_t per 64-key block: dSc[:, block] Kc[block]
+        // dQ_t per 64-key block.  d = 128: dQ_t^T = Kc[block]^T dSc[:, block]^T (M = d,
+        // N = 128 queries; A = K codes read MN-major, B = dS codes K-major), so TMEM lanes are
+        // head-dim channels and the read-out's atomics cover contiguous channels of one row.
+        // d = 64: dQ_t = dSc[:, block] Kc[block] (M = 128 queries, N = d).
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-          for (int kk = 0; kk < 2; ++kk)
-            mma_i8(buf + hh * 128, smem_desc(dsa + hh * 64 + kk * 32, 16, 1024, kSwizzle128B),
-                   smem_desc(kca + (hh * 64 + kk * 32) * D, BKT * D, kSboC, kSwC), id_dq, 1u);
+          for (int kk = 0; kk < 2; ++kk) {
+            if constexpr (D == 128)
+              mma_i8(buf + hh * 128,
+                     smem_desc(kca + (hh * 64 + kk * 32) * D, BKT * D, kSboC, kSwC),
+                     smem_desc(dsa + hh * 64 + kk * 32, 16, 1024, kSwizzle128B), id_dqt, 1u);
+            else
+              mma_i8(buf + hh * 128, smem_desc(dsa + hh * 64 + kk * 32, 16, 1024, kSwizzle128B),
+                     smem_desc(kca + (hh * 64 + kk * 32) * D, BKT * D, kSboC, kSwC), id_dq, 1u);
+          }
         mma_commit(&sm.dq_full);
         mma_commit(&sm.q_empty[s]);
       }
@@ -443,11 +454,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sm.dvdk_free);
         ++dvdk_cnt;
       }
-      // step 4: dQ (thread = query row r, d columns of warpgroup h); afterwards the S region
-      // of this buffer is re-preloaded for tile it+2
+      // step 4: dQ, added to the float32 accumulator with atomics; afterwards the S region of
+      // this buffer is re-preloaded for tile it+2
       mbar_wait(&sm.dq_full, it & 1, 212);
       tc_fence_after();
-      {
+      if constexpr (D == 128) {
+        // thread = head-dim channel r, queries 64h .. 64h+63 of the tile (TMEM columns): each
+        // warp's atomic covers 32 consecutive channels of one dQ row
+        const int g = (64 * h) / args.q_block;
+        const float s0 = scale22(sm.sds[slot][g][0] * sk0 * args.tau);
+        const float s1 = scale22(sm.sds[slot][g][1] * sk1 * args.tau);
+        const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
+        float* dst = args.dq_acc + (static_cast<size_t>(row_base) + qt * BQ + 64 * h) * D + r;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+          uint32_t a0[16], a1[16];
+          tmem_ld16(lane_base + h * 64 + c0, a0);
+          tmem_ld16(lane_base + 128 + h * 64 + c0, a1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            atomicAdd(dst + static_cast<size_t>(c0 + e) * D,
+                      deq(a0[e], s0, n0) + deq(a1[e], s1, n1));
+        }
+#pragma unroll
+        for (int c = 0; c < 64; c += 16) tmem_fill16(lane_base + h * 64 + c, kMagicBits);
+        tmem_st_wait();
+      } else {
+        // thread = query row r, d columns of warpgroup h
         const float s0 = scale22(sm.sds[slot][g_row][0] * sk0 * args.tau);
         const float s1 = scale22(sm.sds[slot][g_row][1] * sk1 * args.tau);
         const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
