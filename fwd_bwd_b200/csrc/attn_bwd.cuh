@@ -30,6 +30,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "ptx.cuh"
@@ -61,20 +62,24 @@ template <int D>
 struct Stage {
   int8_t qc[BQ * D];
   int8_t doc[BQ * D];
-  uint8_t dor[BQ * D * 2];  // raw 16-bit dO, [D/64 atoms][128 rows][128 B]
 };
+
+constexpr int kDqRows = 16;  // queries per dQ staging round (d = 128)
 
 template <int D>
 struct Smem {
   Stage<D> st[2];
+  uint8_t dor[BQ * D * 2];  // raw 16-bit dO of the current tile, [D/64 atoms][128 rows][128 B]
   int8_t kc[BKT * D];
   uint8_t v[BKT * D * 2];  // raw 16-bit V, [D/64 atoms][128 rows][128 B]
   int8_t pc[BQ * BKT];     // P codes  [128 q][128 keys], 128-byte swizzle
   int8_t dsc[BQ * BKT];    // dS codes [128 q][128 keys], 128-byte swizzle
+  // d = 128: dQ staging for the asynchronous bulk reduction, [warpgroup][buffer][row][channel]
+  float dqs[D == 128 ? 2 : 1][2][D == 128 ? kDqRows * 128 : 4];
   float red_p[8], red_ds[8];
   float sp[3][2][2], sds[3][2][2];  // tile scales [tile % 3][q group][key half]
   float dot[BKT];                   // RMSNorm-backward row dot products (warpgroup 1 -> 0)
-  uint64_t kv_full, q_full[2], q_empty[2];
+  uint64_t kv_full, q_full[2], q_empty[2], dor_full, dor_free;
   uint64_t sdp_full[2], pds_ready, dvdk_full, dvdk_free, dq_full, dq_free;
   uint32_t tmem_base;
   int abort;
@@ -84,6 +89,18 @@ template <int D>
 constexpr size_t smem_bytes() {
   return sizeof(Smem<D>) + 1024;
 }
+
+// Every TMA destination / tensor-core operand tile starts on a 1024-byte boundary (the
+// structure itself is placed on one), as the swizzled layouts and descriptors require.
+template <int D>
+constexpr bool tiles_aligned() {
+  return offsetof(Smem<D>, st) % 1024 == 0 && sizeof(Stage<D>) % 1024 == 0 &&
+         offsetof(Stage<D>, doc) % 1024 == 0 && offsetof(Smem<D>, dor) % 1024 == 0 &&
+         offsetof(Smem<D>, kc) % 1024 == 0 && offsetof(Smem<D>, v) % 1024 == 0 &&
+         offsetof(Smem<D>, pc) % 1024 == 0 && offsetof(Smem<D>, dsc) % 1024 == 0 &&
+         offsetof(Smem<D>, dqs) % 1024 == 0;
+}
+static_assert(tiles_aligned<64>() && tiles_aligned<128>(), "shared-memory tiles misaligned");
 
 struct Args {
   const float* q_scale;   // [BH, N/q_block]
@@ -113,7 +130,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_kc,
                     const __grid_constant__ CUtensorMap tm_doc,
                     const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_v, Args args) {
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_dq, Args args) {
   constexpr uint32_t kSwC = (D == 128) ? kSwizzle128B : kSwizzle64B;  // code tiles
   constexpr uint32_t kSboC = 8 * D;
   constexpr int kHalfD = D / 2;
@@ -138,6 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.q_empty[s], 1);
       mbar_init(&sm.sdp_full[s], 1);
     }
+    mbar_init(&sm.dor_full, 1);
+    mbar_init(&sm.dor_free, 1);
     mbar_init(&sm.pds_ready, 256);
     mbar_init(&sm.dvdk_full, 1);
     mbar_init(&sm.dvdk_free, 256);
@@ -187,11 +207,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = it & 1;
         if (it >= 2) mbar_wait(&sm.q_empty[s], ((it >> 1) - 1) & 1, 200);
         const int row = row_base + (i_first + it) * BQ;
-        mbar_arrive_expect_tx(&sm.q_full[s], BQ * D * 4);
+        mbar_arrive_expect_tx(&sm.q_full[s], BQ * D * 2);
         tma_load_2d(sm.st[s].qc, &tm_qc, 0, row, &sm.q_full[s]);
         tma_load_2d(sm.st[s].doc, &tm_doc, 0, row, &sm.q_full[s]);
+        // the raw dO tile is single-buffered: wait until dP of the previous tile has read it
+        if (it >= 1) mbar_wait(&sm.dor_free, (it - 1) & 1, 206);
+        mbar_arrive_expect_tx(&sm.dor_full, BQ * D * 2);
         for (int a = 0; a < D / 64; ++a)
-          tma_load_2d(sm.st[s].dor + a * BQ * 128, &tm_do, a * 64, row, &sm.q_full[s]);
+          tma_load_2d(sm.dor + a * BQ * 128, &tm_do, a * 64, row, &sm.dor_full);
       }
     } else if (warp == kMmaWarp && lane == 0) {
       const uint32_t id_s = instr_desc(2, 1, 1, false, false, BQ, BKT);
@@ -206,8 +229,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_sdp = [&](int it) {
         const int s = it & 1;
         const uint32_t dst = tmem + s * 256;
-        const uint32_t qca = smem_u32(sm.st[s].qc), dora = smem_u32(sm.st[s].dor);
+        const uint32_t qca = smem_u32(sm.st[s].qc), dora = smem_u32(sm.dor);
         mbar_wait(&sm.q_full[s], (it >> 1) & 1, 202);
+        mbar_wait(&sm.dor_full, it & 1, 207);
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
@@ -220,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   smem_desc(va + off, 16, 1024, kSwizzle128B), id_dp, kk > 0 ? 1u : 0u);
         }
         mma_commit(&sm.sdp_full[s]);
+        mma_commit(&sm.dor_free);
       };
       mbar_wait(&sm.kv_full, 0, 201);
       issue_sdp(0);
@@ -295,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int c = 0; c < kHalfD; ++c) accv[c] = acck[c] = 0.0f;
     int dvdk_cnt = 0;
+    int dq_round = 0;  // dQ staging rounds so far (selects the staging buffer)
 
     // per-row inputs of query tile `it`: (c, lse2, D) for this thread's row
     auto row_inputs = [&](int it, float& c, float& lse2, float& dvr) {
@@ -459,26 +485,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&sm.dq_full, it & 1, 212);
       tc_fence_after();
       if constexpr (D == 128) {
-        // thread = head-dim channel r, queries 64h .. 64h+63 of the tile (TMEM columns): each
-        // warp's atomic covers 32 consecutive channels of one dQ row
+        // thread = head-dim channel r, queries 64h .. 64h+63 of the tile (TMEM columns).
+        // Rounds of 16 queries are staged in shared memory (row = query, 128 channels) and
+        // added to the global accumulator by the TMA unit, double-buffered per warpgroup.
         const int g = (64 * h) / args.q_block;
         const float s0 = scale22(sm.sds[slot][g][0] * sk0 * args.tau);
         const float s1 = scale22(sm.sds[slot][g][1] * sk1 * args.tau);
         const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
-        float* dst = args.dq_acc + (static_cast<size_t>(row_base) + qt * BQ + 64 * h) * D + r;
+        const bool issuer = (quarter == 0 && lane == 0);
 #pragma unroll 1
-        for (int c0 = 0; c0 < 64; c0 += 16) {
+        for (int rr = 0; rr < 64 / kDqRows; ++rr) {
+          const int q0 = 64 * h + kDqRows * rr;
+          float* stg = sm.dqs[h][dq_round & 1];
           uint32_t a0[16], a1[16];
-          tmem_ld16(lane_base + h * 64 + c0, a0);
-          tmem_ld16(lane_base + 128 + h * 64 + c0, a1);
+          tmem_ld16(lane_base + q0, a0);
+          tmem_ld16(lane_base + 128 + q0, a1);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            atomicAdd(dst + static_cast<size_t>(c0 + e) * D,
-                      deq(a0[e], s0, n0) + deq(a1[e], s1, n1));
+          for (int e = 0; e < kDqRows; ++e)
+            stg[e * 128 + r] = deq(a0[e], s0, n0) + deq(a1[e], s1, n1);
+          tmem_fill16(lane_base + q0, kMagicBits);
+          tmem_fill16(lane_base + 128 + q0, kMagicBits);
+          fence_proxy_async_smem();
+          named_barrier_sync(5 + h, 128);  // this round's rows are written
+          if (issuer) {
+            tma_reduce_add_2d(&tm_dq, stg, 0, row_base + qt * BQ + q0);
+            bulk_commit();
+            bulk_wait_read_1();  // the previous round's buffer has been read
+          }
+          named_barrier_sync(5 + h, 128);  // the other buffer may be rewritten
+          ++dq_round;
         }
-#pragma unroll
-        for (int c = 0; c < 64; c += 16) tmem_fill16(lane_base + h * 64 + c, kMagicBits);
         tmem_st_wait();
       } else {
         // thread = query row r, d columns of warpgroup h
@@ -560,6 +597,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4*>(dvp + c0) = pack8<T>(fv);
         *reinterpret_cast<uint4*>(dkp + c0) = pack8<T>(fk);
       }
+    }
+    if constexpr (D == 128) {
+      if (quarter == 0 && lane == 0) bulk_wait_all();  // dQ reductions complete
     }
     tc_fence_before();
     named_barrier_sync(15, kThreads);

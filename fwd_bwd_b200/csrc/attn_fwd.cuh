@@ -25,6 +25,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "ptx.cuh"
@@ -62,6 +63,16 @@ template <int D>
 constexpr size_t smem_bytes() {
   return sizeof(Smem<D>) + 1024;  // + alignment slack (tiles need 1024-byte alignment)
 }
+
+// Every TMA destination / tensor-core operand tile starts on a 1024-byte boundary.
+template <int D>
+constexpr bool tiles_aligned() {
+  return offsetof(Smem<D>, q) % 1024 == 0 && (BM * D) % 1024 == 0 &&
+         offsetof(Smem<D>, k) % 1024 == 0 && (BKV * D) % 1024 == 0 &&
+         offsetof(Smem<D>, v) % 1024 == 0 && offsetof(Smem<D>, p) % 1024 == 0 &&
+         (BM * BKV) % 1024 == 0;
+}
+static_assert(tiles_aligned<64>() && tiles_aligned<128>(), "shared-memory tiles misaligned");
 
 struct Args {
   const float* q_scale;

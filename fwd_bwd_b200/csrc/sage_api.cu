@@ -94,20 +94,25 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D map over a row-major [rows][inner] array of 1- or 2-byte elements.
+// Boxes whose rows are 64 or 128 bytes are swizzled to match the tensor cores' shared-memory
+// layouts; `swizzle = false` gives a plain row-major box (float32 reduction staging).
 bool make_map(CUtensorMap* m, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
-              uint32_t box_inner, uint32_t box_rows) {
+              uint32_t box_inner, uint32_t box_rows, bool swizzle = true) {
   auto fn = encode_fn();
   if (!fn) return false;
   const uint32_t row_bytes_box = box_inner * elem_bytes;
-  CUtensorMapSwizzle sw = row_bytes_box == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-                          : row_bytes_box == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                                : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUtensorMapSwizzle sw = !swizzle               ? CU_TENSOR_MAP_SWIZZLE_NONE
+                          : row_bytes_box == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : row_bytes_box == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
+  const CUtensorMapDataType dt = elem_bytes == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {inner * elem_bytes};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
-                  2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -225,12 +230,13 @@ int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const
         p->qknorm);
     return launch_status();
   }
-  CUtensorMap tqc, tkc, tdoc, tdo, tv;
+  CUtensorMap tqc, tkc, tdoc, tdo, tv, tdq;
   if (!make_map(&tqc, qb->q_codes, 1, D, rows, D, sage::bwd::BQ) ||
       !make_map(&tkc, qb->k_codes, 1, D, rows, D, sage::bwd::BKT) ||
       !make_map(&tdoc, doc, 1, D, rows, D, sage::bwd::BQ) ||
       !make_map(&tdo, dout, 2, D, rows, 64, sage::bwd::BQ) ||
-      !make_map(&tv, v, 2, D, rows, 64, sage::bwd::BKT))
+      !make_map(&tv, v, 2, D, rows, 64, sage::bwd::BKT) ||
+      !make_map(&tdq, dqacc, 4, D, rows, D, sage::bwd::kDqRows, false))
     return SAGE_ERR_CUDA;
   sage::bwd::Args a;
   a.q_scale = qb->q_scale;
@@ -257,7 +263,8 @@ int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const
   // allocation of exactly kLaunchRegs per thread.  Any other allocation could leave the
   // increasing warpgroups waiting, so refuse to launch.
   if (launch_regs(kern) != sage::bwd::kLaunchRegs) return SAGE_ERR_UNSUPPORTED;
-  kern<<<BH * (N / sage::bwd::BKT), sage::bwd::kThreads, smem, st>>>(tqc, tkc, tdoc, tdo, tv, a);
+  kern<<<BH * (N / sage::bwd::BKT), sage::bwd::kThreads, smem, st>>>(tqc, tkc, tdoc, tdo, tv, tdq,
+                                                                     a);
   return launch_status();
 }
 
