@@ -44,8 +44,8 @@ constexpr int BKT = 128;  // keys per CTA
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kLaunchRegs = 168;   // registers per thread the kernel must be launched with
-constexpr int kComputeRegs = 232;  // compute warpgroups after setmaxnreg.inc
-constexpr int kOtherRegs = 40;     // producer / MMA warpgroup after setmaxnreg.dec
+constexpr int kComputeRegs = 224;  // compute warpgroups after setmaxnreg.inc
+constexpr int kOtherRegs = 56;     // producer / MMA warpgroup after setmaxnreg.dec
 static_assert(2 * 128 * kComputeRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 
@@ -270,6 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    smem_desc(qca + qr * D, BQ * D, kSboC, kSwC), id_mn, 1u);
           }
           mma_commit(&sm.dvdk_full);
+          // dK_t / dV_t are the last readers of this tile's Q and dO codes: release the stage
+          if (g == G - 1) mma_commit(&sm.q_empty[s]);
           mbar_wait(&sm.dvdk_free, dvdk_cnt & 1, 205);
           ++dvdk_cnt;
           tc_fence_after();
@@ -291,7 +293,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                      smem_desc(kca + (hh * 64 + kk * 32) * D, BKT * D, kSboC, kSwC), id_dq, 1u);
           }
         mma_commit(&sm.dq_full);
-        mma_commit(&sm.q_empty[s]);
       }
     }
     // teardown: every MMA has completed once the compute warps pass this barrier
@@ -349,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sa[16], pa[16];
         tmem_ld16(lane_base + col, sa);
         tmem_ld16(lane_base + 128 + col, pa);
-        tmem_ld_wait();
+        tmem_ld_wait_regs(sa, pa);
         if (diag) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -412,14 +413,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qt = i_first + it;
       const size_t grow = static_cast<size_t>(row_base) + qt * BQ + r;
       if (it + 1 < nq) row_inputs(it + 1, c_n, lse2_n, dvr_n);  // loads in flight during pass B
-      // pass B: INT8 codes into shared memory; the dV_t / dK_t regions re-preloaded
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      // pass B: INT8 codes into shared memory; the dV_t / dK_t regions re-preloaded.  The TMEM
+      // loads of chunk ch+1 are in flight while chunk ch is converted.
+      auto proc_b = [&](uint32_t (&sa)[16], uint32_t (&pa)[16], int ch) {
         const int col = h * 64 + ch * 16;
-        uint32_t sa[16], pa[16];
-        tmem_ld16(lane_base + col, sa);
-        tmem_ld16(lane_base + 128 + col, pa);
-        tmem_ld_wait();
         uint32_t cp[4], cd[4];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -439,6 +436,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_fill16(lane_base + col, kMagicBits);
           tmem_fill16(lane_base + 128 + col, kMagicBits);
         }
+      };
+      {
+        const int c0 = h * 64;
+        uint32_t sa0[16], pa0[16], sa1[16], pa1[16];
+        tmem_ld16(lane_base + c0, sa0);
+        tmem_ld16(lane_base + 128 + c0, pa0);
+        tmem_ld_wait_regs(sa0, pa0);
+        tmem_ld16(lane_base + c0 + 16, sa1);
+        tmem_ld16(lane_base + 128 + c0 + 16, pa1);
+        proc_b(sa0, pa0, 0);
+        tmem_ld_wait_regs(sa1, pa1);
+        tmem_ld16(lane_base + c0 + 32, sa0);
+        tmem_ld16(lane_base + 128 + c0 + 32, pa0);
+        proc_b(sa1, pa1, 1);
+        tmem_ld_wait_regs(sa0, pa0);
+        tmem_ld16(lane_base + c0 + 48, sa1);
+        tmem_ld16(lane_base + 128 + c0 + 48, pa1);
+        proc_b(sa0, pa0, 2);
+        tmem_ld_wait_regs(sa1, pa1);
+        proc_b(sa1, pa1, 3);
       }
       tmem_st_wait();
       fence_proxy_async_smem();
@@ -460,20 +477,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sv22 = scale22(sm.sp[slot][g][kh] * sdo);
         const float sk22 = scale22(sm.sds[slot][g][kh] * sqg * args.tau);
         const float nsv = __fmul_rn(-kMagic, sv22), nsk = __fmul_rn(-kMagic, sk22);
+        // 16-column chunks; the loads of chunk c+1 are in flight while chunk c accumulates
+        uint32_t tv0[16], tk0[16], tv1[16], tk1[16];
+        tmem_ld16(lane_base + h * kHalfD, tv0);
+        tmem_ld16(lane_base + 128 + h * kHalfD, tk0);
+        tmem_ld_wait_regs(tv0, tk0);
 #pragma unroll
         for (int c0 = 0; c0 < kHalfD; c0 += 16) {
           const int col = h * kHalfD + c0;
-          uint32_t tv[16], tk[16];
-          tmem_ld16(lane_base + col, tv);
-          tmem_ld16(lane_base + 128 + col, tk);
-          tmem_ld_wait();
+          const bool odd = (c0 / 16) & 1;
+          if (c0 + 16 < kHalfD) {
+            if (odd) {
+              tmem_ld16(lane_base + col + 16, tv0);
+              tmem_ld16(lane_base + 128 + col + 16, tk0);
+            } else {
+              tmem_ld16(lane_base + col + 16, tv1);
+              tmem_ld16(lane_base + 128 + col + 16, tk1);
+            }
+          }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            accv[c0 + e] += deq(tv[e], sv22, nsv);
-            acck[c0 + e] += deq(tk[e], sk22, nsk);
+            accv[c0 + e] += deq(odd ? tv1[e] : tv0[e], sv22, nsv);
+            acck[c0 + e] += deq(odd ? tk1[e] : tk0[e], sk22, nsk);
           }
           tmem_fill16(lane_base + col, kMagicBits);
           tmem_fill16(lane_base + 128 + col, kMagicBits);
+          if (c0 + 16 < kHalfD) {
+            if (odd)
+              tmem_ld_wait_regs(tv0, tk0);
+            else
+              tmem_ld_wait_regs(tv1, tk1);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
