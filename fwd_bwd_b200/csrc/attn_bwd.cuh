@@ -344,39 +344,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&sm.sdp_full[b], (it >> 1) & 1, 210);
       tc_fence_after();
       float pmax = 0.0f, dsmax = 0.0f;
-#pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
-        const int col = h * 64 + ch * 16;
-        uint32_t sa[16], pa[16];
-        tmem_ld16(lane_base + col, sa);
-        tmem_ld16(lane_base + 128 + col, pa);
-        tmem_ld_wait_regs(sa, pa);
-        if (diag) {
+      // 8-column chunks, double-buffered: the TMEM loads of chunk ch+1 are in flight while
+      // chunk ch computes
+      auto proc_a = [&](uint32_t (&sa)[8], uint32_t (&pa)[8], int col) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int key = key_base + col + e;
-            float p = ex2_approx(deq(sa[e], c22, nc22) - lse2);
-            p = key > qrow ? 0.0f : p;
-            const float ds = p * (__uint_as_float(pa[e]) - dvr);
-            dsmax = fmaxf(dsmax, fabsf(ds));
-            sa[e] = __float_as_uint(p);
-            pa[e] = __float_as_uint(ds);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p = ex2_approx(deq(sa[e], c22, nc22) - lse2);
-            const float ds = p * (__uint_as_float(pa[e]) - dvr);
-            dsmax = fmaxf(dsmax, fabsf(ds));
-            sa[e] = __float_as_uint(p);
-            pa[e] = __float_as_uint(ds);
-          }
+        for (int e = 0; e < 8; ++e) {
+          float p = ex2_approx(deq(sa[e], c22, nc22) - lse2);
+          if (diag && key_base + col + e > qrow) p = 0.0f;
+          const float ds = p * (__uint_as_float(pa[e]) - dvr);
+          dsmax = fmaxf(dsmax, fabsf(ds));
+          sa[e] = __float_as_uint(p);
+          pa[e] = __float_as_uint(ds);
         }
 #pragma unroll
-        for (int e = 0; e < 16; e += 2)
+        for (int e = 0; e < 8; e += 2)
           pmax = fmax3(pmax, __uint_as_float(sa[e]), __uint_as_float(sa[e + 1]));
-        tmem_st16(lane_base + col, sa);
-        tmem_st16(lane_base + 128 + col, pa);
+        tmem_st8(lane_base + col, sa);
+        tmem_st8(lane_base + 128 + col, pa);
+      };
+      {
+        const int c0 = h * 64;
+        uint32_t sa0[8], pa0[8], sa1[8], pa1[8];
+        tmem_ld8(lane_base + c0, sa0);
+        tmem_ld8(lane_base + 128 + c0, pa0);
+        tmem_ld_wait_regs8(sa0, pa0);
+#pragma unroll
+        for (int ch = 0; ch < 8; ch += 2) {
+          tmem_ld8(lane_base + c0 + 8 * ch + 8, sa1);
+          tmem_ld8(lane_base + 128 + c0 + 8 * ch + 8, pa1);
+          proc_a(sa0, pa0, c0 + 8 * ch);
+          tmem_ld_wait_regs8(sa1, pa1);
+          if (ch + 2 < 8) {
+            tmem_ld8(lane_base + c0 + 8 * ch + 16, sa0);
+            tmem_ld8(lane_base + 128 + c0 + 8 * ch + 16, pa0);
+          }
+          proc_a(sa1, pa1, c0 + 8 * ch + 8);
+          if (ch + 2 < 8) tmem_ld_wait_regs8(sa0, pa0);
+        }
       }
       tmem_st_wait();
       // per-tile maxima: tile = q_block rows x 64 keys (this warpgroup's key block)

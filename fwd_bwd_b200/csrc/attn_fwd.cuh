@@ -265,19 +265,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float nb22 = __fmul_rn(-kMagic, b22);
         mbar_wait(&sm.pv_full[g], jj & 1, 110);
         tc_fence_after();
+        // 16-column chunks, double-buffered: the load of chunk c+1 is in flight while chunk c
+        // is folded
+        uint32_t a0[16], a1[16];
+        tmem_ld16(lane_base + 128, a0);
+        tmem_ld_wait_regs(a0, a1);
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t a0[16], a1[16];
-          tmem_ld16(lane_base + 128 + c0, a0);
           tmem_ld16(lane_base + 128 + c0 + 16, a1);
-          tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
+          for (int c = 0; c < 16; ++c)
             O[c0 + c] = fmaf(O[c0 + c], alpha_prev, deq(a0[c], b22, nb22));
-            O[c0 + 16 + c] = fmaf(O[c0 + 16 + c], alpha_prev, deq(a1[c], b22, nb22));
-          }
           tmem_fill16(lane_base + 128 + c0, kMagicBits);
+          tmem_ld_wait_regs(a1, a0);
+          if (c0 + 32 < D) tmem_ld16(lane_base + 128 + c0 + 32, a0);
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            O[c0 + 16 + c] = fmaf(O[c0 + 16 + c], alpha_prev, deq(a1[c], b22, nb22));
           tmem_fill16(lane_base + 128 + c0 + 16, kMagicBits);
+          if (c0 + 32 < D) tmem_ld_wait_regs(a0, a1);
         }
         tmem_st_wait();
         tc_fence_before();
