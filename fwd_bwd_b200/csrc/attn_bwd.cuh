@@ -81,6 +81,7 @@ struct Smem {
   float dot[BKT];                   // RMSNorm-backward row dot products (warpgroup 1 -> 0)
   uint64_t kv_full, q_full[2], q_empty[2], dor_full, dor_free;
   uint64_t sdp_full[2], pds_ready, dvdk_full, dvdk_free, dq_full, dq_free;
+  uint64_t scales_full[2];  // tile parity: the P / dS scales of both warpgroups are written
   uint32_t tmem_base;
   int abort;
 };
@@ -159,6 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.dor_full, 1);
     mbar_init(&sm.dor_free, 1);
     mbar_init(&sm.pds_ready, 256);
+    for (int s = 0; s < 2; ++s)  // writers: one per q group per key half
+      mbar_init(&sm.scales_full[s], 2 * (BQ / args.q_block));
     mbar_init(&sm.dvdk_full, 1);
     mbar_init(&sm.dvdk_free, 256);
     mbar_init(&sm.dq_full, 1);
@@ -400,12 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0 && (quarter % wpg) == 0) {
         sm.sp[slot][g_row][h] = __fdiv_rn(tp, 127.0f);
         sm.sds[slot][g_row][h] = __fdiv_rn(tds, 127.0f);
+        mbar_arrive(&sm.scales_full[it & 1]);  // read by both warpgroups in the read-outs
       }
       ip = tp > 0.0f ? __fdiv_rn(127.0f, tp) : 0.0f;
       ids = tds > 0.0f ? __fdiv_rn(127.0f, tds) : 0.0f;
-      tc_fence_before();
-      named_barrier_sync(3, 256);  // all tile scales written; reads of sm.red_* done
-      tc_fence_after();
+      // No CTA-wide barrier here: the warpgroups may drift apart.  sm.red_* is rewritten only
+      // in pass A of tile it+1, which waits for that tile's S / dP, issued after every thread
+      // released tile it-1's dQ -- i.e. after every warp finished reading sm.red_* of tile it.
     };
 
     float c_n, lse2_n, dvr_n, ip, ids;
@@ -469,7 +473,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       float ip_n = 0.0f, ids_n = 0.0f;
       if (it + 1 < nq) pass_a(it + 1, c_n, lse2_n, dvr_n, ip_n, ids_n);
       // step 3: dV_t, dK_t (thread = key row r, d columns of warpgroup h) into registers;
-      // the read columns are re-preloaded for dQ_t
+      // the read columns are re-preloaded for dQ_t.  The tile scales of both warpgroups are
+      // read from here on.  One barrier per tile parity, so arrivals for tiles it and it+1
+      // never share a phase; a writer cannot reach tile it+2 before this thread released tile
+      // it's dQ (its S / dP are issued only after that).
+      mbar_wait(&sm.scales_full[b], (it >> 1) & 1, 213);
       for (int g = 0; g < G; ++g) {
         const size_t qb = static_cast<size_t>(bh) * nqb + (qt * BQ + g * args.q_block) /
                                                               args.q_block;
