@@ -405,8 +405,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.sds[slot][g_row][h] = __fdiv_rn(tds, 127.0f);
         mbar_arrive(&sm.scales_full[it & 1]);  // read by both warpgroups in the read-outs
       }
-      ip = tp > 0.0f ? __fdiv_rn(127.0f, tp) : 0.0f;
-      ids = tds > 0.0f ? __fdiv_rn(127.0f, tds) : 0.0f;
+      // code multipliers: the codes are not compared bit for bit, so the fast divide (within
+      // 2 ulp) serves; the stored scales above are IEEE quotients
+      ip = tp > 0.0f ? __fdividef(127.0f, tp) : 0.0f;
+      ids = tds > 0.0f ? __fdividef(127.0f, tds) : 0.0f;
       // No CTA-wide barrier here: the warpgroups may drift apart.  sm.red_* is rewritten only
       // in pass A of tile it+1, which waits for that tile's S / dP, issued after every thread
       // released tile it-1's dQ -- i.e. after every warp finished reading sm.red_* of tile it.
