@@ -210,3 +210,63 @@ def qk_int32_debug(qb: QuantBufs, like: torch.Tensor, cfg: Config, bh: int,
 
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+def fwd_bwd_host(q, k, v, dout, cfg: Config, o=None, dq=None, dk=None, dv=None,
+                 chunks: int = 16, device=None):
+    """Prologue + forward + backward on host-resident (pinned) [B, H, N, d] tensors.
+
+    Every (batch, head) is an independent problem, so the batch is cut into ``chunks`` slices
+    that flow through three CUDA streams: host-to-device copies of slice c+1 and
+    device-to-host copies of slice c-1 overlap the kernels of slice c.  Two sets of device
+    buffers alternate between slices.  Results (o, dq, dk, dv) are written into pinned host
+    tensors (allocated when not given); the call returns once they are complete.  Inputs
+    should be pinned (page-locked) for the copies to run asynchronously.
+    """
+    device = torch.device("cuda") if device is None else torch.device(device)
+    B = q.shape[0]
+    chunks = max(1, min(chunks, B))
+    bounds = [(B * c // chunks, B * (c + 1) // chunks) for c in range(chunks)]
+    outs = []
+    for t, ref in ((o, q), (dq, q), (dk, k), (dv, v)):
+        outs.append(t if t is not None else torch.empty(ref.shape, dtype=ref.dtype,
+                                                         pin_memory=True))
+    cb = max(b1 - b0 for b0, b1 in bounds)
+    shape = (cb,) + tuple(q.shape[1:])
+    sets = []
+    for _ in range(2):
+        ins = [torch.empty(shape, dtype=q.dtype, device=device) for _ in range(4)]
+        res = [torch.empty(shape, dtype=q.dtype, device=device) for _ in range(4)]
+        sets.append((ins, res))
+    s_in, s_comp, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
+    for c, (b0, b1) in enumerate(bounds):
+        si = c % 2
+        ins, res = sets[si]
+        n = b1 - b0
+        with torch.cuda.stream(s_in):
+            if used[si]:
+                s_in.wait_event(comp_done[si])  # the kernels of slice c-2 have read the inputs
+            for dst, src in zip(ins, (q, k, v, dout)):
+                dst[:n].copy_(src[b0:b1], non_blocking=True)
+            in_done[si].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(in_done[si])
+            if used[si]:
+                s_comp.wait_event(out_done[si])  # slice c-2's results have left the device
+            qd, kd, vd, dod = (t[:n] for t in ins)
+            qb = quant_prologue(qd, kd, vd, cfg)
+            od, lse = attn_fwd(qb, qd, cfg, o=res[0][:n])
+            attn_bwd(qd, kd, vd, qb, od, lse, dod, cfg, res[1][:n], res[2][:n], res[3][:n])
+            comp_done[si].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[si])
+            for src, dst in zip(res, outs):
+                dst[b0:b1].copy_(src[:n], non_blocking=True)
+            out_done[si].record(s_out)
+        used[si] = True
+    s_out.synchronize()
+    return tuple(outs)
