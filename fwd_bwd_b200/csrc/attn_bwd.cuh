@@ -23,7 +23,8 @@
 // Warps 0-7 compute (warpgroup h owns keys 64h .. 64h+63 in step 2 and d columns h*d/2 ..
 // in steps 3-4), warp 8 is the TMA producer, warp 9 the MMA issuer, warps 10-11 idle.  The
 // producer warpgroup gives registers to the compute warpgroups (setmaxnreg): at launch every
-// thread holds 168, afterwards 256 x 232 + 128 x 40 = 64512 = 384 x 168.
+// thread holds 168, afterwards 256 x 208 + 128 x 80 = 63488 <= 384 x 168.  The MMA thread keeps
+// 80: with fewer it spills, and its reloads delay the tensor-core issue.
 // TMEM (512 columns): buffer b in {0,1} at [256b, 256b+256): [0,128) S -> P -> dV_t ->
 // dQ_t(block 0); [128,256) dP -> dS -> dK_t -> dQ_t(block 1).
 #pragma once
@@ -32,6 +33,8 @@
 #include <cuda_fp16.h>
 #include <stddef.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "ptx.cuh"
 #include "rowops.cuh"
@@ -44,8 +47,8 @@ constexpr int BKT = 128;  // keys per CTA
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kLaunchRegs = 168;   // registers per thread the kernel must be launched with
-constexpr int kComputeRegs = 224;  // compute warpgroups after setmaxnreg.inc
-constexpr int kOtherRegs = 56;     // producer / MMA warpgroup after setmaxnreg.dec
+constexpr int kComputeRegs = 208;  // compute warpgroups after setmaxnreg.inc
+constexpr int kOtherRegs = 80;     // producer / MMA warpgroup after setmaxnreg.dec
 static_assert(2 * 128 * kComputeRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 
@@ -65,6 +68,7 @@ struct Stage {
 };
 
 constexpr int kDqRows = 16;  // queries per dQ staging round (d = 128)
+constexpr int kDqCols = 32;  // channels per warp in a dQ staging round (d = 128)
 
 template <int D>
 struct Smem {
@@ -74,9 +78,11 @@ struct Smem {
   uint8_t v[BKT * D * 2];  // raw 16-bit V, [D/64 atoms][128 rows][128 B]
   int8_t pc[BQ * BKT];     // P codes  [128 q][128 keys], 128-byte swizzle
   int8_t dsc[BQ * BKT];    // dS codes [128 q][128 keys], 128-byte swizzle
-  // d = 128: dQ staging for the asynchronous bulk reduction, [warpgroup][buffer][row][channel]
-  float dqs[D == 128 ? 2 : 1][2][D == 128 ? kDqRows * 128 : 4];
-  float red_p[8], red_ds[8];
+  // d = 128: dQ staging for the asynchronous bulk reduction,
+  // [compute warp][buffer][query row][channel of the warp]
+  float dqs[D == 128 ? 8 : 1][2][D == 128 ? kDqRows * kDqCols : 4];
+  alignas(16) float red_p[2][8];  // per-warp tile maxima of P, [tile parity][warp]
+  alignas(16) float red_ds[2][8];  // and of |dS|
   float sp[3][2][2], sds[3][2][2];  // tile scales [tile % 3][q group][key half]
   float dot[BKT];                   // RMSNorm-backward row dot products (warpgroup 1 -> 0)
   uint64_t kv_full, q_full[2], q_empty[2], dor_full, dor_free;
@@ -340,7 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = it & 1, slot = it % 3;
       const uint32_t lane_base = tmem + lane_off + b * 256;
       const int qt = i_first + it;
-      const int qrow = qt * BQ + r;
       const bool diag = args.causal && (qt == t);
       const float c22 = scale22(c);
       const float nc22 = __fmul_rn(-kMagic, c22);
@@ -348,24 +353,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       float pmax = 0.0f, dsmax = 0.0f;
       // 8-column chunks, double-buffered: the TMEM loads of chunk ch+1 are in flight while
-      // chunk ch computes
-      auto proc_a = [&](uint32_t (&sa)[8], uint32_t (&pa)[8], int col) {
+      // chunk ch computes.  The causal mask (key > query) exists only on the diagonal tile, so
+      // the chunk loop is compiled twice and the off-diagonal copy carries no mask test.
+      auto chunks = [&](auto masked) {
+        auto proc_a = [&](uint32_t (&sa)[8], uint32_t (&pa)[8], int col) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float p = ex2_approx(deq(sa[e], c22, nc22) - lse2);
-          if (diag && key_base + col + e > qrow) p = 0.0f;
-          const float ds = p * (__uint_as_float(pa[e]) - dvr);
-          dsmax = fmaxf(dsmax, fabsf(ds));
-          sa[e] = __float_as_uint(p);
-          pa[e] = __float_as_uint(ds);
-        }
+          for (int e = 0; e < 8; ++e) {
+            float p = ex2_approx(deq(sa[e], c22, nc22) - lse2);
+            if constexpr (decltype(masked)::value) {
+              if (col + e > r) p = 0.0f;  // diagonal tile: key index - query index = col - r
+            }
+            const float ds = p * (__uint_as_float(pa[e]) - dvr);
+            dsmax = fmaxf(dsmax, fabsf(ds));
+            sa[e] = __float_as_uint(p);
+            pa[e] = __float_as_uint(ds);
+          }
 #pragma unroll
-        for (int e = 0; e < 8; e += 2)
-          pmax = fmax3(pmax, __uint_as_float(sa[e]), __uint_as_float(sa[e + 1]));
-        tmem_st8(lane_base + col, sa);
-        tmem_st8(lane_base + 128 + col, pa);
-      };
-      {
+          for (int e = 0; e < 8; e += 2)
+            pmax = fmax3(pmax, __uint_as_float(sa[e]), __uint_as_float(sa[e + 1]));
+          tmem_st8(lane_base + col, sa);
+          tmem_st8(lane_base + 128 + col, pa);
+        };
         const int c0 = h * 64;
         uint32_t sa0[8], pa0[8], sa1[8], pa1[8];
         tmem_ld8(lane_base + c0, sa0);
@@ -384,21 +392,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           proc_a(sa1, pa1, c0 + 8 * ch + 8);
           if (ch + 2 < 8) tmem_ld_wait_regs8(sa0, pa0);
         }
-      }
+      };
+      if (diag)
+        chunks(std::true_type{});
+      else
+        chunks(std::false_type{});
       tmem_st_wait();
       // per-tile maxima: tile = q_block rows x 64 keys (this warpgroup's key block)
       pmax = warp_max(pmax);
       dsmax = warp_max(dsmax);
       if (lane == 0) {
-        sm.red_p[h * 4 + quarter] = pmax;
-        sm.red_ds[h * 4 + quarter] = dsmax;
+        sm.red_p[b][h * 4 + quarter] = pmax;
+        sm.red_ds[b][h * 4 + quarter] = dsmax;
       }
       named_barrier_sync(1 + h, 128);
-      float tp = 0.0f, tds = 0.0f;
-      const int w0 = (quarter / wpg) * wpg;
-      for (int w = w0; w < w0 + wpg; ++w) {
-        tp = fmaxf(tp, sm.red_p[h * 4 + w]);
-        tds = fmaxf(tds, sm.red_ds[h * 4 + w]);
+      // the q_block group's warps: all four (q_block = 128) or this warp's pair (64)
+      const float4 rp = *reinterpret_cast<const float4*>(&sm.red_p[b][h * 4]);
+      const float4 rd = *reinterpret_cast<const float4*>(&sm.red_ds[b][h * 4]);
+      float tp, tds;
+      if (wpg == 4) {
+        tp = fmaxf(fmaxf(rp.x, rp.y), fmaxf(rp.z, rp.w));
+        tds = fmaxf(fmaxf(rd.x, rd.y), fmaxf(rd.z, rd.w));
+      } else {
+        tp = quarter < 2 ? fmaxf(rp.x, rp.y) : fmaxf(rp.z, rp.w);
+        tds = quarter < 2 ? fmaxf(rd.x, rd.y) : fmaxf(rd.z, rd.w);
       }
       if (lane == 0 && (quarter % wpg) == 0) {
         sm.sp[slot][g_row][h] = __fdiv_rn(tp, 127.0f);
@@ -409,9 +426,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // 2 ulp) serves; the stored scales above are IEEE quotients
       ip = tp > 0.0f ? __fdividef(127.0f, tp) : 0.0f;
       ids = tds > 0.0f ? __fdividef(127.0f, tds) : 0.0f;
-      // No CTA-wide barrier here: the warpgroups may drift apart.  sm.red_* is rewritten only
-      // in pass A of tile it+1, which waits for that tile's S / dP, issued after every thread
-      // released tile it-1's dQ -- i.e. after every warp finished reading sm.red_* of tile it.
+      // No CTA-wide barrier here: the warpgroups may drift apart.  sm.red_*[b] is rewritten
+      // only in pass A of tile it+2, which waits for that tile's S / dP, issued after every
+      // thread released tile it's dQ -- i.e. after every warp finished reading it for tile it.
+      // (Tiles 0 and 1 have their S / dP issued back to back, hence the two slots.)
     };
 
     float c_n, lse2_n, dvr_n, ip, ids;
@@ -471,6 +489,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sm.pds_ready);
+      // dO and Q block scales of this tile's q_block groups, used by the dV / dK read-out
+      // (loaded here so that pass A hides their latency)
+      float sdo_t[2], sq_t[2];
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const size_t qb = static_cast<size_t>(bh) * nqb +
+                          (qt * BQ + (g < G ? g : 0) * args.q_block) / args.q_block;
+        sdo_t[g] = args.do_scale[qb];
+        sq_t[g] = args.q_scale[qb];
+      }
       // pass A of the next tile while the tensor core works on this one
       float ip_n = 0.0f, ids_n = 0.0f;
       if (it + 1 < nq) pass_a(it + 1, c_n, lse2_n, dvr_n, ip_n, ids_n);
@@ -481,10 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // it's dQ (its S / dP are issued only after that).
       mbar_wait(&sm.scales_full[b], (it >> 1) & 1, 213);
       for (int g = 0; g < G; ++g) {
-        const size_t qb = static_cast<size_t>(bh) * nqb + (qt * BQ + g * args.q_block) /
-                                                              args.q_block;
-        const float sdo = args.do_scale[qb];
-        const float sqg = args.q_scale[qb];
+        const float sdo = g == 0 ? sdo_t[0] : sdo_t[1];
+        const float sqg = g == 0 ? sq_t[0] : sq_t[1];
         const int kh = r >> 6;
         mbar_wait(&sm.dvdk_full, dvdk_cnt & 1, 211);
         tc_fence_after();
@@ -534,35 +560,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       if constexpr (D == 128) {
         // thread = head-dim channel r, queries 64h .. 64h+63 of the tile (TMEM columns).
-        // Rounds of 16 queries are staged in shared memory (row = query, 128 channels) and
-        // added to the global accumulator by the TMA unit, double-buffered per warpgroup.
+        // Each warp stages rounds of 16 queries x its 32 channels in its own shared-memory
+        // buffers (double-buffered) and its lane 0 hands them to the TMA unit, which adds them
+        // to the global accumulator; no warp waits for another.  The TMEM loads of round rr+1
+        // are in flight while round rr is staged.
         const int g = (64 * h) / args.q_block;
         const float s0 = scale22(sm.sds[slot][g][0] * sk0 * args.tau);
         const float s1 = scale22(sm.sds[slot][g][1] * sk1 * args.tau);
         const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
-        const bool issuer = (quarter == 0 && lane == 0);
-#pragma unroll 1
+        uint32_t a0[16], a1[16];
+        tmem_ld16(lane_base + 64 * h, a0);
+        tmem_ld16(lane_base + 128 + 64 * h, a1);
+        tmem_ld_wait_regs(a0, a1);
+#pragma unroll
         for (int rr = 0; rr < 64 / kDqRows; ++rr) {
           const int q0 = 64 * h + kDqRows * rr;
-          float* stg = sm.dqs[h][dq_round & 1];
-          uint32_t a0[16], a1[16];
-          tmem_ld16(lane_base + q0, a0);
-          tmem_ld16(lane_base + 128 + q0, a1);
-          tmem_ld_wait();
+          float v[kDqRows];
 #pragma unroll
-          for (int e = 0; e < kDqRows; ++e)
-            stg[e * 128 + r] = deq(a0[e], s0, n0) + deq(a1[e], s1, n1);
+          for (int e = 0; e < kDqRows; ++e) v[e] = deq(a0[e], s0, n0) + deq(a1[e], s1, n1);
           tmem_fill16(lane_base + q0, kMagicBits);
           tmem_fill16(lane_base + 128 + q0, kMagicBits);
-          fence_proxy_async_smem();
-          named_barrier_sync(5 + h, 128);  // this round's rows are written
-          if (issuer) {
-            tma_reduce_add_2d(&tm_dq, stg, 0, row_base + qt * BQ + q0);
-            bulk_commit();
-            bulk_wait_read_1();  // the previous round's buffer has been read
+          if (rr + 1 < 64 / kDqRows) {
+            tmem_ld16(lane_base + q0 + kDqRows, a0);
+            tmem_ld16(lane_base + 128 + q0 + kDqRows, a1);
           }
-          named_barrier_sync(5 + h, 128);  // the other buffer may be rewritten
+          float* stg = sm.dqs[warp][dq_round & 1];
+          // the buffer's previous round (two rounds back) has been read by the TMA unit
+          if (lane == 0) bulk_wait_read_1();
+          __syncwarp();
+#pragma unroll
+          for (int e = 0; e < kDqRows; ++e) stg[e * kDqCols + lane] = v[e];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_2d(&tm_dq, stg, quarter * kDqCols, row_base + qt * BQ + q0);
+            bulk_commit();
+          }
           ++dq_round;
+          if (rr + 1 < 64 / kDqRows) tmem_ld_wait_regs(a0, a1);
         }
         tmem_st_wait();
       } else {
@@ -647,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if constexpr (D == 128) {
-      if (quarter == 0 && lane == 0) bulk_wait_all();  // dQ reductions complete
+      if (lane == 0) bulk_wait_all();  // this warp's dQ reductions complete
     }
     tc_fence_before();
     named_barrier_sync(15, kThreads);

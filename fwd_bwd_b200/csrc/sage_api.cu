@@ -236,7 +236,8 @@ int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const
       !make_map(&tdoc, doc, 1, D, rows, D, sage::bwd::BQ) ||
       !make_map(&tdo, dout, 2, D, rows, 64, sage::bwd::BQ) ||
       !make_map(&tv, v, 2, D, rows, 64, sage::bwd::BKT) ||
-      !make_map(&tdq, dqacc, 4, D, rows, D, sage::bwd::kDqRows, false))
+      !make_map(&tdq, dqacc, 4, D, rows, D == 128 ? sage::bwd::kDqCols : D,
+                    sage::bwd::kDqRows, false))
     return SAGE_ERR_CUDA;
   sage::bwd::Args a;
   a.q_scale = qb->q_scale;
