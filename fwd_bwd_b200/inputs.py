@@ -8,7 +8,8 @@ or attention arithmetic.
 Recipe (the same for every workload):
 
 * per flattened head ``bh``, ``numpy.random.Generator(PCG64(SeedSequence([seed, offset,
-  bh])))`` with offsets Q:0, K:1, V:2, dO:3, mu:4 (the K-outlier channel offsets);
+  bh])))`` with offsets Q:0, K:1, V:2, dO:3, mu:4 (the K-outlier channel offsets), muQ:5
+  (the Q-outlier channel offsets);
 * ``standard_normal`` in float64, multiplied by the tensor's sigma, rounded to float32;
 * float32 rounded to the 16-bit storage type with round-half-to-even (bf16 by bit
   manipulation, fp16 by numpy's own RNE cast).
@@ -18,8 +19,8 @@ plus an exact float32 view for CPU consumers.
 
 The workloads are the attention shapes of the SageBwd page ("SageBwd: trainable low-bit
 attention", aitrends.kr): the 325M-Llama attention layer it pretrains, a K-outlier stress case
-for the K-smoothing ablation, a long-sequence case for the small-dS regime and the
-tokens-per-step sweep.
+for the K-smoothing ablation, a Q-outlier case for the Q-smoothing variant, a long-sequence
+case for the small-dS regime and the tokens-per-step sweep.
 """
 from __future__ import annotations
 
@@ -28,7 +29,7 @@ from typing import Dict, Optional, Sequence
 
 import numpy as np
 
-OFFSET_Q, OFFSET_K, OFFSET_V, OFFSET_DO, OFFSET_MU = 0, 1, 2, 3, 4
+OFFSET_Q, OFFSET_K, OFFSET_V, OFFSET_DO, OFFSET_MU, OFFSET_QMU = 0, 1, 2, 3, 4, 5
 
 
 @dataclasses.dataclass(frozen=True)
@@ -49,6 +50,8 @@ class Workload:
     sigma_qkv: float = 1.0
     sigma_do: float = 1.0
     k_outlier: bool = False  # per-channel offsets mu_c ~ N(0, 4^2), 4 channels +20
+    q_outlier: bool = False  # the same kind of offsets on Q (own stream)
+    qsmooth: bool = False    # run with Q-smoothing (an operator flag, carried with the shape)
     seed: int = 0
 
     @property
@@ -73,6 +76,9 @@ WORKLOADS: Dict[str, Workload] = {
     "llama325m": Workload("llama325m", 8, 16, 2048, 64, True, "bf16", sigma_do=1e-3),
     # K-outlier stress (run with the qknorm / ksmooth flags on and off)
     "koutlier": Workload("koutlier", 4, 16, 4096, 128, True, "bf16", k_outlier=True),
+    # Q-outlier stress for the Q-smoothing variant (K outliers too, K-smoothing on)
+    "qoutlier": Workload("qoutlier", 4, 16, 4096, 128, True, "bf16", k_outlier=True,
+                         q_outlier=True, qsmooth=True),
     # long sequence, small-dS regime
     "long16k": Workload("long16k", 1, 32, 16384, 128, True, "bf16", sigma_do=1e-4),
 }
@@ -116,12 +122,13 @@ def make_head(w: Workload, bh: int) -> Dict[str, np.ndarray]:
     for name, off, sig in (("q", OFFSET_Q, w.sigma_qkv), ("k", OFFSET_K, w.sigma_qkv),
                            ("v", OFFSET_V, w.sigma_qkv), ("do", OFFSET_DO, w.sigma_do)):
         out[name] = (_rng(w, off, bh).standard_normal(shape) * sig).astype(np.float32)
-    if w.k_outlier:
-        g = _rng(w, OFFSET_MU, bh)
-        mu = (g.standard_normal(w.d) * 4.0).astype(np.float32)
-        chans = g.choice(w.d, size=4, replace=False)
-        mu[chans] += np.float32(20.0)
-        out["k"] = (out["k"] + mu[None, :]).astype(np.float32)
+    for name, flag, off in (("k", w.k_outlier, OFFSET_MU), ("q", w.q_outlier, OFFSET_QMU)):
+        if flag:
+            g = _rng(w, off, bh)
+            mu = (g.standard_normal(w.d) * 4.0).astype(np.float32)
+            chans = g.choice(w.d, size=4, replace=False)
+            mu[chans] += np.float32(20.0)
+            out[name] = (out[name] + mu[None, :]).astype(np.float32)
     return out
 
 
@@ -162,8 +169,9 @@ def make_inputs_fast(w: Workload, device: str = "cpu"):
                       ("do", w.sigma_do)):
         res[name] = (torch.randn(shape, generator=g, device=device, dtype=torch.float32)
                      * sig).to(tdt)
-    if w.k_outlier:
-        mu = torch.randn((w.B, w.H, 1, w.d), generator=g, device=device) * 4.0
-        mu[..., :4] += 20.0
-        res["k"] = (res["k"].float() + mu).to(tdt)
+    for name, flag in (("k", w.k_outlier), ("q", w.q_outlier)):
+        if flag:
+            mu = torch.randn((w.B, w.H, 1, w.d), generator=g, device=device) * 4.0
+            mu[..., :4] += 20.0
+            res[name] = (res[name].float() + mu).to(tdt)
     return res

@@ -12,6 +12,9 @@ What it follows ("SageBwd: trainable low-bit attention", aitrends.kr):
 * QK-norm paragraph -- RMSNorm applied to every token vector of Q and K;
 * K-smoothing paragraph -- a mean is subtracted from K just before quantization
   (read here as the per-channel mean over tokens, see ``k_smooth``);
+* Q-smoothing paragraph (limitations) -- smoothing Q as well needs the bias correction
+  ``dK_bias = (dS^T 1) mu_Q^T`` (optional ``qsmooth`` flag; see ``bias_dot_f32`` and
+  ``attn_bwd_head``);
 * Triton-kernel paragraph -- per-block quantization;
 * error-propagation paragraph -- dQ = dS K and dK = dS^T Q.
 
@@ -146,14 +149,46 @@ def k_smooth_f32(khat: np.ndarray, k_block: int) -> tuple:
     return (khat - m[..., None, :]).astype(F32), m
 
 
+def bias_dot_f32(m: np.ndarray, x: np.ndarray) -> np.ndarray:
+    """Per-token bias ``b_j = sum_c m_c x_jc`` in float32 (Q-smoothing bias, see ``prologue``).
+
+    ``m`` is ``[..., d]``, ``x`` is ``[..., N, d]``.  Reduction order (a reading; the page gives
+    none): the same lane structure as ``rms_norm_rows_f32`` -- ``d/8`` lanes of 8 consecutive
+    channels, each summing ``m_c * x_c`` (product and sum each rounded to float32) in ascending
+    channel order from +0, then the butterfly over lanes; lane 0 holds the result.
+    """
+    m = np.asarray(m, dtype=F32)
+    x = np.asarray(x, dtype=F32)
+    d = x.shape[-1]
+    L = d // 8
+    xl = x.reshape(*x.shape[:-1], L, 8)
+    ml = m.reshape(*m.shape[:-1], 1, L, 8)
+    p = np.zeros(x.shape[:-1] + (L,), dtype=F32)
+    for c in range(8):
+        p = p + (ml[..., c] * xl[..., c]).astype(F32)
+    lanes = np.arange(L)
+    o = L // 2
+    while o >= 1:
+        p = p + p[..., lanes ^ o]
+        o //= 2
+    return p[..., 0].astype(F32)
+
+
 def prologue(q, k, v, *, q_block: int, k_block: int, qknorm: bool, ksmooth: bool,
-             eps: float = 1e-6) -> Dict[str, np.ndarray]:
-    """QK-norm -> K-smoothing -> per-block INT8 quantization of Q, K and V (float32 exact).
+             eps: float = 1e-6, qsmooth: bool = False) -> Dict[str, np.ndarray]:
+    """QK-norm -> smoothing -> per-block INT8 quantization of Q, K and V (float32 exact).
 
     Inputs are float32 arrays ``[BH, N, d]`` holding the exact values of the 16-bit inputs.
     Order (K-smoothing paragraph: smoothing comes right before quantization): normalize, then
     smooth, then quantize.  Q uses blocks of ``q_block`` tokens, K and V blocks of ``k_block``
     tokens; every block spans all ``d`` channels.
+
+    ``qsmooth`` (Q-smoothing paragraph): ``mu_Q``, the per-channel mean of the normalized Q over
+    all tokens (same summation order as K's, blocks of ``k_block`` tokens), is subtracted before
+    Q is quantized.  Scores then lose the term ``mu_Q . k~_j``, which -- unlike K's row-constant
+    shift -- differs per key and so changes softmax; it is restored as a per-key bias
+    ``k_bias_j = mu_Q . k~_j`` (``bias_dot_f32``, from the unquantized smoothed K) that the
+    attention adds to every score of key j.
     """
     q = np.asarray(q, dtype=F32)
     k = np.asarray(k, dtype=F32)
@@ -167,13 +202,19 @@ def prologue(q, k, v, *, q_block: int, k_block: int, qknorm: bool, ksmooth: bool
     if ksmooth:
         kh, out["k_mean"] = k_smooth_f32(kh, k_block)
     out["q_hat"], out["k_tilde"] = qh, kh
-    out["q_codes"], out["q_scale"] = quantize_token_blocks(qh, q_block)
+    qt = qh
+    if qsmooth:
+        qt, out["q_mean"] = k_smooth_f32(qh, k_block)
+        out["k_bias"] = bias_dot_f32(out["q_mean"], kh)
+    out["q_tilde"] = qt
+    out["q_codes"], out["q_scale"] = quantize_token_blocks(qt, q_block)
     out["k_codes"], out["k_scale"] = quantize_token_blocks(kh, k_block)
     out["v_codes"], out["v_scale"] = quantize_token_blocks(v, k_block)
     return out
 
 
-def prologue_fp64(q, k, v, *, qknorm: bool, ksmooth: bool, eps: float = 1e-6) -> Dict:
+def prologue_fp64(q, k, v, *, qknorm: bool, ksmooth: bool, eps: float = 1e-6,
+                  qsmooth: bool = False) -> Dict:
     """X-mode prologue: RMSNorm and mean subtraction in float64 with no quantization."""
     q = np.asarray(q, dtype=F64)
     k = np.asarray(k, dtype=F64)
@@ -190,6 +231,11 @@ def prologue_fp64(q, k, v, *, qknorm: bool, ksmooth: bool, eps: float = 1e-6) ->
         out["k_mean"] = kh.mean(axis=-2)
         kh = kh - out["k_mean"][..., None, :]
     out["q_hat"], out["k_tilde"] = qh, kh
+    out["q_tilde"] = qh
+    if qsmooth:
+        out["q_mean"] = qh.mean(axis=-2)
+        out["q_tilde"] = qh - out["q_mean"][..., None, :]
+        out["k_bias"] = np.einsum("...nc,...c->...n", kh, out["q_mean"])
     return out
 
 
@@ -224,14 +270,18 @@ class _Quant:
         return c.astype(F64), s.astype(F64)
 
 
-def _scores(qc, sq_row, kc, sk_col, tau, causal, i0):
-    """z = (A * (sQ * sK)) * tau with A = Qc Kc^T exact; causal keys > query get -inf.
+def _scores(qc, sq_row, kc, sk_col, tau, causal, i0, k_bias=None):
+    """z = (A * (sQ * sK) + b) * tau with A = Qc Kc^T exact; causal keys > query get -inf.
 
-    ``qc`` holds the query rows ``i0 .. i0 + rows``; causal alignment is square and top-left
-    (key j is visible to query i iff j <= i).
+    ``k_bias`` (Q-smoothing only) is the per-key bias ``b_j``; without it ``b = 0``.  ``qc``
+    holds the query rows ``i0 .. i0 + rows``; causal alignment is square and top-left (key j is
+    visible to query i iff j <= i).
     """
     A = qc @ kc.T
-    z = (A * (sq_row[:, None] * sk_col[None, :])) * tau
+    z = A * (sq_row[:, None] * sk_col[None, :])
+    if k_bias is not None:
+        z = z + np.asarray(k_bias, F64)[None, :]
+    z = z * tau
     if causal:
         qi = np.arange(i0, i0 + qc.shape[0])[:, None]
         kj = np.arange(kc.shape[0])[None, :]
@@ -240,7 +290,8 @@ def _scores(qc, sq_row, kc, sk_col, tau, causal, i0):
 
 
 def attn_fwd_head(qc, q_scale, kc, k_scale, vc, v_scale, *, q_block: int, k_block: int,
-                  causal: bool, tau: float, quant: bool = True) -> tuple:
+                  causal: bool, tau: float, quant: bool = True, k_bias=None,
+                  q_mean=None) -> tuple:
     """Forward attention of one head: returns ``(O float64 [N,d], LSE float64 [N])``.
 
     Inputs are per-token-block codes and scales (Q mode) or float64 values with unit scales
@@ -251,6 +302,8 @@ def attn_fwd_head(qc, q_scale, kc, k_scale, vc, v_scale, *, q_block: int, k_bloc
     3. for every K block: ``p = exp(z - m)`` is quantized with one scale per query row
        (``sP = max_j p / 127``), and ``O += (Pc Vc) * (sP sV)``;
     4. ``O /= l``, ``LSE = m + ln l`` (natural log, in units of the scaled scores).
+
+    With Q-smoothing, ``k_bias`` is added to the scores of step 1 (``q_mean`` is unused here).
 
     Reading: the page only says "per-block"; P gets one scale per (query row, K block).  The
     codes ``rne(p / (max p / 127))`` depend on ``p`` only through ``p / max p``, so they are the
@@ -269,7 +322,7 @@ def attn_fwd_head(qc, q_scale, kc, k_scale, vc, v_scale, *, q_block: int, k_bloc
     LSE = np.zeros(N, F64)
     for i0 in range(0, N, q_block):
         rows = slice(i0, i0 + q_block)
-        z = _scores(qc[rows], sq_row[rows], kc, sk_col, tau, causal, i0)
+        z = _scores(qc[rows], sq_row[rows], kc, sk_col, tau, causal, i0, k_bias)
         m = z.max(axis=1)
         e = np.exp(z - m[:, None])
         l = e.sum(axis=1)
@@ -285,7 +338,7 @@ def attn_fwd_head(qc, q_scale, kc, k_scale, vc, v_scale, *, q_block: int, k_bloc
 
 def attn_bwd_head(qc, q_scale, kc, k_scale, vc, v_scale, v_raw, o_out, lse, do_raw, *,
                   q_block: int, k_block: int, causal: bool, tau: float,
-                  quant: bool = True) -> tuple:
+                  quant: bool = True, k_bias=None, q_mean=None) -> tuple:
     """Backward attention of one head: returns ``(dQhat, dKtilde, dV)`` as float64 ``[N, d]``.
 
     ``v_raw``/``do_raw`` are the 16-bit inputs' exact values (the FP16 GEMM operands),
@@ -306,6 +359,14 @@ def attn_bwd_head(qc, q_scale, kc, k_scale, vc, v_scale, v_raw, o_out, lse, do_r
     gradient with respect to the normalized K, because the mean-subtraction Jacobian
     contributes ``-(1/N) sum_j dK_j``, and ``sum_j dK_j = tau sum_i q_i sum_j dS_ij = 0`` since
     every row of ``dS`` sums to zero (reading: that term is dropped).
+
+    Q-smoothing (``k_bias`` and ``q_mean`` given; ``qc`` then holds the smoothed Q): the scores
+    carry the bias of the forward, and dK gains the page's correction term
+    ``dK_bias = tau (dS^T 1) mu_Q^T``, the gradient through ``b_j = mu_Q . k~_j``.  Its column
+    sums ``dS^T 1`` are taken over the same quantized dS tile the INT8 GEMM uses (reading: the
+    page names this term as an added quantization-noise path), i.e. ``sdS * sum_i dSc_ij``.
+    dQ needs no term: with respect to the normalized Q, the mean terms of the smoothing and of
+    the bias cancel exactly, as for K.
     """
     qz = _Quant(quant)
     N, d = qc.shape
@@ -323,7 +384,7 @@ def attn_bwd_head(qc, q_scale, kc, k_scale, vc, v_scale, v_raw, o_out, lse, do_r
     dV = np.zeros((N, d), F64)
     for bi, i0 in enumerate(range(0, N, q_block)):
         rows = slice(i0, i0 + q_block)
-        z = _scores(qc[rows], sq_row[rows], kc, sk_col, tau, causal, i0)
+        z = _scores(qc[rows], sq_row[rows], kc, sk_col, tau, causal, i0, k_bias)
         P = np.exp(z - np.asarray(lse, F64)[rows][:, None])
         dP = do_raw[rows] @ v_raw.T
         dS = P * (dP - D[rows][:, None])
@@ -333,6 +394,8 @@ def attn_bwd_head(qc, q_scale, kc, k_scale, vc, v_scale, v_raw, o_out, lse, do_r
             dsc, sds = qz.tile(dS[:, cols])
             dV[cols] += (pc.T @ doc[rows]) * (sp * sdo[bi])
             dK[cols] += (dsc.T @ qc[rows]) * (sds * sq_row[i0]) * tau
+            if q_mean is not None:
+                dK[cols] += np.outer(dsc.sum(axis=0) * sds, np.asarray(q_mean, F64)) * tau
             dQ[rows] += (dsc @ kc[cols]) * (sds * sk_col[j * k_block]) * tau
     return dQ, dK, dV
 
@@ -354,7 +417,8 @@ def rms_norm_bwd(g_hat: np.ndarray, x_hat: np.ndarray, inv: np.ndarray) -> np.nd
 # ----------------------------------------------------------------------------------------------
 def sage_attention(q, k, v, do, *, causal: bool, qknorm: bool, ksmooth: bool, q_block: int,
                    k_block: int, dtype: str, tau: float = 0.0, eps: float = 1e-6,
-                   quant: bool = True, round_outputs: bool = True) -> Dict[str, np.ndarray]:
+                   quant: bool = True, round_outputs: bool = True,
+                   qsmooth: bool = False) -> Dict[str, np.ndarray]:
     """Prologue, forward and backward over all heads.
 
     ``q, k, v, do`` are float32 ``[BH, N, d]`` holding the exact 16-bit input values.  Returns
@@ -366,14 +430,14 @@ def sage_attention(q, k, v, do, *, causal: bool, qknorm: bool, ksmooth: bool, q_
     tau = tau if tau > 0 else 1.0 / math.sqrt(d)
     if quant:
         pro = prologue(q, k, v, q_block=q_block, k_block=k_block, qknorm=qknorm,
-                       ksmooth=ksmooth, eps=eps)
+                       ksmooth=ksmooth, eps=eps, qsmooth=qsmooth)
         ops = (pro["q_codes"], pro["q_scale"], pro["k_codes"], pro["k_scale"],
                pro["v_codes"], pro["v_scale"])
     else:
-        pro = prologue_fp64(q, k, v, qknorm=qknorm, ksmooth=ksmooth, eps=eps)
+        pro = prologue_fp64(q, k, v, qknorm=qknorm, ksmooth=ksmooth, eps=eps, qsmooth=qsmooth)
         ones_q = np.ones((BH, N // q_block))
         ones_k = np.ones((BH, N // k_block))
-        ops = (pro["q_hat"], ones_q, pro["k_tilde"], ones_k, pro["v"], ones_k)
+        ops = (pro["q_tilde"], ones_q, pro["k_tilde"], ones_k, pro["v"], ones_k)
     res = dict(pro)
     o = np.zeros((BH, N, d))
     lse = np.zeros((BH, N))
@@ -383,6 +447,8 @@ def sage_attention(q, k, v, do, *, causal: bool, qknorm: bool, ksmooth: bool, q_
     kw = dict(q_block=q_block, k_block=k_block, causal=causal, tau=tau, quant=quant)
     for h in range(BH):
         head_ops = [x[h] for x in ops]
+        if qsmooth:
+            kw.update(k_bias=pro["k_bias"][h], q_mean=pro["q_mean"][h])
         oh, lse[h] = attn_fwd_head(*head_ops, **kw)
         o[h] = round_to_storage(oh, dtype) if round_outputs else oh
         dqh, dkh, dv[h] = attn_bwd_head(*head_ops, v[h], o[h], lse[h], do[h], **kw)

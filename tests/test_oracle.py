@@ -10,6 +10,10 @@
   with N (the page's dS-magnitude bound);
 * Q mode: exact integer S against brute force, a closed form (uniform attention), an explicit
   error bound for P quantization, cosine >= 0.995 against X mode, and the K-outlier trend.
+* Q-smoothing (the optional variant of the Q-smoothing paragraph): in X mode the bias and the
+  dK correction term make every output identical to Q-smoothing off; the prologue's mean and
+  bias against their float64 definitions; in Q mode, scores of Q-outlier inputs are closer to
+  full precision with Q-smoothing than without.
 * planted mistakes in the oracle are caught by these pins.
 """
 import math
@@ -352,6 +356,104 @@ def test_qmode_k_outlier_trend():
 
 
 # ------------------------------------------------------------------------------------------
+# Q-smoothing
+# ------------------------------------------------------------------------------------------
+def _q_outlier_inputs(seed, BH=2, N=128, d=64):
+    g = np.random.default_rng(seed)
+    q, k, v, do = (g.standard_normal((BH, N, d)) for _ in range(4))
+    mu = 4.0 * g.standard_normal((BH, 1, d))
+    mu[..., [3, 17, 40, 60]] += 20.0
+    q = q + mu
+    k = k + 3.0 * g.standard_normal((BH, 1, d))
+    return q, k, v, do
+
+
+def _qsmooth_xmode_gap(causal, ksmooth, seed=21):
+    """Largest relative difference of the X-mode outputs between Q-smoothing on and off."""
+    q, k, v, do = _q_outlier_inputs(seed)
+    kw = dict(causal=causal, qknorm=True, ksmooth=ksmooth, q_block=64, k_block=32,
+              dtype="bf16", quant=False, round_outputs=False)
+    on = O.sage_attention(q, k, v, do, qsmooth=True, **kw)
+    off = O.sage_attention(q, k, v, do, qsmooth=False, **kw)
+    return max(_rel(on[n], off[n]) for n in ("o", "lse", "dq", "dk", "dv"))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("ksmooth", [False, True])
+def test_qsmooth_xmode_invariance(causal, ksmooth):
+    """Q-smoothing with the score bias and dK_bias = (dS^T 1) mu_Q^T is exact in full precision:
+    the scores q~_i . k_j + mu_Q . k_j equal q^_i . k_j, and dK = tau dS^T q~ + tau (dS^T 1)
+    mu_Q^T = tau dS^T q^, so every output equals Q-smoothing off up to float64 rounding."""
+    assert _qsmooth_xmode_gap(causal, ksmooth) < 1e-12
+
+
+def test_qsmooth_xmode_vs_torch():
+    q, k, v, do = _q_outlier_inputs(22)
+    res = O.sage_attention(q, k, v, do, causal=True, qknorm=True, ksmooth=True, q_block=64,
+                           k_block=32, dtype="bf16", quant=False, round_outputs=False,
+                           qsmooth=True)
+    o, lse, dq, dk, dv = _torch_reference(q, k, v, do, True, True, True)
+    for a, b in ((res["o"], o), (res["lse"], lse), (res["dq"], dq), (res["dk"], dk),
+                 (res["dv"], dv)):
+        assert _rel(a, b) < 1e-12
+
+
+def test_qsmooth_prologue_closed_forms():
+    q, k, v, _ = _q_outlier_inputs(23, BH=3, N=256, d=128)
+    q, k, v = (x.astype(np.float32) for x in (q, k, v))
+    pro = O.prologue(q, k, v, q_block=128, k_block=64, qknorm=True, ksmooth=True, qsmooth=True)
+    qh = pro["q_hat"].astype(np.float64)
+    N, d = qh.shape[-2], qh.shape[-1]
+    eps32 = np.finfo(np.float32).eps
+    # mu_Q is the per-channel token mean: float32 summation error bound N * eps * sum|x|
+    m64 = qh.mean(axis=-2)
+    bound = N * eps32 * np.abs(qh).sum(axis=-2) / N + eps32 * np.abs(m64)
+    assert np.all(np.abs(pro["q_mean"] - m64) <= bound)
+    # smoothed Q has (nearly) zero channel means; the offset channels are removed
+    assert np.abs(pro["q_tilde"].astype(np.float64).mean(axis=-2)).max() < 1e-4
+    assert np.abs(pro["q_tilde"]).max() < np.abs(pro["q_hat"]).max()
+    # k_bias_j = mu_Q . k~_j within the float32 dot-product bound d * eps * sum|m k|
+    kt = pro["k_tilde"].astype(np.float64)
+    mq = pro["q_mean"].astype(np.float64)
+    b64 = np.einsum("bnc,bc->bn", kt, mq)
+    bb = d * eps32 * np.einsum("bnc,bc->bn", np.abs(kt), np.abs(mq))
+    assert np.all(np.abs(pro["k_bias"] - b64) <= bb)
+    # the Q codes are those of the smoothed Q
+    c, s = O.quantize_token_blocks(pro["q_tilde"], 128)
+    assert np.array_equal(c, pro["q_codes"]) and np.array_equal(s, pro["q_scale"])
+
+
+def test_qsmooth_qmode_scores_closer_and_cosine():
+    """With large per-channel Q offsets, Q-smoothing makes the INT8 scores (plus bias) closer
+    to the full-precision scores; the whole operator stays within cosine 0.995 of X mode."""
+    q, k, v, do = _q_outlier_inputs(24, BH=2, N=256, d=64)
+    q, k, v, do = (x.astype(np.float32) for x in (q, k, v, do))
+    tau = 1.0 / 8.0
+    errs = {}
+    for qs in (False, True):
+        pro = O.prologue(q, k, v, q_block=128, k_block=64, qknorm=True, ksmooth=True,
+                         qsmooth=qs)
+        exact = np.einsum("bic,bjc->bij", pro["q_hat"].astype(np.float64),
+                          pro["k_tilde"].astype(np.float64)) * tau
+        err = 0.0
+        for h in range(q.shape[0]):
+            sq = np.repeat(pro["q_scale"][h].astype(np.float64), 128)
+            sk = np.repeat(pro["k_scale"][h].astype(np.float64), 64)
+            z = O._scores(pro["q_codes"][h].astype(np.float64), sq,
+                          pro["k_codes"][h].astype(np.float64), sk, tau, False, 0,
+                          pro["k_bias"][h] if qs else None)
+            err += float(np.linalg.norm(z - exact[h]) ** 2)
+        errs[qs] = math.sqrt(err)
+    assert errs[True] < 0.5 * errs[False], errs
+    kw = dict(causal=True, qknorm=True, ksmooth=True, q_block=128, k_block=64, dtype="bf16",
+              qsmooth=True)
+    qm = O.sage_attention(q, k, v, do, **kw)
+    xm = O.sage_attention(q, k, v, do, quant=False, round_outputs=False, **kw)
+    for n in ("o", "dq", "dk", "dv"):
+        assert _cos(qm[n], xm[n]) >= 0.995, n
+
+
+# ------------------------------------------------------------------------------------------
 # planted mistakes are caught
 # ------------------------------------------------------------------------------------------
 def _xmode_vs_torch_ok():
@@ -376,14 +478,30 @@ def test_planted_mistakes_are_caught(monkeypatch):
 
     real_scores = O._scores
 
-    def dropped_tau(qc, sq, kc, sk, tau, causal, i0):
-        return real_scores(qc, sq, kc, sk, 1.0, causal, i0)
+    def dropped_tau(qc, sq, kc, sk, tau, causal, i0, k_bias=None):
+        return real_scores(qc, sq, kc, sk, 1.0, causal, i0, k_bias)
 
     for name, fake in (("attn_bwd_head", wrong_sign_ds), ("attn_bwd_head", transposed_dv),
                        ("_scores", dropped_tau)):
         with monkeypatch.context() as m:
             m.setattr(O, name, fake)
             assert not _xmode_vs_torch_ok(), name
+    # Q-smoothing: a dropped dK correction term, or a bias with the wrong sign
+    def no_dk_bias(*a, **kw):
+        kw["q_mean"] = None
+        return real_bwd(*a, **kw)
+
+    real_fwd = O.attn_fwd_head
+
+    def neg_bias_fwd(*a, **kw):
+        if kw.get("k_bias") is not None:
+            kw["k_bias"] = -kw["k_bias"]
+        return real_fwd(*a, **kw)
+
+    for name, fake in (("attn_bwd_head", no_dk_bias), ("attn_fwd_head", neg_bias_fwd)):
+        with monkeypatch.context() as m:
+            m.setattr(O, name, fake)
+            assert _qsmooth_xmode_gap(True, True) > 1e-6, name
     real_quant = O.quantize_groups
 
     def round_half_up(x, axes):
