@@ -129,7 +129,7 @@ def cpu_baseline(w, n_heads: int):
     args = [x[n + "_f32"] for n in ("q", "k", "v", "do")]
     t0 = time.perf_counter()
     O.sage_attention(*args, causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth,
-                     q_block=w.q_block, k_block=w.k_block, dtype=w.dtype)
+                     q_block=w.q_block, k_block=w.k_block, dtype=w.dtype, qsmooth=w.qsmooth)
     dt = time.perf_counter() - t0
     ops = w.ops() / (w.B * w.H) * n_heads
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -168,7 +168,7 @@ def run_reference(args, w):
 def config_of(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
             "io_dtype": w.dtype, "q_block": w.q_block, "k_block": w.k_block,
-            "qknorm": w.qknorm, "ksmooth": w.ksmooth,
+            "qknorm": w.qknorm, "ksmooth": w.ksmooth, "qsmooth": w.qsmooth,
             "l2": "no flush: every input tensor (1 GiB at the default workload) exceeds L2"}
 
 
@@ -201,7 +201,7 @@ def main():
                                 device_id=dev)
 
     cfg = ops.Config(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth, q_block=w.q_block,
-                     k_block=w.k_block)
+                     k_block=w.k_block, qsmooth=w.qsmooth)
     x = make_inputs_fast(w.replace(seed=w.seed + rank), device=str(dev))
     q, k, v, do = x["q"], x["k"], x["v"], x["do"]
     prm = cfg.params(q)
@@ -212,7 +212,7 @@ def main():
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = (3 if w.ksmooth else 1) + 1 + 3
+    launches_per_step = 1 + 2 * (int(w.ksmooth) + int(w.qsmooth)) + 1 + 3
 
     def step(ev=None):
         ops.quant_prologue(q, k, v, cfg, out=qb, workspace=ws_pro)

@@ -26,13 +26,14 @@ class SageParams(ctypes.Structure):
                 ("d", ctypes.c_int), ("dtype", ctypes.c_int), ("causal", ctypes.c_int),
                 ("qknorm", ctypes.c_int), ("ksmooth", ctypes.c_int),
                 ("q_block", ctypes.c_int), ("k_block", ctypes.c_int),
-                ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float),
+                ("qsmooth", ctypes.c_int)]
 
 
 class SageQBufs(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("q_codes", "k_codes", "v_codes", "q_scale", "k_scale", "v_scale",
-                 "q_inv_rms", "k_inv_rms", "k_mean")]
+                 "q_inv_rms", "k_inv_rms", "k_mean", "q_mean", "k_bias")]
 
 
 class SageError(RuntimeError):

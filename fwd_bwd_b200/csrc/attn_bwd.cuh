@@ -25,6 +25,9 @@
 // producer warpgroup gives registers to the compute warpgroups (setmaxnreg): at launch every
 // thread holds 168, afterwards 256 x 208 + 128 x 80 = 63488 <= 384 x 168.  The MMA thread keeps
 // 80: with fewer it spills, and its reloads delay the tensor-core issue.
+// Q-smoothing (template flag QS): pass A adds the per-key bias to the recomputed scores, and
+// pass B also sums each key's dS codes over the tile's rows (one warp reduction per key), so
+// the epilogue can add dK_bias = tau * (sum over tiles of sdS * column sum) * mu_Q.
 // TMEM (512 columns): buffer b in {0,1} at [256b, 256b+256): [0,128) S -> P -> dV_t ->
 // dQ_t(block 0); [128,256) dP -> dS -> dK_t -> dQ_t(block 1).
 #pragma once
@@ -85,6 +88,8 @@ struct Smem {
   alignas(16) float red_ds[2][8];  // and of |dS|
   float sp[3][2][2], sds[3][2][2];  // tile scales [tile % 3][q group][key half]
   float dot[BKT];                   // RMSNorm-backward row dot products (warpgroup 1 -> 0)
+  float kb[BKT];                    // Q-smoothing: k_bias of the CTA's keys
+  float cs[BKT];                    // Q-smoothing: sum over tiles of sdS * (column sum of dSc)
   uint64_t kv_full, q_full[2], q_empty[2], dor_full, dor_free;
   uint64_t sdp_full[2], pds_ready, dvdk_full, dvdk_free, dq_full, dq_free;
   uint64_t scales_full[2];  // tile parity: the P / dS scales of both warpgroups are written
@@ -123,6 +128,8 @@ struct Args {
   int BH, N, q_block, causal, qknorm;
   float scale_log2;  // softmax_scale * log2(e)
   float tau;         // softmax_scale
+  const float* k_bias;  // [BH, N] (Q-smoothing)
+  const float* q_mean;  // [BH, D] (Q-smoothing)
 };
 
 template <int D>
@@ -131,7 +138,7 @@ __device__ __forceinline__ Smem<D>& smem_ref(uint8_t* raw) {
   return *reinterpret_cast<Smem<D>*>(raw + ((1024u - (a & 1023u)) & 1023u));
 }
 
-template <typename T, int D>
+template <typename T, int D, bool QS>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_qc,
                     const __grid_constant__ CUtensorMap tm_kc,
@@ -173,6 +180,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.dq_full, 1);
     mbar_init(&sm.dq_free, 256);
     fence_barrier_init();
+  }
+  if constexpr (QS) {
+    for (int i = threadIdx.x; i < BKT; i += kThreads) {
+      sm.kb[i] = args.k_bias[static_cast<size_t>(bh) * N + t * BKT + i];
+      sm.cs[i] = 0.0f;
+    }
   }
   __syncthreads();
   if (sm.abort) return;
@@ -342,7 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       dvr = args.dvec[grow];
     };
     // pass A of tile it: P, dS into TMEM buffer it&1, tile maxima -> scales in slot it%3
-    auto pass_a = [&](int it, float c, float lse2, float dvr, float& ip, float& ids) {
+    auto pass_a = [&](int it, float c, float lse2, float dvr, float& ip, float& ids,
+                      float& sds_own) {
       const int b = it & 1, slot = it % 3;
       const uint32_t lane_base = tmem + lane_off + b * 256;
       const int qt = i_first + it;
@@ -359,7 +373,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto proc_a = [&](uint32_t (&sa)[8], uint32_t (&pa)[8], int col) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            float p = ex2_approx(deq(sa[e], c22, nc22) - lse2);
+            float z = deq(sa[e], c22, nc22);
+            if constexpr (QS) z = fmaf(sm.kb[col + e], args.scale_log2, z);
+            float p = ex2_approx(z - lse2);
             if constexpr (decltype(masked)::value) {
               if (col + e > r) p = 0.0f;  // diagonal tile: key index - query index = col - r
             }
@@ -426,15 +442,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // 2 ulp) serves; the stored scales above are IEEE quotients
       ip = tp > 0.0f ? __fdividef(127.0f, tp) : 0.0f;
       ids = tds > 0.0f ? __fdividef(127.0f, tds) : 0.0f;
+      if constexpr (QS) sds_own = __fdiv_rn(tds, 127.0f);  // this row group's dS scale
       // No CTA-wide barrier here: the warpgroups may drift apart.  sm.red_*[b] is rewritten
       // only in pass A of tile it+2, which waits for that tile's S / dP, issued after every
       // thread released tile it's dQ -- i.e. after every warp finished reading it for tile it.
       // (Tiles 0 and 1 have their S / dP issued back to back, hence the two slots.)
     };
 
-    float c_n, lse2_n, dvr_n, ip, ids;
+    float c_n, lse2_n, dvr_n, ip, ids, sdsc = 0.0f;
     row_inputs(0, c_n, lse2_n, dvr_n);
-    pass_a(0, c_n, lse2_n, dvr_n, ip, ids);
+    pass_a(0, c_n, lse2_n, dvr_n, ip, ids, sdsc);
     for (int it = 0; it < nq; ++it) {
       const int b = it & 1, slot = it % 3;
       const uint32_t lane_base = tmem + lane_off + b * 256;
@@ -460,6 +477,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t off = swz_offset(r, h * 4 + ch, 128);
         *reinterpret_cast<uint4*>(sm.pc + off) = make_uint4(cp[0], cp[1], cp[2], cp[3]);
         *reinterpret_cast<uint4*>(sm.dsc + off) = make_uint4(cd[0], cd[1], cd[2], cd[3]);
+        if constexpr (QS) {
+          // column sums of the dS codes over the warp's 32 rows (one q_block group, so one
+          // scale), added to the per-key total; lane e carries column col + e
+          float mine = 0.0f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int v = static_cast<int>(cd[e >> 2] << (24 - 8 * (e & 3))) >> 24;
+            const int cs = __reduce_add_sync(0xFFFFFFFFu, v);
+            if (lane == e) mine = static_cast<float>(cs);
+          }
+          if (lane < 16) atomicAdd(&sm.cs[col + lane], mine * sdsc);
+        }
         if (col < D) {  // dV_t occupies columns [0, D), dK_t [128, 128 + D)
           tmem_fill16(lane_base + col, kMagicBits);
           tmem_fill16(lane_base + 128 + col, kMagicBits);
@@ -500,8 +529,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         sq_t[g] = args.q_scale[qb];
       }
       // pass A of the next tile while the tensor core works on this one
-      float ip_n = 0.0f, ids_n = 0.0f;
-      if (it + 1 < nq) pass_a(it + 1, c_n, lse2_n, dvr_n, ip_n, ids_n);
+      float ip_n = 0.0f, ids_n = 0.0f, sdsc_n = 0.0f;
+      if (it + 1 < nq) pass_a(it + 1, c_n, lse2_n, dvr_n, ip_n, ids_n, sdsc_n);
       // step 3: dV_t, dK_t (thread = key row r, d columns of warpgroup h) into registers;
       // the read columns are re-preloaded for dQ_t.  The tile scales of both warpgroups are
       // read from here on.  One barrier per tile parity, so arrivals for tiles it and it+1
@@ -636,12 +665,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&sm.dq_free);
       ip = ip_n;
       ids = ids_n;
+      sdsc = sdsc_n;
     }
     // epilogue: dv, dk from the register accumulators (thread = key row r, d half h)
     {
       const size_t krow = static_cast<size_t>(row_base) + key_base + r;
       T* dvp = reinterpret_cast<T*>(args.dv) + krow * D + h * kHalfD;
       T* dkp = reinterpret_cast<T*>(args.dk) + krow * D + h * kHalfD;
+      if constexpr (QS) {
+        // dK_bias = tau * (dS^T 1)_r * mu_Q, the gradient through the score bias
+        named_barrier_sync(4, 256);  // every warp's column-sum additions are in
+        const float csr = sm.cs[r] * args.tau;
+        const float4* mq =
+            reinterpret_cast<const float4*>(args.q_mean + static_cast<size_t>(bh) * D + h * kHalfD);
+#pragma unroll
+        for (int c0 = 0; c0 < kHalfD; c0 += 4) {
+          const float4 m4 = __ldg(mq + c0 / 4);
+          acck[c0 + 0] = fmaf(csr, m4.x, acck[c0 + 0]);
+          acck[c0 + 1] = fmaf(csr, m4.y, acck[c0 + 1]);
+          acck[c0 + 2] = fmaf(csr, m4.z, acck[c0 + 2]);
+          acck[c0 + 3] = fmaf(csr, m4.w, acck[c0 + 3]);
+        }
+      }
       if (args.qknorm) {
         // RMSNorm backward: dk = inv * (dkhat - khat * (sum_c dkhat_c khat_c) / d), with
         // khat = k * inv recomputed from the raw row (bitwise the prologue's value)

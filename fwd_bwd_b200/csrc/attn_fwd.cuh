@@ -18,6 +18,10 @@
 // each MMA (see kMagicBits), so results read back as floats that one FMA dequantizes.
 // O (float32) lives in registers.
 //
+// Q-smoothing (template flag QS): every score of key j gains the per-key bias k_bias_j, copied
+// with the K block into shared memory; the block maximum is then taken over the biased scores
+// rather than over the raw INT32 values.
+//
 // P quantization: one scale per (query row, 64-key block).  The codes rne(127 p / max p) do
 // not depend on which running maximum p was taken against, so computing them against the
 // block's own maximum (as here) equals any other evaluation order in exact arithmetic.
@@ -52,6 +56,7 @@ struct Smem {
   int8_t k[NST][BKV * D];
   int8_t v[NST][BKV * D];
   int8_t p[NT][2][BM * BKV];
+  float kb[NST][BKV];  // Q-smoothing: k_bias of the stage's keys
   uint64_t q_full;
   uint64_t k_full[NST], v_full[NST], kv_empty[NST];
   uint64_t s_full[NT][2], p_full[NT][2], pv_full[NT], pv_free[NT];
@@ -83,6 +88,7 @@ struct Args {
   int BH, N, q_block, causal;
   float scale_log2;  // softmax_scale * log2(e)
   int nsup;          // CTAs per head: ceil(N / 256)
+  const float* k_bias;  // [BH, N] (Q-smoothing)
 };
 
 template <int D>
@@ -107,7 +113,7 @@ __device__ __forceinline__ void issue_scores(uint32_t d_tmem, const int8_t* qs,
   }
 }
 
-template <typename T, int D>
+template <typename T, int D, bool QS>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -186,8 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < nb_max; ++j) {
         const int st = j % NST;
         if (j >= NST) mbar_wait(&sm.kv_empty[st], ((j / NST) - 1) & 1, 100);
-        mbar_arrive_expect_tx(&sm.k_full[st], BKV * D);
+        mbar_arrive_expect_tx(&sm.k_full[st], BKV * D + (QS ? BKV * 4 : 0));
         tma_load_2d(sm.k[st], &tm_k, 0, row_base + j * BKV, &sm.k_full[st]);
+        if constexpr (QS)
+          bulk_load(sm.kb[st], args.k_bias + row_base + j * BKV, BKV * 4, &sm.k_full[st]);
         mbar_arrive_expect_tx(&sm.v_full[st], BKV * D);
         tma_load_2d(sm.v[st], &tm_v, 0, row_base + j * BKV, &sm.v_full[st]);
       }
@@ -303,7 +311,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&sm.s_full[g][j & 1], (j >> 1) & 1, 111);
         tc_fence_after();
         const uint32_t sa = lane_base + (j & 1) * 64;
-        // pass 1: block maximum of kMagic + A (floats, ordered like A) over unmasked keys
+        // Q-smoothing: the block's key biases, bulk-copied with its K codes.  Waiting on the
+        // stage's own barrier makes the copy visible here; the stage cannot be refilled before
+        // this tile's P_j has been consumed, so the phase is still block j's.
+        const float* kbj = sm.kb[j % NST];
+        if constexpr (QS) mbar_wait(&sm.k_full[j % NST], (j / NST) & 1, 112);
+        // pass 1: block maximum of kMagic + A (floats, ordered like A) over unmasked keys; with
+        // Q-smoothing, of the biased scores themselves
         float mx = -INFINITY;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -311,7 +325,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld16(sa + h * 32, a0);
           tmem_ld16(sa + h * 32 + 16, a1);
           tmem_ld_wait();
-          if (diag) {
+          if constexpr (QS) {
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) {
+              const int k0 = key0 + h * 32 + cc;
+              float f0 = fmaf(kbj[h * 32 + cc], args.scale_log2, deq(a0[cc], c22, nc22));
+              float f1 = fmaf(kbj[h * 32 + 16 + cc], args.scale_log2, deq(a1[cc], c22, nc22));
+              if (diag && k0 > i) f0 = -INFINITY;
+              if (diag && k0 + 16 > i) f1 = -INFINITY;
+              mx = fmax3(mx, f0, f1);
+            }
+          } else if (diag) {
 #pragma unroll
             for (int cc = 0; cc < 16; ++cc) {
               const int k0 = key0 + h * 32 + cc;
@@ -326,7 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const bool has = mx != -INFINITY;
-        const float mblk = has ? __fmaf_rn(mx, c22, nc22) : -INFINITY;  // fl(c * A_max)
+        float mblk;
+        if constexpr (QS)
+          mblk = mx;
+        else
+          mblk = has ? __fmaf_rn(mx, c22, nc22) : -INFINITY;  // fl(c * A_max)
         // pass 2: p~ = exp2(z - mblk), codes rne(127 p~), row sum
         float rs = 0.0f;
         int8_t* prow = pbase + (j & 1) * (BM * BKV);
@@ -346,7 +374,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int e = 0; e < 4; ++e) {
                 const int cc = q4 * 4 + e;
                 const uint32_t av = half ? a1[cc] : a0[cc];
-                float p = ex2_approx(deq(av, c22, nc22) - mblk);
+                float z = deq(av, c22, nc22);
+                if constexpr (QS) z = fmaf(kbj[h * 32 + half * 16 + cc], args.scale_log2, z);
+                float p = ex2_approx(z - mblk);
                 if (diag && key0 + h * 32 + half * 16 + cc > i) p = 0.0f;
                 rs += p;
                 f[e] = __fmaf_rn(p, 127.0f, kMagic);

@@ -114,6 +114,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// Contiguous global -> shared copy of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned), completing `bar`'s transaction count.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Asynchronous element-wise add of a shared-memory box into global memory (the TMA unit
 // performs the reduction; float32 add for a float32 tensor map).  Tracked by bulk groups.
 __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int x,

@@ -114,7 +114,8 @@ __device__ __forceinline__ uint2 quant8(const float (&x)[8], float s) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// Prologue pass 1 (only with K-smoothing): per 64-token block of k, the column sums of khat.
+// Prologue pass 1 (only with smoothing): per 64-token block of k (or q), the column sums of
+// khat (qhat).
 // One group of D/8 lanes walks one block's 64 tokens in order.  partials: [BH * N/64, D].
 // ---------------------------------------------------------------------------------------------
 template <typename T, int D>
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(kRowThreads) prologue_kstats_kernel(
   dst[1] = make_float4(c[4], c[5], c[6], c[7]);
 }
 
-// Prologue pass 2 (only with K-smoothing): m[bh][c] = (sum over blocks in order) / N.
+// Prologue pass 2 (only with smoothing): m[bh][c] = (sum over blocks in order) / N.
 template <int D>
 __global__ void prologue_kmean_kernel(const float* __restrict__ partials,
                                       float* __restrict__ k_mean, int nkb, int N) {
@@ -181,7 +182,9 @@ struct PrologueArgs {
   float* scale[3];         // q, k, v scales
   float* inv_rms[2];       // q, k
   const float* k_mean;     // [BH, D] (ksmooth)
-  int BH, N, q_block, qknorm, ksmooth;
+  const float* q_mean;     // [BH, D] (qsmooth)
+  float* k_bias;           // [BH, N] (qsmooth): mu_Q . ktilde_j
+  int BH, N, q_block, qknorm, ksmooth, qsmooth;
   float eps;
 };
 
@@ -218,15 +221,33 @@ __global__ void __launch_bounds__(kRowThreads) prologue_quant_kernel(PrologueArg
       if (sub == 0) a.inv_rms[which][row0 + r] = inv;
     }
   }
-  if (which == 1 && a.ksmooth) {
-    const float4* mp =
-        reinterpret_cast<const float4*>(a.k_mean + static_cast<size_t>(bh) * D + sub * 8);
+  // smoothing: K's mean (ksmooth) or Q's (qsmooth) subtracted just before quantization
+  const float* mean = which == 1 ? (a.ksmooth ? a.k_mean : nullptr)
+                                 : (which == 0 && a.qsmooth ? a.q_mean : nullptr);
+  if (mean) {
+    const float4* mp = reinterpret_cast<const float4*>(mean + static_cast<size_t>(bh) * D + sub * 8);
     const float4 m0 = mp[0], m1 = mp[1];
     const float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
     for (int s = 0; s < STEPS; ++s)
 #pragma unroll
       for (int c = 0; c < 8; ++c) x[s][c] = __fsub_rn(x[s][c], m[c]);
+  }
+  if (which == 1 && a.qsmooth) {
+    // Q-smoothing bias of every key: k_bias_j = mu_Q . ktilde_j (lane partials + butterfly)
+    const float4* mp =
+        reinterpret_cast<const float4*>(a.q_mean + static_cast<size_t>(bh) * D + sub * 8);
+    const float4 m0 = mp[0], m1 = mp[1];
+    const float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+    for (int s = 0; s < STEPS; ++s) {
+      float p = 0.0f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) p = __fadd_rn(p, __fmul_rn(m[c], x[s][c]));
+      const float b = row_sum<D / 8>(p, mask);
+      const int r = warp * 16 + s * GPW + grp;
+      if (sub == 0) a.k_bias[row0 + r] = b;
+    }
   }
   float amax = 0.0f;
 #pragma unroll

@@ -39,6 +39,7 @@ int check_params(const sage_params* p) {
   if (p->k_block != 64) return SAGE_ERR_UNSUPPORTED;
   if (p->q_block != 64 && p->q_block != 128) return SAGE_ERR_UNSUPPORTED;
   if (p->N % 128 != 0) return SAGE_ERR_UNSUPPORTED;
+  if (p->qsmooth != 0 && p->qsmooth != 1) return SAGE_ERR_INVALID_ARG;
   // row indices of [B*H*N, d] tensors are passed to TMA as int32
   if (static_cast<long long>(p->B) * p->H * p->N >= (1ll << 31)) return SAGE_ERR_UNSUPPORTED;
   return SAGE_OK;
@@ -54,9 +55,12 @@ int check_qbufs(const sage_params* p, const sage_qbufs* qb) {
     return SAGE_ERR_INVALID_ARG;
   if (p->qknorm && (!qb->q_inv_rms || !qb->k_inv_rms)) return SAGE_ERR_INVALID_ARG;
   if (p->ksmooth && !qb->k_mean) return SAGE_ERR_INVALID_ARG;
+  if (p->qsmooth && (!qb->q_mean || !qb->k_bias)) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(qb->q_codes) || !aligned16(qb->k_codes) || !aligned16(qb->v_codes))
     return SAGE_ERR_ALIGNMENT;
   if (qb->k_mean && !aligned16(qb->k_mean)) return SAGE_ERR_ALIGNMENT;
+  if (p->qsmooth && (!aligned16(qb->q_mean) || !aligned16(qb->k_bias)))
+    return SAGE_ERR_ALIGNMENT;
   return SAGE_OK;
 }
 
@@ -74,9 +78,13 @@ BwdWs bwd_ws(const sage_params* p) {
   w.total = align_up(w.dq + BH * N * d * 4);
   return w;
 }
+// Column-sum partials of the smoothed tensors: K's (ksmooth) then Q's (qsmooth).
+size_t prologue_partials(const sage_params* p) {
+  return static_cast<size_t>(p->B) * p->H * (p->N / 64) * p->d;
+}
 size_t prologue_ws(const sage_params* p) {
-  if (!p->ksmooth) return 0;
-  return align_up(static_cast<size_t>(p->B) * p->H * (p->N / 64) * p->d * 4);
+  const int n = (p->ksmooth ? 1 : 0) + (p->qsmooth ? 1 : 0);
+  return n == 0 ? 0 : align_up(n * prologue_partials(p) * 4);
 }
 
 // ---- TMA tensor maps --------------------------------------------------------------------
@@ -140,13 +148,18 @@ template <typename T, int D>
 int run_prologue(const sage_params* p, const void* q, const void* k, const void* v,
                  const sage_qbufs* out, void* ws, cudaStream_t st) {
   const int BH = p->B * p->H, N = p->N;
-  if (p->ksmooth) {
-    float* partials = reinterpret_cast<float*>(ws);
-    const int total = BH * (N / 64);
-    const int per_cta = (kRowThreads / 32) * (32 / (D / 8));
+  float* partials = reinterpret_cast<float*>(ws);
+  const int total = BH * (N / 64);
+  const int per_cta = (kRowThreads / 32) * (32 / (D / 8));
+  // smoothing means: K's (ksmooth), then Q's (qsmooth), each from its own partials
+  for (int which = 1; which >= 0; --which) {
+    if (which == 1 ? !p->ksmooth : !p->qsmooth) continue;
     sage::prologue_kstats_kernel<T, D><<<(total + per_cta - 1) / per_cta, kRowThreads, 0, st>>>(
-        reinterpret_cast<const T*>(k), partials, total, p->qknorm, p->rms_eps);
-    sage::prologue_kmean_kernel<D><<<BH, D, 0, st>>>(partials, out->k_mean, N / 64, N);
+        reinterpret_cast<const T*>(which == 1 ? k : q), partials, total, p->qknorm,
+        p->rms_eps);
+    sage::prologue_kmean_kernel<D><<<BH, D, 0, st>>>(
+        partials, which == 1 ? out->k_mean : out->q_mean, N / 64, N);
+    partials += prologue_partials(p);
   }
   sage::PrologueArgs a;
   a.src[0] = q;
@@ -161,11 +174,14 @@ int run_prologue(const sage_params* p, const void* q, const void* k, const void*
   a.inv_rms[0] = out->q_inv_rms;
   a.inv_rms[1] = out->k_inv_rms;
   a.k_mean = out->k_mean;
+  a.q_mean = out->q_mean;
+  a.k_bias = out->k_bias;
   a.BH = BH;
   a.N = N;
   a.q_block = p->q_block;
   a.qknorm = p->qknorm;
   a.ksmooth = p->ksmooth;
+  a.qsmooth = p->qsmooth;
   a.eps = p->rms_eps;
   sage::prologue_quant_kernel<T, D><<<3 * BH * (N / kRowsPerCta), kRowThreads, 0, st>>>(a);
   return launch_status();
@@ -193,8 +209,10 @@ int run_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse, cud
   a.causal = p->causal;
   a.scale_log2 = tau_of(p) * 1.4426950408889634f;
   a.nsup = (N + sage::fwd::NT * sage::fwd::BM - 1) / (sage::fwd::NT * sage::fwd::BM);
+  a.k_bias = qb->k_bias;
   const size_t smem = sage::fwd::smem_bytes<D>();
-  auto kern = sage::fwd::attn_fwd_kernel<T, D>;
+  auto kern = p->qsmooth ? sage::fwd::attn_fwd_kernel<T, D, true>
+                         : sage::fwd::attn_fwd_kernel<T, D, false>;
   if (set_smem(kern, smem) != SAGE_OK) return SAGE_ERR_CUDA;
   // register split between warpgroups (setmaxnreg) assumes exactly kLaunchRegs at launch
   if (launch_regs(kern) != sage::fwd::kLaunchRegs) return SAGE_ERR_UNSUPPORTED;
@@ -257,8 +275,11 @@ int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const
   a.qknorm = p->qknorm;
   a.tau = tau_of(p);
   a.scale_log2 = a.tau * 1.4426950408889634f;
+  a.k_bias = qb->k_bias;
+  a.q_mean = qb->q_mean;
   const size_t smem = sage::bwd::smem_bytes<D>();
-  auto kern = sage::bwd::attn_bwd_kernel<T, D>;
+  auto kern = p->qsmooth ? sage::bwd::attn_bwd_kernel<T, D, true>
+                         : sage::bwd::attn_bwd_kernel<T, D, false>;
   if (set_smem(kern, smem) != SAGE_OK) return SAGE_ERR_CUDA;
   // The kernel moves registers between warpgroups (setmaxnreg); the split is sized for a launch
   // allocation of exactly kLaunchRegs per thread.  Any other allocation could leave the

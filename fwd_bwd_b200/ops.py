@@ -30,12 +30,13 @@ class Config:
     k_block: int = 64
     softmax_scale: float = 0.0  # <= 0: 1/sqrt(d)
     rms_eps: float = 1e-6
+    qsmooth: bool = False
 
     def params(self, x: torch.Tensor) -> SageParams:
         B, H, N, d = x.shape
         return SageParams(B, H, N, d, _DTYPES[x.dtype], int(self.causal), int(self.qknorm),
                           int(self.ksmooth), self.q_block, self.k_block,
-                          float(self.softmax_scale), float(self.rms_eps))
+                          float(self.softmax_scale), float(self.rms_eps), int(self.qsmooth))
 
 
 @dataclasses.dataclass
@@ -51,6 +52,8 @@ class QuantBufs:
     q_inv_rms: Optional[torch.Tensor]
     k_inv_rms: Optional[torch.Tensor]
     k_mean: Optional[torch.Tensor]
+    q_mean: Optional[torch.Tensor] = None
+    k_bias: Optional[torch.Tensor] = None
 
     @staticmethod
     def empty(shape, cfg: Config, device) -> "QuantBufs":
@@ -64,13 +67,15 @@ class QuantBufs:
             torch.empty((B, H, N // cfg.k_block), **f32),
             torch.empty((B, H, N), **f32) if cfg.qknorm else None,
             torch.empty((B, H, N), **f32) if cfg.qknorm else None,
-            torch.empty((B, H, d), **f32) if cfg.ksmooth else None)
+            torch.empty((B, H, d), **f32) if cfg.ksmooth else None,
+            torch.empty((B, H, d), **f32) if cfg.qsmooth else None,
+            torch.empty((B, H, N), **f32) if cfg.qsmooth else None)
 
     def c_struct(self) -> SageQBufs:
         p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
         return SageQBufs(p(self.q_codes), p(self.k_codes), p(self.v_codes), p(self.q_scale),
                          p(self.k_scale), p(self.v_scale), p(self.q_inv_rms),
-                         p(self.k_inv_rms), p(self.k_mean))
+                         p(self.k_inv_rms), p(self.k_mean), p(self.q_mean), p(self.k_bias))
 
 
 def _stream(device) -> int:
@@ -179,9 +184,9 @@ class _SageAttention(torch.autograd.Function):
 
 def sage_attention(q, k, v, causal: bool = True, qknorm: bool = True, ksmooth: bool = True,
                    q_block: int = 128, k_block: int = 64, softmax_scale: float = 0.0,
-                   rms_eps: float = 1e-6):
+                   rms_eps: float = 1e-6, qsmooth: bool = False):
     """SageBwd attention with autograd: q, k, v are CUDA [B, H, N, d] fp16/bf16 tensors."""
-    cfg = Config(causal, qknorm, ksmooth, q_block, k_block, softmax_scale, rms_eps)
+    cfg = Config(causal, qknorm, ksmooth, q_block, k_block, softmax_scale, rms_eps, qsmooth)
     return _SageAttention.apply(q, k, v, cfg)
 
 

@@ -60,6 +60,10 @@ typedef struct {
   int k_block; /* tokens per K and V quantization block: 64                           */
   float softmax_scale;
   float rms_eps;
+  int qsmooth; /* 1: Q-smoothing as well (Q-smoothing paragraph): subtract the per-channel
+                  token mean mu_Q from qhat before quantization, add the per-key bias
+                  k_bias_j = mu_Q . ktilde_j to the scores and the correction
+                  softmax_scale * (dS^T 1) mu_Q^T to dK.  0: off.                           */
 } sage_params;
 
 /* Quantized views of Q, K, V produced once by the prologue and read by both the forward and
@@ -71,6 +75,8 @@ typedef struct {
   float *q_inv_rms, *k_inv_rms;        /* [B,H,N]; written when qknorm (else unused, may be
                                           NULL)                                            */
   float *k_mean;                       /* [B,H,d]; written when ksmooth (else may be NULL) */
+  float *q_mean;                       /* [B,H,d]; written when qsmooth (else may be NULL) */
+  float *k_bias;                       /* [B,H,N]; written when qsmooth (else may be NULL) */
 } sage_qbufs;
 
 /* Bytes of scratch each call needs: which = 0 prologue, 1 forward, 2 backward.  Returns 0 for
@@ -80,10 +86,13 @@ size_t sage_workspace_bytes(const sage_params* p, int which);
 /* Prologue (QK-norm, K-smoothing and quantization paragraphs).  In float32:
  *   qknorm:  inv = 1/sqrt(sum(x^2)/d + eps), xhat = x * inv for every token of q and k;
  *   ksmooth: m_c = (sum over all N tokens of khat_c) / N, ktilde = khat - m;
+ *   qsmooth: mu_Q the same mean of qhat, qtilde = qhat - mu_Q is what gets quantized, and
+ *            k_bias_j = sum_c mu_Q,c * ktilde_jc (8-channel lane partials, products and sums
+ *            rounded, combined by a butterfly over the lanes, as in the RMSNorm sum);
  *   quantize: per block of q_block (q) or k_block (k, v) tokens spanning all d channels,
  *            s = absmax/127, code = round-half-even(x / s); s = 0 and codes 0 if absmax = 0.
- * The float32 operation order is fixed, so codes, scales, inv_rms and k_mean are
- * reproducible bit for bit.  q, k, v: 16-bit inputs [B,H,N,d].  out: all buffers written. */
+ * The float32 operation order is fixed, so codes, scales, inv_rms, k_mean, q_mean and k_bias
+ * are reproducible bit for bit.  q, k, v: 16-bit inputs [B,H,N,d].  out: all buffers written. */
 int sage_quant_prologue(const sage_params* p, const void* q, const void* k, const void* v,
                         const sage_qbufs* out, void* workspace, size_t workspace_bytes,
                         void* stream);
@@ -94,10 +103,10 @@ int sage_quant_prologue(const sage_params* p, const void* q, const void* k, cons
  * allocation through its own memory pool, code running under a fixed device-memory budget set
  * at start-up, and latency-critical host threads that must not risk the device-wide
  * synchronization cudaMalloc / cudaFree can cause.  This entry point takes no workspace: the
- * K-smoothing column sums go to a fixed 32 MiB array in the library's own device memory (every
+ * smoothing column sums go to a fixed 32 MiB array in the library's own device memory (every
  * GPU that loads the library holds it until exit), so it supports shapes with
- * B * H * (N / 64) * d * 4 <= 32 MiB (e.g. B*H*N*d up to 2^29 elements) and returns
- * SAGE_ERR_WORKSPACE beyond that, before launching anything.  Everything else -- arguments,
+ * (ksmooth + qsmooth) * B * H * (N / 64) * d * 4 <= 32 MiB (e.g. B*H*N*d up to 2^29 elements
+ * with one of the two) and returns SAGE_ERR_WORKSPACE beyond that, before launching anything.  Everything else -- arguments,
  * outputs, results (bit for bit) -- is as for sage_quant_prologue.  It allocates nothing.
  * The first call on each device looks up the array's device address (with that device
  * current); make that first call before any stream capture.  All calls share the one array,
@@ -108,7 +117,8 @@ int sage_quant_prologue_noalloc(const sage_params* p, const void* q, const void*
                                 const void* v, const sage_qbufs* out, void* stream);
 
 /* Forward attention with INT8 S = Qc Kc^T and O = Pc Vc (quantization-strategy paragraph).
- * z = A * sQ * sK * softmax_scale; P is quantized with one scale per (query row, K block);
+ * z = (A * sQ * sK + k_bias_j) * softmax_scale (k_bias_j = 0 without qsmooth); P is quantized
+ * with one scale per (query row, K block);
  * o: [B,H,N,d] in dtype; lse: [B,H,N] float32, natural log-sum-exp of the scaled scores. */
 int sage_attn_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse,
                   void* workspace, size_t workspace_bytes, void* stream);
@@ -116,7 +126,9 @@ int sage_attn_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* ls
 /* Backward attention (quantization-strategy and error-propagation paragraphs): recomputes the
  * INT8 scores from the same codes, dP = dO V^T in 16-bit float with float32 accumulation,
  * dS = P (dP - rowsum(dO o O)), P and dS quantized per q_block x k_block tile, dO per q_block
- * tokens; dV = P^T dO, dK = dS^T Q, dQ = dS K in INT8.  q, k, v are the raw 16-bit inputs
+ * tokens; dV = P^T dO, dK = dS^T Q, dQ = dS K in INT8 (with qsmooth, the scores carry the
+ * forward's bias and dK gains softmax_scale * (sum_i dS_ij) mu_Q, the column sums taken over the
+ * quantized dS tiles).  q, k, v are the raw 16-bit inputs
  * (needed for dP and the RMSNorm backward); o, lse the forward's outputs; dout = dL/do.
  * dq, dk, dv: [B,H,N,d] in dtype, gradients with respect to the raw q, k, v. */
 int sage_attn_bwd(const sage_params* p, const void* q, const void* k, const void* v,

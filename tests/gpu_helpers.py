@@ -20,7 +20,7 @@ def to_device(bits: np.ndarray, dtype: str) -> torch.Tensor:
 
 def cfg_of(w: Workload) -> ops.Config:
     return ops.Config(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth, q_block=w.q_block,
-                      k_block=w.k_block)
+                      k_block=w.k_block, qsmooth=w.qsmooth)
 
 
 def gpu_run(w: Workload, x: dict, backward: bool = True) -> dict:
@@ -37,7 +37,7 @@ def gpu_run(w: Workload, x: dict, backward: bool = True) -> dict:
     assert ops.device_status() == 0
     res.update(o=o, lse=lse)
     for name in ("q_codes", "k_codes", "v_codes", "q_scale", "k_scale", "v_scale",
-                 "q_inv_rms", "k_inv_rms", "k_mean"):
+                 "q_inv_rms", "k_inv_rms", "k_mean", "q_mean", "k_bias"):
         t = getattr(qb, name)
         if t is not None:
             res[name] = t
@@ -59,7 +59,7 @@ def oracle_run(w: Workload, x: dict, quant: bool = True) -> dict:
     args = [a.reshape(-1, w.N, w.d) for a in args]
     return O.sage_attention(*args, causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth,
                             q_block=w.q_block, k_block=w.k_block, dtype=w.dtype, quant=quant,
-                            round_outputs=quant)
+                            round_outputs=quant, qsmooth=w.qsmooth)
 
 
 def rel_l2(a, b) -> float:

@@ -5,8 +5,9 @@ Gates (element by element over every output):
   * LSE: max |difference| <= 1e-3;
   * cosine similarity >= 0.995 against full-precision (float64) attention.
 The sizes span several query/key tiles, a ragged number of 256-query CTA tiles, both head
-dims, both 16-bit types, both quantization block sizes for Q, causal and not, and every
-combination of the QK-norm / K-smoothing flags.
+dims, both 16-bit types, both quantization block sizes for Q, causal and not, every
+combination of the QK-norm / K-smoothing flags, and the Q-smoothing variant (score bias and
+dK correction) on Q-outlier inputs.
 """
 import numpy as np
 import pytest
@@ -37,6 +38,12 @@ CASES = {
     "koutlier_off_off": K.replace(B=1, H=2, N=512, qknorm=False, ksmooth=False),
     "small_ds_regime": WORKLOADS["long16k"].replace(H=2, N=1024),
     "single_tile": S.replace(B=1, H=1, N=128),
+    "qsmooth_d128_causal": WORKLOADS["qoutlier"].replace(B=1, H=2, N=512),
+    "qsmooth_d64_fp16_noncausal_qb64": WORKLOADS["tiny"].replace(q_outlier=True, qsmooth=True),
+    "qsmooth_d128_qb64_ksmooth_off": WORKLOADS["qoutlier"].replace(B=1, H=2, N=384, q_block=64,
+                                                                  ksmooth=False),
+    "qsmooth_d64_causal_norm_off": L.replace(B=1, H=2, N=512, qknorm=False, q_outlier=True,
+                                             qsmooth=True),
 }
 
 

@@ -1,4 +1,5 @@
-"""Prologue parity: INT8 codes, block scales, inverse RMS and K means bit-exact vs the oracle."""
+"""Prologue parity: INT8 codes, block scales, inverse RMS, K means and (Q-smoothing) Q means and
+key biases bit-exact vs the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -21,13 +22,17 @@ CASES = {
     "koutlier_smooth_off": WORKLOADS["koutlier"].replace(B=1, H=2, N=512, ksmooth=False),
     "koutlier_all_off": WORKLOADS["koutlier"].replace(B=1, H=2, N=256, qknorm=False,
                                                      ksmooth=False),
+    "qsmooth_d128_bf16": WORKLOADS["qoutlier"].replace(B=1, H=2, N=512),
+    "qsmooth_d64_fp16_qb64": WORKLOADS["tiny"].replace(q_outlier=True, qsmooth=True),
+    "qsmooth_ksmooth_off": WORKLOADS["qoutlier"].replace(B=1, H=2, N=256, ksmooth=False),
+    "qsmooth_norm_off": WORKLOADS["qoutlier"].replace(B=2, H=1, N=256, qknorm=False),
 }
 
 
 def _compare(w, x, res):
     args = [x[n + "_f32"].reshape(-1, w.N, w.d) for n in ("q", "k", "v")]
     ref = O.prologue(*args, q_block=w.q_block, k_block=w.k_block, qknorm=w.qknorm,
-                     ksmooth=w.ksmooth)
+                     ksmooth=w.ksmooth, qsmooth=w.qsmooth)
     BH = w.B * w.H
     for name in ("q_codes", "k_codes", "v_codes"):
         np.testing.assert_array_equal(res[name].reshape(BH, w.N, w.d), ref[name], err_msg=name)
@@ -41,6 +46,11 @@ def _compare(w, x, res):
     if w.ksmooth:
         np.testing.assert_array_equal(res["k_mean"].reshape(BH, w.d).view(np.uint32),
                                       ref["k_mean"].view(np.uint32), err_msg="k_mean")
+    if w.qsmooth:
+        np.testing.assert_array_equal(res["q_mean"].reshape(BH, w.d).view(np.uint32),
+                                      ref["q_mean"].view(np.uint32), err_msg="q_mean")
+        np.testing.assert_array_equal(res["k_bias"].reshape(BH, w.N).view(np.uint32),
+                                      ref["k_bias"].view(np.uint32), err_msg="k_bias")
 
 
 @pytest.mark.parametrize("case", sorted(CASES))

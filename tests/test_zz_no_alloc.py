@@ -23,7 +23,7 @@ pytestmark = pytest.mark.gpu
 
 TORCH_DT = {"bf16": torch.bfloat16, "fp16": torch.float16}
 FIELDS = ("q_codes", "k_codes", "v_codes", "q_scale", "k_scale", "v_scale", "q_inv_rms",
-          "k_inv_rms", "k_mean")
+          "k_inv_rms", "k_mean", "q_mean", "k_bias")
 
 
 def _dev(bits, dtype):
@@ -33,13 +33,14 @@ def _dev(bits, dtype):
 
 def _cfg(w):
     return ops.Config(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth, q_block=w.q_block,
-                      k_block=w.k_block)
+                      k_block=w.k_block, qsmooth=w.qsmooth)
 
 
 def test_noalloc_prologue_matches_workspace_prologue_twice():
     L = _lib.lib()
     cases = [WORKLOADS["koutlier"].replace(B=2, H=4, N=1024),
-             WORKLOADS["llama325m"].replace(B=1, H=3, N=768, seed=7)]
+             WORKLOADS["llama325m"].replace(B=1, H=3, N=768, seed=7),
+             WORKLOADS["qoutlier"].replace(B=1, H=3, N=512)]
     for w in cases:
         x = make_inputs(w)
         q, k, v = (_dev(x[n], w.dtype) for n in ("q", "k", "v"))
