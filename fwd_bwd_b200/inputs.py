@@ -175,3 +175,36 @@ def make_inputs_fast(w: Workload, device: str = "cpu"):
             mu[..., :4] += 20.0
             res[name] = (res[name].float() + mu).to(tdt)
     return res
+
+
+def make_study_inputs(w: Workload, seed: int, device: str = "cpu"):
+    """Inputs for the tokens-per-step study: per-seed noise on top of structure every seed shares.
+
+    Trained activations have fixed outlier channels and gradients with a consistent direction;
+    to give the batch-averaged gradient a non-zero expectation that is the same for every seed,
+    Q, K and dO carry fixed per-channel offsets (drawn once from a generator seeded by ``d``):
+    ``q = e + mu_q`` with ``mu_q ~ N(0, 1)``; ``k = e + mu_k`` with ``mu_k ~ N(0, 4^2)`` and +20 on
+    4 channels (the K-outlier recipe); ``v = e``; ``dO = sigma_do (e + mu_do)`` with
+    ``mu_do ~ N(0, 0.5^2)``; every ``e`` is fresh standard-normal noise from torch's generator
+    seeded by ``seed``.  Values are rounded to the workload's 16-bit type.
+    """
+    import torch
+
+    gf = torch.Generator(device="cpu")
+    gf.manual_seed(10_000 + w.d)
+    mu_q = torch.randn(w.d, generator=gf)
+    mu_k = torch.randn(w.d, generator=gf) * 4.0
+    mu_k[torch.randperm(w.d, generator=gf)[:4]] += 20.0
+    mu_do = torch.randn(w.d, generator=gf) * 0.5
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+    shape = (w.B, w.H, w.N, w.d)
+
+    def noise():
+        return torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+
+    return {"q": (noise() + mu_q.to(device)).to(tdt),
+            "k": (noise() + mu_k.to(device)).to(tdt),
+            "v": noise().to(tdt),
+            "do": ((noise() + mu_do.to(device)) * w.sigma_do).to(tdt)}
