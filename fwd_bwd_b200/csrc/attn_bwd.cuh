@@ -86,13 +86,12 @@ struct Smem {
   float dqs[D == 128 ? 8 : 1][2][D == 128 ? kDqRows * kDqCols : 4];
   alignas(16) float red_p[2][8];  // per-warp tile maxima of P, [tile parity][warp]
   alignas(16) float red_ds[2][8];  // and of |dS|
-  float sp[3][2][2], sds[3][2][2];  // tile scales [tile % 3][q group][key half]
   float dot[BKT];                   // RMSNorm-backward row dot products (warpgroup 1 -> 0)
   float kb[BKT];                    // Q-smoothing: k_bias of the CTA's keys
   float cs[BKT];                    // Q-smoothing: sum over tiles of sdS * (column sum of dSc)
   uint64_t kv_full, q_full[2], q_empty[2], dor_full, dor_free;
   uint64_t sdp_full[2], pds_ready, dvdk_full, dvdk_free, dq_full, dq_free;
-  uint64_t scales_full[2];  // tile parity: the P / dS scales of both warpgroups are written
+  uint64_t red_full[2];  // tile parity: every warp's tile maxima are in red_p / red_ds
   uint32_t tmem_base;
   int abort;
 };
@@ -173,8 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.dor_full, 1);
     mbar_init(&sm.dor_free, 1);
     mbar_init(&sm.pds_ready, 256);
-    for (int s = 0; s < 2; ++s)  // writers: one per q group per key half
-      mbar_init(&sm.scales_full[s], 2 * (BQ / args.q_block));
+    for (int s = 0; s < 2; ++s)  // one arrival per compute warp
+      mbar_init(&sm.red_full[s], 8);
     mbar_init(&sm.dvdk_full, 1);
     mbar_init(&sm.dvdk_free, 256);
     mbar_init(&sm.dq_full, 1);
@@ -354,10 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       lse2 = args.lse[grow] * 1.4426950408889634f;
       dvr = args.dvec[grow];
     };
-    // pass A of tile it: P, dS into TMEM buffer it&1, tile maxima -> scales in slot it%3
-    auto pass_a = [&](int it, float c, float lse2, float dvr, float& ip, float& ids,
-                      float& sds_own) {
-      const int b = it & 1, slot = it % 3;
+    // pass A of tile it: P, dS into TMEM buffer it&1, per-warp maxima into red_*[it&1]
+    auto pass_a = [&](int it, float c, float lse2, float dvr) {
+      const int b = it & 1;
       const uint32_t lane_base = tmem + lane_off + b * 256;
       const int qt = i_first + it;
       const bool diag = args.causal && (qt == t);
@@ -414,50 +412,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       else
         chunks(std::false_type{});
       tmem_st_wait();
-      // per-tile maxima: tile = q_block rows x 64 keys (this warpgroup's key block)
+      // per-warp maxima of P and |dS|; the tile maxima (q_block rows x 64 keys) are formed by
+      // their readers -- pass B and the read-outs of this tile -- once every warp has arrived
       pmax = warp_max(pmax);
       dsmax = warp_max(dsmax);
       if (lane == 0) {
         sm.red_p[b][h * 4 + quarter] = pmax;
         sm.red_ds[b][h * 4 + quarter] = dsmax;
+        mbar_arrive(&sm.red_full[b]);
       }
-      named_barrier_sync(1 + h, 128);
-      // the q_block group's warps: all four (q_block = 128) or this warp's pair (64)
-      const float4 rp = *reinterpret_cast<const float4*>(&sm.red_p[b][h * 4]);
-      const float4 rd = *reinterpret_cast<const float4*>(&sm.red_ds[b][h * 4]);
-      float tp, tds;
-      if (wpg == 4) {
-        tp = fmaxf(fmaxf(rp.x, rp.y), fmaxf(rp.z, rp.w));
-        tds = fmaxf(fmaxf(rd.x, rd.y), fmaxf(rd.z, rd.w));
-      } else {
-        tp = quarter < 2 ? fmaxf(rp.x, rp.y) : fmaxf(rp.z, rp.w);
-        tds = quarter < 2 ? fmaxf(rd.x, rd.y) : fmaxf(rd.z, rd.w);
-      }
-      if (lane == 0 && (quarter % wpg) == 0) {
-        sm.sp[slot][g_row][h] = __fdiv_rn(tp, 127.0f);
-        sm.sds[slot][g_row][h] = __fdiv_rn(tds, 127.0f);
-        mbar_arrive(&sm.scales_full[it & 1]);  // read by both warpgroups in the read-outs
-      }
-      // code multipliers: the codes are not compared bit for bit, so the fast divide (within
-      // 2 ulp) serves; the stored scales above are IEEE quotients
-      ip = tp > 0.0f ? __fdividef(127.0f, tp) : 0.0f;
-      ids = tds > 0.0f ? __fdividef(127.0f, tds) : 0.0f;
-      if constexpr (QS) sds_own = __fdiv_rn(tds, 127.0f);  // this row group's dS scale
-      // No CTA-wide barrier here: the warpgroups may drift apart.  sm.red_*[b] is rewritten
-      // only in pass A of tile it+2, which waits for that tile's S / dP, issued after every
-      // thread released tile it's dQ -- i.e. after every warp finished reading it for tile it.
-      // (Tiles 0 and 1 have their S / dP issued back to back, hence the two slots.)
+      // sm.red_*[b] is rewritten only in pass A of tile it+2, which waits for that tile's
+      // S / dP, issued after every thread released tile it's dQ -- i.e. after every warp
+      // finished reading them for tile it.  (Tiles 0 and 1 have their S / dP issued back to
+      // back, hence the two slots.)
+    };
+    // maximum over the warps of q_block group g in warpgroup kh's key block (the tile's
+    // absmax of P or dS): all four warps (q_block = 128) or a pair (64)
+    auto tile_max = [&](const float* red, int g, int kh) {
+      const float4 v = *reinterpret_cast<const float4*>(red + kh * 4);
+      if (wpg == 4) return fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+      return g == 0 ? fmaxf(v.x, v.y) : fmaxf(v.z, v.w);
     };
 
-    float c_n, lse2_n, dvr_n, ip, ids, sdsc = 0.0f;
+    float c_n, lse2_n, dvr_n;
     row_inputs(0, c_n, lse2_n, dvr_n);
-    pass_a(0, c_n, lse2_n, dvr_n, ip, ids, sdsc);
+    pass_a(0, c_n, lse2_n, dvr_n);
     for (int it = 0; it < nq; ++it) {
-      const int b = it & 1, slot = it % 3;
+      const int b = it & 1;
       const uint32_t lane_base = tmem + lane_off + b * 256;
       const int qt = i_first + it;
       const size_t grow = static_cast<size_t>(row_base) + qt * BQ + r;
       if (it + 1 < nq) row_inputs(it + 1, c_n, lse2_n, dvr_n);  // loads in flight during pass B
+      // this tile's maxima (every warp arrived during pass A, a whole phase ago).  One barrier
+      // per tile parity, so arrivals for tiles it and it+1 never share a phase; a warp cannot
+      // arrive for tile it+2 before every thread released tile it's dQ.
+      mbar_wait(&sm.red_full[b], (it >> 1) & 1, 213);
+      float ip, ids, sdsc = 0.0f;
+      {
+        const float tp = tile_max(sm.red_p[b], g_row, h);
+        const float tds = tile_max(sm.red_ds[b], g_row, h);
+        // code multipliers: the codes are not compared bit for bit, so the fast divide
+        // (within 2 ulp) serves; the scales the read-outs use are IEEE quotients
+        ip = tp > 0.0f ? __fdividef(127.0f, tp) : 0.0f;
+        ids = tds > 0.0f ? __fdividef(127.0f, tds) : 0.0f;
+        if constexpr (QS) sdsc = __fdiv_rn(tds, 127.0f);  // this row group's dS scale
+      }
       // pass B: INT8 codes into shared memory; the dV_t / dK_t regions re-preloaded.  The TMEM
       // loads of chunk ch+1 are in flight while chunk ch is converted.
       auto proc_b = [&](uint32_t (&sa)[16], uint32_t (&pa)[16], int ch) {
@@ -529,22 +528,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         sq_t[g] = args.q_scale[qb];
       }
       // pass A of the next tile while the tensor core works on this one
-      float ip_n = 0.0f, ids_n = 0.0f, sdsc_n = 0.0f;
-      if (it + 1 < nq) pass_a(it + 1, c_n, lse2_n, dvr_n, ip_n, ids_n, sdsc_n);
+      if (it + 1 < nq) pass_a(it + 1, c_n, lse2_n, dvr_n);
       // step 3: dV_t, dK_t (thread = key row r, d columns of warpgroup h) into registers;
-      // the read columns are re-preloaded for dQ_t.  The tile scales of both warpgroups are
-      // read from here on.  One barrier per tile parity, so arrivals for tiles it and it+1
-      // never share a phase; a writer cannot reach tile it+2 before this thread released tile
-      // it's dQ (its S / dP are issued only after that).
-      mbar_wait(&sm.scales_full[b], (it >> 1) & 1, 213);
+      // the read columns are re-preloaded for dQ_t.  The tile scales (P and dS absmax / 127,
+      // IEEE quotients) come from the maxima of the key half this thread's key row is in.
       for (int g = 0; g < G; ++g) {
         const float sdo = g == 0 ? sdo_t[0] : sdo_t[1];
         const float sqg = g == 0 ? sq_t[0] : sq_t[1];
         const int kh = r >> 6;
         mbar_wait(&sm.dvdk_full, dvdk_cnt & 1, 211);
         tc_fence_after();
-        const float sv22 = scale22(sm.sp[slot][g][kh] * sdo);
-        const float sk22 = scale22(sm.sds[slot][g][kh] * sqg * args.tau);
+        // P / dS scales of this key row's half (IEEE quotients absmax / 127)
+        const float sp = __fdiv_rn(tile_max(sm.red_p[b], g, kh), 127.0f);
+        const float sds = __fdiv_rn(tile_max(sm.red_ds[b], g, kh), 127.0f);
+        const float sv22 = scale22(sp * sdo);
+        const float sk22 = scale22(sds * sqg * args.tau);
         const float nsv = __fmul_rn(-kMagic, sv22), nsk = __fmul_rn(-kMagic, sk22);
         // 16-column chunks; the loads of chunk c+1 are in flight while chunk c accumulates
         uint32_t tv0[16], tk0[16], tv1[16], tk1[16];
@@ -594,8 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // to the global accumulator; no warp waits for another.  The TMEM loads of round rr+1
         // are in flight while round rr is staged.
         const int g = (64 * h) / args.q_block;
-        const float s0 = scale22(sm.sds[slot][g][0] * sk0 * args.tau);
-        const float s1 = scale22(sm.sds[slot][g][1] * sk1 * args.tau);
+        const float s0 = scale22(__fdiv_rn(tile_max(sm.red_ds[b], g, 0), 127.0f) * sk0 * args.tau);
+        const float s1 = scale22(__fdiv_rn(tile_max(sm.red_ds[b], g, 1), 127.0f) * sk1 * args.tau);
         const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
         uint32_t a0[16], a1[16];
         tmem_ld16(lane_base + 64 * h, a0);
@@ -631,8 +629,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st_wait();
       } else {
         // thread = query row r, d columns of warpgroup h
-        const float s0 = scale22(sm.sds[slot][g_row][0] * sk0 * args.tau);
-        const float s1 = scale22(sm.sds[slot][g_row][1] * sk1 * args.tau);
+        const float s0 =
+            scale22(__fdiv_rn(tile_max(sm.red_ds[b], g_row, 0), 127.0f) * sk0 * args.tau);
+        const float s1 =
+            scale22(__fdiv_rn(tile_max(sm.red_ds[b], g_row, 1), 127.0f) * sk1 * args.tau);
         const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
         float* dst = args.dq_acc + grow * D + h * kHalfD;
 #pragma unroll 1
@@ -663,9 +663,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&sm.dq_free);
-      ip = ip_n;
-      ids = ids_n;
-      sdsc = sdsc_n;
     }
     // epilogue: dv, dk from the register accumulators (thread = key row r, d half h)
     {
