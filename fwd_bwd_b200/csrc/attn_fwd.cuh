@@ -32,6 +32,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 #include "rowops.cuh"
 
@@ -273,25 +275,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float nb22 = __fmul_rn(-kMagic, b22);
         mbar_wait(&sm.pv_full[g], jj & 1, 110);
         tc_fence_after();
-        // 16-column chunks, double-buffered: the load of chunk c+1 is in flight while chunk c
+        // 32-column chunks, double-buffered: the loads of chunk c+1 are in flight while chunk c
         // is folded
-        uint32_t a0[16], a1[16];
+        uint32_t a0[16], a1[16], b0[16], b1[16];
         tmem_ld16(lane_base + 128, a0);
+        tmem_ld16(lane_base + 128 + 16, a1);
         tmem_ld_wait_regs(a0, a1);
+        auto fold32 = [&](const uint32_t (&x0)[16], const uint32_t (&x1)[16], int c0) {
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          tmem_ld16(lane_base + 128 + c0 + 16, a1);
+          for (int c = 0; c < 16; ++c) O[c0 + c] = fmaf(O[c0 + c], alpha_prev, deq(x0[c], b22, nb22));
 #pragma unroll
           for (int c = 0; c < 16; ++c)
-            O[c0 + c] = fmaf(O[c0 + c], alpha_prev, deq(a0[c], b22, nb22));
+            O[c0 + 16 + c] = fmaf(O[c0 + 16 + c], alpha_prev, deq(x1[c], b22, nb22));
           tmem_fill16(lane_base + 128 + c0, kMagicBits);
-          tmem_ld_wait_regs(a1, a0);
-          if (c0 + 32 < D) tmem_ld16(lane_base + 128 + c0 + 32, a0);
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            O[c0 + 16 + c] = fmaf(O[c0 + 16 + c], alpha_prev, deq(a1[c], b22, nb22));
           tmem_fill16(lane_base + 128 + c0 + 16, kMagicBits);
-          if (c0 + 32 < D) tmem_ld_wait_regs(a0, a1);
+        };
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 64) {
+          if (c0 + 32 < D) {
+            tmem_ld16(lane_base + 128 + c0 + 32, b0);
+            tmem_ld16(lane_base + 128 + c0 + 48, b1);
+          }
+          fold32(a0, a1, c0);
+          if (c0 + 32 < D) {
+            tmem_ld_wait_regs(b0, b1);
+            if (c0 + 64 < D) {
+              tmem_ld16(lane_base + 128 + c0 + 64, a0);
+              tmem_ld16(lane_base + 128 + c0 + 80, a1);
+            }
+            fold32(b0, b1, c0 + 32);
+            if (c0 + 64 < D) tmem_ld_wait_regs(a0, a1);
+          }
         }
         tmem_st_wait();
         tc_fence_before();
@@ -318,36 +332,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (QS) mbar_wait(&sm.k_full[j % NST], (j / NST) & 1, 112);
         // pass 1: block maximum of kMagic + A (floats, ordered like A) over unmasked keys; with
         // Q-smoothing, of the biased scores themselves
-        float mx = -INFINITY;
+        // (all 64 keys loaded at once; two maximum chains)
+        float mx;
+        {
+          uint32_t a0[16], a1[16], b0[16], b1[16];
+          tmem_ld16(sa, a0);
+          tmem_ld16(sa + 16, a1);
+          tmem_ld16(sa + 32, b0);
+          tmem_ld16(sa + 48, b1);
+          tmem_ld_wait_regs(a0, a1);
+          tmem_ld_wait_regs(b0, b1);
+          float m0 = -INFINITY, m1 = -INFINITY;
+          auto maxh = [&](const uint32_t (&x0)[16], const uint32_t (&x1)[16], int h, float& m) {
+            if constexpr (QS) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t a0[16], a1[16];
-          tmem_ld16(sa + h * 32, a0);
-          tmem_ld16(sa + h * 32 + 16, a1);
-          tmem_ld_wait();
-          if constexpr (QS) {
+              for (int cc = 0; cc < 16; ++cc) {
+                const int k0 = key0 + h * 32 + cc;
+                float f0 = fmaf(kbj[h * 32 + cc], args.scale_log2, deq(x0[cc], c22, nc22));
+                float f1 = fmaf(kbj[h * 32 + 16 + cc], args.scale_log2, deq(x1[cc], c22, nc22));
+                if (diag && k0 > i) f0 = -INFINITY;
+                if (diag && k0 + 16 > i) f1 = -INFINITY;
+                m = fmax3(m, f0, f1);
+              }
+            } else if (diag) {
 #pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-              const int k0 = key0 + h * 32 + cc;
-              float f0 = fmaf(kbj[h * 32 + cc], args.scale_log2, deq(a0[cc], c22, nc22));
-              float f1 = fmaf(kbj[h * 32 + 16 + cc], args.scale_log2, deq(a1[cc], c22, nc22));
-              if (diag && k0 > i) f0 = -INFINITY;
-              if (diag && k0 + 16 > i) f1 = -INFINITY;
-              mx = fmax3(mx, f0, f1);
+              for (int cc = 0; cc < 16; ++cc) {
+                const int k0 = key0 + h * 32 + cc;
+                const float f0 = k0 <= i ? __uint_as_float(x0[cc]) : -INFINITY;
+                const float f1 = k0 + 16 <= i ? __uint_as_float(x1[cc]) : -INFINITY;
+                m = fmax3(m, f0, f1);
+              }
+            } else {
+#pragma unroll
+              for (int cc = 0; cc < 16; ++cc)
+                m = fmax3(m, __uint_as_float(x0[cc]), __uint_as_float(x1[cc]));
             }
-          } else if (diag) {
-#pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-              const int k0 = key0 + h * 32 + cc;
-              const float f0 = k0 <= i ? __uint_as_float(a0[cc]) : -INFINITY;
-              const float f1 = k0 + 16 <= i ? __uint_as_float(a1[cc]) : -INFINITY;
-              mx = fmax3(mx, f0, f1);
-            }
-          } else {
-#pragma unroll
-            for (int cc = 0; cc < 16; ++cc)
-              mx = fmax3(mx, __uint_as_float(a0[cc]), __uint_as_float(a1[cc]));
-          }
+          };
+          maxh(a0, a1, 0, m0);
+          maxh(b0, b1, 1, m1);
+          mx = fmaxf(m0, m1);
         }
         const bool has = mx != -INFINITY;
         float mblk;
@@ -355,41 +378,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           mblk = mx;
         else
           mblk = has ? __fmaf_rn(mx, c22, nc22) : -INFINITY;  // fl(c * A_max)
-        // pass 2: p~ = exp2(z - mblk), codes rne(127 p~), row sum
-        float rs = 0.0f;
+        // pass 2: p~ = exp2(z - mblk), codes rne(127 p~), row sum.  The loads of keys 32..63
+        // are in flight while keys 0..31 are converted; four partial row sums keep the adds
+        // off one dependency chain; the causal mask test exists only in the diagonal blocks'
+        // copy of the loop.
         int8_t* prow = pbase + (j & 1) * (BM * BKV);
+        float rsp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        auto pass2 = [&](auto masked) {
+          uint32_t a0[16], a1[16], b0[16], b1[16];
+          tmem_ld16(sa, a0);
+          tmem_ld16(sa + 16, a1);
+          tmem_ld_wait_regs(a0, a1);
+          tmem_ld16(sa + 32, b0);
+          tmem_ld16(sa + 48, b1);
+          auto conv = [&](const uint32_t (&x0)[16], const uint32_t (&x1)[16], int h) {
+            uint32_t pk[8];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t a0[16], a1[16];
-          tmem_ld16(sa + h * 32, a0);
-          tmem_ld16(sa + h * 32 + 16, a1);
-          tmem_ld_wait();
-          uint32_t pk[8];
+            for (int half = 0; half < 2; ++half) {
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
+              for (int q4 = 0; q4 < 4; ++q4) {
+                float f[4];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              float f[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int cc = q4 * 4 + e;
-                const uint32_t av = half ? a1[cc] : a0[cc];
-                float z = deq(av, c22, nc22);
-                if constexpr (QS) z = fmaf(kbj[h * 32 + half * 16 + cc], args.scale_log2, z);
-                float p = ex2_approx(z - mblk);
-                if (diag && key0 + h * 32 + half * 16 + cc > i) p = 0.0f;
-                rs += p;
-                f[e] = __fmaf_rn(p, 127.0f, kMagic);
+                for (int e = 0; e < 4; ++e) {
+                  const int cc = q4 * 4 + e;
+                  const uint32_t av = half ? x1[cc] : x0[cc];
+                  float z = deq(av, c22, nc22);
+                  if constexpr (QS) z = fmaf(kbj[h * 32 + half * 16 + cc], args.scale_log2, z);
+                  float p = ex2_approx(z - mblk);
+                  if constexpr (decltype(masked)::value) {
+                    if (key0 + h * 32 + half * 16 + cc > i) p = 0.0f;
+                  }
+                  rsp[e] += p;
+                  f[e] = __fmaf_rn(p, 127.0f, kMagic);
+                }
+                pk[half * 4 + q4] = pack_magic4(f[0], f[1], f[2], f[3]);
               }
-              pk[half * 4 + q4] = pack_magic4(f[0], f[1], f[2], f[3]);
             }
-          }
-          // keys h*32 .. h*32+31 are 16-byte chunks 2h and 2h+1 of this row
-          *reinterpret_cast<uint4*>(prow + swz_offset(r, 2 * h, 64)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          *reinterpret_cast<uint4*>(prow + swz_offset(r, 2 * h + 1, 64)) =
-              make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
+            // keys h*32 .. h*32+31 are 16-byte chunks 2h and 2h+1 of this row
+            *reinterpret_cast<uint4*>(prow + swz_offset(r, 2 * h, 64)) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            *reinterpret_cast<uint4*>(prow + swz_offset(r, 2 * h + 1, 64)) =
+                make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          };
+          conv(a0, a1, 0);
+          tmem_ld_wait_regs(b0, b1);
+          conv(b0, b1, 1);
+        };
+        if (diag)
+          pass2(std::true_type{});
+        else
+          pass2(std::false_type{});
+        const float rs = (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
         // the S buffer is read: preload it for S_{j+2}
 #pragma unroll
         for (int c = 0; c < 64; c += 16) tmem_fill16(sa + c, kMagicBits);
