@@ -333,9 +333,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // pass 1: block maximum of kMagic + A (floats, ordered like A) over unmasked keys; with
         // Q-smoothing, of the biased scores themselves
         // (all 64 keys loaded at once; two maximum chains)
+        // the block's 64 scores stay in registers for pass 2
         float mx;
+        uint32_t a0[16], a1[16], b0[16], b1[16];
         {
-          uint32_t a0[16], a1[16], b0[16], b1[16];
           tmem_ld16(sa, a0);
           tmem_ld16(sa + 16, a1);
           tmem_ld16(sa + 32, b0);
@@ -378,19 +379,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           mblk = mx;
         else
           mblk = has ? __fmaf_rn(mx, c22, nc22) : -INFINITY;  // fl(c * A_max)
-        // pass 2: p~ = exp2(z - mblk), codes rne(127 p~), row sum.  The loads of keys 32..63
-        // are in flight while keys 0..31 are converted; four partial row sums keep the adds
-        // off one dependency chain; the causal mask test exists only in the diagonal blocks'
-        // copy of the loop.
+        // pass 2: p~ = exp2(z - mblk), codes rne(127 p~), row sum, from the scores pass 1
+        // loaded; four partial row sums keep the adds off one dependency chain; the causal mask
+        // test exists only in the diagonal blocks' copy of the loop.
         int8_t* prow = pbase + (j & 1) * (BM * BKV);
         float rsp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         auto pass2 = [&](auto masked) {
-          uint32_t a0[16], a1[16], b0[16], b1[16];
-          tmem_ld16(sa, a0);
-          tmem_ld16(sa + 16, a1);
-          tmem_ld_wait_regs(a0, a1);
-          tmem_ld16(sa + 32, b0);
-          tmem_ld16(sa + 48, b1);
           auto conv = [&](const uint32_t (&x0)[16], const uint32_t (&x1)[16], int h) {
             uint32_t pk[8];
 #pragma unroll
@@ -421,7 +415,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_uint4(pk[4], pk[5], pk[6], pk[7]);
           };
           conv(a0, a1, 0);
-          tmem_ld_wait_regs(b0, b1);
           conv(b0, b1, 1);
         };
         if (diag)
