@@ -581,8 +581,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sm.dvdk_free);
         ++dvdk_cnt;
       }
-      // step 4: dQ, added to the float32 accumulator with atomics; afterwards the S region of
-      // this buffer is re-preloaded for tile it+2
+      // step 4: dQ, added to the float32 accumulator; afterwards the S region of this buffer is
+      // re-preloaded for tile it+2.  The dS scales of both key halves for this thread's dQ rows
+      // are formed while the dQ MMAs run.
+      const int gq = D == 128 ? (64 * h) / args.q_block : g_row;
+      const float s0 = scale22(__fdiv_rn(tile_max(sm.red_ds[b], gq, 0), 127.0f) * sk0 * args.tau);
+      const float s1 = scale22(__fdiv_rn(tile_max(sm.red_ds[b], gq, 1), 127.0f) * sk1 * args.tau);
+      const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
       mbar_wait(&sm.dq_full, it & 1, 212);
       tc_fence_after();
       if constexpr (D == 128) {
@@ -591,10 +596,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // buffers (double-buffered) and its lane 0 hands them to the TMA unit, which adds them
         // to the global accumulator; no warp waits for another.  The TMEM loads of round rr+1
         // are in flight while round rr is staged.
-        const int g = (64 * h) / args.q_block;
-        const float s0 = scale22(__fdiv_rn(tile_max(sm.red_ds[b], g, 0), 127.0f) * sk0 * args.tau);
-        const float s1 = scale22(__fdiv_rn(tile_max(sm.red_ds[b], g, 1), 127.0f) * sk1 * args.tau);
-        const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
         uint32_t a0[16], a1[16];
         tmem_ld16(lane_base + 64 * h, a0);
         tmem_ld16(lane_base + 128 + 64 * h, a1);
@@ -629,11 +630,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st_wait();
       } else {
         // thread = query row r, d columns of warpgroup h
-        const float s0 =
-            scale22(__fdiv_rn(tile_max(sm.red_ds[b], g_row, 0), 127.0f) * sk0 * args.tau);
-        const float s1 =
-            scale22(__fdiv_rn(tile_max(sm.red_ds[b], g_row, 1), 127.0f) * sk1 * args.tau);
-        const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
         float* dst = args.dq_acc + grow * D + h * kHalfD;
 #pragma unroll 1
         for (int c0 = 0; c0 < kHalfD; c0 += 16) {
