@@ -434,29 +434,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       return g == 0 ? fmaxf(v.x, v.y) : fmaxf(v.z, v.w);
     };
 
-    float c_n, lse2_n, dvr_n;
+    // pass B's code multipliers of tile `it` (its own row group and key half) from the tile
+    // maxima, once every warp has arrived.  Code multipliers use the fast divide (within 2 ulp;
+    // codes are not compared bit for bit); the read-outs' scales are IEEE quotients.  One
+    // barrier per tile parity, so arrivals for tiles it and it+1 never share a phase; a warp
+    // cannot arrive for tile it+2 before every thread released tile it's dQ.
+    auto multipliers = [&](int it, float& ip, float& ids, float& sdsc) {
+      const int b = it & 1;
+      mbar_wait(&sm.red_full[b], (it >> 1) & 1, 213);
+      const float tp = tile_max(sm.red_p[b], g_row, h);
+      const float tds = tile_max(sm.red_ds[b], g_row, h);
+      ip = tp > 0.0f ? __fdividef(127.0f, tp) : 0.0f;
+      ids = tds > 0.0f ? __fdividef(127.0f, tds) : 0.0f;
+      sdsc = QS ? __fdiv_rn(tds, 127.0f) : 0.0f;  // Q-smoothing column sums: this group's scale
+    };
+
+    float c_n, lse2_n, dvr_n, ip, ids, sdsc;
     row_inputs(0, c_n, lse2_n, dvr_n);
     pass_a(0, c_n, lse2_n, dvr_n);
+    multipliers(0, ip, ids, sdsc);
     for (int it = 0; it < nq; ++it) {
       const int b = it & 1;
       const uint32_t lane_base = tmem + lane_off + b * 256;
       const int qt = i_first + it;
       const size_t grow = static_cast<size_t>(row_base) + qt * BQ + r;
       if (it + 1 < nq) row_inputs(it + 1, c_n, lse2_n, dvr_n);  // loads in flight during pass B
-      // this tile's maxima (every warp arrived during pass A, a whole phase ago).  One barrier
-      // per tile parity, so arrivals for tiles it and it+1 never share a phase; a warp cannot
-      // arrive for tile it+2 before every thread released tile it's dQ.
-      mbar_wait(&sm.red_full[b], (it >> 1) & 1, 213);
-      float ip, ids, sdsc = 0.0f;
-      {
-        const float tp = tile_max(sm.red_p[b], g_row, h);
-        const float tds = tile_max(sm.red_ds[b], g_row, h);
-        // code multipliers: the codes are not compared bit for bit, so the fast divide
-        // (within 2 ulp) serves; the scales the read-outs use are IEEE quotients
-        ip = tp > 0.0f ? __fdividef(127.0f, tp) : 0.0f;
-        ids = tds > 0.0f ? __fdividef(127.0f, tds) : 0.0f;
-        if constexpr (QS) sdsc = __fdiv_rn(tds, 127.0f);  // this row group's dS scale
-      }
       // pass B: INT8 codes into shared memory; the dV_t / dK_t regions re-preloaded.  The TMEM
       // loads of chunk ch+1 are in flight while chunk ch is converted.
       auto proc_b = [&](uint32_t (&sa)[16], uint32_t (&pa)[16], int ch) {
@@ -588,6 +590,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float s0 = scale22(__fdiv_rn(tile_max(sm.red_ds[b], gq, 0), 127.0f) * sk0 * args.tau);
       const float s1 = scale22(__fdiv_rn(tile_max(sm.red_ds[b], gq, 1), 127.0f) * sk1 * args.tau);
       const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
+      // and the next tile's code multipliers (its pass A is done in every warp by now)
+      float ip_n = 0.0f, ids_n = 0.0f, sdsc_n = 0.0f;
+      if (it + 1 < nq) multipliers(it + 1, ip_n, ids_n, sdsc_n);
       mbar_wait(&sm.dq_full, it & 1, 212);
       tc_fence_after();
       if constexpr (D == 128) {
@@ -659,6 +664,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&sm.dq_free);
+      ip = ip_n;
+      ids = ids_n;
+      sdsc = sdsc_n;
     }
     // epilogue: dv, dk from the register accumulators (thread = key row r, d half h)
     {
