@@ -98,19 +98,19 @@ __device__ __forceinline__ float rms_norm8(float (&x)[8], float eps, uint32_t ma
   return inv;
 }
 
-// code = clamp(rint(x / s), -127, 127) as a byte (two's complement), 0 when s == 0.
-__device__ __forceinline__ uint32_t quant_code(float x, float s) {
-  if (!(s > 0.0f)) return 0u;
-  int c = __float2int_rn(__fdiv_rn(x, s));
-  c = max(-127, min(127, c));
-  return static_cast<uint32_t>(c) & 0xFFu;
+// code = rint(x / s) (round half to even) as a byte (two's complement), 0 when s == 0.
+// |x| <= absmax and s = RN(absmax / 127) keep |x / s| below 127.5, so no clamp is needed and
+// rint is taken by adding 1.5 * 2^23 (the sum rounds the quotient to the nearest integer, ties
+// to even, into the low mantissa bits), which keeps the conversion off the MUFU/XU pipe.
+__device__ __forceinline__ float quant_magic(float x, float s) {
+  return s > 0.0f ? __fadd_rn(__fdiv_rn(x, s), kMagic) : kMagic;
 }
 
 __device__ __forceinline__ uint2 quant8(const float (&x)[8], float s) {
-  return make_uint2(pack4(quant_code(x[0], s), quant_code(x[1], s), quant_code(x[2], s),
-                          quant_code(x[3], s)),
-                    pack4(quant_code(x[4], s), quant_code(x[5], s), quant_code(x[6], s),
-                          quant_code(x[7], s)));
+  return make_uint2(pack_magic4(quant_magic(x[0], s), quant_magic(x[1], s),
+                                quant_magic(x[2], s), quant_magic(x[3], s)),
+                    pack_magic4(quant_magic(x[4], s), quant_magic(x[5], s),
+                                quant_magic(x[6], s), quant_magic(x[7], s)));
 }
 
 // ---------------------------------------------------------------------------------------------
