@@ -191,7 +191,7 @@ struct PrologueArgs {
 // Prologue pass 3: one CTA per 128-token chunk of q, k or v (grid = 3 * BH * N/128):
 // RMSNorm (q, k), mean subtraction (k), block absmax and quantization.
 template <typename T, int D>
-__global__ void __launch_bounds__(kRowThreads) prologue_quant_kernel(PrologueArgs a) {
+__global__ void __launch_bounds__(kRowThreads, 3) prologue_quant_kernel(PrologueArgs a) {
   constexpr int LPR = D / 8, GPW = 32 / LPR, STEPS = 16 / GPW;
   __shared__ float red[8];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kRowThreads) prologue_quant_kernel(PrologueArg
 // float32 dQ accumulator rows cleared.  One CTA per 128 rows.
 // ---------------------------------------------------------------------------------------------
 template <typename T, int D>
-__global__ void __launch_bounds__(kRowThreads) bwd_preprocess_kernel(
+__global__ void __launch_bounds__(kRowThreads, 3) bwd_preprocess_kernel(
     const T* __restrict__ o, const T* __restrict__ dout, float* __restrict__ Dvec,
     int8_t* __restrict__ do_codes, float* __restrict__ do_scale, float* __restrict__ dq_acc,
     int N, int q_block) {
