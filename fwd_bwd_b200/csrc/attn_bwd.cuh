@@ -6,17 +6,18 @@
 //   1. S = Qc Kc^T (kind::i8) and dP = dO V^T (kind::f16 on the raw 16-bit dO and V, float32
 //      accumulation -- the one matmul the page keeps in 16-bit float) into TMEM;
 //   2. P = exp(z - LSE), dS = P (dP - D) (pass A, each thread one query row of 64 keys; values
-//      stored back to TMEM), per-tile absmax of P and dS over q_block x 64 tiles (named
-//      barriers per warpgroup), then INT8 codes written to shared memory (pass B) in the
-//      128-byte swizzled layout, which the tensor core reads K-major (for dQ) and MN-major
-//      (for dV, dK);
+//      stored back to TMEM), per-warp absmax of P and dS handed to the readers through shared
+//      memory and a per-parity mbarrier (each reader forms the q_block x 64 tile maxima it
+//      needs), then INT8 codes written to shared memory (pass B) in the 128-byte swizzled
+//      layout, which the tensor core reads K-major (for dQ) and MN-major (for dV, dK);
 //   3. dV_t = Pc^T dOc and dK_t = dSc^T Qc (kind::i8, M = 128 keys, one per q_block group),
 //      dequantized by the tile scales and added to float32 accumulators in registers;
 //      every INT32 accumulator region is preloaded with the bits of 1.5 * 2^23 so the results
 //      read back as floats that one exact FMA dequantizes (see kMagicBits);
-//   4. dQ_t = dSc Kc per 64-key block (kind::i8; computed transposed for d = 128 so each
-//      warp's atomics cover contiguous channels of one row), dequantized, summed and added to a
-//      float32 dQ accumulator in global memory with atomics.
+//   4. dQ_t = dSc Kc per 64-key block (kind::i8), dequantized, summed and added to a float32
+//      dQ accumulator in global memory: for d = 128 computed transposed (TMEM lanes = head-dim
+//      channels), staged per warp in shared memory and added by the TMA unit
+//      (cp.reduce.async.bulk); for d = 64 with vector atomics.
 // S and dP are double-buffered in TMEM, so the tensor core computes them for query tile i+1
 // while the compute warps turn tile i into codes.
 //
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // dQ_t per 64-key block.  d = 128: dQ_t^T = Kc[block]^T dSc[:, block]^T (M = d,
         // N = 128 queries; A = K codes read MN-major, B = dS codes K-major), so TMEM lanes are
-        // head-dim channels and the read-out's atomics cover contiguous channels of one row.
+        // head-dim channels and each warp's read-out holds 32 contiguous channels of a row.
         // d = 64: dQ_t = dSc[:, block] Kc[block] (M = 128 queries, N = d).
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
