@@ -89,7 +89,10 @@ struct Smem {
   alignas(16) float red_ds[2][8];  // and of |dS|
   float dot[BKT];                   // RMSNorm-backward row dot products (warpgroup 1 -> 0)
   float kb[BKT];                    // Q-smoothing: k_bias of the CTA's keys
-  float cs[BKT];                    // Q-smoothing: sum over tiles of sdS * (column sum of dSc)
+  // Q-smoothing: per compute warp, the sum over tiles of sdS * (column sum of dSc over the
+  // warp's rows) for the 64 keys of its warpgroup; one writer per element, so the totals do
+  // not depend on timing
+  float cs[8][64];
   uint64_t kv_full, q_full[2], q_empty[2], dor_full, dor_free;
   uint64_t sdp_full[2], pds_ready, dvdk_full, dvdk_free, dq_full, dq_free;
   uint64_t red_full[2];  // tile parity: every warp's tile maxima are in red_p / red_ds
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (QS) {
     for (int i = threadIdx.x; i < BKT; i += kThreads) {
       sm.kb[i] = args.k_bias[static_cast<size_t>(bh) * N + t * BKT + i];
-      sm.cs[i] = 0.0f;
+      for (int w = 0; w < 8; w += 2) sm.cs[w + (i >> 6)][i & 63] = 0.0f;
     }
   }
   __syncthreads();
@@ -489,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int cs = __reduce_add_sync(0xFFFFFFFFu, v);
             if (lane == e) mine = static_cast<float>(cs);
           }
-          if (lane < 16) atomicAdd(&sm.cs[col + lane], mine * sdsc);
+          if (lane < 16) sm.cs[warp][ch * 16 + lane] += mine * sdsc;
         }
         if (col < D) {  // dV_t occupies columns [0, D), dK_t [128, 128 + D)
           tmem_fill16(lane_base + col, kMagicBits);
@@ -677,7 +680,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (QS) {
         // dK_bias = tau * (dS^T 1)_r * mu_Q, the gradient through the score bias
         named_barrier_sync(4, 256);  // every warp's column-sum additions are in
-        const float csr = sm.cs[r] * args.tau;
+        const int kh = r >> 6;
+        const float csr = (((sm.cs[kh * 4][r & 63] + sm.cs[kh * 4 + 1][r & 63]) +
+                             sm.cs[kh * 4 + 2][r & 63]) + sm.cs[kh * 4 + 3][r & 63]) * args.tau;
         const float4* mq =
             reinterpret_cast<const float4*>(args.q_mean + static_cast<size_t>(bh) * D + h * kHalfD);
 #pragma unroll

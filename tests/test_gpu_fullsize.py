@@ -23,6 +23,7 @@ CASES = {
     "llama325m": [0, 127],      # B8 H16 N2048 d64 causal
     "long16k": [31],            # B1 H32 N16384 d128 causal, dO sigma 1e-4
     "koutlier": [5],            # B4 H16 N4096 d128 causal, K outliers
+    "qoutlier": [7],            # the same shape with Q outliers and Q-smoothing
 }
 
 
@@ -49,7 +50,7 @@ def test_full_size_sampled_heads(name):
     assert ops.device_status() == 0
     args = [x[n + "_f32"] for n in ("q", "k", "v", "do")]
     kw = dict(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth, q_block=w.q_block,
-              k_block=w.k_block, dtype=w.dtype)
+              k_block=w.k_block, dtype=w.dtype, qsmooth=w.qsmooth)
     ref = O.sage_attention(*args, **kw)
     full = O.sage_attention(*args, quant=False, round_outputs=False, **kw)
     flat = lambda a: a.reshape(w.B * w.H, *a.shape[2:])  # noqa: E731

@@ -13,7 +13,7 @@ from gpu_helpers import TORCH_DT, cfg_of
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name,chunks", [("llama325m", 3), ("sweep8192", 2)])
+@pytest.mark.parametrize("name,chunks", [("llama325m", 3), ("sweep8192", 2), ("qoutlier", 2)])
 def test_host_pipeline_matches_device_path(name, chunks):
     w = WORKLOADS[name].replace(B=5, H=2, N=512)
     x = make_inputs(w)
