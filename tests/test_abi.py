@@ -51,6 +51,11 @@ def test_workspace_sizes(L):
     p0 = _params(ksmooth=0)
     assert L.sage_workspace_bytes(ctypes.byref(p0), 0) == 0
     assert L.sage_workspace_bytes(ctypes.byref(_params(d=96)), 2) == 0
+    # Q-smoothing adds Q's column-sum partials beside K's
+    pq = _params(qsmooth=1)
+    assert L.sage_workspace_bytes(ctypes.byref(pq), 0) == 2 * BH * (N // 64) * d * 4
+    pq0 = _params(ksmooth=0, qsmooth=1)
+    assert L.sage_workspace_bytes(ctypes.byref(pq0), 0) == BH * (N // 64) * d * 4
 
 
 def test_status_strings(L):
@@ -89,6 +94,22 @@ def test_null_and_misaligned_pointers_rejected(L):
                                  None) == _lib.SAGE_ERR_WORKSPACE
     assert L.sage_attn_bwd(ctypes.byref(p), 16, 16, 16, ctypes.byref(qb), 16, 16, 16, 16, 16,
                            16, 16, 1, None) == _lib.SAGE_ERR_WORKSPACE
+
+
+def test_qsmooth_arguments_checked(L):
+    qb = SageQBufs(*([16] * 11))
+    assert L.sage_attn_fwd(ctypes.byref(_params(qsmooth=2)), ctypes.byref(qb), 16, 16, None, 0,
+                           None) == _lib.SAGE_ERR_INVALID_ARG
+    p = _params(qsmooth=1)
+    no_bias = SageQBufs(*([16] * 10 + [None]))  # Q-smoothing needs k_bias
+    assert L.sage_attn_fwd(ctypes.byref(p), ctypes.byref(no_bias), 16, 16, None, 0,
+                           None) == _lib.SAGE_ERR_INVALID_ARG
+    no_mean = SageQBufs(*([16] * 9 + [None, 16]))  # and q_mean
+    assert L.sage_quant_prologue(ctypes.byref(p), 16, 16, 16, ctypes.byref(no_mean), 16,
+                                 1 << 40, None) == _lib.SAGE_ERR_INVALID_ARG
+    odd = SageQBufs(*([16] * 10 + [20]))  # misaligned k_bias
+    assert L.sage_attn_fwd(ctypes.byref(p), ctypes.byref(odd), 16, 16, None, 0,
+                           None) == _lib.SAGE_ERR_ALIGNMENT
 
 
 def test_debug_entry_validation(L):
