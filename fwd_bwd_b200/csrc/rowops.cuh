@@ -31,6 +31,7 @@ namespace sage {
 
 constexpr int kRowThreads = 256;  // 8 warps; a CTA handles 128 rows (16 per warp)
 constexpr int kRowsPerCta = 128;
+constexpr int kQuantThreads = 512;  // prologue quantization: 16 warps, 8 rows each
 
 template <typename T>
 struct Cvt;
@@ -176,6 +177,25 @@ __device__ __forceinline__ float block_absmax(float local, int blk, float* red) 
   return a;
 }
 
+// The same over NW warps (rows 0-63 in the first half of the warps, 64-127 in the second).
+template <int NW>
+__device__ __forceinline__ float block_absmax_n(float local, int blk, float* red) {
+  const int warp = threadIdx.x >> 5;
+  const float wm = warp_max(local);
+  if ((threadIdx.x & 31) == 0) red[warp] = wm;
+  __syncthreads();
+  float a = 0.0f;
+  if (blk == 128) {
+#pragma unroll
+    for (int w = 0; w < NW; ++w) a = fmaxf(a, red[w]);
+  } else {
+    const int w0 = (warp / (NW / 2)) * (NW / 2);
+#pragma unroll
+    for (int w = 0; w < NW / 2; ++w) a = fmaxf(a, red[w0 + w]);
+  }
+  return a;
+}
+
 struct PrologueArgs {
   const void* src[3];      // q, k, v
   int8_t* codes[3];        // q, k, v codes
@@ -191,9 +211,10 @@ struct PrologueArgs {
 // Prologue pass 3: one CTA per 128-token chunk of q, k or v (grid = 3 * BH * N/128):
 // RMSNorm (q, k), mean subtraction (k), block absmax and quantization.
 template <typename T, int D>
-__global__ void __launch_bounds__(kRowThreads, 3) prologue_quant_kernel(PrologueArgs a) {
-  constexpr int LPR = D / 8, GPW = 32 / LPR, STEPS = 16 / GPW;
-  __shared__ float red[8];
+__global__ void __launch_bounds__(kQuantThreads, 2) prologue_quant_kernel(PrologueArgs a) {
+  constexpr int NW = kQuantThreads / 32, RPW = kRowsPerCta / NW;  // warps, rows per warp
+  constexpr int LPR = D / 8, GPW = 32 / LPR, STEPS = RPW / GPW;
+  __shared__ float red[NW];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = lane / LPR, sub = lane % LPR;
   const uint32_t mask = ((LPR == 32) ? 0xFFFFFFFFu : ((1u << LPR) - 1u)) << (grp * LPR);
@@ -208,7 +229,7 @@ __global__ void __launch_bounds__(kRowThreads, 3) prologue_quant_kernel(Prologue
   float x[STEPS][8];
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
-    const int r = warp * 16 + s * GPW + grp;
+    const int r = warp * RPW + s * GPW + grp;
     const uint4 u =
         __ldg(reinterpret_cast<const uint4*>(src + (row0 + r) * D + sub * 8));
     Cvt<T>::load8(u, x[s]);
@@ -217,7 +238,7 @@ __global__ void __launch_bounds__(kRowThreads, 3) prologue_quant_kernel(Prologue
 #pragma unroll
     for (int s = 0; s < STEPS; ++s) {
       const float inv = rms_norm8<D>(x[s], a.eps, mask);
-      const int r = warp * 16 + s * GPW + grp;
+      const int r = warp * RPW + s * GPW + grp;
       if (sub == 0) a.inv_rms[which][row0 + r] = inv;
     }
   }
@@ -245,7 +266,7 @@ __global__ void __launch_bounds__(kRowThreads, 3) prologue_quant_kernel(Prologue
 #pragma unroll
       for (int c = 0; c < 8; ++c) p = __fadd_rn(p, __fmul_rn(m[c], x[s][c]));
       const float b = row_sum<D / 8>(p, mask);
-      const int r = warp * 16 + s * GPW + grp;
+      const int r = warp * RPW + s * GPW + grp;
       if (sub == 0) a.k_bias[row0 + r] = b;
     }
   }
@@ -255,10 +276,10 @@ __global__ void __launch_bounds__(kRowThreads, 3) prologue_quant_kernel(Prologue
 #pragma unroll
     for (int c = 0; c < 8; ++c) amax = fmaxf(amax, fabsf(x[s][c]));
   const int blk = (which == 0) ? a.q_block : 64;
-  const float am = block_absmax(amax, blk, red);
+  const float am = block_absmax_n<NW>(amax, blk, red);
   const float sc = __fdiv_rn(am, 127.0f);
-  if (threadIdx.x == 0 || (blk == 64 && threadIdx.x == 128)) {
-    const int sub_blk = (blk == 64) ? (threadIdx.x >> 7) : 0;
+  if (threadIdx.x == 0 || (blk == 64 && threadIdx.x == kQuantThreads / 2)) {
+    const int sub_blk = (blk == 64 && threadIdx.x != 0) ? 1 : 0;
     const size_t idx = static_cast<size_t>(bh) * (a.N / blk) +
                        static_cast<size_t>(ch) * (kRowsPerCta / blk) + sub_blk;
     a.scale[which][idx] = sc;
@@ -266,7 +287,7 @@ __global__ void __launch_bounds__(kRowThreads, 3) prologue_quant_kernel(Prologue
   int8_t* dst = a.codes[which];
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
-    const int r = warp * 16 + s * GPW + grp;
+    const int r = warp * RPW + s * GPW + grp;
     *reinterpret_cast<uint2*>(dst + (row0 + r) * D + sub * 8) = quant8(x[s], sc);
   }
 }

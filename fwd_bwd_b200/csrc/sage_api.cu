@@ -183,7 +183,8 @@ int run_prologue(const sage_params* p, const void* q, const void* k, const void*
   a.ksmooth = p->ksmooth;
   a.qsmooth = p->qsmooth;
   a.eps = p->rms_eps;
-  sage::prologue_quant_kernel<T, D><<<3 * BH * (N / kRowsPerCta), kRowThreads, 0, st>>>(a);
+  sage::prologue_quant_kernel<T, D>
+      <<<3 * BH * (N / kRowsPerCta), sage::kQuantThreads, 0, st>>>(a);
   return launch_status();
 }
 
