@@ -294,15 +294,16 @@ __global__ void __launch_bounds__(kQuantThreads, 2) prologue_quant_kernel(Prolog
 
 // ---------------------------------------------------------------------------------------------
 // Backward preprocess: D_i = sum_c dO_ic O_ic (float32), dO codes per q_block tokens, and the
-// float32 dQ accumulator rows cleared.  One CTA per 128 rows.
+// float32 dQ accumulator rows cleared.  One CTA (kQuantThreads threads) per 128 rows.
 // ---------------------------------------------------------------------------------------------
 template <typename T, int D>
-__global__ void __launch_bounds__(kRowThreads, 3) bwd_preprocess_kernel(
+__global__ void __launch_bounds__(kQuantThreads, 2) bwd_preprocess_kernel(
     const T* __restrict__ o, const T* __restrict__ dout, float* __restrict__ Dvec,
     int8_t* __restrict__ do_codes, float* __restrict__ do_scale, float* __restrict__ dq_acc,
     int N, int q_block) {
-  constexpr int LPR = D / 8, GPW = 32 / LPR, STEPS = 16 / GPW;
-  __shared__ float red[8];
+  constexpr int NW = kQuantThreads / 32, RPW = kRowsPerCta / NW;  // warps, rows per warp
+  constexpr int LPR = D / 8, GPW = 32 / LPR, STEPS = RPW / GPW;
+  __shared__ float red[NW];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int grp = lane / LPR, sub = lane % LPR;
   const uint32_t mask = ((LPR == 32) ? 0xFFFFFFFFu : ((1u << LPR) - 1u)) << (grp * LPR);
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(kRowThreads, 3) bwd_preprocess_kernel(
   float amax = 0.0f;
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
-    const int r = warp * 16 + s * GPW + grp;
+    const int r = warp * RPW + s * GPW + grp;
     const size_t off = (row0 + r) * D + sub * 8;
     float y[8];
     Cvt<T>::load8(__ldg(reinterpret_cast<const uint4*>(dout + off)), x[s]);
@@ -328,13 +329,13 @@ __global__ void __launch_bounds__(kRowThreads, 3) bwd_preprocess_kernel(
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  const float am = block_absmax(amax, q_block, red);
+  const float am = block_absmax_n<NW>(amax, q_block, red);
   const float sc = __fdiv_rn(am, 127.0f);
-  if (threadIdx.x == 0 || (q_block == 64 && threadIdx.x == 128))
-    do_scale[(row0 + (threadIdx.x >> 7) * 64) / q_block] = sc;
+  if (threadIdx.x == 0 || (q_block == 64 && threadIdx.x == kQuantThreads / 2))
+    do_scale[(row0 + (threadIdx.x == 0 ? 0 : 64)) / q_block] = sc;
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
-    const int r = warp * 16 + s * GPW + grp;
+    const int r = warp * RPW + s * GPW + grp;
     *reinterpret_cast<uint2*>(do_codes + (row0 + r) * D + sub * 8) = quant8(x[s], sc);
   }
 }

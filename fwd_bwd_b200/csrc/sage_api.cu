@@ -238,7 +238,7 @@ int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const
   float* dqacc = reinterpret_cast<float*>(wsb + w.dq);
   if (stage == 0) {
     sage::bwd_preprocess_kernel<T, D>
-        <<<static_cast<int>(rows / kRowsPerCta), kRowThreads, 0, st>>>(
+        <<<static_cast<int>(rows / kRowsPerCta), sage::kQuantThreads, 0, st>>>(
             reinterpret_cast<const T*>(o), reinterpret_cast<const T*>(dout), dvec, doc, dos,
             dqacc, N, p->q_block);
     return launch_status();
