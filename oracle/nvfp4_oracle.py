@@ -1,0 +1,193 @@
+"""CPU oracle for the NVFP4 Q-Attn variant -- TEST INFRASTRUCTURE, NOT PRODUCT CODE.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this module.  It shares no code with the CUDA path (``fwd_bwd_b200``).
+
+What it follows:
+
+* "Full-Stack FP4" (gist.science 2607.04422), section 2.4 "mixed-precision attention (Q-Attn)":
+  the robust paths, Q K^T and dS, run in NVFP4; the softmax-sensitive paths, P V, P^T dO and
+  dO V^T, stay in BF16; the quantized views of Q, K and V are produced once and reused by the
+  forward and the backward pass.
+* "Quartet II" (allinfo.ai.kr), plain-language section: the NVFP4 format is E2M1 values in
+  blocks of 16 that share one E4M3 (FP8) scale, plus one global scale.
+
+Readings (the pages fix neither rounding rules nor the global scale's extent):
+
+* E2M1 magnitudes are {0, 0.5, 1, 1.5, 2, 3, 4, 6}; rounding is to nearest, ties to the code
+  with an even low bit, and magnitudes above 6 saturate to 6.  A value that rounds to zero
+  gets the +0 code.  (``e2m1_encode``)
+* Block scales are unsigned E4M3 (4 exponent bits, bias 7, 3 mantissa bits, subnormals,
+  largest finite 448): round to nearest, ties to even, values of 448 and above saturate to 448.
+  (``e4m3_encode``)
+* The global scale covers one (batch, head) matrix -- the operand of one attention GEMM -- and
+  maps that matrix's absolute maximum G onto 6 * 448 = 2688, the largest value a block scale
+  times an element can reach: ``genc = 2688 / G`` (``genc = 1`` when G = 0).
+* Per block of 16 consecutive channels, in float32 with IEEE rounding at every step:
+  ``a = max |x|``, ``u = (a * genc) / 6``, ``sd = e4m3(u)`` (the stored scale),
+  ``mult = genc / sd`` and ``code = e2m1(x * mult)``; ``sd = 0`` gives all-zero codes.
+  The value a code stands for is ``e2m1_value(code) * sd / genc``.
+* Q and K are quantized along the head dimension (the contraction of Q K^T), after the same
+  QK-norm and K-smoothing as the INT8 recipe (``sage_oracle.rms_norm_rows_f32``,
+  ``sage_oracle.k_smooth_f32``).  V is not quantized (P V runs in BF16).
+* Forward: scores from the dequantized operands (exact in float64), softmax and
+  ``O = softmax(z) V`` in float64.  The kernel feeds P to the tensor core in BF16; the oracle
+  keeps P exact, and the tests bound the difference that BF16 rounding of P can make.
+"""
+from __future__ import annotations
+
+from typing import Dict
+
+import numpy as np
+
+from . import sage_oracle as S8
+
+F32 = np.float32
+F64 = np.float64
+
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=F64)
+GLOBAL_RANGE = 2688.0  # 6 (largest E2M1 value) * 448 (largest E4M3 value)
+NVFP4_BLOCK = 16
+
+
+def e2m1_encode(y: np.ndarray) -> np.ndarray:
+    """4-bit E2M1 codes (bit 3 = sign) of float32 values: nearest, ties to even, saturating.
+
+    The magnitude code counts the rounding boundaries ``|y|`` has passed.  Between two
+    neighbours the midpoint goes to the one whose code is even: 0.25 -> 0, 0.75 -> 1,
+    1.25 -> 1, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4 (codes 0, 2, 2, 4, 4, 6, 6).
+    """
+    a = np.abs(np.asarray(y, dtype=F32))
+    mag = ((a > 0.25).astype(np.uint8) + (a >= 0.75) + (a > 1.25) + (a >= 1.75) + (a > 2.5)
+           + (a >= 3.5) + (a > 5.0)).astype(np.uint8)
+    neg = (np.asarray(y, dtype=F32) < 0) & (mag > 0)
+    return (mag | (neg.astype(np.uint8) << 3)).astype(np.uint8)
+
+
+def e2m1_decode(code: np.ndarray) -> np.ndarray:
+    code = np.asarray(code, dtype=np.uint8)
+    v = E2M1_VALUES[code & 7]
+    return np.where(code & 8, -v, v)
+
+
+def e4m3_decode(code: np.ndarray) -> np.ndarray:
+    """Value of an unsigned E4M3 byte (bias 7; exponent field 0 is subnormal, m * 2^-9)."""
+    code = np.asarray(code, dtype=np.int64)
+    e = (code >> 3) & 15
+    m = code & 7
+    return np.where(e == 0, m * 2.0 ** -9, (8 + m) * np.exp2(e - 10.0)).astype(F64)
+
+
+def e4m3_encode(u: np.ndarray) -> np.ndarray:
+    """Unsigned E4M3 code of non-negative float32 ``u``: nearest, ties to even, saturating.
+
+    Below 2^-6 the grid is ``m * 2^-9`` (m = 0..8; m = 8 is the smallest normal, whose code
+    is 8 too).  From 2^-6 on, with ``u = f * 2^e`` (1 <= f < 2), ``q = rne(8 f)`` in 8..16
+    (16 carries into the exponent) and the code is ``(e + 7) << 3 | (q - 8)``.  448 and above
+    give 448 (code 0x7E).  Scaling by powers of two is exact, so only ``rne`` rounds.
+    """
+    u = np.asarray(u, dtype=F32).astype(F64)
+    sub = u < 2.0 ** -6
+    q_sub = np.rint(u * 512.0)
+    _, ex = np.frexp(np.where(sub, 1.0, u))  # u = f' 2^ex with f' in [0.5, 1)
+    e = ex - 1
+    q = np.rint(np.where(sub, 8.0, u) * np.exp2(3.0 - e))
+    carry = q == 16
+    e = np.where(carry, e + 1, e)
+    q = np.where(carry, 8, q)
+    normal = ((e + 7) << 3) | (q.astype(np.int64) - 8)
+    code = np.where(sub, q_sub.astype(np.int64), normal)
+    code = np.where(u >= 448.0, 0x7E, code)
+    return code.astype(np.uint8)
+
+
+def nvfp4_quantize(x: np.ndarray) -> Dict[str, np.ndarray]:
+    """NVFP4 quantization of ``x[..., N, d]`` along its last axis (blocks of 16 channels).
+
+    One global scale per matrix (the last two axes).  Returns ``codes`` (uint8 values 0..15,
+    one per element, ``x``'s shape), ``sf`` (E4M3 block-scale bytes, ``[..., N, d/16]``) and
+    ``genc`` (float32 global encode scale, ``x.shape[:-2]``).
+    """
+    x = np.asarray(x, dtype=F32)
+    *lead, N, d = x.shape
+    G = np.max(np.abs(x), axis=(-2, -1)).astype(F32)
+    genc = np.where(G > 0, F32(GLOBAL_RANGE) / np.where(G > 0, G, F32(1)), F32(1)).astype(F32)
+    xb = x.reshape(*lead, N, d // NVFP4_BLOCK, NVFP4_BLOCK)
+    a = np.max(np.abs(xb), axis=-1)
+    g = genc.reshape(*genc.shape, 1, 1)
+    u = ((a * g).astype(F32) / F32(6.0)).astype(F32)
+    sf = e4m3_encode(u)
+    sd = e4m3_decode(sf).astype(F32)
+    mult = np.where(sd > 0, (g / np.where(sd > 0, sd, F32(1))).astype(F32), F32(0)).astype(F32)
+    y = (xb * mult[..., None]).astype(F32)
+    codes = e2m1_encode(y).reshape(x.shape)
+    return {"codes": codes, "sf": sf, "genc": genc}
+
+
+def nvfp4_dequantize(codes: np.ndarray, sf: np.ndarray, genc: np.ndarray) -> np.ndarray:
+    """float64 values ``e2m1(code) * sd / genc`` of ``nvfp4_quantize``'s output."""
+    *lead, N, d = codes.shape
+    v = e2m1_decode(codes).reshape(*lead, N, d // NVFP4_BLOCK, NVFP4_BLOCK)
+    v = v * e4m3_decode(sf)[..., None]
+    return v.reshape(codes.shape) / np.asarray(genc, F64).reshape(*np.shape(genc), 1, 1)
+
+
+def qattn_prologue(q, k, *, qknorm: bool, ksmooth: bool, eps: float = 1e-6,
+                   k_block: int = 64) -> Dict[str, np.ndarray]:
+    """QK-norm and K-smoothing (float32, as in the INT8 recipe), then NVFP4 views of Q and K.
+
+    ``q``, ``k`` are float32 ``[BH, N, d]`` holding the exact 16-bit input values.
+    """
+    out: Dict[str, np.ndarray] = {}
+    qh, kh = np.asarray(q, F32), np.asarray(k, F32)
+    if qknorm:
+        qh, out["q_inv_rms"] = S8.rms_norm_rows_f32(qh, eps)
+        kh, out["k_inv_rms"] = S8.rms_norm_rows_f32(kh, eps)
+    if ksmooth:
+        kh, out["k_mean"] = S8.k_smooth_f32(kh, k_block)
+    out["q_hat"], out["k_tilde"] = qh, kh
+    for name, x in (("q", qh), ("k", kh)):
+        r = nvfp4_quantize(x)
+        out[name + "_codes"], out[name + "_sf"], out[name + "_genc"] = r["codes"], r["sf"], r["genc"]
+    return out
+
+
+def qattn_fwd_head(qd: np.ndarray, kd: np.ndarray, v: np.ndarray, *, causal: bool,
+                   tau: float) -> tuple:
+    """Forward of one head from dequantized Q, K (float64 ``[N, d]``) and V.
+
+    ``z = tau * qd kd^T`` (causal: key j visible to query i iff j <= i), ``m = max_j z``,
+    ``p = exp(z - m)``, ``l = sum_j p``, ``O = (p V) / l``, ``LSE = m + ln l``.
+    Returns ``(O, LSE)`` in float64.  Also returns ``W = (p |V|) / l`` per (row, channel), the
+    weight the tests use to bound the effect of rounding P to BF16.
+    """
+    qd, kd, v = (np.asarray(t, F64) for t in (qd, kd, v))
+    z = (qd @ kd.T) * tau
+    if causal:
+        N = z.shape[0]
+        z = np.where(np.arange(N)[None, :] > np.arange(N)[:, None], -np.inf, z)
+    m = z.max(axis=1)
+    p = np.exp(z - m[:, None])
+    l = p.sum(axis=1)
+    O = (p @ v) / l[:, None]
+    W = (p @ np.abs(v)) / l[:, None]
+    return O, m + np.log(l), W
+
+
+def qattn_forward(q, k, v, *, causal: bool, qknorm: bool, ksmooth: bool,
+                  tau: float | None = None, eps: float = 1e-6) -> Dict[str, np.ndarray]:
+    """Prologue plus forward over every (batch, head); inputs float32 ``[BH, N, d]``."""
+    q = np.asarray(q, F32)
+    d = q.shape[-1]
+    tau = 1.0 / np.sqrt(d) if tau is None else tau
+    pro = qattn_prologue(q, k, qknorm=qknorm, ksmooth=ksmooth, eps=eps)
+    qd = nvfp4_dequantize(pro["q_codes"], pro["q_sf"], pro["q_genc"])
+    kd = nvfp4_dequantize(pro["k_codes"], pro["k_sf"], pro["k_genc"])
+    BH, N, _ = q.shape
+    o = np.zeros((BH, N, d), F64)
+    lse = np.zeros((BH, N), F64)
+    w = np.zeros((BH, N, d), F64)
+    for h in range(BH):
+        o[h], lse[h], w[h] = qattn_fwd_head(qd[h], kd[h], v[h], causal=causal, tau=tau)
+    pro.update(o=o, lse=lse, w=w, q_deq=qd, k_deq=kd)
+    return pro

@@ -1,0 +1,285 @@
+"""Pins of the NVFP4 Q-Attn oracle against facts fixed outside it.
+
+* E2M1 / E4M3 decoding from the bit formats (sign, exponent bias, subnormals) and, for E4M3,
+  torch's own float8_e4m3fn conversion (a library routine);
+* rounding checked by brute force against the whole representable grid (nearest, ties to the
+  even code, saturation);
+* NVFP4 quantization: exact round trip of values planted on the grid, the per-element error
+  bound, exact invariance under power-of-two scaling, the global scale's placement;
+* the forward: torch's float64 scaled-dot-product attention and logsumexp on the same
+  dequantized operands, and the end-to-end wiring on inputs that quantize exactly.
+
+Planted mistakes (at the end) check that these pins catch plausible slips in the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.nvfp4_oracle as F
+
+# ------------------------------------------------------------------------------------------
+# E2M1
+# ------------------------------------------------------------------------------------------
+
+
+def _e2m1_from_bits(c):
+    """E2M1 from its bit fields: 1 sign, 2 exponent (bias 1), 1 mantissa bit."""
+    s, e, m = (c >> 3) & 1, (c >> 1) & 3, c & 1
+    mag = m * 0.5 if e == 0 else (1.0 + m / 2.0) * 2.0 ** (e - 1)
+    return -mag if s else mag
+
+
+def test_e2m1_decode_matches_bit_format():
+    for c in range(16):
+        assert F.e2m1_decode(np.array([c], np.uint8))[0] == _e2m1_from_bits(c)
+
+
+def _e2m1_brute(y):
+    """Nearest grid magnitude, ties to the even code, above 6 -> 6; sign kept unless zero."""
+    a = abs(float(y))
+    if a >= 6.0:
+        mag = 7
+    else:
+        d = np.abs(F.E2M1_VALUES - a)
+        best = np.flatnonzero(d == d.min())
+        mag = int(best[0]) if len(best) == 1 else int([b for b in best if b % 2 == 0][0])
+    return mag | (8 if (y < 0 and mag > 0) else 0)
+
+
+def test_e2m1_encode_brute_force():
+    ys = np.concatenate([np.arange(-8.0, 8.0, 1.0 / 64.0),
+                         [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -5.0, 1e30, -1e30,
+                          -0.0, 0.1, -0.1]]).astype(np.float32)
+    got = F.e2m1_encode(ys)
+    want = np.array([_e2m1_brute(y) for y in ys], np.uint8)
+    assert np.array_equal(got, want)
+
+
+def test_e2m1_ties_and_saturation():
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    assert F.e2m1_decode(F.e2m1_encode(ties)).tolist() == [0, 1, 1, 2, 2, 4, 4]
+    assert F.e2m1_encode(np.array([7.0, 100.0, -6.5], np.float32)).tolist() == [7, 7, 15]
+
+
+# ------------------------------------------------------------------------------------------
+# E4M3
+# ------------------------------------------------------------------------------------------
+def _e4m3_torch(codes):
+    t = torch.tensor(np.asarray(codes, np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def test_e4m3_decode_matches_torch():
+    codes = np.arange(0, 127, dtype=np.uint8)  # every non-negative finite code (0x7F is NaN)
+    assert np.array_equal(F.e4m3_decode(codes), _e4m3_torch(codes))
+    assert F.e4m3_decode(np.array([0x7E]))[0] == 448.0
+    assert F.e4m3_decode(np.array([0x01]))[0] == 2.0 ** -9
+    assert F.e4m3_decode(np.array([0x08]))[0] == 2.0 ** -6
+    assert F.e4m3_decode(np.array([0x38]))[0] == 1.0
+
+
+def test_e4m3_encode_grid_midpoints_and_torch():
+    codes = np.arange(0, 127, dtype=np.uint8)
+    vals = F.e4m3_decode(codes)
+    # every representable value maps to its own code
+    assert np.array_equal(F.e4m3_encode(vals.astype(np.float32)), codes)
+    # midpoints go to the neighbour with the even code
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    assert np.all(mids.astype(np.float64) == (vals[:-1] + vals[1:]) / 2)  # exact in float32
+    got = F.e4m3_encode(mids)
+    lo = codes[:-1]
+    want = np.where(lo % 2 == 0, lo, lo + 1)
+    assert np.array_equal(got, want)
+    # random values below 448: torch's round-to-nearest-even conversion
+    rng = np.random.default_rng(5)
+    u = np.concatenate([rng.uniform(0, 448, 20000), np.exp(rng.uniform(-14, 6, 20000)),
+                        rng.uniform(0, 2.0 ** -6, 5000)]).astype(np.float32)
+    u = u[u < 448]
+    t = torch.tensor(u).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(F.e4m3_encode(u), t)
+    # saturation
+    assert F.e4m3_encode(np.array([448.0, 460.0, 1e9], np.float32)).tolist() == [0x7E] * 3
+
+
+# ------------------------------------------------------------------------------------------
+# NVFP4 quantization
+# ------------------------------------------------------------------------------------------
+def _planted(seed, BH=2, N=64, d=128):
+    """Values exactly on the NVFP4 grid with a global maximum of 2688 (so genc = 1): every
+    block has a largest code of magnitude 6, so the block scale is recovered exactly."""
+    rng = np.random.default_rng(seed)
+    nb = d // 16
+    codes = rng.integers(0, 16, size=(BH, N, nb, 16)).astype(np.uint8)
+    pos = rng.integers(0, 16, size=(BH, N, nb))
+    sgn = rng.integers(0, 2, size=(BH, N, nb)).astype(np.uint8) << 3
+    np.put_along_axis(codes, pos[..., None], (7 | sgn)[..., None], axis=-1)
+    sf = rng.integers(1, 0x7F, size=(BH, N, nb)).astype(np.uint8)
+    sf[:, 0, 0] = 0x7E  # 448: the block holding the global maximum 6 * 448
+    x = F.e2m1_decode(codes) * F.e4m3_decode(sf)[..., None]
+    return x.reshape(BH, N, d).astype(np.float32), codes.reshape(BH, N, d), sf
+
+
+def test_nvfp4_planted_round_trip():
+    x, codes, sf = _planted(1)
+    assert np.all(np.abs(x).max(axis=(1, 2)) == 2688.0)
+    r = F.nvfp4_quantize(x)
+    assert np.all(r["genc"] == 1.0)
+    assert np.array_equal(r["sf"], sf)
+    # -0 codes (sign bit with magnitude 0) come back as +0
+    want = np.where((codes & 7) == 0, 0, codes)
+    assert np.array_equal(r["codes"], want)
+    assert np.array_equal(F.nvfp4_dequantize(r["codes"], r["sf"], r["genc"]), x)
+
+
+def test_nvfp4_error_bound_and_global_scale():
+    rng = np.random.default_rng(2)
+    x = (rng.standard_normal((3, 256, 128)) * np.exp(rng.uniform(-3, 3, (3, 1, 128)))).astype(np.float32)
+    r = F.nvfp4_quantize(x)
+    G = np.abs(x).max(axis=(1, 2))
+    assert np.array_equal(r["genc"], (np.float32(2688.0) / G.astype(np.float32)))
+    sd = F.e4m3_decode(r["sf"])
+    xd = F.nvfp4_dequantize(r["codes"], r["sf"], r["genc"])
+    err = np.abs(xd - x).reshape(3, 256, 8, 16).max(axis=-1)
+    # scaled values stay within 6 (1 + 2^-4) and the E2M1 grid spacing is at most 2, so the
+    # error is at most one scaled unit, sd / genc, wherever the block scale is a normal E4M3
+    normal = sd >= 2.0 ** -6
+    bound = sd / r["genc"][:, None, None].astype(np.float64) * (1 + 1e-6)
+    assert np.all(err[normal] <= bound[normal])
+    assert normal.mean() > 0.99
+    # the element holding the global maximum is coded +-6 with the largest scale
+    for h in range(3):
+        n, c = np.unravel_index(np.argmax(np.abs(x[h])), x[h].shape)
+        assert r["sf"][h, n, c // 16] == 0x7E and (r["codes"][h, n, c] & 7) == 7
+
+
+def test_nvfp4_power_of_two_invariance():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((2, 128, 64)).astype(np.float32)
+    r0 = F.nvfp4_quantize(x)
+    for k in (-7, -1, 3, 11):
+        r = F.nvfp4_quantize((x * np.float32(2.0 ** k)).astype(np.float32))
+        assert np.array_equal(r["codes"], r0["codes"]) and np.array_equal(r["sf"], r0["sf"])
+        assert np.array_equal(r["genc"], (r0["genc"] * np.float32(2.0 ** -k)).astype(np.float32))
+
+
+def test_nvfp4_zero_matrix():
+    r = F.nvfp4_quantize(np.zeros((1, 32, 64), np.float32))
+    assert np.all(r["genc"] == 1.0) and not r["sf"].any() and not r["codes"].any()
+
+
+# ------------------------------------------------------------------------------------------
+# Q-Attn forward
+# ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_qattn_fwd_head_vs_torch(causal):
+    rng = np.random.default_rng(4)
+    N, d = 96, 64
+    q, k, v = (rng.standard_normal((N, d)) for _ in range(3))
+    tau = 0.3
+    o, lse, w = F.qattn_fwd_head(q, k, v, causal=causal, tau=tau)
+    t = [torch.tensor(a)[None, None] for a in (q, k, v)]
+    ref = torch.nn.functional.scaled_dot_product_attention(*t, is_causal=causal, scale=tau)
+    assert np.allclose(o, ref[0, 0].numpy(), rtol=1e-12, atol=1e-12)
+    z = torch.tensor(q) @ torch.tensor(k).T * tau
+    if causal:
+        z = z.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+    assert np.allclose(lse, torch.logsumexp(z, dim=1).numpy(), rtol=1e-12, atol=1e-12)
+    assert np.all(w >= np.abs(o) - 1e-12)
+
+
+def test_qattn_forward_exact_inputs_equal_plain_attention():
+    """Without QK-norm and smoothing, inputs on the NVFP4 grid dequantize to themselves, so
+    the Q-Attn forward is plain attention of the inputs."""
+    x, _, _ = _planted(6, BH=2, N=64, d=64)
+    y, _, _ = _planted(7, BH=2, N=64, d=64)
+    q, k = x / np.float32(512.0), y / np.float32(256.0)  # powers of two keep them on the grid
+    v = np.random.default_rng(8).standard_normal((2, 64, 64)).astype(np.float32)
+    tau = 1.0 / 512.0
+    r = F.qattn_forward(q, k, v, causal=True, qknorm=False, ksmooth=False, tau=tau)
+    assert np.array_equal(r["q_deq"], q.astype(np.float64))
+    assert np.array_equal(r["k_deq"], k.astype(np.float64))
+    t = [torch.tensor(a.astype(np.float64)) for a in (q, k, v)]
+    ref = torch.nn.functional.scaled_dot_product_attention(*t, is_causal=True, scale=tau)
+    assert np.allclose(r["o"], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_qattn_forward_close_to_full_precision():
+    rng = np.random.default_rng(9)
+    BH, N, d = 2, 256, 128
+    q, k, v = (rng.standard_normal((BH, N, d)).astype(np.float32) for _ in range(3))
+    k += 3.0 * rng.standard_normal((BH, 1, d)).astype(np.float32)  # channel offsets on K
+    r = F.qattn_forward(q, k, v, causal=True, qknorm=True, ksmooth=True)
+    t = [torch.tensor(a.astype(np.float64)) for a in (r["q_hat"], r["k_tilde"], v)]
+    ref = torch.nn.functional.scaled_dot_product_attention(*t, is_causal=True).numpy()
+    cos = (r["o"] * ref).sum() / np.sqrt((r["o"] ** 2).sum() * (ref ** 2).sum())
+    assert cos > 0.99, cos
+
+
+# ------------------------------------------------------------------------------------------
+# planted mistakes are caught
+# ------------------------------------------------------------------------------------------
+def _fails(test, *args):
+    try:
+        test(*args)
+        return False
+    except AssertionError:
+        return True
+
+
+def test_planted_mistakes_are_caught(monkeypatch):
+    assert not _fails(test_e2m1_encode_brute_force)
+    real_e2m1 = F.e2m1_encode
+
+    def ties_up(y):  # ties away from zero instead of to even
+        a = np.abs(np.asarray(y, np.float32))
+        mag = ((a >= 0.25).astype(np.uint8) + (a >= 0.75) + (a >= 1.25) + (a >= 1.75)
+               + (a >= 2.5) + (a >= 3.5) + (a >= 5.0)).astype(np.uint8)
+        return (mag | (((np.asarray(y) < 0) & (mag > 0)).astype(np.uint8) << 3)).astype(np.uint8)
+
+    with monkeypatch.context() as m:
+        m.setattr(F, "e2m1_encode", ties_up)
+        assert _fails(test_e2m1_encode_brute_force)
+
+    real_e4m3 = F.e4m3_encode
+
+    def truncating(u):  # rounds toward zero
+        u = np.asarray(u, np.float32).astype(np.float64)
+        codes = np.arange(0, 127, dtype=np.uint8)
+        vals = F.e4m3_decode(codes)
+        idx = np.searchsorted(vals, u, side="right") - 1
+        return codes[np.clip(idx, 0, 126)]
+
+    with monkeypatch.context() as m:
+        m.setattr(F, "e4m3_encode", truncating)
+        assert _fails(test_e4m3_encode_grid_midpoints_and_torch)
+
+    real_q = F.nvfp4_quantize
+
+    def no_global(x):  # global scale left out of the block scale
+        r = real_q(x)
+        r2 = real_q(x / np.maximum(np.abs(x).max(axis=(-2, -1), keepdims=True), 1e-30) * 2688.0)
+        r2["genc"] = np.ones_like(r["genc"])
+        return r2
+
+    def sf_transposed(x):  # scale of block b taken from block (nb - 1 - b)
+        r = real_q(x)
+        r["sf"] = r["sf"][..., ::-1].copy()
+        return r
+
+    for fake, test in ((no_global, test_nvfp4_error_bound_and_global_scale),
+                       (no_global, test_nvfp4_power_of_two_invariance),
+                       (sf_transposed, test_nvfp4_planted_round_trip),
+                       (sf_transposed, test_nvfp4_error_bound_and_global_scale)):
+        with monkeypatch.context() as m:
+            m.setattr(F, "nvfp4_quantize", fake)
+            assert _fails(test), (fake.__name__, test.__name__)
+
+    real_head = F.qattn_fwd_head
+
+    def dropped_tau(qd, kd, v, *, causal, tau):
+        return real_head(qd, kd, v, causal=causal, tau=1.0)
+
+    with monkeypatch.context() as m:
+        m.setattr(F, "qattn_fwd_head", dropped_tau)
+        assert _fails(test_qattn_forward_exact_inputs_equal_plain_attention)
+    assert F.e2m1_encode is real_e2m1 and F.e4m3_encode is real_e4m3
