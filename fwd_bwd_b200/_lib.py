@@ -1,4 +1,4 @@
-"""ctypes view of libsage.so (the C ABI declared in include/sage.h).
+"""ctypes view of libsage.so (the C ABI declared in include/sage.h and include/sage_nvfp4.h).
 
 Loading fails loudly when the shared library is missing: there is no fallback path.
 """
@@ -36,6 +36,12 @@ class SageQBufs(ctypes.Structure):
                  "q_inv_rms", "k_inv_rms", "k_mean", "q_mean", "k_bias")]
 
 
+class SageFp4Bufs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q_fp4", "k_fp4", "q_sf", "k_sf", "q_genc", "k_genc", "q_inv_rms",
+                 "k_inv_rms", "k_mean")]
+
+
 class SageError(RuntimeError):
     def __init__(self, fn: str, status: int, text: str):
         super().__init__(f"{fn} failed: {text} ({status})")
@@ -69,6 +75,12 @@ def lib() -> ctypes.CDLL:
         L.sage_attn_bwd_stage.argtypes = [i, P(SageParams), vp, vp, vp, P(SageQBufs), vp, vp,
                                           vp, vp, vp, vp, vp, sz, vp]
         L.sage_attn_bwd_stage.restype = i
+        L.sage_fp4_workspace_bytes.argtypes = [P(SageParams), i]
+        L.sage_fp4_workspace_bytes.restype = sz
+        L.sage_fp4_quant_prologue.argtypes = [P(SageParams), vp, vp, P(SageFp4Bufs), vp, sz, vp]
+        L.sage_fp4_quant_prologue.restype = i
+        L.sage_fp4_attn_fwd.argtypes = [P(SageParams), P(SageFp4Bufs), vp, vp, vp, vp]
+        L.sage_fp4_attn_fwd.restype = i
         L.sage_last_device_status.argtypes = [vp]
         L.sage_last_device_status.restype = i
         L.sage_status_string.argtypes = [i]

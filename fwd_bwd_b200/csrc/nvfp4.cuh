@@ -1,0 +1,493 @@
+// nvfp4.cuh -- the NVFP4 Q-Attn variant on sm_100a ("Full-Stack FP4", gist.science
+// 2607.04422, section 2.4: Q K^T in NVFP4, P V in BF16; the quantized views of Q and K are made
+// once and reused).  NVFP4 format ("Quartet II", allinfo.ai.kr): E2M1 values in blocks of 16
+// sharing an E4M3 scale, plus one global scale.
+//
+// Prologue (two passes over q and k, after the INT8 path's QK-norm / K-smoothing):
+//   amax pass   per (tensor, batch-head) absolute maximum G of the normalized, smoothed values
+//               (atomicMax on the float bits: non-negative floats order like their bits, so
+//               the result does not depend on the order of the atomics);
+//   quant pass  genc = 2688 / G (1 when G = 0); per 16 channels: a = max|x|,
+//               u = (a * genc) / 6, sd = e4m3(u) (nearest, ties to even, saturating at 448),
+//               code = e2m1(x * (genc / sd)) (nearest, ties to even, saturating at 6; +0 for
+//               values that round to zero); every step a correctly rounded float32 operation.
+// Outputs: codes [BH, N, d/2] (channel 2i in the low nibble of byte i), block scales in the
+// tensor core's scale-factor order (per 128-row tile and 64-channel chunk, 512 bytes: byte
+// (r % 32) * 16 + (r / 32) * 4 + b holds row r's scale of the chunk's 16-channel block b), and
+// genc [BH].
+//
+// Forward: per CTA one tile of 128 query rows of one (batch, head), walking 128-key blocks.
+//   warp 0      TMA producer: Q codes and scales once, then K codes, K scales and V (16-bit)
+//               through a 3-stage ring;
+//   warp 1      MMA issuer (one thread): block scales copied to TMEM (tcgen05.cp), S_j = Q K_j^T
+//               (kind::mxf4nvf4, scale vector 16, FP32 in TMEM, double-buffered), then
+//               PV_{j-1} = P_{j-1} V_{j-1} (kind::f16 in V's type, FP32 in TMEM);
+//   warps 2-5   softmax, one query row per thread: z = S * tau / (genc_Q genc_K), causal mask,
+//               running max, p = exp2(z - m) written to shared memory in V's 16-bit type
+//               (K-major, 128-byte swizzle), running sum of the float32 p, and the fold
+//               O <- alpha O + PV in registers.
+// TMEM (512 columns): S buffers at 0 and 128, PV at 256, Q scales at 384, K scales at 392 and
+// 400 (one set per S buffer).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <type_traits>
+
+#include "ptx.cuh"
+#include "rowops.cuh"
+
+namespace sage {
+namespace fp4 {
+
+// ---------------------------------------------------------------------------------------------
+// Number formats
+// ---------------------------------------------------------------------------------------------
+// Unsigned E4M3 code of u >= 0: nearest, ties to even, 448 and above -> 448 (0x7E).
+__device__ __forceinline__ uint32_t e4m3_code(float u) {
+  if (u >= 448.0f) return 0x7Eu;
+  if (u < 0.015625f) return static_cast<uint32_t>(__float2int_rn(u * 512.0f));  // m * 2^-9
+  const int e = static_cast<int>((__float_as_uint(u) >> 23) & 0xFFu) - 127;
+  // u * 2^(3-e) lies in [8, 16) and is exact (a power-of-two scaling)
+  int q = __float2int_rn(u * __uint_as_float(static_cast<uint32_t>(130 - e) << 23));
+  int ee = e;
+  if (q == 16) {
+    q = 8;
+    ee = e + 1;
+  }
+  return static_cast<uint32_t>(((ee + 7) << 3) | (q - 8));
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const uint32_t e = c >> 3, m = c & 7u;
+  return e == 0 ? static_cast<float>(m) * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// E2M1 code (bit 3 = sign): the number of rounding boundaries |y| has passed; midpoints go to
+// the even code (0.25 -> 0, 0.75 -> 1.0, 1.25 -> 1.0, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4).
+__device__ __forceinline__ uint32_t e2m1_code(float y) {
+  const float a = fabsf(y);
+  const uint32_t m = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
+                     static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
+                     static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) +
+                     static_cast<uint32_t>(a > 5.0f);
+  return (y < 0.0f && m != 0u) ? (m | 8u) : m;
+}
+
+constexpr float kGlobalRange = 2688.0f;  // 6 (largest E2M1) * 448 (largest E4M3)
+
+// ---------------------------------------------------------------------------------------------
+// Prologue
+// ---------------------------------------------------------------------------------------------
+struct PrologueArgs {
+  const void* src[2];     // q, k
+  uint8_t* codes[2];      // [BH, N, D/2]
+  uint8_t* sf[2];         // [BH, N/128, D/64, 512]
+  float* genc[2];         // [BH]
+  float* inv_rms[2];      // [BH, N] (qknorm)
+  const float* k_mean;    // [BH, D] (ksmooth)
+  uint32_t* gmax;         // [2, BH] float bits, zeroed before the amax pass
+  int BH, N, qknorm, ksmooth;
+  float eps;
+};
+
+// The rows of one 128-row chunk, normalized and smoothed exactly as the INT8 prologue does.
+template <typename T, int D, int STEPS, int RPW, int GPW>
+__device__ __forceinline__ void load_rows(const PrologueArgs& a, int which, int bh, size_t row0,
+                                          int warp, int grp, int sub, uint32_t mask,
+                                          bool write_inv, float (&x)[STEPS][8]) {
+  const T* src = reinterpret_cast<const T*>(which == 0 ? a.src[0] : a.src[1]);
+  float* inv_out = which == 0 ? a.inv_rms[0] : a.inv_rms[1];
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int r = warp * RPW + s * GPW + grp;
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + (row0 + r) * D + sub * 8));
+    Cvt<T>::load8(u, x[s]);
+  }
+  if (a.qknorm) {
+#pragma unroll
+    for (int s = 0; s < STEPS; ++s) {
+      const float inv = rms_norm8<D>(x[s], a.eps, mask);
+      const int r = warp * RPW + s * GPW + grp;
+      if (write_inv && sub == 0 && inv_out) inv_out[row0 + r] = inv;
+    }
+  }
+  if (which == 1 && a.ksmooth) {
+    const float4* mp =
+        reinterpret_cast<const float4*>(a.k_mean + static_cast<size_t>(bh) * D + sub * 8);
+    const float4 m0 = mp[0], m1 = mp[1];
+    const float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+    for (int s = 0; s < STEPS; ++s)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) x[s][c] = __fsub_rn(x[s][c], m[c]);
+  }
+}
+
+// Pass 1: per (tensor, batch-head) absolute maximum.  Grid 2 * BH * N/128, kQuantThreads.
+template <typename T, int D>
+__global__ void __launch_bounds__(kQuantThreads, 2) prologue_amax_kernel(PrologueArgs a) {
+  constexpr int NW = kQuantThreads / 32, RPW = kRowsPerCta / NW;
+  constexpr int LPR = D / 8, GPW = 32 / LPR, STEPS = RPW / GPW;
+  __shared__ float red[NW];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = lane / LPR, sub = lane % LPR;
+  const uint32_t mask = ((LPR == 32) ? 0xFFFFFFFFu : ((1u << LPR) - 1u)) << (grp * LPR);
+  const int nchunk = a.N / kRowsPerCta, per = a.BH * nchunk;
+  const int which = blockIdx.x / per, rem = blockIdx.x % per;
+  const int bh = rem / nchunk, ch = rem % nchunk;
+  const size_t row0 = static_cast<size_t>(bh) * a.N + static_cast<size_t>(ch) * kRowsPerCta;
+  float x[STEPS][8];
+  load_rows<T, D, STEPS, RPW, GPW>(a, which, bh, row0, warp, grp, sub, mask, false, x);
+  float am = 0.0f;
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) am = fmaxf(am, fabsf(x[s][c]));
+  am = warp_max(am);
+  if (lane == 0) red[warp] = am;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) m = fmaxf(m, red[w]);
+    atomicMax(a.gmax + which * a.BH + bh, __float_as_uint(m));
+  }
+}
+
+// Pass 2: codes, block scales and the global scale.  Grid 2 * BH * N/128, kQuantThreads.
+template <typename T, int D>
+__global__ void __launch_bounds__(kQuantThreads, 2) prologue_quant_kernel(PrologueArgs a) {
+  constexpr int NW = kQuantThreads / 32, RPW = kRowsPerCta / NW;
+  constexpr int LPR = D / 8, GPW = 32 / LPR, STEPS = RPW / GPW;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = lane / LPR, sub = lane % LPR;
+  const uint32_t mask = ((LPR == 32) ? 0xFFFFFFFFu : ((1u << LPR) - 1u)) << (grp * LPR);
+  const int nchunk = a.N / kRowsPerCta, per = a.BH * nchunk;
+  const int which = blockIdx.x / per, rem = blockIdx.x % per;
+  const int bh = rem / nchunk, ch = rem % nchunk;
+  const size_t row0 = static_cast<size_t>(bh) * a.N + static_cast<size_t>(ch) * kRowsPerCta;
+  float x[STEPS][8];
+  load_rows<T, D, STEPS, RPW, GPW>(a, which, bh, row0, warp, grp, sub, mask, true, x);
+  const float G = __uint_as_float(a.gmax[which * a.BH + bh]);
+  const float genc = G > 0.0f ? __fdiv_rn(kGlobalRange, G) : 1.0f;
+  if (ch == 0 && threadIdx.x == 0) (which == 0 ? a.genc[0] : a.genc[1])[bh] = genc;
+  // this lane's 8 channels are half of the 16-channel block (sub / 2)
+  const int kb = sub >> 1;
+  uint8_t* codes = which == 0 ? a.codes[0] : a.codes[1];
+  uint8_t* sf_tile = (which == 0 ? a.sf[0] : a.sf[1]) + (static_cast<size_t>(bh) * nchunk + ch) * (D / 64) * 512 +
+                     (kb >> 2) * 512 + (kb & 3);
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    float am = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) am = fmaxf(am, fabsf(x[s][c]));
+    am = fmaxf(am, __shfl_xor_sync(mask, am, 1));
+    const float u = __fdiv_rn(__fmul_rn(am, genc), 6.0f);
+    const uint32_t sc = e4m3_code(u);
+    const float sd = e4m3_value(sc);
+    const float mult = sd > 0.0f ? __fdiv_rn(genc, sd) : 0.0f;
+    uint32_t w = 0;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) w |= e2m1_code(__fmul_rn(x[s][c], mult)) << (4 * c);
+    const int r = warp * RPW + s * GPW + grp;
+    *reinterpret_cast<uint32_t*>(codes + (row0 + r) * (D / 2) + sub * 4) = w;
+    if ((sub & 1) == 0) sf_tile[(r & 31) * 16 + (r >> 5) * 4] = static_cast<uint8_t>(sc);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Forward
+// ---------------------------------------------------------------------------------------------
+constexpr int BM = 128;   // query rows per CTA (MMA M)
+constexpr int BKV = 128;  // keys per block
+constexpr int NST = 3;    // K / V pipeline stages
+constexpr int kThreads = 192;
+constexpr int kProducerWarp = 0, kMmaWarp = 1;
+constexpr uint32_t kColPV = 256, kColSfa = 384, kColSfb = 392;  // TMEM columns
+
+template <typename T, int D>
+struct Smem {
+  alignas(1024) uint8_t q[BM * D / 2];
+  alignas(1024) uint8_t k[NST][BKV * D / 2];
+  alignas(1024) T v[NST][BKV * D];   // D/64 boxes of [BKV keys][64 channels]
+  alignas(1024) T p[2][BM * BKV];    // 2 swizzle atoms of [BM rows][64 keys]
+  alignas(128) uint8_t qsf[D / 64 * 512];
+  alignas(128) uint8_t ksf[NST][D / 64 * 512];
+  uint64_t q_full, k_full[NST], v_full[NST], kv_empty[NST];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_full, pv_free;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <typename T, int D>
+constexpr size_t smem_bytes() {
+  return sizeof(Smem<T, D>) + 1024;
+}
+
+template <typename T, int D>
+__device__ __forceinline__ Smem<T, D>& smem_ref(uint8_t* raw) {
+  const uint32_t a = smem_u32(raw);
+  return *reinterpret_cast<Smem<T, D>*>(raw + ((1024u - (a & 1023u)) & 1023u));
+}
+
+struct Args {
+  const uint8_t* q_sf;
+  const uint8_t* k_sf;
+  const float* q_genc;
+  const float* k_genc;
+  void* o;
+  float* lse;
+  int N, causal;
+  float scale_log2;  // softmax_scale * log2(e)
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, Args args) {
+  static_assert(D == 64 || D == 128, "head dimension");
+  extern __shared__ uint8_t smem_raw[];
+  Smem<T, D>& sm = smem_ref<T, D>(smem_raw);
+  constexpr uint32_t kSfBytes = D / 64 * 512;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = args.N, nqt = N / BM;
+  // head-major order; within a head, the query tiles with the most key blocks first (causal)
+  const int bh = blockIdx.x / nqt, t = blockIdx.x % nqt;
+  const int qt = args.causal ? nqt - 1 - t : t;
+  const int q0 = qt * BM;
+  const int nb = args.causal ? qt + 1 : N / BKV;
+
+  if (threadIdx.x == 0) {
+    sm.abort = device_aborted() ? 1 : 0;
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.s_free[b], BM);
+      mbar_init(&sm.p_full[b], BM);
+    }
+    mbar_init(&sm.pv_full, 1);
+    mbar_init(&sm.pv_free, BM);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (sm.abort) return;
+  if (warp == kMmaWarp) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const int row_base = bh * N;
+      mbar_arrive_expect_tx(&sm.q_full, BM * D / 2 + kSfBytes);
+      tma_load_2d(sm.q, &tm_q, 0, row_base + q0, &sm.q_full);
+      bulk_load(sm.qsf, args.q_sf + (static_cast<size_t>(bh) * nqt + qt) * kSfBytes, kSfBytes,
+                &sm.q_full);
+      for (int j = 0; j < nb; ++j) {
+        const int st = j % NST;
+        if (j >= NST) mbar_wait(&sm.kv_empty[st], ((j / NST) - 1) & 1, 201);
+        mbar_arrive_expect_tx(&sm.k_full[st], BKV * D / 2 + kSfBytes);
+        tma_load_2d(sm.k[st], &tm_k, 0, row_base + j * BKV, &sm.k_full[st]);
+        bulk_load(sm.ksf[st], args.k_sf + (static_cast<size_t>(bh) * (N / BKV) + j) * kSfBytes,
+                  kSfBytes, &sm.k_full[st]);
+        mbar_arrive_expect_tx(&sm.v_full[st], BKV * D * 2);
+#pragma unroll
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_2d(sm.v[st] + b * BKV * 64, &tm_v, b * 64, row_base + j * BKV, &sm.v_full[st]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t kSw = (D == 128) ? kSwizzle64B : kSwizzle32B;
+      constexpr uint32_t kSbo = 8 * (D / 2);  // 8 rows of D/2 bytes
+      constexpr uint32_t kFmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+      const uint32_t idesc_s = instr_desc_nvf4(BM, BKV);
+      // P (A, K-major) and V (B, MN-major) share V's 16-bit type
+      const uint32_t idesc_pv = instr_desc(1, kFmt, kFmt, false, true, BM, D);
+      const uint32_t qa = smem_u32(sm.q);
+      mbar_wait(&sm.q_full, 0, 210);
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 64; ++kk)
+        tmem_cp_sf(tmem + kColSfa + 4 * kk,
+                   smem_desc(smem_u32(sm.qsf) + 512 * kk, 128, 128, kSwizzleNone));
+      auto issue_pv = [&](int jj) {
+        const int st = jj % NST;
+        mbar_wait(&sm.v_full[st], (jj / NST) & 1, 213);
+        mbar_wait(&sm.p_full[jj & 1], (jj >> 1) & 1, 214);
+        if (jj >= 1) mbar_wait(&sm.pv_free, (jj - 1) & 1, 215);
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sm.p[jj & 1]);
+        const uint32_t va = smem_u32(sm.v[st]);
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          mma_f16(tmem + kColPV,
+                  smem_desc(pa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024, kSwizzle128B),
+                  smem_desc(va + kk * 16 * 128, BKV * 128, 1024, kSwizzle128B), idesc_pv,
+                  kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sm.pv_full);
+        mma_commit(&sm.kv_empty[st]);
+      };
+      for (int j = 0; j < nb; ++j) {
+        const int st = j % NST, b = j & 1;
+        mbar_wait(&sm.k_full[st], (j / NST) & 1, 211);
+        // S buffer b and its K-scale columns served block j-2: free once its softmax has read
+        // S (s_free), which also orders the scale copy below after block j-2's MMAs
+        if (j >= 2) mbar_wait(&sm.s_free[b], ((j - 2) >> 1) & 1, 212);
+        tc_fence_after();
+        const uint32_t sfb = tmem + kColSfb + 8 * b;
+#pragma unroll
+        for (int kk = 0; kk < D / 64; ++kk)
+          tmem_cp_sf(sfb + 4 * kk, smem_desc(smem_u32(sm.ksf[st]) + 512 * kk, 128, 128,
+                                             kSwizzleNone));
+        const uint32_t ka = smem_u32(sm.k[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 64; ++kk)
+          mma_nvf4(tmem + b * 128, smem_desc(qa + 32 * kk, 16, kSbo, kSw),
+                   smem_desc(ka + 32 * kk, 16, kSbo, kSw), idesc_s, tmem + kColSfa + 4 * kk,
+                   sfb + 4 * kk, kk > 0 ? 1u : 0u);
+        mma_commit(&sm.s_full[b]);
+        if (j >= 1) issue_pv(j - 1);
+      }
+      issue_pv(nb - 1);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- softmax warps ----------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int i = q0 + r;
+    const uint32_t lane_base = tmem + ((quarter * 32u) << 16);
+    const float c = __fdiv_rn(args.scale_log2, args.q_genc[bh] * args.k_genc[bh]);
+    float O[D];
+#pragma unroll
+    for (int cc = 0; cc < D; ++cc) O[cc] = 0.0f;
+    float m = -INFINITY, l = 0.0f, alpha_prev = 1.0f;
+
+    auto fold_pv = [&](int jj, float a) {
+      mbar_wait(&sm.pv_full, jj & 1, 221);
+      tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t x0[16], x1[16];
+        tmem_ld16(lane_base + kColPV + c0, x0);
+        tmem_ld16(lane_base + kColPV + c0 + 16, x1);
+        tmem_ld_wait_regs(x0, x1);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          O[c0 + e] = fmaf(O[c0 + e], a, __uint_as_float(x0[e]));
+          O[c0 + 16 + e] = fmaf(O[c0 + 16 + e], a, __uint_as_float(x1[e]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.pv_free);
+    };
+
+    for (int j = 0; j < nb; ++j) {
+      const int b = j & 1;
+      const bool diag = args.causal && j == qt;
+      const int key0 = j * BKV;
+      mbar_wait(&sm.s_full[b], (j >> 1) & 1, 220);
+      tc_fence_after();
+      const uint32_t sa = lane_base + b * 128;
+      // pass 1: block maximum of the raw scores over visible keys (c > 0 keeps the order)
+      float mx = -INFINITY;
+#pragma unroll
+      for (int h = 0; h < BKV / 32; ++h) {
+        uint32_t x0[16], x1[16];
+        tmem_ld16(sa + h * 32, x0);
+        tmem_ld16(sa + h * 32 + 16, x1);
+        tmem_ld_wait_regs(x0, x1);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float f0 = __uint_as_float(x0[e]), f1 = __uint_as_float(x1[e]);
+          if (diag && key0 + h * 32 + e > i) f0 = -INFINITY;
+          if (diag && key0 + h * 32 + 16 + e > i) f1 = -INFINITY;
+          mx = fmax3(mx, f0, f1);
+        }
+      }
+      const float mn = fmaxf(m, mx * c);
+      const float alpha = ex2_approx(m - mn);
+      // pass 2: p = exp2(S c - mn), row sum, P in V's type into the swizzled K-major tile
+      float rs0 = 0.0f, rs1 = 0.0f;
+      uint8_t* pt = reinterpret_cast<uint8_t*>(sm.p[b]);
+#pragma unroll
+      for (int h = 0; h < BKV / 32; ++h) {
+        uint32_t x0[16], x1[16];
+        tmem_ld16(sa + h * 32, x0);
+        tmem_ld16(sa + h * 32 + 16, x1);
+        tmem_ld_wait_regs(x0, x1);
+        // keys h*32 .. h*32+31 are 16-byte chunks 4(h%2) .. 4(h%2)+3 of swizzle atom h/2;
+        // x0 holds keys +0..15 (chunks q4 = 0, 1), x1 keys +16..31 (q4 = 2, 3)
+        uint8_t* atom = pt + (h >> 1) * (BM * 128);
+        auto conv = [&](const uint32_t (&x)[16], int q4) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const int k0 = key0 + h * 32 + q4 * 8 + e;
+            const int xi = (q4 & 1) * 8 + e;
+            float p0 = ex2_approx(fmaf(__uint_as_float(x[xi]), c, -mn));
+            float p1 = ex2_approx(fmaf(__uint_as_float(x[xi + 1]), c, -mn));
+            if (diag && k0 > i) p0 = 0.0f;
+            if (diag && k0 + 1 > i) p1 = 0.0f;
+            rs0 += p0;
+            rs1 += p1;
+            w[e / 2] = Cvt<T>::pack2(p0, p1);
+          }
+          *reinterpret_cast<uint4*>(atom + swz_offset(r, (h & 1) * 4 + q4, 128)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        };
+        conv(x0, 0);
+        conv(x0, 1);
+        conv(x1, 2);
+        conv(x1, 3);
+      }
+      l = fmaf(l, alpha, rs0 + rs1);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm.s_free[b]);
+      mbar_arrive(&sm.p_full[b]);
+      if (j > 0) fold_pv(j - 1, alpha_prev);
+      alpha_prev = alpha;
+      m = mn;
+    }
+    fold_pv(nb - 1, alpha_prev);
+    // epilogue: O / l in the output type, LSE = (m + log2 l) ln 2
+    const float inv_l = 1.0f / l;
+    T* orow = reinterpret_cast<T*>(args.o) + (static_cast<size_t>(bh) * N + i) * D;
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 8) {
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = O[c0 + e] * inv_l;
+      *reinterpret_cast<uint4*>(orow + c0) = pack8<T>(f);
+    }
+    args.lse[static_cast<size_t>(bh) * N + i] = (m + log2f(l)) * 0.69314718055994531f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace fp4
+}  // namespace sage

@@ -199,6 +199,29 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
 }
 
 // Arrive on `bar` once every tcgen05.mma previously issued by this thread has completed.
+// D[tmem] (+)= (A * SFA)[smem] * (B * SFB)[smem]: NVFP4 operands (packed E2M1, two per byte,
+// K = 64 per instruction) with one unsigned E4M3 scale per 16 elements along K; FP32
+// accumulator.  sfa / sfb are the TMEM addresses of the scale factors (see tmem_cp_sf).
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], "
+      "[%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copy 32 rows x 16 bytes of shared memory (described by a no-swizzle K-major descriptor) into
+// TMEM columns [taddr, taddr + 4) of all four 32-lane sub-partitions.  Ordered with later
+// tcgen05.mma of the same thread.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -321,6 +344,14 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t c_fmt, uint32_t a_fmt
                                                   int M, int N) {
   return (c_fmt << 4) | (a_fmt << 7) | (b_fmt << 10) | (static_cast<uint32_t>(a_mn) << 15) |
          (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor of a block-scaled tcgen05.mma of kind::mxf4nvf4 with E2M1 A and B
+// (format code 1), both K-major, unsigned E4M3 scales (bit 23 = 0), scale-factor IDs 0 and a
+// dense K of 64.
+__host__ __device__ constexpr uint32_t instr_desc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 

@@ -13,9 +13,11 @@
 #include <mutex>
 
 #include "sage.h"
+#include "sage_nvfp4.h"
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "debug_kernels.cuh"
+#include "nvfp4.cuh"
 #include "ptx.cuh"
 #include "rowops.cuh"
 
@@ -315,6 +317,103 @@ int bwd_stage(int stage, const sage_params* p, const void* q, const void* k, con
             : run_bwd<__half, 64>(stage, p, q, k, v, qb, o, lse, dout, dq, dk, dv, workspace, st);
 }
 
+// ---- NVFP4 variant -----------------------------------------------------------------------
+int check_fp4(const sage_params* p) {
+  const int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  return p->qsmooth ? SAGE_ERR_UNSUPPORTED : SAGE_OK;
+}
+
+int check_fp4bufs(const sage_params* p, const sage_fp4_bufs* fb) {
+  if (!fb || !fb->q_fp4 || !fb->k_fp4 || !fb->q_sf || !fb->k_sf || !fb->q_genc || !fb->k_genc)
+    return SAGE_ERR_INVALID_ARG;
+  if (p->ksmooth && !fb->k_mean) return SAGE_ERR_INVALID_ARG;
+  const void* ptrs[] = {fb->q_fp4, fb->k_fp4, fb->q_sf, fb->k_sf, fb->q_genc, fb->k_genc,
+                        fb->k_mean, fb->q_inv_rms, fb->k_inv_rms};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return SAGE_ERR_ALIGNMENT;
+  return SAGE_OK;
+}
+
+// Workspace: K-mean partials (ksmooth) then the 2 x BH global maxima.
+struct Fp4Ws {
+  size_t gmax, total;
+};
+Fp4Ws fp4_ws(const sage_params* p) {
+  Fp4Ws w;
+  w.gmax = p->ksmooth ? align_up(prologue_partials(p) * 4) : 0;
+  w.total = align_up(w.gmax + 2 * static_cast<size_t>(p->B) * p->H * 4);
+  return w;
+}
+
+template <typename T, int D>
+int run_fp4_prologue(const sage_params* p, const void* q, const void* k, const sage_fp4_bufs* fb,
+                     void* ws, cudaStream_t st) {
+  const int BH = p->B * p->H, N = p->N;
+  const Fp4Ws w = fp4_ws(p);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+  if (p->ksmooth) {
+    const int total = BH * (N / 64);
+    const int per_cta = (kRowThreads / 32) * (32 / (D / 8));
+    float* partials = reinterpret_cast<float*>(wsb);
+    sage::prologue_kstats_kernel<T, D><<<(total + per_cta - 1) / per_cta, kRowThreads, 0, st>>>(
+        reinterpret_cast<const T*>(k), partials, total, p->qknorm, p->rms_eps);
+    sage::prologue_kmean_kernel<D><<<BH, D, 0, st>>>(partials, fb->k_mean, N / 64, N);
+  }
+  uint32_t* gmax = reinterpret_cast<uint32_t*>(wsb + w.gmax);
+  if (cudaMemsetAsync(gmax, 0, 2 * static_cast<size_t>(BH) * 4, st) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  sage::fp4::PrologueArgs a;
+  a.src[0] = q;
+  a.src[1] = k;
+  a.codes[0] = fb->q_fp4;
+  a.codes[1] = fb->k_fp4;
+  a.sf[0] = fb->q_sf;
+  a.sf[1] = fb->k_sf;
+  a.genc[0] = fb->q_genc;
+  a.genc[1] = fb->k_genc;
+  a.inv_rms[0] = fb->q_inv_rms;
+  a.inv_rms[1] = fb->k_inv_rms;
+  a.k_mean = fb->k_mean;
+  a.gmax = gmax;
+  a.BH = BH;
+  a.N = N;
+  a.qknorm = p->qknorm;
+  a.ksmooth = p->ksmooth;
+  a.eps = p->rms_eps;
+  const int grid = 2 * BH * (N / kRowsPerCta);
+  sage::fp4::prologue_amax_kernel<T, D><<<grid, sage::kQuantThreads, 0, st>>>(a);
+  sage::fp4::prologue_quant_kernel<T, D><<<grid, sage::kQuantThreads, 0, st>>>(a);
+  return launch_status();
+}
+
+template <typename T, int D>
+int run_fp4_fwd(const sage_params* p, const sage_fp4_bufs* fb, const void* v, void* o,
+                float* lse, cudaStream_t st) {
+  const int BH = p->B * p->H, N = p->N;
+  const uint64_t rows = static_cast<uint64_t>(BH) * N;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, fb->q_fp4, 1, D / 2, rows, D / 2, sage::fp4::BM) ||
+      !make_map(&tk, fb->k_fp4, 1, D / 2, rows, D / 2, sage::fp4::BKV) ||
+      !make_map(&tv, v, 2, D, rows, 64, sage::fp4::BKV))
+    return SAGE_ERR_CUDA;
+  sage::fp4::Args a;
+  a.q_sf = fb->q_sf;
+  a.k_sf = fb->k_sf;
+  a.q_genc = fb->q_genc;
+  a.k_genc = fb->k_genc;
+  a.o = o;
+  a.lse = lse;
+  a.N = N;
+  a.causal = p->causal;
+  a.scale_log2 = tau_of(p) * 1.4426950408889634f;
+  const size_t smem = sage::fp4::smem_bytes<T, D>();
+  auto kern = sage::fp4::attn_fwd_kernel<T, D>;
+  if (set_smem(kern, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+  kern<<<BH * (N / sage::fp4::BM), sage::fp4::kThreads, smem, st>>>(tq, tk, tv, a);
+  return launch_status();
+}
+
 // ---- prologue scratch for callers that cannot allocate -------------------------------------
 // A fixed device array that sage_quant_prologue_noalloc uses instead of a caller workspace for
 // the K-smoothing column sums.  Every device that loads the library holds it until exit.
@@ -430,6 +529,46 @@ int sage_attn_bwd_stage(int stage, const sage_params* p, const void* q, const vo
                         size_t workspace_bytes, void* stream) {
   return bwd_stage(stage, p, q, k, v, qb, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
                    stream);
+}
+
+size_t sage_fp4_workspace_bytes(const sage_params* p, int which) {
+  if (check_fp4(p) != SAGE_OK) return 0;
+  return which == 0 ? fp4_ws(p).total : 0;
+}
+
+int sage_fp4_quant_prologue(const sage_params* p, const void* q, const void* k,
+                            const sage_fp4_bufs* out, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  int s = check_fp4(p);
+  if (s != SAGE_OK) return s;
+  if (!q || !k) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_fp4bufs(p, out)) != SAGE_OK) return s;
+  if (!aligned16(q) || !aligned16(k)) return SAGE_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < fp4_ws(p).total) return SAGE_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SAGE_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_fp4_prologue<__nv_bfloat16, 128>(p, q, k, out, workspace, st)
+              : run_fp4_prologue<__half, 128>(p, q, k, out, workspace, st);
+  return bf ? run_fp4_prologue<__nv_bfloat16, 64>(p, q, k, out, workspace, st)
+            : run_fp4_prologue<__half, 64>(p, q, k, out, workspace, st);
+}
+
+int sage_fp4_attn_fwd(const sage_params* p, const sage_fp4_bufs* fb, const void* v, void* o,
+                      float* lse, void* stream) {
+  int s = check_fp4(p);
+  if (s != SAGE_OK) return s;
+  if ((s = check_fp4bufs(p, fb)) != SAGE_OK) return s;
+  if (!v || !o || !lse) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(v) || !aligned16(o) || !aligned16(lse)) return SAGE_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_fp4_fwd<__nv_bfloat16, 128>(p, fb, v, o, lse, st)
+              : run_fp4_fwd<__half, 128>(p, fb, v, o, lse, st);
+  return bf ? run_fp4_fwd<__nv_bfloat16, 64>(p, fb, v, o, lse, st)
+            : run_fp4_fwd<__half, 64>(p, fb, v, o, lse, st);
 }
 
 int sage_last_device_status(void* stream) {

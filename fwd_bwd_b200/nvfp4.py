@@ -1,0 +1,83 @@
+"""Python binding of the NVFP4 Q-Attn variant (include/sage_nvfp4.h): argument marshalling only.
+
+Every step runs in libsage's CUDA kernels; there is no other path.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional
+
+import torch
+
+from ._lib import SageFp4Bufs, check, lib
+from .ops import Config, _check_inputs, _stream
+
+
+@dataclasses.dataclass
+class Fp4Bufs:
+    """NVFP4 views of Q and K (codes, E4M3 block scales, global scales), made once, reused."""
+
+    q_fp4: torch.Tensor
+    k_fp4: torch.Tensor
+    q_sf: torch.Tensor
+    k_sf: torch.Tensor
+    q_genc: torch.Tensor
+    k_genc: torch.Tensor
+    q_inv_rms: Optional[torch.Tensor]
+    k_inv_rms: Optional[torch.Tensor]
+    k_mean: Optional[torch.Tensor]
+
+    @staticmethod
+    def empty(shape, cfg: Config, device) -> "Fp4Bufs":
+        B, H, N, d = shape
+        u8 = dict(dtype=torch.uint8, device=device)
+        f32 = dict(dtype=torch.float32, device=device)
+        sf = (B, H, N // 128, d // 64, 512)
+        return Fp4Bufs(torch.empty((B, H, N, d // 2), **u8), torch.empty((B, H, N, d // 2), **u8),
+                       torch.empty(sf, **u8), torch.empty(sf, **u8),
+                       torch.empty((B, H), **f32), torch.empty((B, H), **f32),
+                       torch.empty((B, H, N), **f32) if cfg.qknorm else None,
+                       torch.empty((B, H, N), **f32) if cfg.qknorm else None,
+                       torch.empty((B, H, d), **f32) if cfg.ksmooth else None)
+
+    def c_struct(self) -> SageFp4Bufs:
+        p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        return SageFp4Bufs(p(self.q_fp4), p(self.k_fp4), p(self.q_sf), p(self.k_sf),
+                           p(self.q_genc), p(self.k_genc), p(self.q_inv_rms), p(self.k_inv_rms),
+                           p(self.k_mean))
+
+
+def workspace_bytes(cfg: Config, like: torch.Tensor) -> int:
+    return int(lib().sage_fp4_workspace_bytes(ctypes.byref(cfg.params(like)), 0))
+
+
+def quant_prologue(q, k, cfg: Config, out: Optional[Fp4Bufs] = None,
+                   workspace: Optional[torch.Tensor] = None) -> Fp4Bufs:
+    """QK-norm, K-smoothing and NVFP4 quantization of q and k (sage_fp4_quant_prologue)."""
+    _check_inputs(q, k)
+    prm = cfg.params(q)
+    fb = out if out is not None else Fp4Bufs.empty(tuple(q.shape), cfg, q.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(cfg, q), dtype=torch.uint8, device=q.device)
+    st = fb.c_struct()
+    check("sage_fp4_quant_prologue", lib().sage_fp4_quant_prologue(
+        ctypes.byref(prm), q.data_ptr(), k.data_ptr(), ctypes.byref(st), workspace.data_ptr(),
+        workspace.numel(), _stream(q.device)))
+    return fb
+
+
+def attn_fwd(fb: Fp4Bufs, v: torch.Tensor, cfg: Config, o=None, lse=None):
+    """NVFP4 Q K^T, 16-bit P V forward (sage_fp4_attn_fwd): returns (o, lse)."""
+    _check_inputs(v)
+    prm = cfg.params(v)
+    B, H, N, d = v.shape
+    if o is None:
+        o = torch.empty_like(v)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=v.device)
+    st = fb.c_struct()
+    check("sage_fp4_attn_fwd", lib().sage_fp4_attn_fwd(
+        ctypes.byref(prm), ctypes.byref(st), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+        _stream(v.device)))
+    return o, lse

@@ -1,0 +1,67 @@
+/*
+ * sage_nvfp4.h -- C ABI of the NVFP4 Q-Attn variant of libsage (B200, sm_100a).
+ *
+ * The operation ("Full-Stack FP4", gist.science 2607.04422, section 2.4 "mixed-precision
+ * attention (Q-Attn)"): the robust product Q K^T runs in NVFP4, the softmax-sensitive product
+ * P V in BF16 (here: in the inputs' 16-bit type); the quantized views of Q and K are produced
+ * once by sage_fp4_quant_prologue and reused.  NVFP4 ("Quartet II", allinfo.ai.kr): E2M1
+ * values in blocks of 16 along the head dimension, one E4M3 scale per block, plus a global
+ * scale, here one per (batch, head) matrix.
+ *
+ * Quantization (float32, every step correctly rounded, reproducible bit for bit):
+ *   x      q or k after the optional QK-norm and K-smoothing of sage.h (same arithmetic);
+ *   G      max |x| over the (batch, head) matrix; genc = 2688 / G (1 when G == 0);
+ *   block  a = max |x| over 16 channels; u = (a * genc) / 6;
+ *          sd = E4M3(u): round to nearest, ties to even, subnormals, 448 and above -> 448;
+ *          code = E2M1(x * (genc / sd)): magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}, nearest, ties
+ *          to the even code, above 6 -> 6, values rounding to zero -> +0; sd == 0 -> code 0.
+ *   value  E2M1(code) * sd / genc.
+ *
+ * Conventions are those of sage.h (device pointers owned by the caller, 16-byte alignment,
+ * asynchronous on `stream`, negative sage_status on argument errors, no exceptions).
+ * Supported: d in {64, 128}, N a multiple of 128, qsmooth == 0 (else SAGE_ERR_UNSUPPORTED);
+ * q_block and k_block are validated as in sage.h but unused (NVFP4 blocks are 16 channels).
+ */
+#ifndef SAGE_NVFP4_H_
+#define SAGE_NVFP4_H_
+
+#include "sage.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* NVFP4 views of Q and K.  Sizes per (batch, head); all owned by the caller. */
+typedef struct {
+  uint8_t *q_fp4, *k_fp4;       /* [B,H,N,d/2]: E2M1 codes, channel 2i in the low nibble of
+                                   byte i, channel 2i+1 in the high nibble                   */
+  uint8_t *q_sf, *k_sf;         /* [B,H,N/128,d/64,512]: E4M3 block scales; per 128-row tile
+                                   and 64-channel chunk, byte (r%32)*16 + (r/32)*4 + b holds
+                                   row r's scale of the chunk's 16-channel block b           */
+  float *q_genc, *k_genc;       /* [B,H]: global encode scales genc                         */
+  float *q_inv_rms, *k_inv_rms; /* [B,H,N]: 1/rms per token (qknorm; may be NULL otherwise) */
+  float *k_mean;                /* [B,H,d]: K channel means (ksmooth; else unused)          */
+} sage_fp4_bufs;
+
+/* Workspace bytes: which = 0 prologue (K-mean partials when ksmooth, plus 2*B*H words for the
+ * global maxima), 1 forward (0).  Returns 0 for invalid parameters. */
+size_t sage_fp4_workspace_bytes(const sage_params* p, int which);
+
+/* QK-norm -> K-smoothing -> NVFP4 views of q and k (an absolute-maximum pass, then the
+ * quantization pass).  q, k: [B,H,N,d] in p->dtype. */
+int sage_fp4_quant_prologue(const sage_params* p, const void* q, const void* k,
+                            const sage_fp4_bufs* out, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Forward: S = tau * (Q K^T) from the NVFP4 views (tensor-core block-scaled MMA, FP32
+ * accumulation), causal mask, online softmax, O = P V with P rounded to the 16-bit type of v
+ * and FP32 accumulation.  v: [B,H,N,d] in p->dtype; o: [B,H,N,d] in p->dtype;
+ * lse: [B,H,N] float32, natural log of sum_j exp(z_ij). */
+int sage_fp4_attn_fwd(const sage_params* p, const sage_fp4_bufs* fb, const void* v, void* o,
+                      float* lse, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_NVFP4_H_ */

@@ -21,8 +21,8 @@ def L():
     return _lib.lib()
 
 
-def _declared():
-    src = open(os.path.join(ROOT, "include", "sage.h")).read()
+def _declared(header="sage.h"):
+    src = open(os.path.join(ROOT, "include", header)).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(sage_[a-z0-9_]+)\s*\(", src)))
 
@@ -30,8 +30,39 @@ def _declared():
 def test_exports_every_declared_symbol(L):
     names = _declared()
     assert len(names) == 10
-    for n in names:
+    fp4 = _declared("sage_nvfp4.h")
+    assert fp4 == ["sage_fp4_attn_fwd", "sage_fp4_quant_prologue", "sage_fp4_workspace_bytes"]
+    for n in names + fp4:
         assert hasattr(L, n), n
+
+
+def test_fp4_workspace_and_argument_checks(L):
+    from fwd_bwd_b200._lib import SageFp4Bufs
+
+    BH, N, d = 8, 1024, 128
+    p = _params()
+    assert L.sage_fp4_workspace_bytes(ctypes.byref(p), 0) == BH * (N // 64) * d * 4 + 256
+    assert L.sage_fp4_workspace_bytes(ctypes.byref(p), 1) == 0
+    assert L.sage_fp4_workspace_bytes(ctypes.byref(_params(ksmooth=0)), 0) == 256
+    assert L.sage_fp4_workspace_bytes(ctypes.byref(_params(qsmooth=1)), 0) == 0
+    fake = 1 << 20  # never dereferenced: every call below fails its host-side checks
+    fb = SageFp4Bufs(*([fake] * 9))
+    ws = BH * (N // 64) * d * 4 + 256
+    assert L.sage_fp4_quant_prologue(ctypes.byref(_params(qsmooth=1)), fake, fake,
+                                     ctypes.byref(fb), fake, ws, None) == _lib.SAGE_ERR_UNSUPPORTED
+    assert L.sage_fp4_quant_prologue(ctypes.byref(_params(d=96)), fake, fake, ctypes.byref(fb),
+                                     fake, ws, None) == _lib.SAGE_ERR_UNSUPPORTED
+    assert L.sage_fp4_quant_prologue(ctypes.byref(p), None, fake, ctypes.byref(fb), fake, ws,
+                                     None) == _lib.SAGE_ERR_INVALID_ARG
+    assert L.sage_fp4_quant_prologue(ctypes.byref(p), fake, fake, ctypes.byref(fb), fake, ws - 1,
+                                     None) == _lib.SAGE_ERR_WORKSPACE
+    assert L.sage_fp4_quant_prologue(ctypes.byref(p), fake + 8, fake, ctypes.byref(fb), fake, ws,
+                                     None) == _lib.SAGE_ERR_ALIGNMENT
+    nosf = SageFp4Bufs(fake, fake, None, fake, fake, fake, fake, fake, fake)
+    assert L.sage_fp4_attn_fwd(ctypes.byref(p), ctypes.byref(nosf), fake, fake, fake,
+                               None) == _lib.SAGE_ERR_INVALID_ARG
+    assert L.sage_fp4_attn_fwd(ctypes.byref(p), ctypes.byref(fb), fake, fake + 4, fake,
+                               None) == _lib.SAGE_ERR_ALIGNMENT
 
 
 def _params(**kw):

@@ -1,0 +1,112 @@
+"""NVFP4 Q-Attn parity: the CUDA path against the NVFP4 oracle on the same seeded inputs.
+
+* Prologue: E2M1 codes, E4M3 block scales, global scales, inverse RMS and K means bit-exact
+  (every quantization decision is a correctly rounded float32 step on both sides).
+* Forward: O and LSE element by element.  The kernel rounds P to the 16-bit type of V before
+  P V (the tensor-core operand precision) while the oracle keeps P exact; with
+  W = sum_j p_j |v_j| / l that rounding moves O by at most u16 * W (u16 = 2^-8 for bf16,
+  2^-11 for fp16, relative half-ulp), the 16-bit output rounding by u16 |O|, and the FP32
+  accumulation of S and PV and the exp2 approximation by far less.  The test allows twice
+  those bounds plus 1e-5 W.  LSE depends only on FP32 sums: |dLSE| <= 1e-4.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.nvfp4_oracle as F
+from fwd_bwd_b200 import nvfp4, ops
+from fwd_bwd_b200.inputs import WORKLOADS
+
+from gpu_helpers import to_device
+from fwd_bwd_b200.inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+BASE = WORKLOADS["sweep8192"]
+CASES = {
+    "d128_bf16_causal": BASE.replace(B=1, H=3, N=384),
+    "d128_bf16_full": BASE.replace(B=1, H=2, N=256, causal=False),
+    "d128_fp16_causal": BASE.replace(B=2, H=1, N=512, dtype="fp16"),
+    "d64_bf16_causal": WORKLOADS["llama325m"].replace(B=1, H=3, N=384),
+    "d64_fp16_full": WORKLOADS["llama325m"].replace(B=1, H=2, N=256, dtype="fp16",
+                                                   causal=False),
+    "koutlier_norm_off": WORKLOADS["koutlier"].replace(B=1, H=2, N=256, qknorm=False),
+    "koutlier_all_off": WORKLOADS["koutlier"].replace(B=1, H=2, N=384, qknorm=False,
+                                                     ksmooth=False),
+    "single_tile": BASE.replace(B=1, H=1, N=128),
+}
+
+
+def _cfg(w):
+    return ops.Config(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth, q_block=w.q_block,
+                      k_block=w.k_block)
+
+
+def unpack_codes(packed: np.ndarray) -> np.ndarray:
+    """[..., d/2] bytes -> [..., d] 4-bit codes (channel 2i in the low nibble of byte i)."""
+    out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), np.uint8)
+    out[..., 0::2] = packed & 15
+    out[..., 1::2] = packed >> 4
+    return out
+
+
+def unpack_sf(sf: np.ndarray, N: int, d: int) -> np.ndarray:
+    """[BH, N/128, d/64, 512] scale atoms -> [BH, N, d/16] (row r, 16-channel block b)."""
+    sf = sf.reshape(-1, N // 128, d // 64, 512)
+    BH = sf.shape[0]
+    r = np.arange(128)
+    b = np.arange(4)
+    idx = (r[:, None] % 32) * 16 + (r[:, None] // 32) * 4 + b[None, :]  # [128, 4]
+    t = sf[..., idx]  # [BH, N/128, d/64, 128, 4]
+    return t.transpose(0, 1, 3, 2, 4).reshape(BH, N, d // 16)
+
+
+def _run(w):
+    x = make_inputs(w)
+    q, k, v = (to_device(x[n], w.dtype) for n in ("q", "k", "v"))
+    cfg = _cfg(w)
+    fb = nvfp4.quant_prologue(q, k, cfg)
+    o, lse = nvfp4.attn_fwd(fb, v, cfg)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    return x, fb, o, lse
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_nvfp4_prologue_and_forward(name):
+    w = CASES[name]
+    BH, N, d = w.B * w.H, w.N, w.d
+    x, fb, o, lse = _run(w)
+    qf, kf, vf = (x[n + "_f32"].reshape(BH, N, d) for n in ("q", "k", "v"))
+    ref = F.qattn_forward(qf, kf, vf, causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth)
+    for t in ("q", "k"):
+        codes = unpack_codes(getattr(fb, t + "_fp4").cpu().numpy().reshape(BH, N, d // 2))
+        np.testing.assert_array_equal(codes, ref[t + "_codes"], err_msg=t + " codes")
+        sf = unpack_sf(getattr(fb, t + "_sf").cpu().numpy(), N, d)
+        np.testing.assert_array_equal(sf, ref[t + "_sf"], err_msg=t + " scales")
+        np.testing.assert_array_equal(getattr(fb, t + "_genc").cpu().numpy().reshape(BH),
+                                      ref[t + "_genc"], err_msg=t + " genc")
+        if w.qknorm:
+            np.testing.assert_array_equal(
+                getattr(fb, t + "_inv_rms").cpu().numpy().reshape(BH, N), ref[t + "_inv_rms"])
+    if w.ksmooth:
+        np.testing.assert_array_equal(fb.k_mean.cpu().numpy().reshape(BH, d), ref["k_mean"])
+    u16 = 2.0 ** -8 if w.dtype == "bf16" else 2.0 ** -11
+    og = o.float().cpu().numpy().astype(np.float64).reshape(BH, N, d)
+    err = np.abs(og - ref["o"])
+    tol = 2 * u16 * (ref["w"] + np.abs(ref["o"])) + 1e-5 * ref["w"] + 1e-7
+    bad = err > tol
+    assert not bad.any(), (f"{bad.sum()} of {bad.size} outside; worst excess "
+                           f"{(err - tol).max():.3g}; max err {err.max():.3g}")
+    lg = lse.cpu().numpy().astype(np.float64).reshape(BH, N)
+    np.testing.assert_allclose(lg, ref["lse"], rtol=0, atol=1e-4)
+
+
+def test_nvfp4_unsupported_qsmooth():
+    w = CASES["single_tile"]
+    x = make_inputs(w)
+    q, k = (to_device(x[n], w.dtype) for n in ("q", "k"))
+    cfg = _cfg(w)
+    cfg.qsmooth = True
+    with pytest.raises(Exception, match="UNSUPPORTED"):
+        nvfp4.quant_prologue(q, k, cfg)
