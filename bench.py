@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--chunks", type=int, default=16,
                     help="batch slices of the end-to-end host-buffer pipeline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", default="int8", choices=["int8", "nvfp4"],
+                    help="int8: the SageBwd step (default); nvfp4: the NVFP4 Q-Attn forward")
     return ap.parse_args()
 
 
@@ -165,6 +167,123 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+METRIC_FP4 = "NVFP4 Q-Attn forward effective TOPS at 1 B200 and % of FP4/16-bit TC roofline"
+
+
+def cpu_baseline_fp4(w, n_heads: int):
+    """Time the NVFP4 oracle (as it stands) on the first n_heads heads: prologue + forward."""
+    from threadpoolctl import threadpool_info
+
+    import oracle.nvfp4_oracle as F
+    from fwd_bwd_b200.inputs import make_inputs
+
+    x = make_inputs(w, heads=range(n_heads))
+    t0 = time.perf_counter()
+    F.qattn_forward(x["q_f32"], x["k_f32"], x["v_f32"], causal=w.causal, qknorm=w.qknorm,
+                    ksmooth=w.ksmooth)
+    dt = time.perf_counter() - t0
+    ops = w.ops("fwd") / (w.B * w.H) * n_heads
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{n_heads} of {w.B * w.H} heads (flattened b*H+h = 0..{n_heads - 1}) of "
+                      f"the workload, NVFP4 prologue+forward, numpy oracle"}
+
+
+def run_nvfp4(args, w):
+    """The NVFP4 Q-Attn forward: step = NVFP4 prologue (amax + quantization) + forward."""
+    import torch
+
+    from fwd_bwd_b200 import nvfp4, ops
+    from fwd_bwd_b200.inputs import make_inputs_fast
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--variant nvfp4 runs on one GPU")
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    cfg = ops.Config(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth)
+    x = make_inputs_fast(w, device=str(dev))
+    q, k, v = x["q"], x["k"], x["v"]
+    fb = nvfp4.Fp4Bufs.empty(tuple(q.shape), cfg, dev)
+    ws = torch.empty(nvfp4.workspace_bytes(cfg, q), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 2 * int(w.ksmooth) + 2 + 1
+
+    def step(ev=None):
+        nvfp4.quant_prologue(q, k, cfg, out=fb, workspace=ws)
+        if ev is not None:
+            ev[0].record(stream)
+        nvfp4.attn_fwd(fb, v, cfg, o=o, lse=lse)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    time.sleep(0.3)
+    t0.record(stream)
+    for s_ in range(args.steps):
+        step(evs[s_])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if ops.device_status(dev) != 0:
+        raise RuntimeError("device status reports a kernel timeout in the timed region")
+    ms = t0.elapsed_time(t1) / args.steps
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    fwd_ops = w.ops("fwd")
+    value = fwd_ops / (ms * 1e-3) / 1e12
+    pk = peaks()
+    # Q K^T at the FP4 rate (4x bf16, the nominal dense ratio 9 : 2.25 POPS), P V at the bf16
+    # rate; equal op counts
+    p_bf16 = pk["bf16_sustained"]
+    p_fwd = 1.0 / (0.5 / (4.0 * p_bf16) + 0.5 / p_bf16)
+    achieved = fwd_ops / (fwd_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "fp4::attn_fwd_kernel", "achieved": achieved,
+                "peak": p_fwd, "unit": "TFLOP/s", "frac": achieved / p_fwd, "traffic": None,
+                "peak_note": f"{pk['basis']} sustained bf16; NVFP4 = 4x bf16, weighted 1:1 "
+                             f"with the 16-bit P V"}
+    e2e = None
+    if not args.no_e2e:
+        hin = [t.cpu().pin_memory() for t in (q, k, v)]
+        hout = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        qd, kd, vd = (torch.empty_like(t) for t in (q, k, v))
+
+        def host_step():
+            for h, d_ in zip(hin, (qd, kd, vd)):
+                d_.copy_(h, non_blocking=True)
+            nvfp4.quant_prologue(qd, kd, cfg, out=fb, workspace=ws)
+            nvfp4.attn_fwd(fb, vd, cfg, o=o, lse=lse)
+            hout.copy_(o, non_blocking=True)
+            torch.cuda.synchronize(dev)
+
+        host_step()
+        w0 = time.perf_counter()
+        for _ in range(args.steps):
+            host_step()
+        e_ms = (time.perf_counter() - w0) * 1e3 / args.steps
+        e2e = {"value": fwd_ops / (e_ms * 1e-3) / 1e12, "unit": "TOPS",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hin),
+               "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+    line = {"metric": METRIC_FP4, "value": value, "unit": "TOPS", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4+bf16", "data": "synthetic",
+            "config": dict(config_of(w), variant="nvfp4 forward"),
+            "kernels": {"fp4::attn_fwd_kernel": {"ms": round(fwd_ms, 4),
+                                                 "tops": round(achieved, 2),
+                                                 "frac": round(achieved / p_fwd, 4)}},
+            "roofline": roofline, "clocks": clocks, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps}
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_fp4(w, 4)
+    print(json.dumps(line), flush=True)
+
+
 def config_of(w):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
             "io_dtype": w.dtype, "q_block": w.q_block, "k_block": w.k_block,
@@ -181,6 +300,9 @@ def main():
         w = w.replace(B=args.B)
     if args.impl == "reference":
         run_reference(args, w)
+        return
+    if args.variant == "nvfp4":
+        run_nvfp4(args, w)
         return
 
     import torch

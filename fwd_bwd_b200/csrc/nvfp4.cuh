@@ -17,15 +17,19 @@
 // genc [BH].
 //
 // Forward: per CTA one tile of 128 query rows of one (batch, head), walking 128-key blocks.
-//   warp 0      TMA producer: Q codes and scales once, then K codes, K scales and V (16-bit)
+//   warp 8      TMA producer: Q codes and scales once, then K codes, K scales and V (16-bit)
 //               through a 3-stage ring;
-//   warp 1      MMA issuer (one thread): block scales copied to TMEM (tcgen05.cp), S_j = Q K_j^T
+//   warp 9      MMA issuer (one thread): block scales copied to TMEM (tcgen05.cp), S_j = Q K_j^T
 //               (kind::mxf4nvf4, scale vector 16, FP32 in TMEM, double-buffered), then
 //               PV_{j-1} = P_{j-1} V_{j-1} (kind::f16 in V's type, FP32 in TMEM);
-//   warps 2-5   softmax, one query row per thread: z = S * tau / (genc_Q genc_K), causal mask,
-//               running max, p = exp2(z - m) written to shared memory in V's 16-bit type
-//               (K-major, 128-byte swizzle), running sum of the float32 p, and the fold
-//               O <- alpha O + PV in registers.
+//   warps 0-7   softmax, two warps per query row (one per 64-key half of each block and per
+//               half of the output channels): z = S * tau / (genc_Q genc_K), causal mask,
+//               running max (the pair exchanges its block maxima through shared memory),
+//               p = exp2(z - m) written to shared memory in V's 16-bit type (K-major, 128-byte
+//               swizzle), running sum of the float32 p, and the fold O <- alpha O + PV in
+//               registers.
+//   warps 10-11 idle (they complete the producer warpgroup, which gives its registers to the
+//               softmax warpgroups).
 // TMEM (512 columns): S buffers at 0 and 128, PV at 256, Q scales at 384, K scales at 392 and
 // 400 (one set per S buffer).
 #pragma once
@@ -205,8 +209,15 @@ __global__ void __launch_bounds__(kQuantThreads, 2) prologue_quant_kernel(Prolog
 constexpr int BM = 128;   // query rows per CTA (MMA M)
 constexpr int BKV = 128;  // keys per block
 constexpr int NST = 3;    // K / V pipeline stages
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 0, kMmaWarp = 1;
+constexpr int kThreads = 384;  // 8 softmax warps, producer, MMA, 2 idle warps
+constexpr int kSoftmaxThreads = 256;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+// register split (setmaxnreg): the softmax warpgroups rise to 232, the producer warpgroup
+// (producer, MMA and two idle warps) drops to 40; the launch gives every thread 168
+constexpr int kLaunchRegs = 168, kSoftmaxRegs = 232, kOtherRegs = 40;
+static_assert(kSoftmaxThreads * kSoftmaxRegs + (kThreads - kSoftmaxThreads) * kOtherRegs <=
+                  kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr uint32_t kColPV = 256, kColSfa = 384, kColSfb = 392;  // TMEM columns
 
 template <typename T, int D>
@@ -217,6 +228,8 @@ struct Smem {
   alignas(1024) T p[2][BM * BKV];    // 2 swizzle atoms of [BM rows][64 keys]
   alignas(128) uint8_t qsf[D / 64 * 512];
   alignas(128) uint8_t ksf[NST][D / 64 * 512];
+  float mx[2][2][BM];   // per S buffer, per key half: the rows' block maxima (x c)
+  float lsum[2][BM];    // per key half: the rows' final partial sums
   uint64_t q_full, k_full[NST], v_full[NST], kv_empty[NST];
   uint64_t s_full[2], s_free[2], p_full[2], pv_full, pv_free;
   uint32_t tmem_base;
@@ -272,11 +285,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], BM);
-      mbar_init(&sm.p_full[b], BM);
+      mbar_init(&sm.s_free[b], kSoftmaxThreads);
+      mbar_init(&sm.p_full[b], kSoftmaxThreads);
     }
     mbar_init(&sm.pv_full, 1);
-    mbar_init(&sm.pv_free, BM);
+    mbar_init(&sm.pv_free, kSoftmaxThreads);
     fence_barrier_init();
   }
   __syncthreads();
@@ -290,107 +303,121 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == kProducerWarp) {
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      const int row_base = bh * N;
-      mbar_arrive_expect_tx(&sm.q_full, BM * D / 2 + kSfBytes);
-      tma_load_2d(sm.q, &tm_q, 0, row_base + q0, &sm.q_full);
-      bulk_load(sm.qsf, args.q_sf + (static_cast<size_t>(bh) * nqt + qt) * kSfBytes, kSfBytes,
-                &sm.q_full);
-      for (int j = 0; j < nb; ++j) {
-        const int st = j % NST;
-        if (j >= NST) mbar_wait(&sm.kv_empty[st], ((j / NST) - 1) & 1, 201);
-        mbar_arrive_expect_tx(&sm.k_full[st], BKV * D / 2 + kSfBytes);
-        tma_load_2d(sm.k[st], &tm_k, 0, row_base + j * BKV, &sm.k_full[st]);
-        bulk_load(sm.ksf[st], args.k_sf + (static_cast<size_t>(bh) * (N / BKV) + j) * kSfBytes,
-                  kSfBytes, &sm.k_full[st]);
-        mbar_arrive_expect_tx(&sm.v_full[st], BKV * D * 2);
-#pragma unroll
-        for (int b = 0; b < D / 64; ++b)
-          tma_load_2d(sm.v[st] + b * BKV * 64, &tm_v, b * 64, row_base + j * BKV, &sm.v_full[st]);
-      }
-    }
-    __syncwarp();
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) {
-      constexpr uint32_t kSw = (D == 128) ? kSwizzle64B : kSwizzle32B;
-      constexpr uint32_t kSbo = 8 * (D / 2);  // 8 rows of D/2 bytes
-      constexpr uint32_t kFmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
-      const uint32_t idesc_s = instr_desc_nvf4(BM, BKV);
-      // P (A, K-major) and V (B, MN-major) share V's 16-bit type
-      const uint32_t idesc_pv = instr_desc(1, kFmt, kFmt, false, true, BM, D);
-      const uint32_t qa = smem_u32(sm.q);
-      mbar_wait(&sm.q_full, 0, 210);
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < D / 64; ++kk)
-        tmem_cp_sf(tmem + kColSfa + 4 * kk,
-                   smem_desc(smem_u32(sm.qsf) + 512 * kk, 128, 128, kSwizzleNone));
-      auto issue_pv = [&](int jj) {
-        const int st = jj % NST;
-        mbar_wait(&sm.v_full[st], (jj / NST) & 1, 213);
-        mbar_wait(&sm.p_full[jj & 1], (jj >> 1) & 1, 214);
-        if (jj >= 1) mbar_wait(&sm.pv_free, (jj - 1) & 1, 215);
-        tc_fence_after();
-        const uint32_t pa = smem_u32(sm.p[jj & 1]);
-        const uint32_t va = smem_u32(sm.v[st]);
-#pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          mma_f16(tmem + kColPV,
-                  smem_desc(pa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024, kSwizzle128B),
-                  smem_desc(va + kk * 16 * 128, BKV * 128, 1024, kSwizzle128B), idesc_pv,
-                  kk > 0 ? 1u : 0u);
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
+    if (warp == kProducerWarp) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        const int row_base = bh * N;
+        mbar_arrive_expect_tx(&sm.q_full, BM * D / 2 + kSfBytes);
+        tma_load_2d(sm.q, &tm_q, 0, row_base + q0, &sm.q_full);
+        bulk_load(sm.qsf, args.q_sf + (static_cast<size_t>(bh) * nqt + qt) * kSfBytes, kSfBytes,
+                  &sm.q_full);
+        for (int j = 0; j < nb; ++j) {
+          const int st = j % NST;
+          if (j >= NST) mbar_wait(&sm.kv_empty[st], ((j / NST) - 1) & 1, 201);
+          mbar_arrive_expect_tx(&sm.k_full[st], BKV * D / 2 + kSfBytes);
+          tma_load_2d(sm.k[st], &tm_k, 0, row_base + j * BKV, &sm.k_full[st]);
+          bulk_load(sm.ksf[st], args.k_sf + (static_cast<size_t>(bh) * (N / BKV) + j) * kSfBytes,
+                    kSfBytes, &sm.k_full[st]);
+          mbar_arrive_expect_tx(&sm.v_full[st], BKV * D * 2);
+  #pragma unroll
+          for (int b = 0; b < D / 64; ++b)
+            tma_load_2d(sm.v[st] + b * BKV * 64, &tm_v, b * 64, row_base + j * BKV, &sm.v_full[st]);
         }
-        mma_commit(&sm.pv_full);
-        mma_commit(&sm.kv_empty[st]);
-      };
-      for (int j = 0; j < nb; ++j) {
-        const int st = j % NST, b = j & 1;
-        mbar_wait(&sm.k_full[st], (j / NST) & 1, 211);
-        // S buffer b and its K-scale columns served block j-2: free once its softmax has read
-        // S (s_free), which also orders the scale copy below after block j-2's MMAs
-        if (j >= 2) mbar_wait(&sm.s_free[b], ((j - 2) >> 1) & 1, 212);
-        tc_fence_after();
-        const uint32_t sfb = tmem + kColSfb + 8 * b;
-#pragma unroll
-        for (int kk = 0; kk < D / 64; ++kk)
-          tmem_cp_sf(sfb + 4 * kk, smem_desc(smem_u32(sm.ksf[st]) + 512 * kk, 128, 128,
-                                             kSwizzleNone));
-        const uint32_t ka = smem_u32(sm.k[st]);
-#pragma unroll
-        for (int kk = 0; kk < D / 64; ++kk)
-          mma_nvf4(tmem + b * 128, smem_desc(qa + 32 * kk, 16, kSbo, kSw),
-                   smem_desc(ka + 32 * kk, 16, kSbo, kSw), idesc_s, tmem + kColSfa + 4 * kk,
-                   sfb + 4 * kk, kk > 0 ? 1u : 0u);
-        mma_commit(&sm.s_full[b]);
-        if (j >= 1) issue_pv(j - 1);
       }
-      issue_pv(nb - 1);
+      __syncwarp();
+    } else if (warp == kMmaWarp) {
+      if (lane == 0) {
+        constexpr uint32_t kSw = (D == 128) ? kSwizzle64B : kSwizzle32B;
+        constexpr uint32_t kSbo = 8 * (D / 2);  // 8 rows of D/2 bytes
+        constexpr uint32_t kFmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+        const uint32_t idesc_s = instr_desc_nvf4(BM, BKV);
+        // P (A, K-major) and V (B, MN-major) share V's 16-bit type
+        const uint32_t idesc_pv = instr_desc(1, kFmt, kFmt, false, true, BM, D);
+        const uint32_t qa = smem_u32(sm.q);
+        mbar_wait(&sm.q_full, 0, 210);
+        tc_fence_after();
+  #pragma unroll
+        for (int kk = 0; kk < D / 64; ++kk)
+          tmem_cp_sf(tmem + kColSfa + 4 * kk,
+                     smem_desc(smem_u32(sm.qsf) + 512 * kk, 128, 128, kSwizzleNone));
+        auto issue_pv = [&](int jj) {
+          const int st = jj % NST;
+          mbar_wait(&sm.v_full[st], (jj / NST) & 1, 213);
+          mbar_wait(&sm.p_full[jj & 1], (jj >> 1) & 1, 214);
+          if (jj >= 1) mbar_wait(&sm.pv_free, (jj - 1) & 1, 215);
+          tc_fence_after();
+          const uint32_t pa = smem_u32(sm.p[jj & 1]);
+          const uint32_t va = smem_u32(sm.v[st]);
+  #pragma unroll
+          for (int kk = 0; kk < BKV / 16; ++kk) {
+            mma_f16(tmem + kColPV,
+                    smem_desc(pa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024, kSwizzle128B),
+                    smem_desc(va + kk * 16 * 128, BKV * 128, 1024, kSwizzle128B), idesc_pv,
+                    kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&sm.pv_full);
+          mma_commit(&sm.kv_empty[st]);
+        };
+        for (int j = 0; j < nb; ++j) {
+          const int st = j % NST, b = j & 1;
+          mbar_wait(&sm.k_full[st], (j / NST) & 1, 211);
+          // S buffer b and its K-scale columns served block j-2: free once its softmax has read
+          // S (s_free), which also orders the scale copy below after block j-2's MMAs
+          if (j >= 2) mbar_wait(&sm.s_free[b], ((j - 2) >> 1) & 1, 212);
+          tc_fence_after();
+          const uint32_t sfb = tmem + kColSfb + 8 * b;
+  #pragma unroll
+          for (int kk = 0; kk < D / 64; ++kk)
+            tmem_cp_sf(sfb + 4 * kk, smem_desc(smem_u32(sm.ksf[st]) + 512 * kk, 128, 128,
+                                               kSwizzleNone));
+          const uint32_t ka = smem_u32(sm.k[st]);
+  #pragma unroll
+          for (int kk = 0; kk < D / 64; ++kk)
+            mma_nvf4(tmem + b * 128, smem_desc(qa + 32 * kk, 16, kSbo, kSw),
+                     smem_desc(ka + 32 * kk, 16, kSbo, kSw), idesc_s, tmem + kColSfa + 4 * kk,
+                     sfb + 4 * kk, kk > 0 ? 1u : 0u);
+          mma_commit(&sm.s_full[b]);
+          if (j >= 1) issue_pv(j - 1);
+        }
+        issue_pv(nb - 1);
+      }
+      __syncwarp();
     }
-    __syncwarp();
+    tc_fence_before();
+    named_barrier_sync(15, kThreads);
+    tc_fence_after();
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
     // ---------------- softmax warps ----------------
+    // Two warps per TMEM lane quarter: `half` 0 takes keys 0-63 of every block and output
+    // channels 0 .. D/2-1, half 1 keys 64-127 and channels D/2 .. D-1.  The pair shares each
+    // block's row maximum through shared memory; the row sums are combined at the end.
     const int quarter = warp & 3;
+    const int half = warp >> 2;
     const int r = quarter * 32 + lane;
     const int i = q0 + r;
     const uint32_t lane_base = tmem + ((quarter * 32u) << 16);
+    const int pair_bar = 1 + quarter;  // named barrier of the two warps of this quarter
     const float c = __fdiv_rn(args.scale_log2, args.q_genc[bh] * args.k_genc[bh]);
-    float O[D];
+    constexpr int DH = D / 2;
+    float O[DH];
 #pragma unroll
-    for (int cc = 0; cc < D; ++cc) O[cc] = 0.0f;
+    for (int cc = 0; cc < DH; ++cc) O[cc] = 0.0f;
     float m = -INFINITY, l = 0.0f, alpha_prev = 1.0f;
 
     auto fold_pv = [&](int jj, float a) {
       mbar_wait(&sm.pv_full, jj & 1, 221);
       tc_fence_after();
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < DH; c0 += 32) {
         uint32_t x0[16], x1[16];
-        tmem_ld16(lane_base + kColPV + c0, x0);
-        tmem_ld16(lane_base + kColPV + c0 + 16, x1);
+        tmem_ld16(lane_base + kColPV + half * DH + c0, x0);
+        tmem_ld16(lane_base + kColPV + half * DH + c0 + 16, x1);
         tmem_ld_wait_regs(x0, x1);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -405,88 +432,92 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < nb; ++j) {
       const int b = j & 1;
       const bool diag = args.causal && j == qt;
-      const int key0 = j * BKV;
+      const int key0 = j * BKV + half * 64;
       mbar_wait(&sm.s_full[b], (j >> 1) & 1, 220);
       tc_fence_after();
-      const uint32_t sa = lane_base + b * 128;
-      // pass 1: block maximum of the raw scores over visible keys (c > 0 keeps the order)
-      float mx = -INFINITY;
-#pragma unroll
-      for (int h = 0; h < BKV / 32; ++h) {
-        uint32_t x0[16], x1[16];
-        tmem_ld16(sa + h * 32, x0);
-        tmem_ld16(sa + h * 32 + 16, x1);
-        tmem_ld_wait_regs(x0, x1);
+      // this warp's 64 scores, read from TMEM once
+      const uint32_t sa = lane_base + b * 128 + half * 64;
+      uint32_t x0[16], x1[16], x2[16], x3[16];
+      tmem_ld16(sa, x0);
+      tmem_ld16(sa + 16, x1);
+      tmem_ld16(sa + 32, x2);
+      tmem_ld16(sa + 48, x3);
+      tmem_ld_wait_regs(x0, x1);
+      tmem_ld_wait_regs(x2, x3);
+      tc_fence_before();
+      mbar_arrive(&sm.s_free[b]);
+      // block maximum of the raw scores over visible keys (c > 0 keeps the order)
+      float m0 = -INFINITY, m1 = -INFINITY;
+      auto maxh = [&](const uint32_t (&xa)[16], const uint32_t (&xb)[16], int k0, float& mm) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          float f0 = __uint_as_float(x0[e]), f1 = __uint_as_float(x1[e]);
-          if (diag && key0 + h * 32 + e > i) f0 = -INFINITY;
-          if (diag && key0 + h * 32 + 16 + e > i) f1 = -INFINITY;
-          mx = fmax3(mx, f0, f1);
+          float f0 = __uint_as_float(xa[e]), f1 = __uint_as_float(xb[e]);
+          if (diag && key0 + k0 + e > i) f0 = -INFINITY;
+          if (diag && key0 + k0 + 16 + e > i) f1 = -INFINITY;
+          mm = fmax3(mm, f0, f1);
         }
-      }
-      const float mn = fmaxf(m, mx * c);
+      };
+      maxh(x0, x1, 0, m0);
+      maxh(x2, x3, 32, m1);
+      const float mine = fmaxf(m0, m1) * c;
+      sm.mx[b][half][r] = mine;
+      named_barrier_sync(pair_bar, 64);
+      const float mn = fmaxf(m, fmaxf(mine, sm.mx[b][half ^ 1][r]));
       const float alpha = ex2_approx(m - mn);
-      // pass 2: p = exp2(S c - mn), row sum, P in V's type into the swizzled K-major tile
+      // p = exp2(S c - mn) in V's type into this half's swizzle atom (64 keys), row sum
       float rs0 = 0.0f, rs1 = 0.0f;
-      uint8_t* pt = reinterpret_cast<uint8_t*>(sm.p[b]);
+      uint8_t* atom = reinterpret_cast<uint8_t*>(sm.p[b]) + half * (BM * 128);
+      auto conv = [&](const uint32_t (&x)[16], int k16) {
 #pragma unroll
-      for (int h = 0; h < BKV / 32; ++h) {
-        uint32_t x0[16], x1[16];
-        tmem_ld16(sa + h * 32, x0);
-        tmem_ld16(sa + h * 32 + 16, x1);
-        tmem_ld_wait_regs(x0, x1);
-        // keys h*32 .. h*32+31 are 16-byte chunks 4(h%2) .. 4(h%2)+3 of swizzle atom h/2;
-        // x0 holds keys +0..15 (chunks q4 = 0, 1), x1 keys +16..31 (q4 = 2, 3)
-        uint8_t* atom = pt + (h >> 1) * (BM * 128);
-        auto conv = [&](const uint32_t (&x)[16], int q4) {
+        for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
-            const int k0 = key0 + h * 32 + q4 * 8 + e;
-            const int xi = (q4 & 1) * 8 + e;
-            float p0 = ex2_approx(fmaf(__uint_as_float(x[xi]), c, -mn));
-            float p1 = ex2_approx(fmaf(__uint_as_float(x[xi + 1]), c, -mn));
-            if (diag && k0 > i) p0 = 0.0f;
-            if (diag && k0 + 1 > i) p1 = 0.0f;
+            const int kk = k16 * 16 + q2 * 8 + e;  // key within this half
+            float p0 = ex2_approx(fmaf(__uint_as_float(x[q2 * 8 + e]), c, -mn));
+            float p1 = ex2_approx(fmaf(__uint_as_float(x[q2 * 8 + e + 1]), c, -mn));
+            if (diag && key0 + kk > i) p0 = 0.0f;
+            if (diag && key0 + kk + 1 > i) p1 = 0.0f;
             rs0 += p0;
             rs1 += p1;
             w[e / 2] = Cvt<T>::pack2(p0, p1);
           }
-          *reinterpret_cast<uint4*>(atom + swz_offset(r, (h & 1) * 4 + q4, 128)) =
+          *reinterpret_cast<uint4*>(atom + swz_offset(r, k16 * 2 + q2, 128)) =
               make_uint4(w[0], w[1], w[2], w[3]);
-        };
-        conv(x0, 0);
-        conv(x0, 1);
-        conv(x1, 2);
-        conv(x1, 3);
-      }
+        }
+      };
+      conv(x0, 0);
+      conv(x1, 1);
+      conv(x2, 2);
+      conv(x3, 3);
       l = fmaf(l, alpha, rs0 + rs1);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&sm.s_free[b]);
       mbar_arrive(&sm.p_full[b]);
       if (j > 0) fold_pv(j - 1, alpha_prev);
       alpha_prev = alpha;
       m = mn;
     }
     fold_pv(nb - 1, alpha_prev);
-    // epilogue: O / l in the output type, LSE = (m + log2 l) ln 2
-    const float inv_l = 1.0f / l;
-    T* orow = reinterpret_cast<T*>(args.o) + (static_cast<size_t>(bh) * N + i) * D;
+    // row sum over both halves (same order on both warps), then the epilogue: O / l in the
+    // output type, LSE = (m + log2 l) ln 2
+    sm.lsum[half][r] = l;
+    named_barrier_sync(pair_bar, 64);
+    const float lt = sm.lsum[0][r] + sm.lsum[1][r];
+    const float inv_l = 1.0f / lt;
+    T* orow = reinterpret_cast<T*>(args.o) + (static_cast<size_t>(bh) * N + i) * D + half * DH;
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 8) {
+    for (int c0 = 0; c0 < DH; c0 += 8) {
       float f[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) f[e] = O[c0 + e] * inv_l;
       *reinterpret_cast<uint4*>(orow + c0) = pack8<T>(f);
     }
-    args.lse[static_cast<size_t>(bh) * N + i] = (m + log2f(l)) * 0.69314718055994531f;
+    if (half == 0)
+      args.lse[static_cast<size_t>(bh) * N + i] = (m + log2f(lt)) * 0.69314718055994531f;
+    tc_fence_before();
+    named_barrier_sync(15, kThreads);
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace fp4

@@ -410,6 +410,8 @@ int run_fp4_fwd(const sage_params* p, const sage_fp4_bufs* fb, const void* v, vo
   const size_t smem = sage::fp4::smem_bytes<T, D>();
   auto kern = sage::fp4::attn_fwd_kernel<T, D>;
   if (set_smem(kern, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+  // register split between warpgroups (setmaxnreg) assumes exactly kLaunchRegs at launch
+  if (launch_regs(kern) != sage::fp4::kLaunchRegs) return SAGE_ERR_UNSUPPORTED;
   kern<<<BH * (N / sage::fp4::BM), sage::fp4::kThreads, smem, st>>>(tq, tk, tv, a);
   return launch_status();
 }
