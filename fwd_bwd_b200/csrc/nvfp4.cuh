@@ -20,8 +20,9 @@
 //   warp 8      TMA producer: Q codes and scales once, then K codes, K scales and V (16-bit)
 //               through a 3-stage ring;
 //   warp 9      MMA issuer (one thread): block scales copied to TMEM (tcgen05.cp), S_j = Q K_j^T
-//               (kind::mxf4nvf4, scale vector 16, FP32 in TMEM, double-buffered), then
-//               PV_{j-1} = P_{j-1} V_{j-1} (kind::f16 in V's type, FP32 in TMEM);
+//               (kind::mxf4nvf4, scale vector 16, FP32 in TMEM; S is read into registers as
+//               soon as it lands, so one buffer suffices), then PV_{j-1} = P_{j-1} V_{j-1}
+//               (kind::f16 in V's type, FP32 in TMEM, double-buffered);
 //   warps 0-7   softmax, two warps per query row (one per 64-key half of each block and per
 //               half of the output channels): z = S * tau / (genc_Q genc_K), causal mask,
 //               running max (the pair exchanges its block maxima through shared memory),
@@ -30,8 +31,8 @@
 //               registers.
 //   warps 10-11 idle (they complete the producer warpgroup, which gives its registers to the
 //               softmax warpgroups).
-// TMEM (512 columns): S buffers at 0 and 128, PV at 256, Q scales at 384, K scales at 392 and
-// 400 (one set per S buffer).
+// TMEM (512 columns): S at 0, PV buffers at 128 and 256, Q scales at 384, K scales at 392 and
+// 400 (alternating by block).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -218,7 +219,7 @@ constexpr int kLaunchRegs = 168, kSoftmaxRegs = 232, kOtherRegs = 40;
 static_assert(kSoftmaxThreads * kSoftmaxRegs + (kThreads - kSoftmaxThreads) * kOtherRegs <=
                   kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
-constexpr uint32_t kColPV = 256, kColSfa = 384, kColSfb = 392;  // TMEM columns
+constexpr uint32_t kColS = 0, kColPV = 128, kColSfa = 384, kColSfb = 392;  // TMEM columns
 
 template <typename T, int D>
 struct Smem {
@@ -228,10 +229,10 @@ struct Smem {
   alignas(1024) T p[2][BM * BKV];    // 2 swizzle atoms of [BM rows][64 keys]
   alignas(128) uint8_t qsf[D / 64 * 512];
   alignas(128) uint8_t ksf[NST][D / 64 * 512];
-  float mx[2][2][BM];   // per S buffer, per key half: the rows' block maxima (x c)
+  float mx[2][2][BM];   // per block parity, per key half: the rows' block maxima (x c)
   float lsum[2][BM];    // per key half: the rows' final partial sums
   uint64_t q_full, k_full[NST], v_full[NST], kv_empty[NST];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_full, pv_free;
+  uint64_t s_full, s_free, p_full[2], pv_full[2], pv_free[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -283,13 +284,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.s_free, kSoftmaxThreads);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&sm.s_full[b], 1);
-      mbar_init(&sm.s_free[b], kSoftmaxThreads);
       mbar_init(&sm.p_full[b], kSoftmaxThreads);
+      mbar_init(&sm.pv_full[b], 1);
+      mbar_init(&sm.pv_free[b], kSoftmaxThreads);
     }
-    mbar_init(&sm.pv_full, 1);
-    mbar_init(&sm.pv_free, kSoftmaxThreads);
     fence_barrier_init();
   }
   __syncthreads();
@@ -348,26 +349,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = jj % NST;
           mbar_wait(&sm.v_full[st], (jj / NST) & 1, 213);
           mbar_wait(&sm.p_full[jj & 1], (jj >> 1) & 1, 214);
-          if (jj >= 1) mbar_wait(&sm.pv_free, (jj - 1) & 1, 215);
+          if (jj >= 2) mbar_wait(&sm.pv_free[jj & 1], ((jj - 2) >> 1) & 1, 215);
           tc_fence_after();
           const uint32_t pa = smem_u32(sm.p[jj & 1]);
           const uint32_t va = smem_u32(sm.v[st]);
   #pragma unroll
           for (int kk = 0; kk < BKV / 16; ++kk) {
-            mma_f16(tmem + kColPV,
+            mma_f16(tmem + kColPV + (jj & 1) * 128,
                     smem_desc(pa + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024, kSwizzle128B),
                     smem_desc(va + kk * 16 * 128, BKV * 128, 1024, kSwizzle128B), idesc_pv,
                     kk > 0 ? 1u : 0u);
           }
-          mma_commit(&sm.pv_full);
+          mma_commit(&sm.pv_full[jj & 1]);
           mma_commit(&sm.kv_empty[st]);
         };
         for (int j = 0; j < nb; ++j) {
           const int st = j % NST, b = j & 1;
           mbar_wait(&sm.k_full[st], (j / NST) & 1, 211);
-          // S buffer b and its K-scale columns served block j-2: free once its softmax has read
-          // S (s_free), which also orders the scale copy below after block j-2's MMAs
-          if (j >= 2) mbar_wait(&sm.s_free[b], ((j - 2) >> 1) & 1, 212);
+          // S and the K-scale columns b served block j-1 / j-2: S is free once block j-1's
+          // softmax has read it (s_free), which also orders the scale copy below after the
+          // MMAs of block j-2 (s_free of block j-1 follows s_full of block j-2)
+          if (j >= 1) mbar_wait(&sm.s_free, (j - 1) & 1, 212);
           tc_fence_after();
           const uint32_t sfb = tmem + kColSfb + 8 * b;
   #pragma unroll
@@ -377,10 +379,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ka = smem_u32(sm.k[st]);
   #pragma unroll
           for (int kk = 0; kk < D / 64; ++kk)
-            mma_nvf4(tmem + b * 128, smem_desc(qa + 32 * kk, 16, kSbo, kSw),
+            mma_nvf4(tmem + kColS, smem_desc(qa + 32 * kk, 16, kSbo, kSw),
                      smem_desc(ka + 32 * kk, 16, kSbo, kSw), idesc_s, tmem + kColSfa + 4 * kk,
                      sfb + 4 * kk, kk > 0 ? 1u : 0u);
-          mma_commit(&sm.s_full[b]);
+          mma_commit(&sm.s_full);
           if (j >= 1) issue_pv(j - 1);
         }
         issue_pv(nb - 1);
@@ -411,13 +413,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY, l = 0.0f, alpha_prev = 1.0f;
 
     auto fold_pv = [&](int jj, float a) {
-      mbar_wait(&sm.pv_full, jj & 1, 221);
+      const uint32_t pv = lane_base + kColPV + (jj & 1) * 128 + half * DH;
+      mbar_wait(&sm.pv_full[jj & 1], (jj >> 1) & 1, 221);
       tc_fence_after();
 #pragma unroll
       for (int c0 = 0; c0 < DH; c0 += 32) {
         uint32_t x0[16], x1[16];
-        tmem_ld16(lane_base + kColPV + half * DH + c0, x0);
-        tmem_ld16(lane_base + kColPV + half * DH + c0 + 16, x1);
+        tmem_ld16(pv + c0, x0);
+        tmem_ld16(pv + c0 + 16, x1);
         tmem_ld_wait_regs(x0, x1);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -426,17 +429,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&sm.pv_free);
+      mbar_arrive(&sm.pv_free[jj & 1]);
     };
 
     for (int j = 0; j < nb; ++j) {
       const int b = j & 1;
       const bool diag = args.causal && j == qt;
       const int key0 = j * BKV + half * 64;
-      mbar_wait(&sm.s_full[b], (j >> 1) & 1, 220);
+      mbar_wait(&sm.s_full, j & 1, 220);
       tc_fence_after();
       // this warp's 64 scores, read from TMEM once
-      const uint32_t sa = lane_base + b * 128 + half * 64;
+      const uint32_t sa = lane_base + kColS + half * 64;
       uint32_t x0[16], x1[16], x2[16], x3[16];
       tmem_ld16(sa, x0);
       tmem_ld16(sa + 16, x1);
@@ -445,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait_regs(x0, x1);
       tmem_ld_wait_regs(x2, x3);
       tc_fence_before();
-      mbar_arrive(&sm.s_free[b]);
+      mbar_arrive(&sm.s_free);
       // block maximum of the raw scores over visible keys (c > 0 keeps the order)
       float m0 = -INFINITY, m1 = -INFINITY;
       auto maxh = [&](const uint32_t (&xa)[16], const uint32_t (&xb)[16], int k0, float& mm) {
