@@ -25,7 +25,7 @@
 //               (kind::f16 in V's type, FP32 in TMEM, double-buffered);
 //   warps 0-7   softmax, two warps per query row (one per 64-key half of each block and per
 //               half of the output channels): z = S * tau / (genc_Q genc_K), causal mask,
-//               running max (the pair exchanges its block maxima through shared memory),
+//               running max (both warps of a row take it over all 128 scores of the block),
 //               p = exp2(z - m) written to shared memory in V's 16-bit type (K-major, 128-byte
 //               swizzle), running sum of the float32 p, and the fold O <- alpha O + PV in
 //               registers.
@@ -229,7 +229,6 @@ struct Smem {
   alignas(1024) T p[2][BM * BKV];    // 2 swizzle atoms of [BM rows][64 keys]
   alignas(128) uint8_t qsf[D / 64 * 512];
   alignas(128) uint8_t ksf[NST][D / 64 * 512];
-  float mx[2][2][BM];   // per block parity, per key half: the rows' block maxima (x c)
   float lsum[2][BM];    // per key half: the rows' final partial sums
   uint64_t q_full, k_full[NST], v_full[NST], kv_empty[NST];
   uint64_t s_full, s_free, p_full[2], pv_full[2], pv_free[2];
@@ -397,8 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSoftmaxRegs));
     // ---------------- softmax warps ----------------
     // Two warps per TMEM lane quarter: `half` 0 takes keys 0-63 of every block and output
-    // channels 0 .. D/2-1, half 1 keys 64-127 and channels D/2 .. D-1.  The pair shares each
-    // block's row maximum through shared memory; the row sums are combined at the end.
+    // channels 0 .. D/2-1, half 1 keys 64-127 and channels D/2 .. D-1.  The row sums are
+    // combined at the end through shared memory.
     const int quarter = warp & 3;
     const int half = warp >> 2;
     const int r = quarter * 32 + lane;
@@ -432,40 +431,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&sm.pv_free[jj & 1]);
     };
 
-    for (int j = 0; j < nb; ++j) {
+    // One 128-key block.  Both warps of a row read all 128 scores for the block maximum
+    // (identical on both: max does not depend on the order), so they need no exchange; each
+    // keeps only its own 64 for the exponentials.  MASK: the causal test, compiled only into
+    // the diagonal block's copy.
+    auto block = [&](int j, auto masked) {
+      constexpr bool MASK = decltype(masked)::value;
       const int b = j & 1;
-      const bool diag = args.causal && j == qt;
-      const int key0 = j * BKV + half * 64;
+      const int key0 = j * BKV + half * 64, okey0 = j * BKV + (half ^ 1) * 64;
       mbar_wait(&sm.s_full, j & 1, 220);
       tc_fence_after();
-      // this warp's 64 scores, read from TMEM once
       const uint32_t sa = lane_base + kColS + half * 64;
-      uint32_t x0[16], x1[16], x2[16], x3[16];
+      const uint32_t so = lane_base + kColS + (half ^ 1) * 64;
+      uint32_t x0[16], x1[16], x2[16], x3[16], y0[16], y1[16];
       tmem_ld16(sa, x0);
       tmem_ld16(sa + 16, x1);
       tmem_ld16(sa + 32, x2);
       tmem_ld16(sa + 48, x3);
+      tmem_ld16(so, y0);
+      tmem_ld16(so + 16, y1);
       tmem_ld_wait_regs(x0, x1);
       tmem_ld_wait_regs(x2, x3);
-      tc_fence_before();
-      mbar_arrive(&sm.s_free);
-      // block maximum of the raw scores over visible keys (c > 0 keeps the order)
+      tmem_ld_wait_regs(y0, y1);
       float m0 = -INFINITY, m1 = -INFINITY;
       auto maxh = [&](const uint32_t (&xa)[16], const uint32_t (&xb)[16], int k0, float& mm) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           float f0 = __uint_as_float(xa[e]), f1 = __uint_as_float(xb[e]);
-          if (diag && key0 + k0 + e > i) f0 = -INFINITY;
-          if (diag && key0 + k0 + 16 + e > i) f1 = -INFINITY;
+          if (MASK && k0 + e > i) f0 = -INFINITY;
+          if (MASK && k0 + 16 + e > i) f1 = -INFINITY;
           mm = fmax3(mm, f0, f1);
         }
       };
-      maxh(x0, x1, 0, m0);
-      maxh(x2, x3, 32, m1);
-      const float mine = fmaxf(m0, m1) * c;
-      sm.mx[b][half][r] = mine;
-      named_barrier_sync(pair_bar, 64);
-      const float mn = fmaxf(m, fmaxf(mine, sm.mx[b][half ^ 1][r]));
+      maxh(y0, y1, okey0, m1);
+      tmem_ld16(so + 32, y0);
+      tmem_ld16(so + 48, y1);
+      maxh(x0, x1, key0, m0);
+      maxh(x2, x3, key0 + 32, m0);
+      tmem_ld_wait_regs(y0, y1);
+      tc_fence_before();
+      mbar_arrive(&sm.s_free);
+      maxh(y0, y1, okey0 + 32, m1);
+      // block maximum of the raw scores over visible keys (c > 0 keeps the order)
+      const float mn = fmaxf(m, fmaxf(m0, m1) * c);
       const float alpha = ex2_approx(m - mn);
       // p = exp2(S c - mn) in V's type into this half's swizzle atom (64 keys), row sum
       float rs0 = 0.0f, rs1 = 0.0f;
@@ -476,11 +484,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
-            const int kk = k16 * 16 + q2 * 8 + e;  // key within this half
+            const int kk = key0 + k16 * 16 + q2 * 8 + e;
             float p0 = ex2_approx(fmaf(__uint_as_float(x[q2 * 8 + e]), c, -mn));
             float p1 = ex2_approx(fmaf(__uint_as_float(x[q2 * 8 + e + 1]), c, -mn));
-            if (diag && key0 + kk > i) p0 = 0.0f;
-            if (diag && key0 + kk + 1 > i) p1 = 0.0f;
+            if (MASK && kk > i) p0 = 0.0f;
+            if (MASK && kk + 1 > i) p1 = 0.0f;
             rs0 += p0;
             rs1 += p1;
             w[e / 2] = Cvt<T>::pack2(p0, p1);
@@ -500,6 +508,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (j > 0) fold_pv(j - 1, alpha_prev);
       alpha_prev = alpha;
       m = mn;
+    };
+    for (int j = 0; j < nb; ++j) {
+      if (args.causal && j == qt)
+        block(j, std::true_type{});
+      else
+        block(j, std::false_type{});
     }
     fold_pv(nb - 1, alpha_prev);
     // row sum over both halves (same order on both warps), then the epilogue: O / l in the
