@@ -110,3 +110,51 @@ def test_nvfp4_unsupported_qsmooth():
     cfg.qsmooth = True
     with pytest.raises(Exception, match="UNSUPPORTED"):
         nvfp4.quant_prologue(q, k, cfg)
+
+
+FULL = {
+    "sweep8192": [0, 511],   # the bench workload: B32 H16 N8192 d128 causal bf16
+    "llama325m": [0, 127],   # B8 H16 N2048 d64 causal bf16
+}
+
+
+@pytest.mark.parametrize("name", sorted(FULL))
+def test_nvfp4_full_size_sampled_heads(name):
+    """The whole batch in the launch configuration bench.py --variant nvfp4 times; sampled
+    (batch, head) pairs carry the seeded per-head inputs and are checked one head at a time
+    (each head is independent: its global scales, codes and outputs depend on it alone)."""
+    w = WORKLOADS[name]
+    heads = FULL[name]
+    dev = torch.device("cuda")
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+    g = torch.Generator(device=dev).manual_seed(2)
+    shape = (w.B * w.H, w.N, w.d)
+    t = {n: (torch.randn(shape, generator=g, device=dev) * w.sigma_qkv).to(dt)
+         for n in ("q", "k", "v")}
+    x = make_inputs(w, heads=heads)
+    for n in ("q", "k", "v"):
+        for i, bh in enumerate(heads):
+            t[n][bh] = torch.from_numpy(x[n][i].view(np.int16)).view(dt).to(dev)
+    q, k, v = (t[n].view(w.B, w.H, w.N, w.d) for n in ("q", "k", "v"))
+    cfg = _cfg(w)
+    fb = nvfp4.quant_prologue(q, k, cfg)
+    o, lse = nvfp4.attn_fwd(fb, v, cfg)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    N, d = w.N, w.d
+    u16 = 2.0 ** -8 if w.dtype == "bf16" else 2.0 ** -11
+    for i, bh in enumerate(heads):
+        one = [x[n + "_f32"][i:i + 1] for n in ("q", "k", "v")]
+        ref = F.qattn_forward(*one, causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth)
+        b_, h_ = divmod(bh, w.H)
+        for tname in ("q", "k"):
+            codes = unpack_codes(getattr(fb, tname + "_fp4")[b_, h_].cpu().numpy())
+            np.testing.assert_array_equal(codes, ref[tname + "_codes"][0], err_msg=tname)
+            sf = unpack_sf(getattr(fb, tname + "_sf")[b_, h_].cpu().numpy(), N, d)
+            np.testing.assert_array_equal(sf[0], ref[tname + "_sf"][0], err_msg=tname)
+            assert getattr(fb, tname + "_genc")[b_, h_].item() == ref[tname + "_genc"][0]
+        og = o[b_, h_].float().cpu().numpy().astype(np.float64)
+        err = np.abs(og - ref["o"][0])
+        tol = 2 * u16 * (ref["w"][0] + np.abs(ref["o"][0])) + 1e-5 * ref["w"][0] + 1e-7
+        assert not (err > tol).any(), f"head {bh}: {(err > tol).sum()} outside"
+        np.testing.assert_allclose(lse[b_, h_].cpu().numpy(), ref["lse"][0], rtol=0, atol=1e-4)
