@@ -9,8 +9,8 @@
 //               the result does not depend on the order of the atomics);
 //   quant pass  genc = 2688 / G (1 when G = 0); per 16 channels: a = max|x|,
 //               u = (a * genc) / 6, sd = e4m3(u) (nearest, ties to even, saturating at 448),
-//               code = e2m1(x * (genc / sd)) (nearest, ties to even, saturating at 6; +0 for
-//               values that round to zero); every step a correctly rounded float32 operation.
+//               code = e2m1(x * (genc / sd)) (nearest, ties to even, saturating at 6, the sign
+//               bit the product's); every step a correctly rounded float32 operation.
 // Outputs: codes [BH, N, d/2] (channel 2i in the low nibble of byte i), block scales in the
 // tensor core's scale-factor order (per 128-row tile and 64-channel chunk, 512 bytes: byte
 // (r % 32) * 16 + (r / 32) * 4 + b holds row r's scale of the chunk's 16-channel block b), and
@@ -71,15 +71,17 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
   return e == 0 ? static_cast<float>(m) * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
-// E2M1 code (bit 3 = sign): the number of rounding boundaries |y| has passed; midpoints go to
-// the even code (0.25 -> 0, 0.75 -> 1.0, 1.25 -> 1.0, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4).
-__device__ __forceinline__ uint32_t e2m1_code(float y) {
-  const float a = fabsf(y);
-  const uint32_t m = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
-                     static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
-                     static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) +
-                     static_cast<uint32_t>(a > 5.0f);
-  return (y < 0.0f && m != 0u) ? (m | 8u) : m;
+// Two E2M1 codes in one byte (lo in bits 0-3, hi in bits 4-7) by the hardware conversion:
+// round to nearest, ties to even, saturating at +-6, the sign bit that of the input (a
+// negative value that rounds to zero gives -0, code 8).
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(lo), "f"(hi));
+  return r;
 }
 
 constexpr float kGlobalRange = 2688.0f;  // 6 (largest E2M1) * 448 (largest E4M3)
@@ -197,7 +199,8 @@ __global__ void __launch_bounds__(kQuantThreads, 2) prologue_quant_kernel(Prolog
     const float mult = sd > 0.0f ? __fdiv_rn(genc, sd) : 0.0f;
     uint32_t w = 0;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) w |= e2m1_code(__fmul_rn(x[s][c], mult)) << (4 * c);
+    for (int c = 0; c < 8; c += 2)
+      w |= e2m1x2(__fmul_rn(x[s][c], mult), __fmul_rn(x[s][c + 1], mult)) << (4 * c);
     const int r = warp * RPW + s * GPW + grp;
     *reinterpret_cast<uint32_t*>(codes + (row0 + r) * (D / 2) + sub * 4) = w;
     if ((sub & 1) == 0) sf_tile[(r & 31) * 16 + (r >> 5) * 4] = static_cast<uint8_t>(sc);

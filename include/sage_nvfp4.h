@@ -14,7 +14,8 @@
  *   block  a = max |x| over 16 channels; u = (a * genc) / 6;
  *          sd = E4M3(u): round to nearest, ties to even, subnormals, 448 and above -> 448;
  *          code = E2M1(x * (genc / sd)): magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}, nearest, ties
- *          to the even code, above 6 -> 6, values rounding to zero -> +0; sd == 0 -> code 0.
+ *          to the even code, above 6 -> 6, the sign bit that of the product (a negative value
+ *          rounding to zero gives -0, code 8); sd == 0 -> genc / sd taken as 0 (codes +-0).
  *   value  E2M1(code) * sd / genc.
  *
  * Conventions are those of sage.h (device pointers owned by the caller, 16-byte alignment,

@@ -15,8 +15,9 @@ What it follows:
 Readings (the pages fix neither rounding rules nor the global scale's extent):
 
 * E2M1 magnitudes are {0, 0.5, 1, 1.5, 2, 3, 4, 6}; rounding is to nearest, ties to the code
-  with an even low bit, and magnitudes above 6 saturate to 6.  A value that rounds to zero
-  gets the +0 code.  (``e2m1_encode``)
+  with an even low bit, and magnitudes above 6 saturate to 6.  The sign bit is the input's, so
+  a negative value (or -0) that rounds to zero gets the -0 code 8, as IEEE rounding keeps the
+  sign of a result that rounds to zero.  (``e2m1_encode``)
 * Block scales are unsigned E4M3 (4 exponent bits, bias 7, 3 mantissa bits, subnormals,
   largest finite 448): round to nearest, ties to even, values of 448 and above saturate to 448.
   (``e4m3_encode``)
@@ -25,7 +26,8 @@ Readings (the pages fix neither rounding rules nor the global scale's extent):
   times an element can reach: ``genc = 2688 / G`` (``genc = 1`` when G = 0).
 * Per block of 16 consecutive channels, in float32 with IEEE rounding at every step:
   ``a = max |x|``, ``u = (a * genc) / 6``, ``sd = e4m3(u)`` (the stored scale),
-  ``mult = genc / sd`` and ``code = e2m1(x * mult)``; ``sd = 0`` gives all-zero codes.
+  ``mult = genc / sd`` and ``code = e2m1(x * mult)``; ``sd = 0`` gives codes of value zero
+  (``mult = 0``, so +0 or -0 by the sign of x).
   The value a code stands for is ``e2m1_value(code) * sd / genc``.
 * Q and K are quantized along the head dimension (the contraction of Q K^T), after the same
   QK-norm and K-smoothing as the INT8 recipe (``sage_oracle.rms_norm_rows_f32``,
@@ -55,13 +57,14 @@ def e2m1_encode(y: np.ndarray) -> np.ndarray:
 
     The magnitude code counts the rounding boundaries ``|y|`` has passed.  Between two
     neighbours the midpoint goes to the one whose code is even: 0.25 -> 0, 0.75 -> 1,
-    1.25 -> 1, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4 (codes 0, 2, 2, 4, 4, 6, 6).
+    1.25 -> 1, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4 (codes 0, 2, 2, 4, 4, 6, 6).  The sign
+    bit is the sign bit of ``y`` (so -0.1 and -0.0 give the -0 code 8).
     """
-    a = np.abs(np.asarray(y, dtype=F32))
+    y = np.asarray(y, dtype=F32)
+    a = np.abs(y)
     mag = ((a > 0.25).astype(np.uint8) + (a >= 0.75) + (a > 1.25) + (a >= 1.75) + (a > 2.5)
            + (a >= 3.5) + (a > 5.0)).astype(np.uint8)
-    neg = (np.asarray(y, dtype=F32) < 0) & (mag > 0)
-    return (mag | (neg.astype(np.uint8) << 3)).astype(np.uint8)
+    return (mag | (np.signbit(y).astype(np.uint8) << 3)).astype(np.uint8)
 
 
 def e2m1_decode(code: np.ndarray) -> np.ndarray:

@@ -35,7 +35,7 @@ def test_e2m1_decode_matches_bit_format():
 
 
 def _e2m1_brute(y):
-    """Nearest grid magnitude, ties to the even code, above 6 -> 6; sign kept unless zero."""
+    """Nearest grid magnitude, ties to the even code, above 6 -> 6; the sign bit is y's."""
     a = abs(float(y))
     if a >= 6.0:
         mag = 7
@@ -43,7 +43,7 @@ def _e2m1_brute(y):
         d = np.abs(F.E2M1_VALUES - a)
         best = np.flatnonzero(d == d.min())
         mag = int(best[0]) if len(best) == 1 else int([b for b in best if b % 2 == 0][0])
-    return mag | (8 if (y < 0 and mag > 0) else 0)
+    return mag | (8 if np.signbit(np.float32(y)) else 0)
 
 
 def test_e2m1_encode_brute_force():
@@ -59,6 +59,8 @@ def test_e2m1_ties_and_saturation():
     ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
     assert F.e2m1_decode(F.e2m1_encode(ties)).tolist() == [0, 1, 1, 2, 2, 4, 4]
     assert F.e2m1_encode(np.array([7.0, 100.0, -6.5], np.float32)).tolist() == [7, 7, 15]
+    # rounding to zero keeps the sign, as IEEE rounding does
+    assert F.e2m1_encode(np.array([0.1, -0.1, 0.0, -0.0], np.float32)).tolist() == [0, 8, 0, 8]
 
 
 # ------------------------------------------------------------------------------------------
@@ -125,9 +127,8 @@ def test_nvfp4_planted_round_trip():
     r = F.nvfp4_quantize(x)
     assert np.all(r["genc"] == 1.0)
     assert np.array_equal(r["sf"], sf)
-    # -0 codes (sign bit with magnitude 0) come back as +0
-    want = np.where((codes & 7) == 0, 0, codes)
-    assert np.array_equal(r["codes"], want)
+    # every planted code comes back, -0 (code 8) included
+    assert np.array_equal(r["codes"], codes)
     assert np.array_equal(F.nvfp4_dequantize(r["codes"], r["sf"], r["genc"]), x)
 
 
@@ -234,7 +235,7 @@ def test_planted_mistakes_are_caught(monkeypatch):
         a = np.abs(np.asarray(y, np.float32))
         mag = ((a >= 0.25).astype(np.uint8) + (a >= 0.75) + (a >= 1.25) + (a >= 1.75)
                + (a >= 2.5) + (a >= 3.5) + (a >= 5.0)).astype(np.uint8)
-        return (mag | (((np.asarray(y) < 0) & (mag > 0)).astype(np.uint8) << 3)).astype(np.uint8)
+        return (mag | (np.signbit(np.asarray(y, np.float32)).astype(np.uint8) << 3)).astype(np.uint8)
 
     with monkeypatch.context() as m:
         m.setattr(F, "e2m1_encode", ties_up)
