@@ -243,8 +243,10 @@ def run_nvfp4(args, w):
     p_bf16 = pk["bf16_sustained"]
     p_fwd = 1.0 / (0.5 / (4.0 * p_bf16) + 0.5 / p_bf16)
     achieved = fwd_ops / (fwd_ms * 1e-3) / 1e12
+    traffic = (traffic_per_launch("fp4::attn_fwd_kernel", "fwd_bwd_b200/csrc/nvfp4.cuh")
+               if w.name == "sweep8192" and w.B == 32 else None)
     roofline = {"bound": "tensor", "kernel": "fp4::attn_fwd_kernel", "achieved": achieved,
-                "peak": p_fwd, "unit": "TFLOP/s", "frac": achieved / p_fwd, "traffic": None,
+                "peak": p_fwd, "unit": "TFLOP/s", "frac": achieved / p_fwd, "traffic": traffic,
                 "peak_note": f"{pk['basis']} sustained bf16; NVFP4 = 4x bf16, weighted 1:1 "
                              f"with the 16-bit P V"}
     e2e = None
