@@ -158,3 +158,55 @@ def test_nvfp4_full_size_sampled_heads(name):
         tol = 2 * u16 * (ref["w"][0] + np.abs(ref["o"][0])) + 1e-5 * ref["w"][0] + 1e-7
         assert not (err > tol).any(), f"head {bh}: {(err > tol).sum()} outside"
         np.testing.assert_allclose(lse[b_, h_].cpu().numpy(), ref["lse"][0], rtol=0, atol=1e-4)
+
+
+def _degenerate_inputs(kind, BH=2, N=256, d=128):
+    rng = np.random.default_rng(11)
+    q, k, v = (rng.standard_normal((BH, N, d)).astype(np.float32) for _ in range(3))
+    if kind == "zero_head":        # G = 0 for head 0: genc = 1, zero scales, uniform attention
+        q[0] = 0.0
+        k[0] = 0.0
+    elif kind == "wide_range":     # rows from 2^-20 to 2^4: subnormal and zero E4M3 scales
+        q *= np.exp2(rng.uniform(-20, 4, (BH, N, 1))).astype(np.float32)
+        k *= np.exp2(rng.uniform(-20, 4, (BH, N, 1))).astype(np.float32)
+    elif kind == "fp16_large":     # fp16 near its largest values (|x| up to ~3e4 of 65504)
+        q *= 6000.0
+        k *= 3000.0
+    return q, k, v
+
+
+@pytest.mark.parametrize("kind,dtype,qknorm", [("zero_head", "bf16", True),
+                                              ("zero_head", "bf16", False),
+                                              ("wide_range", "bf16", False),
+                                              ("fp16_large", "fp16", False)])
+def test_nvfp4_degenerate(kind, dtype, qknorm):
+    q, k, v = _degenerate_inputs(kind)
+    BH, N, d = q.shape
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    tq, tk, tv = (torch.from_numpy(a).to(tdt) for a in (q, k, v))
+    qf, kf, vf = (t.float().numpy() for t in (tq, tk, tv))  # exact 16-bit values
+    assert np.isfinite(qf).all() and np.isfinite(kf).all()
+    cfg = ops.Config(causal=True, qknorm=qknorm, ksmooth=True)
+    dev = torch.device("cuda")
+    shape = (1, BH, N, d)
+    fb = nvfp4.quant_prologue(tq.reshape(shape).to(dev), tk.reshape(shape).to(dev), cfg)
+    o, lse = nvfp4.attn_fwd(fb, tv.reshape(shape).to(dev), cfg)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    ref = F.qattn_forward(qf, kf, vf, causal=True, qknorm=qknorm, ksmooth=True)
+    for t in ("q", "k"):
+        codes = unpack_codes(getattr(fb, t + "_fp4").cpu().numpy().reshape(BH, N, d // 2))
+        np.testing.assert_array_equal(codes, ref[t + "_codes"], err_msg=t)
+        np.testing.assert_array_equal(unpack_sf(getattr(fb, t + "_sf").cpu().numpy(), N, d),
+                                      ref[t + "_sf"], err_msg=t)
+        np.testing.assert_array_equal(getattr(fb, t + "_genc").cpu().numpy().reshape(BH),
+                                      ref[t + "_genc"], err_msg=t)
+    if kind == "wide_range":  # the case exercises subnormal and zero block scales (Q is not
+        # smoothed; K-smoothing lifts K's small rows to the mean's size)
+        assert (ref["q_sf"] < 8).any() and (ref["q_sf"] == 0).any()
+    u16 = 2.0 ** -8 if dtype == "bf16" else 2.0 ** -11
+    og = o.float().cpu().numpy().astype(np.float64).reshape(BH, N, d)
+    tol = 2 * u16 * (ref["w"] + np.abs(ref["o"])) + 1e-5 * ref["w"] + 1e-7
+    assert not (np.abs(og - ref["o"]) > tol).any()
+    # fp16_large has scores near 1e8: float32 rounding of S and of S * c is relative there
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(BH, N), ref["lse"], rtol=2e-6, atol=1e-4)
