@@ -35,6 +35,11 @@ Readings (the pages fix neither rounding rules nor the global scale's extent):
 * Forward: scores from the dequantized operands (exact in float64), softmax and
   ``O = softmax(z) V`` in float64.  The kernel feeds P to the tensor core in BF16; the oracle
   keeps P exact, and the tests bound the difference that BF16 rounding of P can make.
+* Backward (``qattn_bwd_head``): S recomputed from the same views, ``dP = dO V^T`` and
+  ``dV = P^T dO`` from 16-bit operands, ``dS = P o (dP - D)``; dS is quantized per 128 x 128
+  tile with the tile's maximum as its global scale, in 16-key blocks for ``dQ = tau dS K`` and
+  in 16-query blocks for ``dK = tau dS^T Q``, whose K and Q operands are NVFP4 views along the
+  sequence (blocks of 16 tokens, one global scale per head).
 """
 from __future__ import annotations
 
@@ -146,6 +151,7 @@ def qattn_prologue(q, k, *, qknorm: bool, ksmooth: bool, eps: float = 1e-6,
     if qknorm:
         qh, out["q_inv_rms"] = S8.rms_norm_rows_f32(qh, eps)
         kh, out["k_inv_rms"] = S8.rms_norm_rows_f32(kh, eps)
+    out["k_hat"] = kh
     if ksmooth:
         kh, out["k_mean"] = S8.k_smooth_f32(kh, k_block)
     out["q_hat"], out["k_tilde"] = qh, kh
@@ -194,3 +200,117 @@ def qattn_forward(q, k, v, *, causal: bool, qknorm: bool, ksmooth: bool,
         o[h], lse[h], w[h] = qattn_fwd_head(qd[h], kd[h], v[h], causal=causal, tau=tau)
     pro.update(o=o, lse=lse, w=w, q_deq=qd, k_deq=kd)
     return pro
+
+
+# ----------------------------------------------------------------------------------------------
+# Backward (Full-Stack FP4 section 2.4: dS in NVFP4, P^T dO and dO V^T in BF16)
+# ----------------------------------------------------------------------------------------------
+def nvfp4_quantize_tile(x: np.ndarray, axis: int) -> np.ndarray:
+    """Dequantized NVFP4 value of a tile ``x`` (2-D, float32) with ONE global scale for the
+    whole tile and blocks of 16 along ``axis``; same float32 steps as ``nvfp4_quantize``.
+
+    Reading (the pages fix no granularity for the operand made inside the backward): dS is
+    quantized per 128 x 128 (query, key) tile -- the unit the kernel holds -- with the tile's
+    absolute maximum as its global scale, so that both orientations (16-key blocks for
+    ``dQ = dS K``, 16-query blocks for ``dK = dS^T Q``) share it.
+    """
+    x = np.asarray(x, F32)
+    t = np.moveaxis(x, axis, -1)[None]
+    r = nvfp4_quantize(t)
+    deq = nvfp4_dequantize(r["codes"], r["sf"], r["genc"])[0]
+    return np.moveaxis(deq, -1, axis)
+
+
+def qattn_bwd_head(qd, kd, q_seq, k_seq, v, o, lse, do, *, causal: bool, tau: float,
+                   quant: bool = True, tile: int = 128) -> tuple:
+    """Backward of one head: returns ``(dQhat, dKtilde, dV)`` float64 ``[N, d]``.
+
+    ``qd``/``kd``: the forward's dequantized NVFP4 views (along d); ``q_seq``/``k_seq``: the
+    dequantized NVFP4 views along the sequence (blocks of 16 tokens, ``nvfp4_quantize`` of the
+    transposed matrix, one global scale per head) -- the K-major operands of dQ and dK; ``v``,
+    ``do``: exact 16-bit inputs; ``o``, ``lse``: the forward's outputs.  Steps:
+
+    1. ``z = tau qd kd^T`` (causal mask), ``P = exp(z - LSE)``;
+    2. ``dP = dO V^T`` (16-bit operands, exact products), ``D_i = sum_c dO_ic O_ic``,
+       ``dS = P o (dP - D)``;
+    3. per 128 x 128 tile, dS (rounded to float32, the kernel's precision) is quantized twice
+       with the tile's global scale: in 16-key blocks (``dS_k``) and in 16-query blocks
+       (``dS_q``) -- ``nvfp4_quantize_tile``;
+    4. ``dV = P^T dO`` (16-bit operands: P exact here, the tests bound its BF16 rounding),
+       ``dQ = tau dS_k k_seq``, ``dK = tau dS_q^T q_seq``.
+
+    With ``quant=False`` every quantizer is the identity (``qd = q_seq`` = the exact Q etc.),
+    which is plain attention's gradient.  The gradient for K is the one for the smoothed K,
+    which equals the one for the normalized K (every row of dS sums to zero).
+    """
+    qd, kd, q_seq, k_seq, v, o, do = (np.asarray(t, F64) for t in (qd, kd, q_seq, k_seq, v, o, do))
+    N, d = qd.shape
+    z = (qd @ kd.T) * tau
+    if causal:
+        z = np.where(np.arange(N)[None, :] > np.arange(N)[:, None], -np.inf, z)
+    P = np.exp(z - np.asarray(lse, F64)[:, None])
+    dP = do @ v.T
+    D = (do * o).sum(axis=1)
+    dS = P * (dP - D[:, None])
+    dV = P.T @ do
+    if quant:
+        dS_k = np.zeros_like(dS)
+        dS_q = np.zeros_like(dS)
+        for i0 in range(0, N, tile):
+            for j0 in range(0, N, tile):
+                t = dS[i0:i0 + tile, j0:j0 + tile].astype(F32)
+                dS_k[i0:i0 + tile, j0:j0 + tile] = nvfp4_quantize_tile(t, axis=1)
+                dS_q[i0:i0 + tile, j0:j0 + tile] = nvfp4_quantize_tile(t, axis=0)
+    else:
+        dS_k = dS_q = dS
+    dQ = (dS_k @ k_seq) * tau
+    dK = (dS_q.T @ q_seq) * tau
+    return dQ, dK, dV
+
+
+def qattn_attention(q, k, v, do, *, causal: bool, qknorm: bool, ksmooth: bool,
+                    tau: float | None = None, eps: float = 1e-6,
+                    quant: bool = True) -> Dict[str, np.ndarray]:
+    """NVFP4 Q-Attn forward and backward over every (batch, head).
+
+    Inputs float32 ``[BH, N, d]`` (exact 16-bit values).  Returns the forward's results
+    (``qattn_forward``) plus ``dq, dk, dv`` with respect to the raw q, k, v (RMSNorm backward
+    applied when ``qknorm``).  ``quant=False``: full precision (float64, no quantizer).
+    """
+    q, k, v, do = (np.asarray(t, F32) for t in (q, k, v, do))
+    BH, N, d = q.shape
+    tau = 1.0 / np.sqrt(d) if tau is None else tau
+    if quant:
+        res = qattn_forward(q, k, v, causal=causal, qknorm=qknorm, ksmooth=ksmooth, tau=tau,
+                            eps=eps)
+        qs = nvfp4_quantize(np.swapaxes(res["q_hat"], -1, -2))
+        ks = nvfp4_quantize(np.swapaxes(res["k_tilde"], -1, -2))
+        q_seq = np.swapaxes(nvfp4_dequantize(qs["codes"], qs["sf"], qs["genc"]), -1, -2)
+        k_seq = np.swapaxes(nvfp4_dequantize(ks["codes"], ks["sf"], ks["genc"]), -1, -2)
+        res.update(q_seq=q_seq, k_seq=k_seq)
+        qd, kd = res["q_deq"], res["k_deq"]
+    else:
+        pro = S8.prologue_fp64(q, k, v, qknorm=qknorm, ksmooth=ksmooth, eps=eps)
+        res = {"q_hat": pro["q_hat"], "k_hat": pro["k_hat"], "k_tilde": pro["k_tilde"]}
+        if qknorm:
+            res.update(q_inv_rms=pro["q_inv_rms"], k_inv_rms=pro["k_inv_rms"])
+        qd = q_seq = pro["q_hat"]
+        kd = k_seq = pro["k_tilde"]
+        o = np.zeros((BH, N, d))
+        lse = np.zeros((BH, N))
+        for h in range(BH):
+            o[h], lse[h], _ = qattn_fwd_head(qd[h], kd[h], v[h], causal=causal, tau=tau)
+        res.update(o=o, lse=lse)
+    dq = np.zeros((BH, N, d))
+    dk = np.zeros((BH, N, d))
+    dv = np.zeros((BH, N, d))
+    for h in range(BH):
+        dqh, dkh, dv[h] = qattn_bwd_head(qd[h], kd[h], q_seq[h], k_seq[h], v[h], res["o"][h],
+                                         res["lse"][h], do[h], causal=causal, tau=tau,
+                                         quant=quant)
+        if qknorm:  # the RMSNorm backward takes the normalized (unsmoothed) rows
+            dqh = S8.rms_norm_bwd(dqh, res["q_hat"][h], res["q_inv_rms"][h])
+            dkh = S8.rms_norm_bwd(dkh, res["k_hat"][h], res["k_inv_rms"][h])
+        dq[h], dk[h] = dqh, dkh
+    res.update(dq=dq, dk=dk, dv=dv, tau=tau)
+    return res

@@ -284,3 +284,124 @@ def test_planted_mistakes_are_caught(monkeypatch):
         m.setattr(F, "qattn_fwd_head", dropped_tau)
         assert _fails(test_qattn_forward_exact_inputs_equal_plain_attention)
     assert F.e2m1_encode is real_e2m1 and F.e4m3_encode is real_e4m3
+
+
+# ------------------------------------------------------------------------------------------
+# Backward
+# ------------------------------------------------------------------------------------------
+def _torch_grads(q, k, v, do, causal, qknorm, ksmooth, tau=None):
+    t = [torch.tensor(a.astype(np.float64), requires_grad=True) for a in (q, k, v)]
+    qq, kk = t[0], t[1]
+    if qknorm:
+        qq = qq * torch.rsqrt((qq * qq).mean(-1, keepdim=True) + 1e-6)
+        kk = kk * torch.rsqrt((kk * kk).mean(-1, keepdim=True) + 1e-6)
+    if ksmooth:
+        kk = kk - kk.mean(-2, keepdim=True)
+    o = torch.nn.functional.scaled_dot_product_attention(qq, kk, t[2], is_causal=causal,
+                                                         scale=tau)
+    o.backward(torch.tensor(do.astype(np.float64)))
+    return o.detach().numpy(), [g.grad.numpy() for g in t]
+
+
+@pytest.mark.parametrize("causal,qknorm,ksmooth", [(True, True, True), (False, False, False),
+                                                   (True, False, True), (False, True, False)])
+def test_qattn_bwd_full_precision_vs_torch_autograd(causal, qknorm, ksmooth):
+    rng = np.random.default_rng(21)
+    q, k, v, do = (rng.standard_normal((2, 256, 64)).astype(np.float32) for _ in range(4))
+    k += 2.0 * rng.standard_normal((2, 1, 64)).astype(np.float32)
+    r = F.qattn_attention(q, k, v, do, causal=causal, qknorm=qknorm, ksmooth=ksmooth,
+                          quant=False)
+    o, grads = _torch_grads(q, k, v, do, causal, qknorm, ksmooth)
+    assert np.allclose(r["o"], o, rtol=0, atol=1e-12)
+    for name, g in zip(("dq", "dk", "dv"), grads):
+        assert np.allclose(r[name], g, rtol=0, atol=1e-11), name
+
+
+def _quant_tile_brute(t, axis):
+    """Per-tile NVFP4 of a float32 tile, element loops (blocks of 16 along `axis`)."""
+    G = float(np.max(np.abs(t)))
+    genc = np.float32(2688.0) / np.float32(G) if G > 0 else np.float32(1.0)
+    out = np.zeros(t.shape, np.float64)
+    tt = t if axis == 1 else t.T
+    res = np.zeros(tt.shape, np.float64)
+    for r in range(tt.shape[0]):
+        for b0 in range(0, tt.shape[1], 16):
+            blk = tt[r, b0:b0 + 16]
+            a = np.float32(np.max(np.abs(blk)))
+            u = np.float32(np.float32(a * genc) / np.float32(6.0))
+            sd = np.float32(F.e4m3_decode(F.e4m3_encode(np.array([u], np.float32)))[0])
+            mult = np.float32(genc / sd) if sd > 0 else np.float32(0.0)
+            for c in range(16):
+                code = F.e2m1_encode(np.array([np.float32(blk[c] * mult)], np.float32))[0]
+                res[r, b0 + c] = F.e2m1_decode(np.array([code]))[0] * float(sd) / float(genc)
+    out[:] = res if axis == 1 else res.T
+    return out
+
+
+def test_qattn_bwd_tile_quantizer_brute_force():
+    rng = np.random.default_rng(22)
+    t = (rng.standard_normal((128, 128)) * np.exp(rng.uniform(-4, 2, (128, 1)))).astype(np.float32)
+    for axis in (0, 1):
+        assert np.array_equal(F.nvfp4_quantize_tile(t, axis), _quant_tile_brute(t, axis)), axis
+
+
+def test_qattn_bwd_quantized_products_brute_force():
+    """One 128-key tile, d = 32: dQ and dK from explicit sums over the brute-force quantized
+    dS (16-key blocks for dQ, 16-query blocks for dK) and the sequence views."""
+    rng = np.random.default_rng(23)
+    N, d, tau = 128, 32, 0.25
+    q, k, v, do = (rng.standard_normal((1, N, d)).astype(np.float32) for _ in range(4))
+    r = F.qattn_attention(q, k, v, do, causal=True, qknorm=False, ksmooth=False, tau=tau)
+    z = (r["q_deq"][0] @ r["k_deq"][0].T) * tau
+    z = np.where(np.arange(N)[None, :] > np.arange(N)[:, None], -np.inf, z)
+    P = np.exp(z - r["lse"][0][:, None])
+    dS = P * (do[0].astype(np.float64) @ v[0].T.astype(np.float64)
+              - (do[0] * r["o"][0]).sum(1)[:, None])
+    dS32 = dS.astype(np.float32)
+    dSk, dSq = _quant_tile_brute(dS32, 1), _quant_tile_brute(dS32, 0)
+    dq = np.zeros((N, d))
+    dk = np.zeros((N, d))
+    for i in range(N):
+        for j in range(N):
+            dq[i] += dSk[i, j] * r["k_seq"][0][j]
+            dk[j] += dSq[i, j] * r["q_seq"][0][i]
+    assert np.allclose(r["dq"][0], dq * tau, rtol=1e-12, atol=1e-12)
+    assert np.allclose(r["dk"][0], dk * tau, rtol=1e-12, atol=1e-12)
+    assert np.allclose(r["dv"][0], P.T @ do[0].astype(np.float64), rtol=1e-12, atol=1e-12)
+
+
+def test_qattn_bwd_close_to_full_precision():
+    rng = np.random.default_rng(24)
+    q, k, v, do = (rng.standard_normal((2, 256, 128)).astype(np.float32) for _ in range(4))
+    k += 3.0 * rng.standard_normal((2, 1, 128)).astype(np.float32)
+    kw = dict(causal=True, qknorm=True, ksmooth=True)
+    qm = F.qattn_attention(q, k, v, do, **kw)
+    xm = F.qattn_attention(q, k, v, do, quant=False, **kw)
+    cos = lambda a, b: (a * b).sum() / np.sqrt((a * a).sum() * (b * b).sum())  # noqa: E731
+    for n in ("o", "dq", "dk", "dv"):
+        assert cos(qm[n], xm[n]) > 0.98, n
+
+
+def test_qattn_bwd_planted_mistakes_are_caught(monkeypatch):
+    real_tile = F.nvfp4_quantize_tile
+
+    def wrong_axis(x, axis):  # dS quantized along the other axis
+        return real_tile(x, 1 - axis)
+
+    with monkeypatch.context() as m:
+        m.setattr(F, "nvfp4_quantize_tile", wrong_axis)
+        assert _fails(test_qattn_bwd_quantized_products_brute_force)
+    real_bwd = F.qattn_bwd_head
+
+    def dropped_tau_dk(*a, **kw):
+        dq, dk, dv = real_bwd(*a, **kw)
+        return dq, dk / kw["tau"], dv
+
+    def transposed_ds(*a, **kw):
+        dq, dk, dv = real_bwd(*a, **kw)
+        return dq, dk[::-1], dv
+
+    for fake in (dropped_tau_dk, transposed_ds):
+        with monkeypatch.context() as m:
+            m.setattr(F, "qattn_bwd_head", fake)
+            assert _fails(test_qattn_bwd_full_precision_vs_torch_autograd, True, True, True)
