@@ -39,7 +39,7 @@ class SageQBufs(ctypes.Structure):
 class SageFp4Bufs(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("q_fp4", "k_fp4", "q_sf", "k_sf", "q_genc", "k_genc", "q_inv_rms",
-                 "k_inv_rms", "k_mean")]
+                 "k_inv_rms", "k_mean", "q_fp4_t", "k_fp4_t", "q_sf_t", "k_sf_t")]
 
 
 class SageError(RuntimeError):

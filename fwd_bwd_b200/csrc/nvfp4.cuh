@@ -97,9 +97,18 @@ struct PrologueArgs {
   float* inv_rms[2];      // [BH, N] (qknorm)
   const float* k_mean;    // [BH, D] (ksmooth)
   uint32_t* gmax;         // [2, BH] float bits, zeroed before the amax pass
+  uint8_t* codes_t[2];    // sequence views (or null): [BH, D, N/2], 16-token blocks per channel
+  uint8_t* sf_t[2];       // [BH, ceil(D/128), N/64, 512]
   int BH, N, qknorm, ksmooth;
   float eps;
 };
+
+// Shared memory of the quantization pass when it also writes the sequence views: the chunk's
+// normalized, smoothed values (128 tokens x D channels, rows padded by one float).
+template <int D>
+constexpr size_t seq_smem_bytes() {
+  return static_cast<size_t>(kRowsPerCta) * (D + 1) * sizeof(float);
+}
 
 // The rows of one 128-row chunk, normalized and smoothed exactly as the INT8 prologue does.
 template <typename T, int D, int STEPS, int RPW, int GPW>
@@ -204,6 +213,50 @@ __global__ void __launch_bounds__(kQuantThreads, 2) prologue_quant_kernel(Prolog
     const int r = warp * RPW + s * GPW + grp;
     *reinterpret_cast<uint32_t*>(codes + (row0 + r) * (D / 2) + sub * 4) = w;
     if ((sub & 1) == 0) sf_tile[(r & 31) * 16 + (r >> 5) * 4] = static_cast<uint8_t>(sc);
+  }
+  uint8_t* codes_t = which == 0 ? a.codes_t[0] : a.codes_t[1];
+  if (codes_t == nullptr) return;
+  // Sequence views: the same values quantized in blocks of 16 tokens per channel (the global
+  // scale is the matrix maximum, as for the row views).  Item (channel c, block tb) of the
+  // chunk: codes of tokens 16 tb .. 16 tb + 15 at row c, scale at the channel's atom row.
+  extern __shared__ float tile[];  // [kRowsPerCta][D + 1]
+#pragma unroll
+  for (int s = 0; s < STEPS; ++s) {
+    const int r = warp * RPW + s * GPW + grp;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) tile[r * (D + 1) + sub * 8 + c] = x[s][c];
+  }
+  __syncthreads();
+  uint8_t* sf_t = which == 0 ? a.sf_t[0] : a.sf_t[1];
+  constexpr int NTB = kRowsPerCta / 16;  // token blocks per chunk
+  constexpr int NCG = (D + 127) / 128;   // 128-channel groups (scale atoms)
+  const int nq64 = a.N / 64;
+#pragma unroll
+  for (int item = threadIdx.x; item < D * NTB; item += kQuantThreads) {
+    const int c = item / NTB, tb = item % NTB;
+    float v[16];
+    float am = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      v[e] = tile[(tb * 16 + e) * (D + 1) + c];
+      am = fmaxf(am, fabsf(v[e]));
+    }
+    const float u = __fdiv_rn(__fmul_rn(am, genc), 6.0f);
+    const uint32_t sc = e4m3_code(u);
+    const float sd = e4m3_value(sc);
+    const float mult = sd > 0.0f ? __fdiv_rn(genc, sd) : 0.0f;
+    uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      w0 |= e2m1x2(__fmul_rn(v[e], mult), __fmul_rn(v[e + 1], mult)) << (4 * e);
+      w1 |= e2m1x2(__fmul_rn(v[8 + e], mult), __fmul_rn(v[9 + e], mult)) << (4 * e);
+    }
+    const int t0 = ch * kRowsPerCta + tb * 16;  // first token of the block
+    *reinterpret_cast<uint2*>(codes_t + (static_cast<size_t>(bh) * D + c) * (a.N / 2) + t0 / 2) =
+        make_uint2(w0, w1);
+    const size_t atom = (static_cast<size_t>(bh) * NCG + c / 128) * nq64 + t0 / 64;
+    sf_t[atom * 512 + (c & 31) * 16 + ((c & 127) >> 5) * 4 + ((t0 >> 4) & 3)] =
+        static_cast<uint8_t>(sc);
   }
 }
 

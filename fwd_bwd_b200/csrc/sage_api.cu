@@ -328,8 +328,12 @@ int check_fp4bufs(const sage_params* p, const sage_fp4_bufs* fb) {
   if (!fb || !fb->q_fp4 || !fb->k_fp4 || !fb->q_sf || !fb->k_sf || !fb->q_genc || !fb->k_genc)
     return SAGE_ERR_INVALID_ARG;
   if (p->ksmooth && !fb->k_mean) return SAGE_ERR_INVALID_ARG;
+  if ((fb->q_fp4_t == nullptr) != (fb->q_sf_t == nullptr) ||
+      (fb->k_fp4_t == nullptr) != (fb->k_sf_t == nullptr))
+    return SAGE_ERR_INVALID_ARG;
   const void* ptrs[] = {fb->q_fp4, fb->k_fp4, fb->q_sf, fb->k_sf, fb->q_genc, fb->k_genc,
-                        fb->k_mean, fb->q_inv_rms, fb->k_inv_rms};
+                        fb->k_mean, fb->q_inv_rms, fb->k_inv_rms, fb->q_fp4_t, fb->k_fp4_t,
+                        fb->q_sf_t, fb->k_sf_t};
   for (const void* ptr : ptrs)
     if (ptr && !aligned16(ptr)) return SAGE_ERR_ALIGNMENT;
   return SAGE_OK;
@@ -376,6 +380,10 @@ int run_fp4_prologue(const sage_params* p, const void* q, const void* k, const s
   a.inv_rms[1] = fb->k_inv_rms;
   a.k_mean = fb->k_mean;
   a.gmax = gmax;
+  a.codes_t[0] = fb->q_fp4_t;
+  a.codes_t[1] = fb->k_fp4_t;
+  a.sf_t[0] = fb->q_sf_t;
+  a.sf_t[1] = fb->k_sf_t;
   a.BH = BH;
   a.N = N;
   a.qknorm = p->qknorm;
@@ -383,7 +391,12 @@ int run_fp4_prologue(const sage_params* p, const void* q, const void* k, const s
   a.eps = p->rms_eps;
   const int grid = 2 * BH * (N / kRowsPerCta);
   sage::fp4::prologue_amax_kernel<T, D><<<grid, sage::kQuantThreads, 0, st>>>(a);
-  sage::fp4::prologue_quant_kernel<T, D><<<grid, sage::kQuantThreads, 0, st>>>(a);
+  // the sequence views stage each chunk through shared memory
+  const bool seq = fb->q_fp4_t != nullptr || fb->k_fp4_t != nullptr;
+  const size_t smem = seq ? sage::fp4::seq_smem_bytes<D>() : 0;
+  if (seq && set_smem(sage::fp4::prologue_quant_kernel<T, D>, smem) != SAGE_OK)
+    return SAGE_ERR_CUDA;
+  sage::fp4::prologue_quant_kernel<T, D><<<grid, sage::kQuantThreads, smem, st>>>(a);
   return launch_status();
 }
 

@@ -27,25 +27,34 @@ class Fp4Bufs:
     q_inv_rms: Optional[torch.Tensor]
     k_inv_rms: Optional[torch.Tensor]
     k_mean: Optional[torch.Tensor]
+    # sequence views (16-token blocks per channel), made only when requested
+    q_fp4_t: Optional[torch.Tensor] = None
+    k_fp4_t: Optional[torch.Tensor] = None
+    q_sf_t: Optional[torch.Tensor] = None
+    k_sf_t: Optional[torch.Tensor] = None
 
     @staticmethod
-    def empty(shape, cfg: Config, device) -> "Fp4Bufs":
+    def empty(shape, cfg: Config, device, seq: bool = False) -> "Fp4Bufs":
         B, H, N, d = shape
         u8 = dict(dtype=torch.uint8, device=device)
         f32 = dict(dtype=torch.float32, device=device)
         sf = (B, H, N // 128, d // 64, 512)
+        sf_t = (B, H, (d + 127) // 128, N // 64, 512)
+        opt = (lambda s_: torch.empty(s_, **u8)) if seq else (lambda s_: None)
         return Fp4Bufs(torch.empty((B, H, N, d // 2), **u8), torch.empty((B, H, N, d // 2), **u8),
                        torch.empty(sf, **u8), torch.empty(sf, **u8),
                        torch.empty((B, H), **f32), torch.empty((B, H), **f32),
                        torch.empty((B, H, N), **f32) if cfg.qknorm else None,
                        torch.empty((B, H, N), **f32) if cfg.qknorm else None,
-                       torch.empty((B, H, d), **f32) if cfg.ksmooth else None)
+                       torch.empty((B, H, d), **f32) if cfg.ksmooth else None,
+                       opt((B, H, d, N // 2)), opt((B, H, d, N // 2)), opt(sf_t), opt(sf_t))
 
     def c_struct(self) -> SageFp4Bufs:
         p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
         return SageFp4Bufs(p(self.q_fp4), p(self.k_fp4), p(self.q_sf), p(self.k_sf),
                            p(self.q_genc), p(self.k_genc), p(self.q_inv_rms), p(self.k_inv_rms),
-                           p(self.k_mean))
+                           p(self.k_mean), p(self.q_fp4_t), p(self.k_fp4_t), p(self.q_sf_t),
+                           p(self.k_sf_t))
 
 
 def workspace_bytes(cfg: Config, like: torch.Tensor) -> int:
@@ -53,11 +62,12 @@ def workspace_bytes(cfg: Config, like: torch.Tensor) -> int:
 
 
 def quant_prologue(q, k, cfg: Config, out: Optional[Fp4Bufs] = None,
-                   workspace: Optional[torch.Tensor] = None) -> Fp4Bufs:
-    """QK-norm, K-smoothing and NVFP4 quantization of q and k (sage_fp4_quant_prologue)."""
+                   workspace: Optional[torch.Tensor] = None, seq: bool = False) -> Fp4Bufs:
+    """QK-norm, K-smoothing and NVFP4 quantization of q and k (sage_fp4_quant_prologue);
+    ``seq`` also makes the sequence views (when ``out`` is None)."""
     _check_inputs(q, k)
     prm = cfg.params(q)
-    fb = out if out is not None else Fp4Bufs.empty(tuple(q.shape), cfg, q.device)
+    fb = out if out is not None else Fp4Bufs.empty(tuple(q.shape), cfg, q.device, seq=seq)
     if workspace is None:
         workspace = torch.empty(workspace_bytes(cfg, q), dtype=torch.uint8, device=q.device)
     st = fb.c_struct()

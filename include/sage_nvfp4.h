@@ -42,6 +42,13 @@ typedef struct {
   float *q_genc, *k_genc;       /* [B,H]: global encode scales genc                         */
   float *q_inv_rms, *k_inv_rms; /* [B,H,N]: 1/rms per token (qknorm; may be NULL otherwise) */
   float *k_mean;                /* [B,H,d]: K channel means (ksmooth; else unused)          */
+  /* Optional sequence views (NULL: not produced): the same values quantized along the tokens,
+   * the K-major operands of dK = dS^T Q and dQ = dS K.  Global scales as above.               */
+  uint8_t *q_fp4_t, *k_fp4_t;   /* [B,H,d,N/2]: channel rows, token 2i in the low nibble     */
+  uint8_t *q_sf_t, *k_sf_t;     /* [B,H,ceil(d/128),N/64,512]: per 128-channel group and
+                                   64-token chunk, byte (c%32)*16 + ((c%128)/32)*4 + b holds
+                                   channel c's scale of the chunk's 16-token block b (rows
+                                   c >= d of a group are left unwritten)                     */
 } sage_fp4_bufs;
 
 /* Workspace bytes: which = 0 prologue (K-mean partials when ksmooth, plus 2*B*H words for the

@@ -46,7 +46,7 @@ def test_fp4_workspace_and_argument_checks(L):
     assert L.sage_fp4_workspace_bytes(ctypes.byref(_params(ksmooth=0)), 0) == 256
     assert L.sage_fp4_workspace_bytes(ctypes.byref(_params(qsmooth=1)), 0) == 0
     fake = 1 << 20  # never dereferenced: every call below fails its host-side checks
-    fb = SageFp4Bufs(*([fake] * 9))
+    fb = SageFp4Bufs(*([fake] * 9 + [None] * 4))
     ws = BH * (N // 64) * d * 4 + 256
     assert L.sage_fp4_quant_prologue(ctypes.byref(_params(qsmooth=1)), fake, fake,
                                      ctypes.byref(fb), fake, ws, None) == _lib.SAGE_ERR_UNSUPPORTED
@@ -59,6 +59,9 @@ def test_fp4_workspace_and_argument_checks(L):
     assert L.sage_fp4_quant_prologue(ctypes.byref(p), fake + 8, fake, ctypes.byref(fb), fake, ws,
                                      None) == _lib.SAGE_ERR_ALIGNMENT
     nosf = SageFp4Bufs(fake, fake, None, fake, fake, fake, fake, fake, fake)
+    half_seq = SageFp4Bufs(*([fake] * 9 + [fake, None, None, None]))  # codes without scales
+    assert L.sage_fp4_quant_prologue(ctypes.byref(p), fake, fake, ctypes.byref(half_seq), fake,
+                                     ws, None) == _lib.SAGE_ERR_INVALID_ARG
     assert L.sage_fp4_attn_fwd(ctypes.byref(p), ctypes.byref(nosf), fake, fake, fake,
                                None) == _lib.SAGE_ERR_INVALID_ARG
     assert L.sage_fp4_attn_fwd(ctypes.byref(p), ctypes.byref(fb), fake, fake + 4, fake,

@@ -210,3 +210,42 @@ def test_nvfp4_degenerate(kind, dtype, qknorm):
     assert not (np.abs(og - ref["o"]) > tol).any()
     # fp16_large has scores near 1e8: float32 rounding of S and of S * c is relative there
     np.testing.assert_allclose(lse.cpu().numpy().reshape(BH, N), ref["lse"], rtol=2e-6, atol=1e-4)
+
+
+def unpack_sf_t(sf_t: np.ndarray, BH: int, N: int, d: int) -> np.ndarray:
+    """[BH, ceil(d/128), N/64, 512] scale atoms -> [BH, d, N/16] (channel c, 16-token block)."""
+    sf_t = sf_t.reshape(BH, (d + 127) // 128, N // 64, 512)
+    c = np.arange(d)[:, None]
+    b = np.arange(N // 16)[None, :]
+    byte = (c % 32) * 16 + ((c % 128) // 32) * 4 + b % 4
+    return sf_t[:, c // 128, b // 4, byte]
+
+
+@pytest.mark.parametrize("name", ["d128_bf16_causal", "d64_bf16_causal", "d128_fp16_causal",
+                                  "koutlier_all_off"])
+def test_nvfp4_sequence_views(name):
+    """The views along the tokens (16-token blocks per channel), bit-exact: the oracle's
+    nvfp4_quantize of the transposed normalized / smoothed matrices."""
+    w = CASES[name]
+    BH, N, d = w.B * w.H, w.N, w.d
+    x = make_inputs(w)
+    q, k = (to_device(x[n], w.dtype) for n in ("q", "k"))
+    cfg = _cfg(w)
+    fb = nvfp4.quant_prologue(q, k, cfg, seq=True)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    qf, kf = (x[n + "_f32"].reshape(BH, N, d) for n in ("q", "k"))
+    pro = F.qattn_prologue(qf, kf, qknorm=w.qknorm, ksmooth=w.ksmooth)
+    for t, src in (("q", pro["q_hat"]), ("k", pro["k_tilde"])):
+        ref = F.nvfp4_quantize(np.swapaxes(src, -1, -2))
+        codes = unpack_codes(getattr(fb, t + "_fp4_t").cpu().numpy().reshape(BH, d, N // 2))
+        np.testing.assert_array_equal(codes, ref["codes"], err_msg=t + " codes")
+        sf = unpack_sf_t(getattr(fb, t + "_sf_t").cpu().numpy(), BH, N, d)
+        np.testing.assert_array_equal(sf, ref["sf"], err_msg=t + " scales")
+        np.testing.assert_array_equal(getattr(fb, t + "_genc").cpu().numpy().reshape(BH),
+                                      ref["genc"], err_msg=t + " genc")
+    # the row views are unchanged by also producing the sequence views
+    for t in ("q", "k"):
+        np.testing.assert_array_equal(
+            unpack_codes(getattr(fb, t + "_fp4").cpu().numpy().reshape(BH, N, d // 2)),
+            pro[t + "_codes"])
