@@ -118,8 +118,10 @@ __device__ __forceinline__ uint2 quant8(const float (&x)[8], float s) {
 // Prologue pass 1 (only with smoothing): per 64-token block of k (or q), the column sums of
 // khat (qhat).
 // One group of D/8 lanes walks one block's 64 tokens in order.  partials: [BH * N/64, D].
+// MINMAX (NVFP4 prologue): also the block's column maxima and minima, at partials +
+// total_blocks * D and + 2 * total_blocks * D.
 // ---------------------------------------------------------------------------------------------
-template <typename T, int D>
+template <typename T, int D, bool MINMAX = false>
 __global__ void __launch_bounds__(kRowThreads) prologue_kstats_kernel(
     const T* __restrict__ k, float* __restrict__ partials, int total_blocks, int qknorm,
     float eps) {
@@ -130,9 +132,13 @@ __global__ void __launch_bounds__(kRowThreads) prologue_kstats_kernel(
   if (blk >= total_blocks) return;  // whole lane groups leave together
   const uint32_t mask = ((LPR == 32) ? 0xFFFFFFFFu : ((1u << LPR) - 1u)) << (grp * LPR);
   const T* src = k + static_cast<size_t>(blk) * 64 * D + sub * 8;
-  float c[8];
+  float c[8], hi[8], lo[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) c[i] = 0.0f;
+  for (int i = 0; i < 8; ++i) {
+    c[i] = 0.0f;
+    hi[i] = -INFINITY;
+    lo[i] = INFINITY;
+  }
 #pragma unroll 4
   for (int t = 0; t < 64; ++t) {
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(src + static_cast<size_t>(t) * D));
@@ -140,22 +146,59 @@ __global__ void __launch_bounds__(kRowThreads) prologue_kstats_kernel(
     Cvt<T>::load8(u, x);
     if (qknorm) rms_norm8<D>(x, eps, mask);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) c[i] = __fadd_rn(c[i], x[i]);
+    for (int i = 0; i < 8; ++i) {
+      c[i] = __fadd_rn(c[i], x[i]);
+      if constexpr (MINMAX) {
+        hi[i] = fmaxf(hi[i], x[i]);
+        lo[i] = fminf(lo[i], x[i]);
+      }
+    }
   }
   float4* dst = reinterpret_cast<float4*>(partials + static_cast<size_t>(blk) * D + sub * 8);
   dst[0] = make_float4(c[0], c[1], c[2], c[3]);
   dst[1] = make_float4(c[4], c[5], c[6], c[7]);
+  if constexpr (MINMAX) {
+    const size_t plane = static_cast<size_t>(total_blocks) * D;
+    dst[plane / 4] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+    dst[plane / 4 + 1] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+    dst[plane / 2] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+    dst[plane / 2 + 1] = make_float4(lo[4], lo[5], lo[6], lo[7]);
+  }
 }
 
 // Prologue pass 2 (only with smoothing): m[bh][c] = (sum over blocks in order) / N.
-template <int D>
+// MINMAX (NVFP4 prologue): also the head's maximum of |fl(khat - m)|, as float bits in
+// gmax[bh].  fl(x - m) is monotone in x, so per channel that maximum is reached at the
+// channel's largest or smallest khat: no pass over the smoothed values is needed.
+template <int D, bool MINMAX = false>
 __global__ void prologue_kmean_kernel(const float* __restrict__ partials,
-                                      float* __restrict__ k_mean, int nkb, int N) {
+                                      float* __restrict__ k_mean, int nkb, int N,
+                                      int total_blocks = 0, uint32_t* gmax = nullptr) {
   const int bh = blockIdx.x, c = threadIdx.x;
   const float* src = partials + static_cast<size_t>(bh) * nkb * D + c;
   float s = 0.0f;
   for (int t = 0; t < nkb; ++t) s = __fadd_rn(s, src[static_cast<size_t>(t) * D]);
-  k_mean[static_cast<size_t>(bh) * D + c] = __fdiv_rn(s, static_cast<float>(N));
+  const float m = __fdiv_rn(s, static_cast<float>(N));
+  k_mean[static_cast<size_t>(bh) * D + c] = m;
+  if constexpr (MINMAX) {
+    const size_t plane = static_cast<size_t>(total_blocks) * D;
+    float hi = -INFINITY, lo = INFINITY;
+    for (int t = 0; t < nkb; ++t) {
+      hi = fmaxf(hi, src[plane + static_cast<size_t>(t) * D]);
+      lo = fminf(lo, src[2 * plane + static_cast<size_t>(t) * D]);
+    }
+    float a = fmaxf(fabsf(__fsub_rn(hi, m)), fabsf(__fsub_rn(lo, m)));
+    __shared__ float red[D / 32];
+    a = warp_max(a);
+    if ((c & 31) == 0) red[c >> 5] = a;
+    __syncthreads();
+    if (c == 0) {
+      float g = 0.0f;
+#pragma unroll
+      for (int w = 0; w < D / 32; ++w) g = fmaxf(g, red[w]);
+      gmax[bh] = __float_as_uint(g);
+    }
+  }
 }
 
 // Block absmax over the CTA's 128 rows: rows 0-63 are warps 0-3, rows 64-127 warps 4-7.

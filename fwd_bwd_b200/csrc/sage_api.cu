@@ -345,7 +345,8 @@ struct Fp4Ws {
 };
 Fp4Ws fp4_ws(const sage_params* p) {
   Fp4Ws w;
-  w.gmax = p->ksmooth ? align_up(prologue_partials(p) * 4) : 0;
+  // K statistics: column sums, maxima and minima per 64-token block (ksmooth)
+  w.gmax = p->ksmooth ? align_up(3 * prologue_partials(p) * 4) : 0;
   w.total = align_up(w.gmax + 2 * static_cast<size_t>(p->B) * p->H * 4);
   return w;
 }
@@ -356,17 +357,20 @@ int run_fp4_prologue(const sage_params* p, const void* q, const void* k, const s
   const int BH = p->B * p->H, N = p->N;
   const Fp4Ws w = fp4_ws(p);
   uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
-  if (p->ksmooth) {
-    const int total = BH * (N / 64);
-    const int per_cta = (kRowThreads / 32) * (32 / (D / 8));
-    float* partials = reinterpret_cast<float*>(wsb);
-    sage::prologue_kstats_kernel<T, D><<<(total + per_cta - 1) / per_cta, kRowThreads, 0, st>>>(
-        reinterpret_cast<const T*>(k), partials, total, p->qknorm, p->rms_eps);
-    sage::prologue_kmean_kernel<D><<<BH, D, 0, st>>>(partials, fb->k_mean, N / 64, N);
-  }
   uint32_t* gmax = reinterpret_cast<uint32_t*>(wsb + w.gmax);
   if (cudaMemsetAsync(gmax, 0, 2 * static_cast<size_t>(BH) * 4, st) != cudaSuccess)
     return SAGE_ERR_CUDA;
+  if (p->ksmooth) {
+    // K's mean and, from its column extremes, K's global maximum (gmax[BH + bh])
+    const int total = BH * (N / 64);
+    const int per_cta = (kRowThreads / 32) * (32 / (D / 8));
+    float* partials = reinterpret_cast<float*>(wsb);
+    sage::prologue_kstats_kernel<T, D, true>
+        <<<(total + per_cta - 1) / per_cta, kRowThreads, 0, st>>>(
+            reinterpret_cast<const T*>(k), partials, total, p->qknorm, p->rms_eps);
+    sage::prologue_kmean_kernel<D, true><<<BH, D, 0, st>>>(partials, fb->k_mean, N / 64, N,
+                                                           total, gmax + BH);
+  }
   sage::fp4::PrologueArgs a;
   a.src[0] = q;
   a.src[1] = k;
@@ -390,7 +394,10 @@ int run_fp4_prologue(const sage_params* p, const void* q, const void* k, const s
   a.ksmooth = p->ksmooth;
   a.eps = p->rms_eps;
   const int grid = 2 * BH * (N / kRowsPerCta);
-  sage::fp4::prologue_amax_kernel<T, D><<<grid, sage::kQuantThreads, 0, st>>>(a);
+  // the absolute-maximum pass covers Q, and K too unless the K statistics gave its maximum
+  // (blocks [0, grid/2) are Q's)
+  sage::fp4::prologue_amax_kernel<T, D>
+      <<<p->ksmooth ? grid / 2 : grid, sage::kQuantThreads, 0, st>>>(a);
   // the sequence views stage each chunk through shared memory
   const bool seq = fb->q_fp4_t != nullptr || fb->k_fp4_t != nullptr;
   const size_t smem = seq ? sage::fp4::seq_smem_bytes<D>() : 0;

@@ -41,13 +41,13 @@ def test_fp4_workspace_and_argument_checks(L):
 
     BH, N, d = 8, 1024, 128
     p = _params()
-    assert L.sage_fp4_workspace_bytes(ctypes.byref(p), 0) == BH * (N // 64) * d * 4 + 256
+    assert L.sage_fp4_workspace_bytes(ctypes.byref(p), 0) == 3 * BH * (N // 64) * d * 4 + 256
     assert L.sage_fp4_workspace_bytes(ctypes.byref(p), 1) == 0
     assert L.sage_fp4_workspace_bytes(ctypes.byref(_params(ksmooth=0)), 0) == 256
     assert L.sage_fp4_workspace_bytes(ctypes.byref(_params(qsmooth=1)), 0) == 0
     fake = 1 << 20  # never dereferenced: every call below fails its host-side checks
     fb = SageFp4Bufs(*([fake] * 9 + [None] * 4))
-    ws = BH * (N // 64) * d * 4 + 256
+    ws = 3 * BH * (N // 64) * d * 4 + 256
     assert L.sage_fp4_quant_prologue(ctypes.byref(_params(qsmooth=1)), fake, fake,
                                      ctypes.byref(fb), fake, ws, None) == _lib.SAGE_ERR_UNSUPPORTED
     assert L.sage_fp4_quant_prologue(ctypes.byref(_params(d=96)), fake, fake, ctypes.byref(fb),
