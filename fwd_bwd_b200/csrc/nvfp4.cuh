@@ -3,10 +3,12 @@
 // once and reused).  NVFP4 format ("Quartet II", allinfo.ai.kr): E2M1 values in blocks of 16
 // sharing an E4M3 scale, plus one global scale.
 //
-// Prologue (two passes over q and k, after the INT8 path's QK-norm / K-smoothing):
+// Prologue (after the INT8 path's QK-norm / K-smoothing):
 //   amax pass   per (tensor, batch-head) absolute maximum G of the normalized, smoothed values
 //               (atomicMax on the float bits: non-negative floats order like their bits, so
-//               the result does not depend on the order of the atomics);
+//               the result does not depend on the order of the atomics).  With K-smoothing,
+//               K's G comes instead from the K-statistics pass (column extremes, see
+//               prologue_kmean_kernel) and this pass reads Q only;
 //   quant pass  genc = 2688 / G (1 when G = 0); per 16 channels: a = max|x|,
 //               u = (a * genc) / 6, sd = e4m3(u) (nearest, ties to even, saturating at 448),
 //               code = e2m1(x * (genc / sd)) (nearest, ties to even, saturating at 6, the sign
@@ -14,7 +16,9 @@
 // Outputs: codes [BH, N, d/2] (channel 2i in the low nibble of byte i), block scales in the
 // tensor core's scale-factor order (per 128-row tile and 64-channel chunk, 512 bytes: byte
 // (r % 32) * 16 + (r / 32) * 4 + b holds row r's scale of the chunk's 16-channel block b), and
-// genc [BH].
+// genc [BH].  Optionally the sequence views: the same values quantized in blocks of 16 tokens
+// per channel (codes [BH, d, N/2], scale atoms per 128-channel group and 64-token chunk), the
+// K-major operands of the backward's dK = dS^T Q and dQ = dS K.
 //
 // Forward: per CTA one tile of 128 query rows of one (batch, head), walking 128-key blocks.
 //   warp 8      TMA producer: Q codes and scales once, then K codes, K scales and V (16-bit)
