@@ -58,6 +58,17 @@ def test_fp4_workspace_and_argument_checks(L):
                                      None) == _lib.SAGE_ERR_WORKSPACE
     assert L.sage_fp4_quant_prologue(ctypes.byref(p), fake + 8, fake, ctypes.byref(fb), fake, ws,
                                      None) == _lib.SAGE_ERR_ALIGNMENT
+    # ragged and empty shapes are refused before any launch
+    for bad, want in ((dict(N=1000), _lib.SAGE_ERR_UNSUPPORTED),
+                      (dict(N=0), _lib.SAGE_ERR_INVALID_ARG),
+                      (dict(B=0), _lib.SAGE_ERR_INVALID_ARG),
+                      (dict(d=32), _lib.SAGE_ERR_UNSUPPORTED)):
+        pb = _params(**bad)
+        assert L.sage_fp4_quant_prologue(ctypes.byref(pb), fake, fake, ctypes.byref(fb), fake,
+                                         ws, None) == want, bad
+        assert L.sage_fp4_attn_fwd(ctypes.byref(pb), ctypes.byref(fb), fake, fake, fake,
+                                   None) == want, bad
+        assert L.sage_fp4_workspace_bytes(ctypes.byref(pb), 0) == 0
     nosf = SageFp4Bufs(fake, fake, None, fake, fake, fake, fake, fake, fake)
     half_seq = SageFp4Bufs(*([fake] * 9 + [fake, None, None, None]))  # codes without scales
     assert L.sage_fp4_quant_prologue(ctypes.byref(p), fake, fake, ctypes.byref(half_seq), fake,
