@@ -10,7 +10,6 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
-#include <mutex>
 
 #include "sage.h"
 #include "sage_nvfp4.h"
@@ -442,24 +441,18 @@ int run_fp4_fwd(const sage_params* p, const sage_fp4_bufs* fb, const void* v, vo
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of g_noalloc_scratch on the current device, looked up once per device.  In
-// host code the array's name is only a host-side stand-in, so kernels must be given this
-// address instead.
+// Device address of g_noalloc_scratch in the calling thread's current context.  In host code
+// the array's name is only a host-side stand-in, so kernels must be given this address.  The
+// address belongs to the copy of the library's device code loaded in that context: a driver
+// context other than the device's primary one, or the primary context re-created after
+// cudaDeviceReset, holds its own copy at another address.  So it is looked up on every call
+// (a host-side table lookup once the code is loaded there, which allocates nothing) rather than
+// cached per device.
 int noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SAGE_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
-      return SAGE_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+    return SAGE_ERR_CUDA;
+  *out = ptr;
   return SAGE_OK;
 }
 

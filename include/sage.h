@@ -104,15 +104,21 @@ int sage_quant_prologue(const sage_params* p, const void* q, const void* k, cons
  * at start-up, and latency-critical host threads that must not risk the device-wide
  * synchronization cudaMalloc / cudaFree can cause.  This entry point takes no workspace: the
  * smoothing column sums go to a fixed 32 MiB array in the library's own device memory (every
- * GPU that loads the library holds it until exit), so it supports shapes with
- * (ksmooth + qsmooth) * B * H * (N / 64) * d * 4 <= 32 MiB (e.g. B*H*N*d up to 2^29 elements
- * with one of the two) and returns SAGE_ERR_WORKSPACE beyond that, before launching anything.  Everything else -- arguments,
- * outputs, results (bit for bit) -- is as for sage_quant_prologue.  It allocates nothing.
- * The first call on each device looks up the array's device address (with that device
- * current); make that first call before any stream capture.  All calls share the one array,
- * which keeps the last call's contents; every value a call reads from it is written by that
- * same call first, so nothing needs clearing, but calls whose kernels overlap on the GPU (on
- * different streams) race on it and must be ordered by the caller. */
+ * context that loads the library's device code holds it until the context is destroyed), so
+ * it supports shapes with (ksmooth + qsmooth) * B * H * (N / 64) * d * 4 <= 32 MiB (e.g.
+ * B*H*N*d up to 2^29 elements with one of the two) and returns SAGE_ERR_WORKSPACE beyond
+ * that, before launching anything.  Everything else -- arguments, outputs, results (bit for
+ * bit) -- is as for sage_quant_prologue.  It allocates nothing.
+ * Every call looks up the array's device address in the calling thread's current context (a
+ * host-side lookup that allocates nothing), so calls from any context -- the device's primary
+ * one or a driver context of the caller's own -- use that context's copy of the array.  The
+ * library's device code, and the 32 MiB array with it, is loaded into a context by the first
+ * call of any libsage entry point there (lazy module loading), and that load allocates device
+ * memory and may synchronize the device: callers that cannot afford either later should make
+ * one warm-up call per context at start-up, before any stream capture.  All calls in one
+ * context share its array, which keeps the last call's contents; every value a call reads from
+ * it is written by that same call first, so nothing needs clearing, but calls whose kernels
+ * overlap on the GPU (on different streams) race on it and must be ordered by the caller. */
 int sage_quant_prologue_noalloc(const sage_params* p, const void* q, const void* k,
                                 const void* v, const sage_qbufs* out, void* stream);
 
