@@ -3,9 +3,14 @@
 
 One step = the whole hot path on one batch: the quantization prologue (QK-norm, K-smoothing,
 INT8 codes), the forward kernel and the three backward stages, on synthetic bf16 inputs that
-are resident in HBM (each input tensor is 1 GiB, far larger than the 126 MB L2, so no flush is
-needed between steps).  Metric: effective tensor-core TOPS over the step, counting the seven
-attention GEMMs (FlashAttention convention, causal half not credited).
+are resident in HBM.  Metric: effective tensor-core TOPS over the step, counting the seven
+attention GEMMs (FlashAttention convention, causal half not credited).  Each step is timed with
+CUDA events on the launching stream; when an input tensor is smaller than 4x the 126 MB L2,
+L2 is flushed (a 512 MiB buffer written) before every step, outside the timed events.
+
+Roofline denominators are measured in the same run on the same GPU: the tensor cores' INT8
+(kind::i8) and 16-bit (kind::f16) throughput from the library's own back-to-back tcgen05 MMA
+loop (sage_mma_peak), weighted by each kernel's mix of INT8 and 16-bit GEMMs.
 
 Multi-GPU (torchrun): every (batch, head) is independent and the operator has no weights, so
 each rank runs its own full-size batch with no collective on the data path (weak scaling); the
@@ -28,6 +33,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd+bwd effective TOPS at 1 B200 and % of INT8/FP16 TC roofline"
+METRIC_FP4 = "NVFP4 Q-Attn forward effective TOPS at 1 B200 and % of FP4/16-bit TC roofline"
+L2_BYTES = 126 * 2 ** 20
 
 
 def parse():
@@ -42,13 +49,16 @@ def parse():
     ap.add_argument("--chunks", type=int, default=16,
                     help="batch slices of the end-to-end host-buffer pipeline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-peaks", action="store_true",
+                    help="skip the tensor-core peak loop (profiling runs; no roofline fraction)")
     ap.add_argument("--variant", default="int8", choices=["int8", "nvfp4"],
                     help="int8: the SageBwd step (default); nvfp4: the NVFP4 Q-Attn forward")
     return ap.parse_args()
 
 
 def peaks():
-    """Roofline denominators: measured bf16 peaks; INT8 = 2x bf16 (nominal dense ratio)."""
+    """cuBLAS bf16 and HBM copy figures from MEASURED_PEAKS.json (driver-measured): context for
+    the tensor cores, and the HBM roofline of the prologue."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         m = json.load(open(path))
@@ -74,11 +84,10 @@ def traffic_per_launch(kernel: str, src: str):
     return None
 
 
-def weighted_peak(p_bf16: float, n_i8: int, n_f16: int) -> float:
-    """Peak of a mix of equal-size INT8 and 16-bit GEMMs (INT8 at twice the bf16 rate)."""
-    p_i8 = 2.0 * p_bf16
-    n = n_i8 + n_f16
-    return 1.0 / (n_i8 / n / p_i8 + n_f16 / n / p_bf16)
+def mixed_peak(p_a: float, p_b: float, n_a: int, n_b: int) -> float:
+    """Peak of a mix of equal-size GEMMs at two rates: total ops over total minimum time."""
+    n = n_a + n_b
+    return 1.0 / (n_a / n / p_a + (n_b / n / p_b if n_b else 0.0))
 
 
 class ClockSampler:
@@ -119,9 +128,59 @@ class ClockSampler:
                 else None, "reasons": reasons, "samples": len(rows)}
 
 
+def uuid_of(dev) -> str:
+    import torch
+
+    return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+
+
+def measure_tc_peaks(dev, dtype16: str, seconds: float = 0.6) -> dict:
+    """The tensor cores' own INT8 (kind::i8) and 16-bit (kind::f16) throughput on this GPU, now:
+    one CTA per SM issuing back-to-back 128 x 256 MMAs from shared memory (sage_mma_peak), timed
+    with CUDA events while nvidia-smi samples the SM clock.  Returns TOPS per kind (median of
+    three launches) with the median SM clock seen."""
+    import torch
+
+    from fwd_bwd_b200 import ops
+
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    kind16 = 2 if dtype16 == "bf16" else 1
+    fills = {0: torch.randint(-127, 128, (49152,), generator=g, device=dev).to(torch.int8),
+             kind16: torch.randn(24576, generator=g, device=dev).to(
+                 torch.bfloat16 if kind16 == 2 else torch.float16)}
+    out = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for kind in (0, kind16):
+        groups = 2000
+        ops.mma_peak(kind, nsm, groups, fills[kind])
+        e0.record()
+        ops.mma_peak(kind, nsm, groups, fills[kind])
+        e1.record()
+        torch.cuda.synchronize(dev)
+        groups = max(1000, int(groups * (seconds / 3) * 1e3 / e0.elapsed_time(e1)))
+        sampler = ClockSampler(uuid_of(dev))
+        time.sleep(0.25)
+        rates = []
+        for _ in range(3):
+            e0.record()
+            ops.mma_peak(kind, nsm, groups, fills[kind])
+            e1.record()
+            torch.cuda.synchronize(dev)
+            rates.append(ops.mma_peak_ops(kind, nsm, groups)
+                         / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+        clk = sampler.stop() or {}
+        if ops.device_status(dev) != 0:
+            raise RuntimeError("the tensor-core peak loop reported a timeout")
+        out["i8" if kind == 0 else "f16"] = {"tops": statistics.median(rates),
+                                             "sm_mhz": clk.get("sm_mhz"),
+                                             "reasons": clk.get("reasons")}
+    return out
+
+
 def cpu_baseline(w, n_heads: int):
     """Time the oracle (as it stands) on the first n_heads heads of the workload."""
-    import numpy as np
     from threadpoolctl import threadpool_info
 
     import oracle.sage_oracle as O
@@ -135,7 +194,6 @@ def cpu_baseline(w, n_heads: int):
     dt = time.perf_counter() - t0
     ops = w.ops() / (w.B * w.H) * n_heads
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    del np
     return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
             "seconds": dt,
             "sample": f"{n_heads} of {w.B * w.H} heads (flattened b*H+h = 0..{n_heads - 1}) of "
@@ -167,9 +225,6 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-METRIC_FP4 = "NVFP4 Q-Attn forward effective TOPS at 1 B200 and % of FP4/16-bit TC roofline"
-
-
 def cpu_baseline_fp4(w, n_heads: int):
     """Time the NVFP4 oracle (as it stands) on the first n_heads heads: prologue + forward."""
     from threadpoolctl import threadpool_info
@@ -187,6 +242,38 @@ def cpu_baseline_fp4(w, n_heads: int):
     return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
             "sample": f"{n_heads} of {w.B * w.H} heads (flattened b*H+h = 0..{n_heads - 1}) of "
                       f"the workload, NVFP4 prologue+forward, numpy oracle"}
+
+
+def l2_policy(w) -> tuple:
+    """(flush, label): flush L2 before each step unless every input is >= 4x L2."""
+    tensor = w.B * w.H * w.N * w.d * 2
+    if tensor >= 4 * L2_BYTES:
+        return False, f"no flush: every input tensor ({tensor / 2 ** 20:.0f} MiB) exceeds 4x L2"
+    return True, (f"L2 flushed before every step (input tensors {tensor / 2 ** 20:.0f} MiB "
+                  f"< 4x L2)")
+
+
+def config_of(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "io_dtype": w.dtype, "q_block": w.q_block, "k_block": w.k_block,
+            "qknorm": w.qknorm, "ksmooth": w.ksmooth, "qsmooth": w.qsmooth,
+            "l2": l2_policy(w)[1]}
+
+
+def timed_steps(step, nev: int, steps: int, dev, flush_buf=None):
+    """Run `steps` steps, each bracketed by its own CUDA events (`step(ev)` records ev[1..]);
+    L2 is flushed between steps (outside the events) when `flush_buf` is given.  Returns the
+    per-step event lists."""
+    import torch
+
+    stream = torch.cuda.current_stream(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(steps)]
+    for s in range(steps):
+        if flush_buf is not None:
+            flush_buf.add_(1)
+        evs[s][0].record(stream)
+        step(evs[s])
+    return evs
 
 
 def run_nvfp4(args, w):
@@ -209,49 +296,48 @@ def run_nvfp4(args, w):
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     launches_per_step = 2 * int(w.ksmooth) + 2 + 1
+    flush, _ = l2_policy(w)
+    flush_buf = torch.empty(2 ** 27, dtype=torch.float32, device=dev) if flush else None
 
-    def step(ev=None):
+    def step(ev):
         nvfp4.quant_prologue(q, k, cfg, out=fb, workspace=ws)
-        if ev is not None:
-            ev[0].record(stream)
+        ev[1].record(stream)
         nvfp4.attn_fwd(fb, v, cfg, o=o, lse=lse)
-        if ev is not None:
-            ev[1].record(stream)
+        ev[2].record(stream)
 
     for _ in range(args.warmup):
-        step()
+        step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
     torch.cuda.synchronize(dev)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    tc = None if args.no_peaks else measure_tc_peaks(dev, w.dtype)
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(uuid_of(dev))
     time.sleep(0.3)
-    t0.record(stream)
-    for s_ in range(args.steps):
-        step(evs[s_])
-    t1.record(stream)
+    evs = timed_steps(step, 3, args.steps, dev, flush_buf)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     if ops.device_status(dev) != 0:
         raise RuntimeError("device status reports a kernel timeout in the timed region")
-    ms = t0.elapsed_time(t1) / args.steps
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    ms = statistics.mean(e[0].elapsed_time(e[2]) for e in evs)
+    fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     fwd_ops = w.ops("fwd")
     value = fwd_ops / (ms * 1e-3) / 1e12
-    pk = peaks()
-    # Q K^T at the FP4 rate (4x bf16, the nominal dense ratio 9 : 2.25 POPS), P V at the bf16
-    # rate; equal op counts
-    p_bf16 = pk["bf16_sustained"]
-    p_fwd = 1.0 / (0.5 / (4.0 * p_bf16) + 0.5 / p_bf16)
     achieved = fwd_ops / (fwd_ms * 1e-3) / 1e12
     traffic = (traffic_per_launch("fp4::attn_fwd_kernel", "fwd_bwd_b200/csrc/nvfp4.cuh")
                if w.name == "sweep8192" and w.B == 32 else None)
     roofline = {"bound": "tensor", "kernel": "fp4::attn_fwd_kernel", "achieved": achieved,
-                "peak": p_fwd, "unit": "TFLOP/s", "frac": achieved / p_fwd, "traffic": traffic,
-                "peak_note": f"{pk['basis']} sustained bf16; NVFP4 = 4x bf16, weighted 1:1 "
-                             f"with the 16-bit P V"}
+                "unit": "TFLOP/s", "traffic": traffic}
+    if tc is not None:
+        # Q K^T at the FP4 rate (4x the measured 16-bit rate: the nominal dense ratio 9 : 2.25
+        # POPS), P V at the measured 16-bit rate; equal op counts
+        p16 = tc["f16"]["tops"]
+        p_fwd = mixed_peak(4.0 * p16, p16, 1, 1)
+        roofline.update(peak=p_fwd, frac=achieved / p_fwd,
+                        peak_note=f"measured in this run: own tcgen05 kind::f16 loop "
+                                  f"{p16:.0f} TOPS; NVFP4 = 4x that (nominal ratio), weighted "
+                                  f"1:1 with the 16-bit P V")
     e2e = None
     if not args.no_e2e:
-        hin = [t.cpu().pin_memory() for t in (q, k, v)]
+        hin = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t) for t in (q, k, v)]
         hout = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
         qd, kd, vd = (torch.empty_like(t) for t in (q, k, v))
 
@@ -277,20 +363,12 @@ def run_nvfp4(args, w):
             "dtype": "nvfp4+bf16", "data": "synthetic",
             "config": dict(config_of(w), variant="nvfp4 forward"),
             "kernels": {"fp4::attn_fwd_kernel": {"ms": round(fwd_ms, 4),
-                                                 "tops": round(achieved, 2),
-                                                 "frac": round(achieved / p_fwd, 4)}},
-            "roofline": roofline, "clocks": clocks, "e2e": e2e,
+                                                 "tops": round(achieved, 2)}},
+            "tensor_peaks": tc, "roofline": roofline, "clocks": clocks, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps}
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_fp4(w, 4)
     print(json.dumps(line), flush=True)
-
-
-def config_of(w):
-    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
-            "io_dtype": w.dtype, "q_block": w.q_block, "k_block": w.k_block,
-            "qknorm": w.qknorm, "ksmooth": w.ksmooth, "qsmooth": w.qsmooth,
-            "l2": "no flush: every input tensor (1 GiB at the default workload) exceeds L2"}
 
 
 def main():
@@ -337,47 +415,44 @@ def main():
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     stream = torch.cuda.current_stream(dev)
     launches_per_step = 1 + 2 * (int(w.ksmooth) + int(w.qsmooth)) + 1 + 3
+    flush, _ = l2_policy(w)
+    flush_buf = torch.empty(2 ** 27, dtype=torch.float32, device=dev) if flush else None
 
-    def step(ev=None):
+    # events: [0] step start, [1] prologue done, [2] forward done, [3] preprocess done,
+    # [4] backward kernel done, [5] step done
+    def step(ev):
         ops.quant_prologue(q, k, v, cfg, out=qb, workspace=ws_pro)
-        if ev is not None:
-            ev[0].record(stream)
+        ev[1].record(stream)
         ops.attn_fwd(qb, q, cfg, o=o, lse=lse)
-        if ev is not None:
-            ev[1].record(stream)
+        ev[2].record(stream)
         ops.attn_bwd(q, k, v, qb, o, lse, do, cfg, dq, dk, dv, workspace=ws_bwd, stage=0)
-        if ev is not None:
-            ev[2].record(stream)
+        ev[3].record(stream)
         ops.attn_bwd(q, k, v, qb, o, lse, do, cfg, dq, dk, dv, workspace=ws_bwd, stage=1)
-        if ev is not None:
-            ev[3].record(stream)
+        ev[4].record(stream)
         ops.attn_bwd(q, k, v, qb, o, lse, do, cfg, dq, dk, dv, workspace=ws_bwd, stage=2)
+        ev[5].record(stream)
 
     for _ in range(args.warmup):
-        step()
+        step([torch.cuda.Event(enable_timing=True) for _ in range(6)])
     torch.cuda.synchronize(dev)
     if ops.device_status(dev) != 0:
         raise RuntimeError("device status reports a kernel timeout during warm-up")
+    tc = None if args.no_peaks else measure_tc_peaks(dev, w.dtype)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    sampler = ClockSampler(uuid_of(dev))
     time.sleep(0.3)
-    t_start.record(stream)
-    for s in range(args.steps):
-        step(evs[s])
-    t_end.record(stream)
+    evs = timed_steps(step, 6, args.steps, dev, flush_buf)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    elapsed = t_start.elapsed_time(t_end)
-    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    bwd_main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    elapsed = sum(e[0].elapsed_time(e[5]) for e in evs)
+    part = {name: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)
+            for name, a, b in (("prologue", 0, 1), ("fwd", 1, 2), ("bwd_pre", 2, 3),
+                               ("bwd", 3, 4), ("dq_finalize", 4, 5))}
     if world > 1:
         t = torch.tensor([elapsed], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -388,15 +463,20 @@ def main():
     total_ops = w.ops() * world
     value = total_ops / (ms * 1e-3) / 1e12
 
-    # end to end through the public host-buffer API: pinned host inputs in, pinned host results
-    # out, with the copies (and their overlap with the kernels) inside the timed region
+    # end to end through the C ABI's host-buffer call (sage_fwd_bwd_host): pinned host inputs
+    # in, pinned host results out, the copies and their overlap with the kernels inside the
+    # timed region.  Under torchrun every rank streams a 1/world slice of its batch, so the
+    # pinned host memory per node stays that of one full batch.
     e2e = None
     if not args.no_e2e:
-        hin = [t.cpu().pin_memory() for t in (q, k, v, do)]
-        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, dq, dk, dv)]
-        del q, k, v, do, o, dq, dk, dv, qb, ws_pro, ws_bwd, lse, x
+        bsl = max(1, w.B // world)
+        hin = [torch.empty((bsl,) + tuple(t.shape[1:]), dtype=t.dtype,
+                           pin_memory=True).copy_(t[:bsl]) for t in (q, k, v, do)]
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in hin]
+        del q, k, v, do, o, dq, dk, dv, qb, ws_pro, ws_bwd, lse, x, flush_buf
         torch.cuda.empty_cache()
-        ops.fwd_bwd_host(*hin, cfg, *hout, chunks=args.chunks, device=dev)  # warm-up
+        pipe = ops.HostPipeline(hin[0], cfg, args.chunks, dev)
+        ops.fwd_bwd_host(*hin, cfg, *hout, pipeline=pipe)  # warm-up
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
@@ -405,55 +485,78 @@ def main():
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(torch.cuda.current_stream(dev))
         for _ in range(args.steps):
-            ops.fwd_bwd_host(*hin, cfg, *hout, chunks=args.chunks, device=dev)
+            ops.fwd_bwd_host(*hin, cfg, *hout, pipeline=pipe)
         e1.record(torch.cuda.current_stream(dev))
         torch.cuda.synchronize(dev)
         wall_ms = (time.perf_counter() - t0) * 1e3
-        # every call ends with a host-side synchronize, so the events on the default stream
-        # bracket the whole sequence; take the larger of event and wall time
+        # every call returns after the results reached host memory, so the events on the
+        # default stream bracket the whole sequence; take the larger of event and wall time
         e_ms = max(e0.elapsed_time(e1), wall_ms)
         if world > 1:
             t = torch.tensor([e_ms], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
-        e2e = {"value": total_ops / (e_ms / args.steps * 1e-3) / 1e12, "unit": "TOPS",
+        if ops.device_status(dev) != 0:
+            raise RuntimeError("device status reports a kernel timeout in the e2e run")
+        e_ops = w.ops() * bsl / w.B * world
+        e2e = {"value": e_ops / (e_ms / args.steps * 1e-3) / 1e12, "unit": "TOPS",
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hin),
                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout),
-               "chunks": args.chunks}
+               "chunks": args.chunks, "api": "sage_fwd_bwd_host",
+               "batch_per_rank": bsl}
 
     pk = peaks()
-    basis = pk["basis"]
-    p_bwd = weighted_peak(pk["bf16_sustained"], 4, 1)
-    p_fwd = weighted_peak(pk["bf16_sustained"], 2, 0)
-    p_all = weighted_peak(pk["bf16_sustained"], 6, 1)
-    bwd_ops = w.ops("bwd")
-    fwd_ops = w.ops("fwd")
-    kernels = {
-        "attn_bwd_kernel": {"ms": bwd_main_ms, "achieved": bwd_ops / (bwd_main_ms * 1e-3) / 1e12,
-                            "peak": p_bwd},
-        "attn_fwd_kernel": {"ms": fwd_ms, "achieved": fwd_ops / (fwd_ms * 1e-3) / 1e12,
-                            "peak": p_fwd},
-    }
-    dom = max(kernels, key=lambda n: kernels[n]["ms"])
-    kd = kernels[dom]
-    src = {"attn_bwd_kernel": "fwd_bwd_b200/csrc/attn_bwd.cuh",
-           "attn_fwd_kernel": "fwd_bwd_b200/csrc/attn_fwd.cuh"}[dom]
-    traffic = traffic_per_launch(dom, src) if w.name == "sweep8192" and w.B == 32 else None
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": kd["achieved"],
-                "peak": kd["peak"], "unit": "TFLOP/s", "frac": kd["achieved"] / kd["peak"],
-                "traffic": traffic,
-                "peak_note": f"{basis} sustained bf16 x (INT8 = 2x bf16), weighted by the "
-                             f"kernel's INT8:16-bit GEMM mix"}
+    bwd_ops, fwd_ops = w.ops("bwd"), w.ops("fwd")
+    kernels = {"attn_bwd_kernel": {"ms": part["bwd"], "tops": bwd_ops / (part["bwd"] * 1e-3) / 1e12},
+               "attn_fwd_kernel": {"ms": part["fwd"], "tops": fwd_ops / (part["fwd"] * 1e-3) / 1e12}}
+    roofline = {"bound": "tensor", "kernel": "attn_bwd_kernel", "unit": "TFLOP/s",
+                "achieved": kernels["attn_bwd_kernel"]["tops"],
+                "traffic": traffic_per_launch("attn_bwd_kernel", "fwd_bwd_b200/csrc/attn_bwd.cuh")
+                if w.name == "sweep8192" and w.B == 32 else None}
+    line_extra = {}
+    if tc is not None:
+        p8, p16 = tc["i8"]["tops"], tc["f16"]["tops"]
+        mix = {"attn_bwd_kernel": (4, 1), "attn_fwd_kernel": (2, 0)}
+        step_mhz = (clocks or {}).get("sm_mhz")
+        for name, (a, b) in mix.items():
+            pk_k = mixed_peak(p8, p16, a, b)
+            kernels[name].update(peak=pk_k, frac=kernels[name]["tops"] / pk_k)
+        p_all = mixed_peak(p8, p16, 6, 1)
+        roofline.update(peak=kernels["attn_bwd_kernel"]["peak"],
+                        frac=kernels["attn_bwd_kernel"]["frac"],
+                        peak_note=f"measured in this run on this GPU: own tcgen05 loops "
+                                  f"kind::i8 {p8:.0f} TOPS at {tc['i8']['sm_mhz']} MHz, "
+                                  f"kind::f16 {p16:.0f} TOPS at {tc['f16']['sm_mhz']} MHz; "
+                                  f"weighted 4:1 for the backward kernel's GEMMs")
+        # the same peaks scaled to the SM clock the step ran at (the loops draw more power and
+        # run at a lower clock than the attention kernels)
+        if step_mhz and tc["i8"]["sm_mhz"] and tc["f16"]["sm_mhz"]:
+            p8c = p8 * step_mhz / tc["i8"]["sm_mhz"]
+            p16c = p16 * step_mhz / tc["f16"]["sm_mhz"]
+            roofline["frac_at_step_clock"] = (kernels["attn_bwd_kernel"]["tops"]
+                                              / mixed_peak(p8c, p16c, 4, 1))
+            line_extra["frac_of_weighted_peak_at_step_clock"] = (
+                value / world / mixed_peak(p8c, p16c, 6, 1))
+        line_extra.update(frac_of_weighted_peak=value / world / p_all, weighted_peak_tops=p_all)
+    # the prologue's HBM roofline: 9 algorithmic bytes per (token, channel) -- q, k, v read at
+    # 2 bytes and their INT8 codes written at 1 byte
+    pro_bytes = 9.0 * w.B * w.H * w.N * w.d
+    pro_gbs = pro_bytes / (part["prologue"] * 1e-3) / 1e9
+    prologue = {"ms": part["prologue"], "algorithmic_bytes": pro_bytes, "gbs": pro_gbs,
+                "peak_gbs": pk["hbm_gbs"], "frac": pro_gbs / pk["hbm_gbs"],
+                "peak_note": f"{pk['basis']} HBM copy bandwidth"}
 
     line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8+bf16", "data": "synthetic", "config": config_of(w),
-            "frac_of_weighted_peak": value / world / p_all,
-            "weighted_peak_tops": p_all,
-            "kernels": {n: {"ms": round(v_["ms"], 4), "tops": round(v_["achieved"], 2),
-                            "frac": round(v_["achieved"] / v_["peak"], 4)}
-                        for n, v_ in kernels.items()},
+            **line_extra,
+            "kernels": {n: {k_: round(v_, 4) for k_, v_ in d.items()}
+                        for n, d in kernels.items()},
+            "stages_ms": {n: round(v_, 4) for n, v_ in part.items()},
+            "prologue": prologue, "tensor_peaks": tc,
+            "cublas_bf16_tflops": {"burst": pk["bf16_burst"], "sustained": pk["bf16_sustained"],
+                                   "basis": pk["basis"]},
             "roofline": roofline, "clocks": clocks, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -81,6 +81,11 @@ def lib() -> ctypes.CDLL:
         L.sage_fp4_quant_prologue.restype = i
         L.sage_fp4_attn_fwd.argtypes = [P(SageParams), P(SageFp4Bufs), vp, vp, vp, vp]
         L.sage_fp4_attn_fwd.restype = i
+        L.sage_fwd_bwd_host_workspace_bytes.argtypes = [P(SageParams), i]
+        L.sage_fwd_bwd_host_workspace_bytes.restype = sz
+        L.sage_fwd_bwd_host.argtypes = [P(SageParams), vp, vp, vp, vp, vp, vp, vp, vp, i, vp, sz,
+                                        vp, vp, vp]
+        L.sage_fwd_bwd_host.restype = i
         L.sage_last_device_status.argtypes = [vp]
         L.sage_last_device_status.restype = i
         L.sage_status_string.argtypes = [i]
@@ -89,6 +94,10 @@ def lib() -> ctypes.CDLL:
         L.sage_debug_qk_int32.restype = i
         L.sage_debug_umma_gemm.argtypes = [i, i, i, i, i, vp, vp, vp, vp]
         L.sage_debug_umma_gemm.restype = i
+        L.sage_debug_wait_timeout.argtypes = [i, vp]
+        L.sage_debug_wait_timeout.restype = i
+        L.sage_mma_peak.argtypes = [i, i, i, vp, sz, vp]
+        L.sage_mma_peak.restype = i
         _lib = L
     return _lib
 

@@ -432,16 +432,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       // back, hence the two slots.)
     };
     // maximum over the warps of q_block group g in warpgroup kh's key block (the tile's
-    // absmax of P or dS): all four warps (q_block = 128) or a pair (64)
+    // absmax of P or dS): all four warps (q_block = 128) or a pair (64).  Maxima below 2^-121,
+    // where the code multiplier 127 / max would overflow float32, are raised to 2^-121: such a
+    // tile is quantized (and dequantized) with the scale 2^-121 / 127 instead of max / 127, so
+    // its codes and scales stay finite and consistent (a zero tile keeps all-zero codes).
     auto tile_max = [&](const float* red, int g, int kh) {
       const float4 v = *reinterpret_cast<const float4*>(red + kh * 4);
-      if (wpg == 4) return fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
-      return g == 0 ? fmaxf(v.x, v.y) : fmaxf(v.z, v.w);
+      const float m = wpg == 4 ? fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w))
+                               : (g == 0 ? fmaxf(v.x, v.y) : fmaxf(v.z, v.w));
+      return fmaxf(m, 0x1p-121f);
     };
 
-    // pass B's code multipliers of tile `it` (its own row group and key half) from the tile
-    // maxima, once every warp has arrived.  Code multipliers use the fast divide (within 2 ulp;
-    // codes are not compared bit for bit); the read-outs' scales are IEEE quotients.  One
+    // pass B's code multipliers 127 / max of tile `it` (its own row group and key half) from
+    // the tile maxima, once every warp has arrived; IEEE quotients, like the read-outs' scales
+    // max / 127 (an approximate reciprocal would flush a subnormal maximum to zero).  One
     // barrier per tile parity, so arrivals for tiles it and it+1 never share a phase; a warp
     // cannot arrive for tile it+2 before every thread released tile it's dQ.
     auto multipliers = [&](int it, float& ip, float& ids, float& sdsc) {
@@ -449,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&sm.red_full[b], (it >> 1) & 1, 213);
       const float tp = tile_max(sm.red_p[b], g_row, h);
       const float tds = tile_max(sm.red_ds[b], g_row, h);
-      ip = tp > 0.0f ? __fdividef(127.0f, tp) : 0.0f;
-      ids = tds > 0.0f ? __fdividef(127.0f, tds) : 0.0f;
+      ip = __fdiv_rn(127.0f, tp);
+      ids = __fdiv_rn(127.0f, tds);
       sdsc = QS ? __fdiv_rn(tds, 127.0f) : 0.0f;  // Q-smoothing column sums: this group's scale
     };
 

@@ -4,7 +4,13 @@
 //     tcgen05 MMAs the attention kernels use, for every operand form they use (INT8 K-major
 //     and MN-major A and B; FP16/BF16 K-major);
 //   * debug_qk_kernel: the forward kernel's INT8 score product for one query tile against all
-//     keys of one head, through the forward kernel's own issue_scores().
+//     keys of one head, through the forward kernel's own issue_scores();
+//   * mma_peak_kernel: back-to-back tcgen05 MMAs from resident shared memory, one CTA per SM,
+//     so the host can time the tensor cores' sustained INT8 and 16-bit throughput (the
+//     denominators of the attention kernels' rooflines);
+//   * debug_wait_kernel: a bounded wait on an mbarrier that nothing arrives on, so tests can
+//     drive the kernels' failure path (timeout recorded in the status word, TMEM freed, the
+//     kernel returns) without hanging anything.
 #pragma once
 
 #include <stdint.h>
@@ -173,6 +179,93 @@ __global__ void __launch_bounds__(128, 1)
     tc_fence_after();
   }
   if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+struct PeakSmem {
+  uint8_t a[128 * 128];  // A: 128 rows x 128 bytes, 128-byte swizzle, K-major
+  uint8_t b[256 * 128];  // B: 256 rows x 128 bytes
+  uint64_t done;
+  uint32_t tmem_base;
+};
+constexpr int kPeakFillBytes = 128 * 128 + 256 * 128;
+
+// One thread issues `groups` x 4 MMAs of M = 128, N = 256 and K = 32 bytes (kind::i8: 32
+// elements; kind::f16: 16) back to back, alternating two 256-column accumulators; the
+// operands are `fill`'s first 48 KB, staged once.  kind 0: int8 -> int32; 1: fp16 -> fp32;
+// 2: bf16 -> fp32.
+__global__ void __launch_bounds__(128, 1)
+    mma_peak_kernel(const uint4* __restrict__ fill, int kind, int groups) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);
+  PeakSmem& sm = *reinterpret_cast<PeakSmem*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
+  const int warp = threadIdx.x >> 5;
+  uint4* dst = reinterpret_cast<uint4*>(sm.a);  // a and b are contiguous
+  for (int i = threadIdx.x; i < kPeakFillBytes / 16; i += blockDim.x) dst[i] = fill[i];
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.done, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (threadIdx.x == 0) {
+    const uint32_t ab = kind == 2 ? 1u : 0u;
+    const uint32_t id = kind == 0 ? instr_desc(2, 1, 1, false, false, 128, 256)
+                                  : instr_desc(1, ab, ab, false, false, 128, 256);
+    const uint32_t aa = smem_u32(sm.a), ba = smem_u32(sm.b);
+    for (int g = 0; g < groups; ++g) {
+      const uint32_t acc = tmem + (g & 1) * 256;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = smem_desc(aa + kk * 32, 16, 1024, kSwizzle128B);
+        const uint64_t bd = smem_desc(ba + kk * 32, 16, 1024, kSwizzle128B);
+        const uint32_t accum = (g >= 2 || kk > 0) ? 1u : 0u;
+        if (kind == 0)
+          mma_i8(acc, ad, bd, id, accum);
+        else
+          mma_f16(acc, ad, bd, id, accum);
+      }
+    }
+    mma_commit(&sm.done);
+    mbar_wait(&sm.done, 0, 320);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// One CTA holding TMEM waits (thread 0) on a barrier whose arrival never comes, for at most
+// limit_ns; the wait records SAGE_ERR_TIMEOUT (site 330), then the CTA frees its TMEM and
+// returns -- the same exit every pipeline kernel takes when one of its waits runs out.
+__global__ void __launch_bounds__(128, 1) debug_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tmem_base;
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0) mbar_wait_ns(&bar, 0, 330, limit_ns);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem_base, 32);
 }
 
 }  // namespace dbg

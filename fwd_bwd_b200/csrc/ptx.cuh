@@ -73,22 +73,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits until the phase with the given parity has completed.  Returns false on timeout.
-// Fully inlined: kernels that move registers between warpgroups (setmaxnreg) must not make
-// calls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site) {
+// Waits until the phase with the given parity has completed, for at most limit_ns
+// nanoseconds; on timeout records SAGE_ERR_TIMEOUT (with `site`) and returns false.  Fully
+// inlined: kernels that move registers between warpgroups (setmaxnreg) must not make calls.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, int site,
+                                             uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  const uint64_t limit = device_aborted() ? 1000000ull : 2000000000ull;  // 1 ms / 2 s
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > limit) {
+    if (global_timer_ns() - t0 > limit_ns) {
       record_timeout(site);
       return false;
     }
   }
+}
+
+// The kernels' wait: 2 s, or 1 ms once any wait on the device has failed (so the whole grid
+// drains quickly).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_ns(bar, parity, site, device_aborted() ? 1000000ull : 2000000000ull);
 }
 
 // Named barrier among `nthreads` threads (a multiple of 32) of the CTA.

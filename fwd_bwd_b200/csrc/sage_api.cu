@@ -435,6 +435,48 @@ int run_fp4_fwd(const sage_params* p, const sage_fp4_bufs* fb, const void* v, vo
   return launch_status();
 }
 
+// ---- end-to-end pipeline over host buffers -------------------------------------------------
+// One chunk slot of sage_fwd_bwd_host's device workspace: the chunk's 16-bit inputs and
+// outputs, its quantized views, LSE and the prologue / backward scratch; offsets from the
+// slot's start, each 256-byte aligned.
+struct HostSlot {
+  size_t in[4], out[4], qc, kc, vc, qs, ks, vs, qinv, kinv, kmean, qmean, kbias, lse, wpro, wbwd;
+  size_t total;
+};
+HostSlot host_slot(const sage_params* cp) {  // cp->B = the largest chunk's batch
+  const size_t BH = static_cast<size_t>(cp->B) * cp->H, N = cp->N, d = cp->d, e = BH * N * d;
+  HostSlot s;
+  size_t at = 0;
+  auto take = [&](size_t bytes) {
+    const size_t here = at;
+    at = align_up(at + bytes);
+    return here;
+  };
+  for (int i = 0; i < 4; ++i) s.in[i] = take(e * 2);
+  for (int i = 0; i < 4; ++i) s.out[i] = take(e * 2);
+  s.qc = take(e);
+  s.kc = take(e);
+  s.vc = take(e);
+  s.qs = take(BH * (N / cp->q_block) * 4);
+  s.ks = take(BH * (N / cp->k_block) * 4);
+  s.vs = take(BH * (N / cp->k_block) * 4);
+  s.qinv = take(BH * N * 4);
+  s.kinv = take(BH * N * 4);
+  s.kmean = take(BH * d * 4);
+  s.qmean = take(BH * d * 4);
+  s.kbias = take(BH * N * 4);
+  s.lse = take(BH * N * 4);
+  s.wpro = take(prologue_ws(cp));
+  s.wbwd = take(bwd_ws(cp).total);
+  s.total = at;
+  return s;
+}
+sage_params largest_chunk(const sage_params* p, int chunks) {
+  sage_params cp = *p;
+  cp.B = (p->B + chunks - 1) / chunks;
+  return cp;
+}
+
 // ---- prologue scratch for callers that cannot allocate -------------------------------------
 // A fixed device array that sage_quant_prologue_noalloc uses instead of a caller workspace for
 // the K-smoothing column sums.  Every device that loads the library holds it until exit.
@@ -546,6 +588,101 @@ int sage_attn_bwd_stage(int stage, const sage_params* p, const void* q, const vo
                    stream);
 }
 
+size_t sage_fwd_bwd_host_workspace_bytes(const sage_params* p, int chunks) {
+  if (check_params(p) != SAGE_OK || chunks < 1) return 0;
+  chunks = chunks < p->B ? chunks : p->B;
+  const sage_params cp = largest_chunk(p, chunks);
+  return 2 * host_slot(&cp).total;
+}
+
+int sage_fwd_bwd_host(const sage_params* p, const void* q, const void* k, const void* v,
+                      const void* dout, void* o, void* dq, void* dk, void* dv, int chunks,
+                      void* workspace, size_t workspace_bytes, void* stream_in,
+                      void* stream_compute, void* stream_out) {
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if (!q || !k || !v || !dout || !o || !dq || !dk || !dv || chunks < 1)
+    return SAGE_ERR_INVALID_ARG;
+  chunks = chunks < p->B ? chunks : p->B;
+  const sage_params cp = largest_chunk(p, chunks);
+  const HostSlot L = host_slot(&cp);
+  if (!workspace || workspace_bytes < 2 * L.total) return SAGE_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return SAGE_ERR_ALIGNMENT;
+  cudaStream_t sin = reinterpret_cast<cudaStream_t>(stream_in);
+  cudaStream_t scomp = reinterpret_cast<cudaStream_t>(stream_compute);
+  cudaStream_t sout = reinterpret_cast<cudaStream_t>(stream_out);
+  // [0]: a slot's inputs are on the device, [1]: its kernels are done, [2]: its results left
+  cudaEvent_t ev[3][2] = {};
+  for (auto& row : ev)
+    for (auto& e : row)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) s = SAGE_ERR_CUDA;
+  const void* hin[4] = {q, k, v, dout};
+  void* hout[4] = {o, dq, dk, dv};
+  const size_t per_b = static_cast<size_t>(p->H) * p->N * p->d * 2;  // bytes per batch entry
+  for (int c = 0; c < chunks && s == SAGE_OK; ++c) {
+    const int b0 = static_cast<int>(static_cast<long long>(p->B) * c / chunks);
+    const int b1 = static_cast<int>(static_cast<long long>(p->B) * (c + 1) / chunks);
+    const int slot = c & 1;
+    uint8_t* base = reinterpret_cast<uint8_t*>(workspace) + slot * L.total;
+    sage_params pc = *p;
+    pc.B = b1 - b0;
+    const size_t bytes = static_cast<size_t>(b1 - b0) * per_b, off = b0 * per_b;
+    auto ok = [&](cudaError_t e) {
+      if (e != cudaSuccess && s == SAGE_OK) s = SAGE_ERR_CUDA;
+    };
+    // host -> device: the slot's previous chunk (c - 2) must have finished reading its inputs
+    if (c >= 2) ok(cudaStreamWaitEvent(sin, ev[1][slot], 0));
+    for (int i = 0; i < 4; ++i)
+      ok(cudaMemcpyAsync(base + L.in[i], static_cast<const uint8_t*>(hin[i]) + off, bytes,
+                         cudaMemcpyHostToDevice, sin));
+    ok(cudaEventRecord(ev[0][slot], sin));
+    // kernels: after the inputs arrived and chunk c - 2's results left the slot
+    ok(cudaStreamWaitEvent(scomp, ev[0][slot], 0));
+    if (c >= 2) ok(cudaStreamWaitEvent(scomp, ev[2][slot], 0));
+    if (s != SAGE_OK) break;
+    sage_qbufs qb;
+    qb.q_codes = reinterpret_cast<int8_t*>(base + L.qc);
+    qb.k_codes = reinterpret_cast<int8_t*>(base + L.kc);
+    qb.v_codes = reinterpret_cast<int8_t*>(base + L.vc);
+    qb.q_scale = reinterpret_cast<float*>(base + L.qs);
+    qb.k_scale = reinterpret_cast<float*>(base + L.ks);
+    qb.v_scale = reinterpret_cast<float*>(base + L.vs);
+    qb.q_inv_rms = reinterpret_cast<float*>(base + L.qinv);
+    qb.k_inv_rms = reinterpret_cast<float*>(base + L.kinv);
+    qb.k_mean = reinterpret_cast<float*>(base + L.kmean);
+    qb.q_mean = reinterpret_cast<float*>(base + L.qmean);
+    qb.k_bias = reinterpret_cast<float*>(base + L.kbias);
+    float* lse = reinterpret_cast<float*>(base + L.lse);
+    void* din[4];
+    void* dres[4];
+    for (int i = 0; i < 4; ++i) {
+      din[i] = base + L.in[i];
+      dres[i] = base + L.out[i];
+    }
+    s = sage_quant_prologue(&pc, din[0], din[1], din[2], &qb, base + L.wpro, prologue_ws(&pc),
+                            scomp);
+    if (s == SAGE_OK) s = sage_attn_fwd(&pc, &qb, dres[0], lse, nullptr, 0, scomp);
+    if (s == SAGE_OK)
+      s = sage_attn_bwd(&pc, din[0], din[1], din[2], &qb, dres[0], lse, din[3], dres[1],
+                        dres[2], dres[3], base + L.wbwd, bwd_ws(&pc).total, scomp);
+    if (s != SAGE_OK) break;
+    ok(cudaEventRecord(ev[1][slot], scomp));
+    // device -> host once the kernels are done
+    ok(cudaStreamWaitEvent(sout, ev[1][slot], 0));
+    for (int i = 0; i < 4; ++i)
+      ok(cudaMemcpyAsync(static_cast<uint8_t*>(hout[i]) + off, base + L.out[i], bytes,
+                         cudaMemcpyDeviceToHost, sout));
+    ok(cudaEventRecord(ev[2][slot], sout));
+  }
+  // whatever happened, nothing of this call is left in flight when it returns
+  for (cudaStream_t st : {sin, scomp, sout})
+    if (cudaStreamSynchronize(st) != cudaSuccess && s == SAGE_OK) s = SAGE_ERR_CUDA;
+  for (auto& row : ev)
+    for (auto& e : row)
+      if (e) cudaEventDestroy(e);
+  return s;
+}
+
 size_t sage_fp4_workspace_bytes(const sage_params* p, int which) {
   if (check_fp4(p) != SAGE_OK) return 0;
   return which == 0 ? fp4_ws(p).total : 0;
@@ -655,6 +792,27 @@ int sage_debug_umma_gemm(int kind, int a_mn_major, int b_mn_major, int N, int K,
   if (set_smem(sage::dbg::debug_gemm_kernel, smem) != SAGE_OK) return SAGE_ERR_CUDA;
   sage::dbg::debug_gemm_kernel<<<1, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
       ta, tb, kind, a_mn_major, b_mn_major, N, K, C);
+  return launch_status();
+}
+
+int sage_debug_wait_timeout(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return SAGE_ERR_INVALID_ARG;
+  sage::dbg::debug_wait_kernel<<<1, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_us) * 1000ull);
+  return launch_status();
+}
+
+int sage_mma_peak(int kind, int n_ctas, int groups, const void* fill, size_t fill_bytes,
+                  void* stream) {
+  if (kind < 0 || kind > 2 || !fill) return SAGE_ERR_INVALID_ARG;
+  if (n_ctas < 1 || n_ctas > 65535 || groups < 1 || groups > (1 << 26))
+    return SAGE_ERR_INVALID_ARG;
+  if (fill_bytes < static_cast<size_t>(sage::dbg::kPeakFillBytes)) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(fill)) return SAGE_ERR_ALIGNMENT;
+  const size_t smem = sizeof(sage::dbg::PeakSmem) + 1024;
+  if (set_smem(sage::dbg::mma_peak_kernel, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+  sage::dbg::mma_peak_kernel<<<n_ctas, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint4*>(fill), kind, groups);
   return launch_status();
 }
 

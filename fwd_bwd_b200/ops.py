@@ -201,6 +201,29 @@ def umma_gemm_debug(kind: int, a: torch.Tensor, b: torch.Tensor, a_mn: bool, b_m
     return c
 
 
+def wait_timeout_debug(limit_us: int, device=None) -> None:
+    """Launch a kernel whose bounded barrier wait runs out (sage_debug_wait_timeout)."""
+    check("sage_debug_wait_timeout",
+          lib().sage_debug_wait_timeout(int(limit_us), _stream(device)))
+
+
+def mma_peak(kind: int, n_ctas: int, groups: int, fill: torch.Tensor) -> None:
+    """Launch the tensor-core throughput loop (sage_mma_peak) on the current stream.
+
+    ``kind`` 0 = INT8, 1 = fp16, 2 = bf16; ``fill`` is a device tensor of at least 48 KB whose
+    bytes become the operands.  Ops per launch: see ``mma_peak_ops``.
+    """
+    check("sage_mma_peak", lib().sage_mma_peak(kind, n_ctas, groups, fill.data_ptr(),
+                                               fill.numel() * fill.element_size(),
+                                               _stream(fill.device)))
+
+
+def mma_peak_ops(kind: int, n_ctas: int, groups: int) -> float:
+    """Operations of one sage_mma_peak launch: 4 MMAs of 128 x 256 x K per group and CTA."""
+    k = 32 if kind == 0 else 16
+    return float(n_ctas) * groups * 4 * 2 * 128 * 256 * k
+
+
 def qk_int32_debug(qb: QuantBufs, like: torch.Tensor, cfg: Config, bh: int,
                    q_tile: int) -> torch.Tensor:
     """INT8 score tile Qc Kc^T of the forward kernel's MMA path (sage_debug_qk_int32)."""
@@ -217,61 +240,46 @@ def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
 
 
-def fwd_bwd_host(q, k, v, dout, cfg: Config, o=None, dq=None, dk=None, dv=None,
-                 chunks: int = 16, device=None):
-    """Prologue + forward + backward on host-resident (pinned) [B, H, N, d] tensors.
+def host_workspace_bytes(cfg: Config, like: torch.Tensor, chunks: int) -> int:
+    """Device workspace of fwd_bwd_host (sage_fwd_bwd_host_workspace_bytes)."""
+    return int(lib().sage_fwd_bwd_host_workspace_bytes(ctypes.byref(cfg.params(like)), chunks))
 
-    Every (batch, head) is an independent problem, so the batch is cut into ``chunks`` slices
-    that flow through three CUDA streams: host-to-device copies of slice c+1 and
-    device-to-host copies of slice c-1 overlap the kernels of slice c.  Two sets of device
-    buffers alternate between slices.  Results (o, dq, dk, dv) are written into pinned host
-    tensors (allocated when not given); the call returns once they are complete.  Inputs
-    should be pinned (page-locked) for the copies to run asynchronously.
+
+class HostPipeline:
+    """Device workspace and streams for repeated ``fwd_bwd_host`` calls on one device."""
+
+    def __init__(self, like: torch.Tensor, cfg: Config, chunks: int = 16, device=None):
+        self.device = torch.device("cuda") if device is None else torch.device(device)
+        self.chunks = chunks
+        n = host_workspace_bytes(cfg, like, chunks)
+        self.workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=self.device)
+        self.streams = [torch.cuda.Stream(self.device) for _ in range(3)]
+
+
+def fwd_bwd_host(q, k, v, dout, cfg: Config, o=None, dq=None, dk=None, dv=None,
+                 chunks: int = 16, device=None, pipeline: Optional[HostPipeline] = None):
+    """Prologue + forward + backward on host-resident [B, H, N, d] tensors (sage_fwd_bwd_host).
+
+    The C entry point cuts the batch into ``chunks`` slices and overlaps each slice's
+    host-to-device copies, kernels and device-to-host copies on three streams; it returns once
+    the results (o, dq, dk, dv; pinned host tensors, allocated when not given) are complete.
+    Inputs should be pinned for the copies to run asynchronously.  ``pipeline`` reuses a device
+    workspace and streams across calls.
     """
-    device = torch.device("cuda") if device is None else torch.device(device)
-    B = q.shape[0]
-    chunks = max(1, min(chunks, B))
-    bounds = [(B * c // chunks, B * (c + 1) // chunks) for c in range(chunks)]
+    for t in (q, k, v, dout):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("fwd_bwd_host takes contiguous host tensors")
     outs = []
     for t, ref in ((o, q), (dq, q), (dk, k), (dv, v)):
         outs.append(t if t is not None else torch.empty(ref.shape, dtype=ref.dtype,
                                                          pin_memory=True))
-    cb = max(b1 - b0 for b0, b1 in bounds)
-    shape = (cb,) + tuple(q.shape[1:])
-    sets = []
-    for _ in range(2):
-        ins = [torch.empty(shape, dtype=q.dtype, device=device) for _ in range(4)]
-        res = [torch.empty(shape, dtype=q.dtype, device=device) for _ in range(4)]
-        sets.append((ins, res))
-    s_in, s_comp, s_out = (torch.cuda.Stream(device) for _ in range(3))
-    in_done = [torch.cuda.Event() for _ in range(2)]
-    comp_done = [torch.cuda.Event() for _ in range(2)]
-    out_done = [torch.cuda.Event() for _ in range(2)]
-    used = [False, False]
-    for c, (b0, b1) in enumerate(bounds):
-        si = c % 2
-        ins, res = sets[si]
-        n = b1 - b0
-        with torch.cuda.stream(s_in):
-            if used[si]:
-                s_in.wait_event(comp_done[si])  # the kernels of slice c-2 have read the inputs
-            for dst, src in zip(ins, (q, k, v, dout)):
-                dst[:n].copy_(src[b0:b1], non_blocking=True)
-            in_done[si].record(s_in)
-        with torch.cuda.stream(s_comp):
-            s_comp.wait_event(in_done[si])
-            if used[si]:
-                s_comp.wait_event(out_done[si])  # slice c-2's results have left the device
-            qd, kd, vd, dod = (t[:n] for t in ins)
-            qb = quant_prologue(qd, kd, vd, cfg)
-            od, lse = attn_fwd(qb, qd, cfg, o=res[0][:n])
-            attn_bwd(qd, kd, vd, qb, od, lse, dod, cfg, res[1][:n], res[2][:n], res[3][:n])
-            comp_done[si].record(s_comp)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(comp_done[si])
-            for src, dst in zip(res, outs):
-                dst[b0:b1].copy_(src[:n], non_blocking=True)
-            out_done[si].record(s_out)
-        used[si] = True
-    s_out.synchronize()
+    if pipeline is None:
+        pipeline = HostPipeline(q, cfg, chunks, device)
+    prm = cfg.params(q)
+    ws = pipeline.workspace
+    with torch.cuda.device(pipeline.device):
+        check("sage_fwd_bwd_host", lib().sage_fwd_bwd_host(
+            ctypes.byref(prm), q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
+            *(t.data_ptr() for t in outs), pipeline.chunks, ws.data_ptr(), ws.numel(),
+            *(s_.cuda_stream for s_ in pipeline.streams)))
     return tuple(outs)

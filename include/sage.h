@@ -14,8 +14,9 @@
  * Conventions shared by every entry point
  *   Layout     All tensors are contiguous [B, H, N, d] with d innermost; per-block scales are
  *              [B, H, N / block]; per-token vectors [B, H, N]; K means [B, H, d].
- *   Pointers   Every pointer is a DEVICE pointer, allocated and owned by the caller; the
- *              library never allocates, frees or retains memory.  Tensor pointers must be
+ *   Pointers   Every pointer is a DEVICE pointer, allocated and owned by the caller, except
+ *              the tensors of sage_fwd_bwd_host (host memory); the library never allocates,
+ *              frees or retains memory.  Tensor pointers must be
  *              16-byte aligned.  Work is asynchronous on `stream` (a cudaStream_t; NULL = the
  *              legacy default stream); buffers must stay valid until the stream reaches it.
  *   Shapes     d in {64, 128}; k_block == 64; q_block in {64, 128}; N a multiple of 128.
@@ -154,6 +155,28 @@ int sage_attn_bwd_stage(int stage, const sage_params* p, const void* q, const vo
                         const void* dout, void* dq, void* dk, void* dv, void* workspace,
                         size_t workspace_bytes, void* stream);
 
+/* The whole step -- prologue, forward, backward -- on HOST buffers (end to end: the operator as
+ * a host program calls it).  q, k, v, dout and the results o, dq, dk, dv are host pointers to
+ * [B,H,N,d] 16-bit tensors; pin them (cudaHostAlloc / cudaHostRegister) for the copies to run
+ * asynchronously (pageable memory works, with copies that block the host).  Every (batch, head)
+ * is independent, so the batch is cut into `chunks` contiguous slices of B*c/chunks ..
+ * B*(c+1)/chunks (chunks is capped at B) that flow through two device slots: slice c's
+ * host-to-device copies run on stream_in, its kernels on stream_compute and its device-to-host
+ * copies on stream_out, so the copies of neighbouring slices overlap slice c's kernels.  One
+ * cudaMemcpyAsync per tensor and slice.  `workspace` is caller-owned device memory of at least
+ * sage_fwd_bwd_host_workspace_bytes(p, chunks) bytes (16-byte aligned) holding both slots.  The
+ * three streams are caller-owned (distinct streams overlap; NULL serializes everything on the
+ * legacy default stream); the library creates six CUDA events for the call and destroys them
+ * before returning.  The call returns once the results are in host memory (or on the first
+ * error, after draining the streams); results equal sage_quant_prologue + sage_attn_fwd +
+ * sage_attn_bwd run on the same data on the device.  Read sage_last_device_status() afterwards
+ * for device-side timeouts. */
+size_t sage_fwd_bwd_host_workspace_bytes(const sage_params* p, int chunks);
+int sage_fwd_bwd_host(const sage_params* p, const void* q, const void* k, const void* v,
+                      const void* dout, void* o, void* dq, void* dk, void* dv, int chunks,
+                      void* workspace, size_t workspace_bytes, void* stream_in,
+                      void* stream_compute, void* stream_out);
+
 /* Synchronizes `stream`, returns the device status word of the current device (SAGE_OK or
  * SAGE_ERR_TIMEOUT) and clears it.  Returns SAGE_ERR_CUDA if the synchronization fails. */
 int sage_last_device_status(void* stream);
@@ -173,6 +196,32 @@ int sage_debug_qk_int32(const sage_params* p, const sage_qbufs* qb, int bh, int 
                         int32_t* s_out, void* stream);
 int sage_debug_umma_gemm(int kind, int a_mn_major, int b_mn_major, int N, int K, const void* A,
                          const void* B, void* C, void* stream);
+
+/* sage_debug_wait_timeout: drives the kernels' failure path on purpose, without a fault.  One
+ * CTA allocates tensor memory and waits on a shared-memory barrier that nothing ever arrives
+ * on, for at most limit_us microseconds (1 .. 1e6); the wait then records SAGE_ERR_TIMEOUT in
+ * the device status word, the CTA frees its tensor memory and returns, exactly as a pipeline
+ * kernel does when one of its bounded waits runs out.  Until the status word is read and
+ * cleared by sage_last_device_status(), the attention kernels launched afterwards on the same
+ * device see the recorded failure and return at once without writing their outputs.  Returns
+ * SAGE_ERR_INVALID_ARG for limit_us out of range, before launching. */
+int sage_debug_wait_timeout(int limit_us, void* stream);
+
+/* ---- measurement support: the tensor cores' own peak ---------------------------------------
+ * sage_mma_peak launches n_ctas CTAs (one per SM: pass the SM count), each of which stages
+ * the first 48 KB of `fill` (a device buffer of at least 49152 bytes, 16-byte aligned; give it
+ * random int8 codes for kind 0 and random fp16 / bf16 values for kinds 1 / 2 so the operands
+ * toggle like real data) in shared memory and issues `groups` x 4 back-to-back tcgen05 MMAs of
+ * M = 128, N = 256 from it: kind 0 = kind::i8 (K = 32 per MMA, INT32 accumulation), 1 = fp16
+ * and 2 = bf16 (kind::f16, K = 16, float32 accumulation).  Each CTA performs
+ * groups * 4 * 2 * 128 * 256 * K operations; the caller times the launch on `stream` with CUDA
+ * events.  This is the denominator of the attention kernels' rooflines (the quantization-
+ * strategy paragraph's six INT8 and one 16-bit matmul run at these two rates); it computes
+ * nothing the attention uses.  groups in [1, 2^26]; keep one launch well under a second (the
+ * issuing thread's completion wait gives up after two seconds and records SAGE_ERR_TIMEOUT).
+ * Returns SAGE_ERR_INVALID_ARG / SAGE_ERR_ALIGNMENT for bad arguments before launching. */
+int sage_mma_peak(int kind, int n_ctas, int groups, const void* fill, size_t fill_bytes,
+                  void* stream);
 
 #ifdef __cplusplus
 }

@@ -29,11 +29,49 @@ def _declared(header="sage.h"):
 
 def test_exports_every_declared_symbol(L):
     names = _declared()
-    assert len(names) == 10
+    assert len(names) == 14
     fp4 = _declared("sage_nvfp4.h")
     assert fp4 == ["sage_fp4_attn_fwd", "sage_fp4_quant_prologue", "sage_fp4_workspace_bytes"]
     for n in names + fp4:
         assert hasattr(L, n), n
+
+
+def test_host_pipeline_workspace_and_argument_checks(L):
+    p = _params()  # B2 H4 N1024 d128 bf16, ksmooth
+    n1 = L.sage_fwd_bwd_host_workspace_bytes(ctypes.byref(p), 1)
+    n2 = L.sage_fwd_bwd_host_workspace_bytes(ctypes.byref(p), 2)
+    assert n1 > n2 > 0  # two slots of the largest slice: B/1 vs B/2 batch entries
+    assert L.sage_fwd_bwd_host_workspace_bytes(ctypes.byref(p), 99) == n2  # capped at B
+    assert L.sage_fwd_bwd_host_workspace_bytes(ctypes.byref(p), 0) == 0
+    # 16-bit inputs and outputs (8 tensors) dominate each slot
+    e = 1 * 4 * 1024 * 128 * 2
+    assert n2 >= 2 * 8 * e
+    fake = 1 << 20  # never dereferenced: every call below fails its host-side checks
+    ten = [fake] * 8
+    f = L.sage_fwd_bwd_host
+    assert f(ctypes.byref(p), *ten, 0, fake, n2, None, None, None) == _lib.SAGE_ERR_INVALID_ARG
+    assert f(ctypes.byref(p), None, *ten[1:], 2, fake, n2, None, None, None) == \
+        _lib.SAGE_ERR_INVALID_ARG
+    assert f(ctypes.byref(p), *ten, 2, fake, n2 - 1, None, None, None) == _lib.SAGE_ERR_WORKSPACE
+    assert f(ctypes.byref(p), *ten, 2, None, n2, None, None, None) == _lib.SAGE_ERR_WORKSPACE
+    assert f(ctypes.byref(p), *ten, 2, fake + 8, n2, None, None, None) == _lib.SAGE_ERR_ALIGNMENT
+    assert f(ctypes.byref(_params(d=96)), *ten, 2, fake, n2, None, None, None) == \
+        _lib.SAGE_ERR_UNSUPPORTED
+
+
+def test_wait_timeout_argument_checks(L):
+    for bad in (0, -5, 1000001):
+        assert L.sage_debug_wait_timeout(bad, None) == _lib.SAGE_ERR_INVALID_ARG
+
+
+def test_mma_peak_argument_checks(L):
+    fake = 1 << 20  # never dereferenced: every call below fails its host-side checks
+    bad = [(3, 148, 10, fake, 49152), (-1, 148, 10, fake, 49152), (0, 0, 10, fake, 49152),
+           (0, 148, 0, fake, 49152), (0, 148, (1 << 26) + 1, fake, 49152),
+           (0, 148, 10, None, 49152), (1, 148, 10, fake, 49151)]
+    for args in bad:
+        assert L.sage_mma_peak(*args, None) == _lib.SAGE_ERR_INVALID_ARG, args
+    assert L.sage_mma_peak(2, 148, 10, fake + 4, 49152, None) == _lib.SAGE_ERR_ALIGNMENT
 
 
 def test_fp4_workspace_and_argument_checks(L):

@@ -4,7 +4,11 @@
   attention is uniform, O = 0 and every gradient is 0;
 * identical keys with K-smoothing: smoothed K is exactly 0, so the scores vanish and O is the
   running mean of V (causal) -- the closed form the oracle is also pinned to;
-* large magnitudes (|x| ~ 1e3, bf16): the quantization is scale-invariant, so parity holds.
+* large magnitudes (|x| ~ 1e3, bf16): the quantization is scale-invariant, so parity holds;
+* tiny gradients (dO ~ 2^-100) and key blocks whose probabilities -- and so the backward's P and
+  dS tile maxima -- lie in float32's subnormal range: every output stays finite and parity
+  holds (the code multipliers 127 / max are IEEE quotients; the NVFP4 page on Quartet II
+  reports an approximate reciprocal that flushed subnormals to zero and produced NaN).
 """
 import numpy as np
 import pytest
@@ -79,4 +83,45 @@ def test_extreme_magnitudes(case):
     o = oracle_run(w, x)
     BH = w.B * w.H
     for n in ("o", "dq", "dk", "dv"):
+        assert rel_l2(g[n].reshape(BH, w.N, w.d), o[n]) <= 2e-3, n
+
+
+def test_tiny_gradients():
+    """dO ~ 2^-100 (bf16 keeps float32's exponent range): the dS and dO scales are ~2^-107,
+    their products with the Q / K / P scales stay normal floats, and parity holds."""
+    w = BASE.replace(qknorm=False, ksmooth=False)
+    x = make_inputs(w)
+    x = _with(x, w, do=x["do_f32"] * 2.0 ** -100)
+    g = gpu_run(w, x)
+    o = oracle_run(w, x)
+    BH = w.B * w.H
+    for n in ("o", "dq", "dk", "dv"):
+        assert np.all(np.isfinite(g[n])), n
+        assert rel_l2(g[n].reshape(BH, w.N, w.d), o[n]) <= 2e-3, n
+
+
+def test_subnormal_tile_maxima():
+    """Channel 0 of every query is +30 and key blocks 1, 3 and 5 have channel 0 at -33.5, so their
+    scores sit ~89 below the rows' maxima: P ~ e^-89 and dS there are float32 subnormals, and so
+    are those tiles' maxima.  Outputs must stay finite and match the oracle (the tiles below
+    2^-121 contribute only ~1e-38 to any output)."""
+    w = BASE.replace(qknorm=False, ksmooth=False, causal=False)
+    x = make_inputs(w)
+    q = x["q_f32"].copy()
+    k = x["k_f32"].copy()
+    q[..., 0] = 30.0
+    for blk in (1, 3, 5):
+        k[..., blk * 64:(blk + 1) * 64, 0] = -33.5
+    x = _with(x, w, q=q, k=k)
+    g = gpu_run(w, x)
+    o = oracle_run(w, x)
+    BH = w.B * w.H
+    # the case is what it claims: the far blocks' probabilities are subnormal in float32
+    z = np.einsum("hnd,hmd->hnm", q.reshape(BH, w.N, w.d).astype(np.float64),
+                  k.reshape(BH, w.N, w.d).astype(np.float64)) / np.sqrt(w.d)
+    p = np.exp(z - o["lse"][:, :, None])
+    far = p[:, :, 64:128]
+    assert far.max() < 1.1754944e-38 and far.max() > 1e-44
+    for n in ("o", "dq", "dk", "dv"):
+        assert np.all(np.isfinite(g[n])), n
         assert rel_l2(g[n].reshape(BH, w.N, w.d), o[n]) <= 2e-3, n

@@ -1,6 +1,7 @@
-"""The host-buffer API (batch slices streamed through copy / compute / copy streams) gives the
-same results as the device-resident path: O, dK, dV bit for bit (each head's arithmetic is
-independent of how the batch is sliced), dQ up to the order of its float32 atomics."""
+"""The host-buffer entry point sage_fwd_bwd_host (batch slices streamed through copy / compute /
+copy streams inside the C library) gives the same results as the device-resident path: O, dK,
+dV bit for bit (each head's arithmetic is independent of how the batch is sliced), dQ up to the
+order of its float32 reductions.  Two calls in a row reuse one workspace and stream set."""
 import numpy as np
 import pytest
 import torch
@@ -21,7 +22,9 @@ def test_host_pipeline_matches_device_path(name, chunks):
     host = [torch.from_numpy(x[n].view(np.int16)).view(dt).pin_memory()
             for n in ("q", "k", "v", "do")]
     cfg = cfg_of(w)
-    o_h, dq_h, dk_h, dv_h = ops.fwd_bwd_host(*host, cfg, chunks=chunks)
+    pipe = ops.HostPipeline(host[0], cfg, chunks)
+    for _ in range(2):
+        o_h, dq_h, dk_h, dv_h = ops.fwd_bwd_host(*host, cfg, pipeline=pipe)
     q, k, v, do = (t.cuda() for t in host)
     qb = ops.quant_prologue(q, k, v, cfg)
     o, lse = ops.attn_fwd(qb, q, cfg)
