@@ -14,7 +14,8 @@ loop (sage_mma_peak), weighted by each kernel's mix of INT8 and 16-bit GEMMs.
 
 Multi-GPU (torchrun): every (batch, head) is independent and the operator has no weights, so
 each rank runs its own full-size batch with no collective on the data path (weak scaling); the
-harness takes the maximum elapsed time over ranks.
+harness takes the maximum elapsed time over ranks.  The end-to-end leg streams one global batch
+from host memory, split across the ranks in contiguous batch ranges.
 
 ``--impl reference`` times the CPU oracle (the plain restatement of the method the tests
 check the kernels against) on a bounded sample of the same workload.
@@ -465,13 +466,16 @@ def main():
 
     # end to end through the C ABI's host-buffer call (sage_fwd_bwd_host): pinned host inputs
     # in, pinned host results out, the copies and their overlap with the kernels inside the
-    # timed region.  Under torchrun every rank streams a 1/world slice of its batch, so the
-    # pinned host memory per node stays that of one full batch.
+    # timed region.  One global batch of B entries is split across the ranks (contiguous batch
+    # ranges, shard.head_range), so the pinned host memory per node stays that of one batch.
     e2e = None
     if not args.no_e2e:
-        bsl = max(1, w.B // world)
+        from fwd_bwd_b200.shard import head_range
+
+        mine = head_range(w.B, world, rank)
+        bsl = len(mine)
         hin = [torch.empty((bsl,) + tuple(t.shape[1:]), dtype=t.dtype,
-                           pin_memory=True).copy_(t[:bsl]) for t in (q, k, v, do)]
+                           pin_memory=True).copy_(t[mine.start:mine.stop]) for t in (q, k, v, do)]
         hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in hin]
         del q, k, v, do, o, dq, dk, dv, qb, ws_pro, ws_bwd, lse, x, flush_buf
         torch.cuda.empty_cache()
@@ -498,12 +502,12 @@ def main():
             e_ms = float(t.item())
         if ops.device_status(dev) != 0:
             raise RuntimeError("device status reports a kernel timeout in the e2e run")
-        e_ops = w.ops() * bsl / w.B * world
-        e2e = {"value": e_ops / (e_ms / args.steps * 1e-3) / 1e12, "unit": "TOPS",
+        e2e = {"value": w.ops() / (e_ms / args.steps * 1e-3) / 1e12, "unit": "TOPS",
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hin),
                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout),
                "chunks": args.chunks, "api": "sage_fwd_bwd_host",
-               "batch_per_rank": bsl}
+               "global_batch": w.B, "batch_per_rank": bsl,
+               "bytes_note": "per rank; one global batch split across the ranks"}
 
     pk = peaks()
     bwd_ops, fwd_ops = w.ops("bwd"), w.ops("fwd")

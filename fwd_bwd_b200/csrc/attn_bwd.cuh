@@ -13,7 +13,9 @@
 //   3. dV_t = Pc^T dOc and dK_t = dSc^T Qc (kind::i8, M = 128 keys, one per q_block group),
 //      dequantized by the tile scales and added to float32 accumulators in registers;
 //      every INT32 accumulator region is preloaded with the bits of 1.5 * 2^23 so the results
-//      read back as floats that one exact FMA dequantizes (see kMagicBits);
+//      read back as floats that one exact FMA dequantizes (see kMagicBits); the MMA thread
+//      writes every preload with one bf16 MMA (mma_fill_magic), so the compute warps store to
+//      TMEM only P and dS in pass A;
 //   4. dQ_t = dSc Kc per 64-key block (kind::i8), dequantized, summed and added to a float32
 //      dQ accumulator in global memory: for d = 128 computed transposed (TMEM lanes = head-dim
 //      channels), staged per warp in shared memory and added by the TMA unit
@@ -86,6 +88,7 @@ struct Smem {
   // d = 128: dQ staging for the asynchronous bulk reduction,
   // [compute warp][buffer][query row][channel of the warp]
   float dqs[D == 128 ? 8 : 1][2][D == 128 ? kDqRows * kDqCols : 4];
+  alignas(256) uint8_t fill[kFillBytes];  // operands of the preload MMA (mma_fill_magic)
   alignas(16) float red_p[2][8];  // per-warp tile maxima of P, [tile parity][warp]
   alignas(16) float red_ds[2][8];  // and of |dS|
   float dot[BKT];                   // RMSNorm-backward row dot products (warpgroup 1 -> 0)
@@ -114,8 +117,9 @@ constexpr bool tiles_aligned() {
          offsetof(Stage<D>, doc) % 1024 == 0 && offsetof(Smem<D>, dor) % 1024 == 0 &&
          offsetof(Smem<D>, kc) % 1024 == 0 && offsetof(Smem<D>, v) % 1024 == 0 &&
          offsetof(Smem<D>, pc) % 1024 == 0 && offsetof(Smem<D>, dsc) % 1024 == 0 &&
-         offsetof(Smem<D>, dqs) % 1024 == 0;
+         offsetof(Smem<D>, dqs) % 1024 == 0 && offsetof(Smem<D>, fill) % 256 == 0;
 }
+static_assert(smem_bytes<128>() <= 232448, "shared memory exceeds the per-block limit");
 static_assert(tiles_aligned<64>() && tiles_aligned<128>(), "shared-memory tiles misaligned");
 
 struct Args {
@@ -166,6 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nq = N / BQ - i_first;
   const int G = BQ / args.q_block;  // q_block groups per query tile (1 or 2)
 
+  write_fill_operands(sm.fill, threadIdx.x, kThreads);
+  fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     sm.abort = device_aborted() ? 1 : 0;
     mbar_init(&sm.kv_full, 1);
@@ -202,20 +208,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   const int row_base = bh * N;
-  if (warp < 8) {
-    // INT32 accumulators are preloaded with the bits of 1.5 * 2^23 (see kMagicBits): the S
-    // regions of both TMEM buffers, this thread's lane, this warpgroup's 64-column half
-    const uint32_t lb = tmem + (((warp & 3) * 32u) << 16) + (warp >> 2) * 64;
-#pragma unroll
-    for (int c = 0; c < 64; c += 16) {
-      tmem_fill16(lb + c, kMagicBits);
-      tmem_fill16(lb + 256 + c, kMagicBits);
-    }
-    tmem_st_wait();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
 
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
@@ -259,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&sm.q_full[s], (it >> 1) & 1, 202);
         mbar_wait(&sm.dor_full, it & 1, 207);
         tc_fence_after();
+        mma_fill_magic(dst, sm.fill, BKT);  // the S accumulator's preload
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
           mma_i8(dst, smem_desc(qca + kk * 32, 16, kSboC, kSwC),
@@ -288,6 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int g = 0; g < G; ++g) {
           const int q0 = g * args.q_block;
+          // preload dV_t ([0, D)) and dK_t ([128, 128 + D)); P / dS (pass B) and the previous
+          // group's products (read-out) have been read from these columns
+          if constexpr (D == 128) {
+            mma_fill_magic(buf, sm.fill, 256);
+          } else {
+            mma_fill_magic(buf, sm.fill, D);
+            mma_fill_magic(buf + 128, sm.fill, D);
+          }
           for (int kk = 0; kk < args.q_block / 32; ++kk) {
             const int qr = q0 + kk * 32;
             mma_i8(buf, smem_desc(pca + qr * 128, BQ * BKT, 1024, kSwizzle128B),
@@ -306,6 +307,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // N = 128 queries; A = K codes read MN-major, B = dS codes K-major), so TMEM lanes are
         // head-dim channels and each warp's read-out holds 32 contiguous channels of a row.
         // d = 64: dQ_t = dSc[:, block] Kc[block] (M = 128 queries, N = d).
+        if constexpr (D == 128) {
+          mma_fill_magic(buf, sm.fill, 256);
+        } else {
+          mma_fill_magic(buf, sm.fill, D);
+          mma_fill_magic(buf + 128, sm.fill, D);
+        }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
@@ -343,9 +350,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int key_base = t * BKT;
     const int wpg = args.q_block / 32;  // warps per q_block group
     const int g_row = r / args.q_block;
-    float accv[kHalfD], acck[kHalfD];
+    // float32 dV / dK accumulators of this thread's key row, column pairs (f32x2 updates)
+    float2 accv[kHalfD / 2], acck[kHalfD / 2];
 #pragma unroll
-    for (int c = 0; c < kHalfD; ++c) accv[c] = acck[c] = 0.0f;
+    for (int c = 0; c < kHalfD / 2; ++c) accv[c] = acck[c] = make_float2(0.0f, 0.0f);
     int dvdk_cnt = 0;
     int dq_round = 0;  // dQ staging rounds so far (selects the staging buffer)
 
@@ -366,6 +374,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool diag = args.causal && (qt == t);
       const float c22 = scale22(c);
       const float nc22 = __fmul_rn(-kMagic, c22);
+      const float2 c2 = make_float2(c22, c22), nc2 = make_float2(nc22, nc22);
+      const float2 nlse2 = make_float2(-lse2, -lse2), ndvr2 = make_float2(-dvr, -dvr);
+      const float2 sl2 = make_float2(args.scale_log2, args.scale_log2);
       mbar_wait(&sm.sdp_full[b], (it >> 1) & 1, 210);
       tc_fence_after();
       float pmax = 0.0f, dsmax = 0.0f;
@@ -373,19 +384,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       // chunk ch computes.  The causal mask (key > query) exists only on the diagonal tile, so
       // the chunk loop is compiled twice and the off-diagonal copy carries no mask test.
       auto chunks = [&](auto masked) {
+        // two keys per FMA-pipe instruction (f32x2); the exponentials stay one per key
         auto proc_a = [&](uint32_t (&sa)[8], uint32_t (&pa)[8], int col) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float z = deq(sa[e], c22, nc22);
-            if constexpr (QS) z = fmaf(sm.kb[col + e], args.scale_log2, z);
-            float p = ex2_approx(z - lse2);
+          for (int e = 0; e < 8; e += 2) {
+            float2 z = __ffma2_rn(make_float2(__uint_as_float(sa[e]), __uint_as_float(sa[e + 1])),
+                                  c2, nc2);  // exact dequantization, as deq()
+            if constexpr (QS)
+              z = __ffma2_rn(make_float2(sm.kb[col + e], sm.kb[col + e + 1]), sl2, z);
+            const float2 t = __fadd2_rn(z, nlse2);
+            float2 p = make_float2(ex2_approx(t.x), ex2_approx(t.y));
             if constexpr (decltype(masked)::value) {
-              if (col + e > r) p = 0.0f;  // diagonal tile: key index - query index = col - r
+              // diagonal tile: key index - query index = col - r
+              if (col + e > r) p.x = 0.0f;
+              if (col + e + 1 > r) p.y = 0.0f;
             }
-            const float ds = p * (__uint_as_float(pa[e]) - dvr);
-            dsmax = fmaxf(dsmax, fabsf(ds));
-            sa[e] = __float_as_uint(p);
-            pa[e] = __float_as_uint(ds);
+            const float2 ds = __fmul2_rn(
+                p, __fadd2_rn(make_float2(__uint_as_float(pa[e]), __uint_as_float(pa[e + 1])),
+                              ndvr2));
+            dsmax = fmax3(dsmax, fabsf(ds.x), fabsf(ds.y));
+            sa[e] = __float_as_uint(p.x);
+            sa[e + 1] = __float_as_uint(p.y);
+            pa[e] = __float_as_uint(ds.x);
+            pa[e + 1] = __float_as_uint(ds.y);
           }
 #pragma unroll
           for (int e = 0; e < 8; e += 2)
@@ -468,21 +489,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qt = i_first + it;
       const size_t grow = static_cast<size_t>(row_base) + qt * BQ + r;
       if (it + 1 < nq) row_inputs(it + 1, c_n, lse2_n, dvr_n);  // loads in flight during pass B
-      // pass B: INT8 codes into shared memory; the dV_t / dK_t regions re-preloaded.  The TMEM
-      // loads of chunk ch+1 are in flight while chunk ch is converted.
+      // pass B: INT8 codes into shared memory.  The TMEM loads of chunk ch+1 are in flight while
+      // chunk ch is converted (two keys per FMA).
+      const float2 ip2 = make_float2(ip, ip), ids2 = make_float2(ids, ids);
+      const float2 km2 = make_float2(kMagic, kMagic);
       auto proc_b = [&](uint32_t (&sa)[16], uint32_t (&pa)[16], int ch) {
         const int col = h * 64 + ch * 16;
         uint32_t cp[4], cd[4];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          float fp[4], fd[4];
+          float2 fp[2], fd[2];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            fp[e] = __fmaf_rn(__uint_as_float(sa[q4 * 4 + e]), ip, kMagic);
-            fd[e] = __fmaf_rn(__uint_as_float(pa[q4 * 4 + e]), ids, kMagic);
+          for (int e = 0; e < 4; e += 2) {
+            const int x = q4 * 4 + e;
+            fp[e >> 1] = __ffma2_rn(make_float2(__uint_as_float(sa[x]), __uint_as_float(sa[x + 1])),
+                                    ip2, km2);
+            fd[e >> 1] = __ffma2_rn(make_float2(__uint_as_float(pa[x]), __uint_as_float(pa[x + 1])),
+                                    ids2, km2);
           }
-          cp[q4] = pack_magic4(fp[0], fp[1], fp[2], fp[3]);
-          cd[q4] = pack_magic4(fd[0], fd[1], fd[2], fd[3]);
+          cp[q4] = pack_magic4(fp[0].x, fp[0].y, fp[1].x, fp[1].y);
+          cd[q4] = pack_magic4(fd[0].x, fd[0].y, fd[1].x, fd[1].y);
         }
         const uint32_t off = swz_offset(r, h * 4 + ch, 128);
         *reinterpret_cast<uint4*>(sm.pc + off) = make_uint4(cp[0], cp[1], cp[2], cp[3]);
@@ -498,10 +524,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == e) mine = static_cast<float>(cs);
           }
           if (lane < 16) sm.cs[warp][ch * 16 + lane] += mine * sdsc;
-        }
-        if (col < D) {  // dV_t occupies columns [0, D), dK_t [128, 128 + D)
-          tmem_fill16(lane_base + col, kMagicBits);
-          tmem_fill16(lane_base + 128 + col, kMagicBits);
         }
       };
       {
@@ -540,8 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // pass A of the next tile while the tensor core works on this one
       if (it + 1 < nq) pass_a(it + 1, c_n, lse2_n, dvr_n);
-      // step 3: dV_t, dK_t (thread = key row r, d columns of warpgroup h) into registers;
-      // the read columns are re-preloaded for dQ_t.  The tile scales (P and dS absmax / 127,
+      // step 3: dV_t, dK_t (thread = key row r, d columns of warpgroup h) into registers.  The tile scales (P and dS absmax / 127,
       // IEEE quotients) come from the maxima of the key half this thread's key row is in.
       for (int g = 0; g < G; ++g) {
         const float sdo = g == 0 ? sdo_t[0] : sdo_t[1];
@@ -555,6 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sv22 = scale22(sp * sdo);
         const float sk22 = scale22(sds * sqg * args.tau);
         const float nsv = __fmul_rn(-kMagic, sv22), nsk = __fmul_rn(-kMagic, sk22);
+        const float2 sv2 = make_float2(sv22, sv22), nsv2 = make_float2(nsv, nsv);
+        const float2 sk2 = make_float2(sk22, sk22), nsk2 = make_float2(nsk, nsk);
         // 16-column chunks; the loads of chunk c+1 are in flight while chunk c accumulates
         uint32_t tv0[16], tk0[16], tv1[16], tk1[16];
         tmem_ld16(lane_base + h * kHalfD, tv0);
@@ -574,12 +597,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            accv[c0 + e] += deq(odd ? tv1[e] : tv0[e], sv22, nsv);
-            acck[c0 + e] += deq(odd ? tk1[e] : tk0[e], sk22, nsk);
+          for (int e = 0; e < 16; e += 2) {
+            const uint32_t* tv = odd ? tv1 : tv0;
+            const uint32_t* tk = odd ? tk1 : tk0;
+            const float2 dv2 = __ffma2_rn(
+                make_float2(__uint_as_float(tv[e]), __uint_as_float(tv[e + 1])), sv2, nsv2);
+            const float2 dk2 = __ffma2_rn(
+                make_float2(__uint_as_float(tk[e]), __uint_as_float(tk[e + 1])), sk2, nsk2);
+            accv[(c0 + e) / 2] = __fadd2_rn(accv[(c0 + e) / 2], dv2);
+            acck[(c0 + e) / 2] = __fadd2_rn(acck[(c0 + e) / 2], dk2);
           }
-          tmem_fill16(lane_base + col, kMagicBits);
-          tmem_fill16(lane_base + 128 + col, kMagicBits);
           if (c0 + 16 < kHalfD) {
             if (odd)
               tmem_ld_wait_regs(tv0, tk0);
@@ -587,18 +614,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_ld_wait_regs(tv1, tk1);
           }
         }
-        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sm.dvdk_free);
         ++dvdk_cnt;
       }
-      // step 4: dQ, added to the float32 accumulator; afterwards the S region of this buffer is
-      // re-preloaded for tile it+2.  The dS scales of both key halves for this thread's dQ rows
+      // step 4: dQ, added to the float32 accumulator.  The dS scales of both key halves for this thread's dQ rows
       // are formed while the dQ MMAs run.
       const int gq = D == 128 ? (64 * h) / args.q_block : g_row;
       const float s0 = scale22(__fdiv_rn(tile_max(sm.red_ds[b], gq, 0), 127.0f) * sk0 * args.tau);
       const float s1 = scale22(__fdiv_rn(tile_max(sm.red_ds[b], gq, 1), 127.0f) * sk1 * args.tau);
       const float n0 = __fmul_rn(-kMagic, s0), n1 = __fmul_rn(-kMagic, s1);
+      const float2 s02 = make_float2(s0, s0), n02 = make_float2(n0, n0);
+      const float2 s12 = make_float2(s1, s1), n12 = make_float2(n1, n1);
       // and the next tile's code multipliers (its pass A is done in every warp by now)
       float ip_n = 0.0f, ids_n = 0.0f, sdsc_n = 0.0f;
       if (it + 1 < nq) multipliers(it + 1, ip_n, ids_n, sdsc_n);
@@ -617,11 +644,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int rr = 0; rr < 64 / kDqRows; ++rr) {
           const int q0 = 64 * h + kDqRows * rr;
-          float v[kDqRows];
+          float2 v[kDqRows / 2];
 #pragma unroll
-          for (int e = 0; e < kDqRows; ++e) v[e] = deq(a0[e], s0, n0) + deq(a1[e], s1, n1);
-          tmem_fill16(lane_base + q0, kMagicBits);
-          tmem_fill16(lane_base + 128 + q0, kMagicBits);
+          for (int e = 0; e < kDqRows; e += 2)
+            v[e / 2] = __fadd2_rn(
+                __ffma2_rn(make_float2(__uint_as_float(a0[e]), __uint_as_float(a0[e + 1])),
+                           s02, n02),
+                __ffma2_rn(make_float2(__uint_as_float(a1[e]), __uint_as_float(a1[e + 1])),
+                           s12, n12));
           if (rr + 1 < 64 / kDqRows) {
             tmem_ld16(lane_base + q0 + kDqRows, a0);
             tmem_ld16(lane_base + 128 + q0 + kDqRows, a1);
@@ -631,7 +661,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) bulk_wait_read_1();
           __syncwarp();
 #pragma unroll
-          for (int e = 0; e < kDqRows; ++e) stg[e * kDqCols + lane] = v[e];
+          for (int e = 0; e < kDqRows; e += 2) {
+            stg[e * kDqCols + lane] = v[e / 2].x;
+            stg[(e + 1) * kDqCols + lane] = v[e / 2].y;
+          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -641,7 +674,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++dq_round;
           if (rr + 1 < 64 / kDqRows) tmem_ld_wait_regs(a0, a1);
         }
-        tmem_st_wait();
       } else {
         // thread = query row r, d columns of warpgroup h
         float* dst = args.dq_acc + grow * D + h * kHalfD;
@@ -661,15 +693,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicAdd(reinterpret_cast<float4*>(dst + c0 + e), v4);
           }
         }
-        // S occupies columns [0, 128): each thread refills the dQ_t0 columns it read
-        // ([h*d/2, (h+1)*d/2)) and its warpgroup's half of [d, 128), so no thread writes a
-        // column the other warpgroup may still be reading
-#pragma unroll
-        for (int c = 0; c < kHalfD; c += 16) tmem_fill16(lane_base + h * kHalfD + c, kMagicBits);
-#pragma unroll
-        for (int c = 0; c < (128 - D) / 2; c += 16)
-          tmem_fill16(lane_base + D + h * ((128 - D) / 2) + c, kMagicBits);
-        tmem_st_wait();
       }
       tc_fence_before();
       mbar_arrive(&sm.dq_free);
@@ -693,10 +716,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c0 = 0; c0 < kHalfD; c0 += 4) {
           const float4 m4 = __ldg(mq + c0 / 4);
-          acck[c0 + 0] = fmaf(csr, m4.x, acck[c0 + 0]);
-          acck[c0 + 1] = fmaf(csr, m4.y, acck[c0 + 1]);
-          acck[c0 + 2] = fmaf(csr, m4.z, acck[c0 + 2]);
-          acck[c0 + 3] = fmaf(csr, m4.w, acck[c0 + 3]);
+          acck[c0 / 2].x = fmaf(csr, m4.x, acck[c0 / 2].x);
+          acck[c0 / 2].y = fmaf(csr, m4.y, acck[c0 / 2].y);
+          acck[c0 / 2 + 1].x = fmaf(csr, m4.z, acck[c0 / 2 + 1].x);
+          acck[c0 / 2 + 1].y = fmaf(csr, m4.w, acck[c0 / 2 + 1].y);
         }
       }
       if (args.qknorm) {
@@ -710,7 +733,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float x[8];
           Cvt<T>::load8(__ldg(reinterpret_cast<const uint4*>(kp + c0)), x);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) part = fmaf(acck[c0 + e], __fmul_rn(x[e], inv), part);
+          for (int e = 0; e < 8; ++e) {
+            const float a = (e & 1) ? acck[(c0 + e) / 2].y : acck[(c0 + e) / 2].x;
+            part = fmaf(a, __fmul_rn(x[e], inv), part);
+          }
         }
         if (h == 1) sm.dot[r] = part;
         named_barrier_sync(3, 256);
@@ -722,17 +748,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           float x[8];
           Cvt<T>::load8(__ldg(reinterpret_cast<const uint4*>(kp + c0)), x);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            acck[c0 + e] = inv * fmaf(-__fmul_rn(x[e], inv), dotd, acck[c0 + e]);
+          for (int e = 0; e < 8; e += 2) {
+            float2& a = acck[(c0 + e) / 2];
+            a.x = inv * fmaf(-__fmul_rn(x[e], inv), dotd, a.x);
+            a.y = inv * fmaf(-__fmul_rn(x[e + 1], inv), dotd, a.y);
+          }
         }
       }
 #pragma unroll
       for (int c0 = 0; c0 < kHalfD; c0 += 8) {
         float fv[8], fk[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          fv[e] = accv[c0 + e];
-          fk[e] = acck[c0 + e];
+        for (int e = 0; e < 8; e += 2) {
+          fv[e] = accv[(c0 + e) / 2].x;
+          fv[e + 1] = accv[(c0 + e) / 2].y;
+          fk[e] = acck[(c0 + e) / 2].x;
+          fk[e + 1] = acck[(c0 + e) / 2].y;
         }
         *reinterpret_cast<uint4*>(dvp + c0) = pack8<T>(fv);
         *reinterpret_cast<uint4*>(dkp + c0) = pack8<T>(fk);

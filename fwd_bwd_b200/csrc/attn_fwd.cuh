@@ -15,7 +15,9 @@
 //               softmax warpgroups: 256 x 232 + 128 x 40 = 64512 = 384 x 168).
 // TMEM (512 columns): tile g uses columns [256g, 256g+256): S buffers at +0 and +64, PV at
 // +128 (d columns, INT32).  The INT32 regions are preloaded with the bits of 1.5 * 2^23 before
-// each MMA (see kMagicBits), so results read back as floats that one FMA dequantizes.
+// each MMA (see kMagicBits), so results read back as floats that one FMA dequantizes; the MMA
+// thread writes the preload with one bf16 MMA (mma_fill_magic), so the softmax warps only read
+// TMEM.
 // O (float32) lives in registers.
 //
 // Q-smoothing (template flag QS): every score of key j gains the per-key bias k_bias_j, copied
@@ -58,6 +60,7 @@ struct Smem {
   int8_t k[NST][BKV * D];
   int8_t v[NST][BKV * D];
   int8_t p[NT][2][BM * BKV];
+  alignas(256) uint8_t fill[kFillBytes];  // operands of the preload MMA (mma_fill_magic)
   float kb[NST][BKV];  // Q-smoothing: k_bias of the stage's keys
   uint64_t q_full;
   uint64_t k_full[NST], v_full[NST], kv_empty[NST];
@@ -77,7 +80,7 @@ constexpr bool tiles_aligned() {
   return offsetof(Smem<D>, q) % 1024 == 0 && (BM * D) % 1024 == 0 &&
          offsetof(Smem<D>, k) % 1024 == 0 && (BKV * D) % 1024 == 0 &&
          offsetof(Smem<D>, v) % 1024 == 0 && offsetof(Smem<D>, p) % 1024 == 0 &&
-         (BM * BKV) % 1024 == 0;
+         (BM * BKV) % 1024 == 0 && offsetof(Smem<D>, fill) % 256 == 0;
 }
 static_assert(tiles_aligned<64>() && tiles_aligned<128>(), "shared-memory tiles misaligned");
 
@@ -140,6 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     nb_max = max(nb_max, nb[g]);
   }
 
+  write_fill_operands(sm.fill, threadIdx.x, kThreads);
+  fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     sm.abort = device_aborted() ? 1 : 0;
     mbar_init(&sm.q_full, 1);
@@ -168,16 +173,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  if (warp < 8) {
-    // preload both S buffers and the PV region of this thread's lane with the magic value
-    const uint32_t lb = tmem + (((warp & 3) * 32u) << 16) + (warp >> 2) * 256;
-#pragma unroll
-    for (int c = 0; c < 128 + D; c += 16) tmem_fill16(lb + c, kMagicBits);
-    tmem_st_wait();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
 
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kOtherRegs));
@@ -210,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       for (int g = 0; g < NT; ++g)
         if (nb[g] > 0) {
+          mma_fill_magic(tmem + g * 256, sm.fill, BKV);
           issue_scores<D>(tmem + g * 256, sm.q[g], sm.k[0], BKV, 1u);
           mma_commit(&sm.s_full[g][0]);
         }
@@ -221,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           for (int g = 0; g < NT; ++g)
             if (j + 1 < nb[g]) {
-              // buffer (j+1)&1 held S_{j-1}: read and re-preloaded before p_full[j-1]
+              // buffer (j+1)&1 held S_{j-1}: read before p_full[j-1]; preloaded here
+              mma_fill_magic(tmem + g * 256 + ((j + 1) & 1) * 64, sm.fill, BKV);
               issue_scores<D>(tmem + g * 256 + ((j + 1) & 1) * 64, sm.q[g], sm.k[st1], BKV,
                               1u);
               mma_commit(&sm.s_full[g][(j + 1) & 1]);
@@ -235,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t pa = smem_u32(sm.p[g][j & 1]);
           const uint32_t va = smem_u32(sm.v[st]);
+          mma_fill_magic(tmem + g * 256 + 128, sm.fill, D);
 #pragma unroll
           for (int kk = 0; kk < BKV / 32; ++kk) {
             mma_i8(tmem + g * 256 + 128, smem_desc(pa + kk * 32, 16, 8 * BKV, kSwizzle64B),
@@ -262,9 +260,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* ksc = args.k_scale + static_cast<size_t>(bh) * nkb;
       const float* vsc = args.v_scale + static_cast<size_t>(bh) * nkb;
       const uint32_t lane_base = tmem + ((quarter * 32u) << 16) + g * 256;
-      float O[D];
+      // O in column pairs: the fold runs on the FMA pipe's paired (f32x2) instructions
+      float2 O[D / 2];
 #pragma unroll
-      for (int c = 0; c < D; ++c) O[c] = 0.0f;
+      for (int c = 0; c < D / 2; ++c) O[c] = make_float2(0.0f, 0.0f);
       float m2 = -INFINITY, l = 0.0f, alpha_prev = 1.0f, beta_prev = 0.0f;
       int8_t* pbase = sm.p[g][0];
       float sk_next = ksc[0], sv_next = vsc[0];
@@ -281,14 +280,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16(lane_base + 128, a0);
         tmem_ld16(lane_base + 128 + 16, a1);
         tmem_ld_wait_regs(a0, a1);
+        const float2 al2 = make_float2(alpha_prev, alpha_prev);
+        const float2 b2 = make_float2(b22, b22), nb2 = make_float2(nb22, nb22);
+        // O = alpha O + deq(PV) for two columns per instruction (deq exact, as in deq())
         auto fold32 = [&](const uint32_t (&x0)[16], const uint32_t (&x1)[16], int c0) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) O[c0 + c] = fmaf(O[c0 + c], alpha_prev, deq(x0[c], b22, nb22));
+          for (int c = 0; c < 16; c += 2) {
+            const float2 t = __ffma2_rn(make_float2(__uint_as_float(x0[c]),
+                                                    __uint_as_float(x0[c + 1])), b2, nb2);
+            O[(c0 + c) / 2] = __ffma2_rn(O[(c0 + c) / 2], al2, t);
+          }
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            O[c0 + 16 + c] = fmaf(O[c0 + 16 + c], alpha_prev, deq(x1[c], b22, nb22));
-          tmem_fill16(lane_base + 128 + c0, kMagicBits);
-          tmem_fill16(lane_base + 128 + c0 + 16, kMagicBits);
+          for (int c = 0; c < 16; c += 2) {
+            const float2 t = __ffma2_rn(make_float2(__uint_as_float(x1[c]),
+                                                    __uint_as_float(x1[c + 1])), b2, nb2);
+            O[(c0 + 16 + c) / 2] = __ffma2_rn(O[(c0 + 16 + c) / 2], al2, t);
+          }
         };
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 64) {
@@ -383,7 +390,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // loaded; four partial row sums keep the adds off one dependency chain; the causal mask
         // test exists only in the diagonal blocks' copy of the loop.
         int8_t* prow = pbase + (j & 1) * (BM * BKV);
-        float rsp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        // Two keys per FMA-pipe instruction (f32x2); the exponentials stay one per key.
+        float2 rs2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+        const float2 c2 = make_float2(c22, c22), nc2 = make_float2(nc22, nc22);
+        const float2 nm2 = make_float2(-mblk, -mblk);
+        const float2 k127 = make_float2(127.0f, 127.0f), km2 = make_float2(kMagic, kMagic);
         auto pass2 = [&](auto masked) {
           auto conv = [&](const uint32_t (&x0)[16], const uint32_t (&x1)[16], int h) {
             uint32_t pk[8];
@@ -391,21 +402,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int half = 0; half < 2; ++half) {
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4) {
-                float f[4];
+                float2 f[2];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
+                for (int e = 0; e < 4; e += 2) {
                   const int cc = q4 * 4 + e;
-                  const uint32_t av = half ? x1[cc] : x0[cc];
-                  float z = deq(av, c22, nc22);
-                  if constexpr (QS) z = fmaf(kbj[h * 32 + half * 16 + cc], args.scale_log2, z);
-                  float p = ex2_approx(z - mblk);
-                  if constexpr (decltype(masked)::value) {
-                    if (key0 + h * 32 + half * 16 + cc > i) p = 0.0f;
+                  const uint32_t a_0 = half ? x1[cc] : x0[cc];
+                  const uint32_t a_1 = half ? x1[cc + 1] : x0[cc + 1];
+                  float2 z = __ffma2_rn(make_float2(__uint_as_float(a_0), __uint_as_float(a_1)),
+                                        c2, nc2);  // exact dequantization, as deq()
+                  if constexpr (QS) {
+                    const float2 kb = make_float2(kbj[h * 32 + half * 16 + cc],
+                                                  kbj[h * 32 + half * 16 + cc + 1]);
+                    z = __ffma2_rn(kb, make_float2(args.scale_log2, args.scale_log2), z);
                   }
-                  rsp[e] += p;
-                  f[e] = __fmaf_rn(p, 127.0f, kMagic);
+                  const float2 t = __fadd2_rn(z, nm2);
+                  float2 p = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                  if constexpr (decltype(masked)::value) {
+                    const int key = key0 + h * 32 + half * 16 + cc;
+                    if (key > i) p.x = 0.0f;
+                    if (key + 1 > i) p.y = 0.0f;
+                  }
+                  rs2[e >> 1] = __fadd2_rn(rs2[e >> 1], p);
+                  f[e >> 1] = __ffma2_rn(p, k127, km2);
                 }
-                pk[half * 4 + q4] = pack_magic4(f[0], f[1], f[2], f[3]);
+                pk[half * 4 + q4] = pack_magic4(f[0].x, f[0].y, f[1].x, f[1].y);
               }
             }
             // keys h*32 .. h*32+31 are 16-byte chunks 2h and 2h+1 of this row
@@ -421,10 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pass2(std::true_type{});
         else
           pass2(std::false_type{});
-        const float rs = (rsp[0] + rsp[1]) + (rsp[2] + rsp[3]);
-        // the S buffer is read: preload it for S_{j+2}
-#pragma unroll
-        for (int c = 0; c < 64; c += 16) tmem_fill16(sa + c, kMagicBits);
+        const float rs = (rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y);
         const float m2n = fmaxf(m2, mblk);
         const float alpha = ex2_approx(m2 - m2n);
         const float eblk = has ? ex2_approx(mblk - m2n) : 0.0f;
@@ -447,7 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c0 = 0; c0 < D; c0 += 8) {
         float f[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = O[c0 + e] * inv_l;
+        for (int e = 0; e < 8; e += 2) {
+          f[e] = O[(c0 + e) / 2].x * inv_l;
+          f[e + 1] = O[(c0 + e) / 2].y * inv_l;
+        }
         *reinterpret_cast<uint4*>(orow + c0) = pack8<T>(f);
       }
       args.lse[static_cast<size_t>(bh) * N + i] = (m2 + log2f(l)) * 0.69314718055994531f;

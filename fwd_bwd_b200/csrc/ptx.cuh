@@ -380,6 +380,38 @@ __device__ __forceinline__ uint32_t swz_offset(uint32_t row, uint32_t chunk,
 constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr float kMagic = 12582912.0f;
 
+// ---------------------------------------------------------------------------------------------
+// Preloading accumulators with the tensor core
+// ---------------------------------------------------------------------------------------------
+// A kind::f16 MMA with accumulate = 0 can write the preload value itself, so the compute warps
+// never store it into TMEM: with A[i][k] = 1 and B[j][k] = 1.5 * 2^22 (both exact in bf16) at
+// k = 0 and k = 8 and zero elsewhere, D[i][j] = 2 * 1.5 * 2^22 = 1.5 * 2^23 exactly, whose float32
+// bits are kMagicBits.  Every 16-byte chunk of the operand tiles holds the same 8 elements
+// (element 0 set, 7 zeros), so each tile row reads k = 0 and k = 8 as set whatever the layout's
+// row and chunk order: only the tiles' extent matters.
+constexpr uint32_t kFillA = 0x00003F80u;  // bf16 1.0 in the chunk's first element
+constexpr uint32_t kFillB = 0x00004AC0u;  // bf16 6291456.0 = 1.5 * 2^22
+constexpr int kFillRowsA = 128;           // M rows of A
+constexpr int kFillRowsB = 256;           // up to N = 256 rows of B
+constexpr int kFillBytes = (kFillRowsA + kFillRowsB) * 32;
+
+// Writes the fill operands (A then B, rows of 32 bytes) into `dst` (256-byte aligned); every
+// thread of the calling group takes its share; the caller fences to the async proxy.
+__device__ __forceinline__ void write_fill_operands(uint8_t* dst, int tid, int nthreads) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  for (int i = tid; i < kFillBytes / 16; i += nthreads)
+    d4[i] = make_uint4(i < kFillRowsA * 2 ? kFillA : kFillB, 0u, 0u, 0u);
+}
+
+// D[tmem, columns 0 .. n) = 1.5 * 2^23 (bits kMagicBits) for all 128 lanes; n in {16 .. 256}, a
+// multiple of 16.  `fill` is the operand tile pair written by write_fill_operands.  Issued by the
+// MMA thread, in order with its other MMAs.
+__device__ __forceinline__ void mma_fill_magic(uint32_t d_tmem, const uint8_t* fill, int n) {
+  const uint32_t a = smem_u32(fill), b = a + kFillRowsA * 32;
+  const uint32_t id = instr_desc(1, 1, 1, false, false, 128, n);  // F32 <- BF16 x BF16
+  mma_f16(d_tmem, smem_desc(a, 16, 256, kSwizzle32B), smem_desc(b, 16, 256, kSwizzle32B), id, 0u);
+}
+
 // s rounded toward zero to 22 significant bits: kMagic * scale22(s) is then exact in float32.
 __device__ __forceinline__ float scale22(float s) {
   return __uint_as_float(__float_as_uint(s) & 0xFFFFFFFCu);

@@ -1,8 +1,9 @@
 """World-size-2 (gloo, CPU) check of the data-parallel partition: each rank computes its own
-contiguous range of heads (here with the CPU oracle standing in for a GPU), and the gathered
-shards equal the single-process result exactly -- every head is an independent problem, so
-there is nothing to exchange but the results.  Also checks the harness's max-over-ranks timing
-reduction."""
+contiguous range of flattened heads -- or, as bench.py's end-to-end leg splits one global batch,
+its own range of batch entries -- (here with the CPU oracle standing in for a GPU), and the
+gathered shards equal the single-process result exactly: every head is an independent problem,
+so there is nothing to exchange but the results.  Also checks the harness's max-over-ranks
+timing reduction."""
 import os
 import socket
 
@@ -32,14 +33,21 @@ def test_head_range_partition():
             assert max(sizes) - min(sizes) <= 1
 
 
-def _worker(rank, world, port, out_q):
+WL = {"heads": dict(B=1, H=5, N=256), "batch": dict(B=3, H=2, N=256)}
+
+
+def _worker(rank, world, port, out_q, unit):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     import oracle.sage_oracle as O
     from fwd_bwd_b200.inputs import WORKLOADS, make_inputs
 
-    w = WORKLOADS["llama325m"].replace(B=1, H=5, N=256)
-    mine = head_range(w.B * w.H, world, rank)
+    w = WORKLOADS["llama325m"].replace(**WL[unit])
+    if unit == "heads":
+        mine = head_range(w.B * w.H, world, rank)
+    else:  # contiguous batch entries (bench.py's end-to-end split), as flattened heads
+        b = head_range(w.B, world, rank)
+        mine = range(b.start * w.H, b.stop * w.H)
     x = make_inputs(w, heads=mine)
     res = O.sage_attention(*(x[n + "_f32"] for n in ("q", "k", "v", "do")), causal=w.causal,
                            qknorm=w.qknorm, ksmooth=w.ksmooth, q_block=w.q_block,
@@ -55,14 +63,15 @@ def _worker(rank, world, port, out_q):
     dist.destroy_process_group()
 
 
-def test_two_rank_shards_concatenate_to_single_result():
+@pytest.mark.parametrize("unit", ["heads", "batch"])
+def test_two_rank_shards_concatenate_to_single_result(unit):
     import oracle.sage_oracle as O
     from fwd_bwd_b200.inputs import WORKLOADS, make_inputs
 
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q, unit)) for r in range(2)]
     for p in procs:
         p.start()
     gathered, tmax = q.get(timeout=240)
@@ -70,7 +79,7 @@ def test_two_rank_shards_concatenate_to_single_result():
         p.join(timeout=60)
         assert p.exitcode == 0
     assert tmax == 2.0
-    w = WORKLOADS["llama325m"].replace(B=1, H=5, N=256)
+    w = WORKLOADS["llama325m"].replace(**WL[unit])
     x = make_inputs(w)
     full = O.sage_attention(*(x[n + "_f32"].reshape(-1, w.N, w.d)
                               for n in ("q", "k", "v", "do")), causal=w.causal,
