@@ -494,7 +494,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 ip2 = make_float2(ip, ip), ids2 = make_float2(ids, ids);
       const float2 km2 = make_float2(kMagic, kMagic);
       auto proc_b = [&](uint32_t (&sa)[16], uint32_t (&pa)[16], int ch) {
-        const int col = h * 64 + ch * 16;
         uint32_t cp[4], cd[4];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {

@@ -274,11 +274,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float nb22 = __fmul_rn(-kMagic, b22);
         mbar_wait(&sm.pv_full[g], jj & 1, 110);
         tc_fence_after();
-        // 32-column chunks, double-buffered: the loads of chunk c+1 are in flight while chunk c
-        // is folded
+        // 32-column chunks (one load each), double-buffered: the load of chunk c+1 is in flight
+        // while chunk c is folded
         uint32_t a0[16], a1[16], b0[16], b1[16];
-        tmem_ld16(lane_base + 128, a0);
-        tmem_ld16(lane_base + 128 + 16, a1);
+        tmem_ld32x(lane_base + 128, a0, a1);
         tmem_ld_wait_regs(a0, a1);
         const float2 al2 = make_float2(alpha_prev, alpha_prev);
         const float2 b2 = make_float2(b22, b22), nb2 = make_float2(nb22, nb22);
@@ -299,22 +298,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 64) {
-          if (c0 + 32 < D) {
-            tmem_ld16(lane_base + 128 + c0 + 32, b0);
-            tmem_ld16(lane_base + 128 + c0 + 48, b1);
-          }
+          if (c0 + 32 < D) tmem_ld32x(lane_base + 128 + c0 + 32, b0, b1);
           fold32(a0, a1, c0);
           if (c0 + 32 < D) {
             tmem_ld_wait_regs(b0, b1);
-            if (c0 + 64 < D) {
-              tmem_ld16(lane_base + 128 + c0 + 64, a0);
-              tmem_ld16(lane_base + 128 + c0 + 80, a1);
-            }
+            if (c0 + 64 < D) tmem_ld32x(lane_base + 128 + c0 + 64, a0, a1);
             fold32(b0, b1, c0 + 32);
             if (c0 + 64 < D) tmem_ld_wait_regs(a0, a1);
           }
         }
-        tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sm.pv_free[g]);
       };
@@ -344,12 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float mx;
         uint32_t a0[16], a1[16], b0[16], b1[16];
         {
-          tmem_ld16(sa, a0);
-          tmem_ld16(sa + 16, a1);
-          tmem_ld16(sa + 32, b0);
-          tmem_ld16(sa + 48, b1);
-          tmem_ld_wait_regs(a0, a1);
-          tmem_ld_wait_regs(b0, b1);
+          tmem_ld64x(sa, a0, a1, b0, b1);  // the block's 64 scores in one load
+          tmem_ld_wait_regs4(a0, a1, b0, b1);
           float m0 = -INFINITY, m1 = -INFINITY;
           auto maxh = [&](const uint32_t (&x0)[16], const uint32_t (&x1)[16], int h, float& m) {
             if constexpr (QS) {
@@ -447,7 +435,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float eblk = has ? ex2_approx(mblk - m2n) : 0.0f;
         l = fmaf(l, alpha, eblk * rs);
         const float beta = eblk * sv * (1.0f / 127.0f);
-        tmem_st_wait();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sm.p_full[g][j & 1]);
