@@ -336,8 +336,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2) prologue_quant_kernel(Prolog
 }
 
 // ---------------------------------------------------------------------------------------------
-// Backward preprocess: D_i = sum_c dO_ic O_ic (float32), dO codes per q_block tokens, and the
-// float32 dQ accumulator rows cleared.  One CTA (kQuantThreads threads) per 128 rows.
+// Backward preprocess: D_i = sum_c dO_ic O_ic (float32), dO codes per q_block tokens (skipped
+// when do_codes is null), and the float32 dQ accumulator rows cleared.  One CTA
+// (kQuantThreads threads) per 128 rows.
 // ---------------------------------------------------------------------------------------------
 template <typename T, int D>
 __global__ void __launch_bounds__(kQuantThreads, 2) bwd_preprocess_kernel(
@@ -372,6 +373,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) bwd_preprocess_kernel(
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  if (do_codes == nullptr) return;  // D and the cleared accumulator only
   const float am = block_absmax_n<NW>(amax, q_block, red);
   const float sc = __fdiv_rn(am, 127.0f);
   if (threadIdx.x == 0 || (q_block == 64 && threadIdx.x == kQuantThreads / 2))

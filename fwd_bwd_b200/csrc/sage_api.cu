@@ -17,6 +17,7 @@
 #include "attn_fwd.cuh"
 #include "debug_kernels.cuh"
 #include "nvfp4.cuh"
+#include "nvfp4_bwd.cuh"
 #include "ptx.cuh"
 #include "rowops.cuh"
 
@@ -435,6 +436,76 @@ int run_fp4_fwd(const sage_params* p, const sage_fp4_bufs* fb, const void* v, vo
   return launch_status();
 }
 
+// Backward workspace: D = rowsum(dO o O) [BH, N] then the float32 dQ accumulator [BH, N, d].
+struct Fp4BwdWs {
+  size_t dvec, dq, total;
+};
+Fp4BwdWs fp4_bwd_ws(const sage_params* p) {
+  const size_t BH = static_cast<size_t>(p->B) * p->H, N = p->N, d = p->d;
+  Fp4BwdWs w;
+  w.dvec = 0;
+  w.dq = align_up(BH * N * 4);
+  w.total = align_up(w.dq + BH * N * d * 4);
+  return w;
+}
+
+template <typename T, int D>
+int run_fp4_bwd(const sage_params* p, const void* q, const void* k, const void* v,
+                const sage_fp4_bufs* fb, const void* o, const float* lse, const void* dout,
+                void* dq, void* dk, void* dv, void* ws, cudaStream_t st) {
+  const int BH = p->B * p->H, N = p->N;
+  const uint64_t rows = static_cast<uint64_t>(BH) * N;
+  const Fp4BwdWs w = fp4_bwd_ws(p);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+  float* dvec = reinterpret_cast<float*>(wsb + w.dvec);
+  float* dqacc = reinterpret_cast<float*>(wsb + w.dq);
+  // D and the cleared dQ accumulator (no INT8 dO codes: dO enters the MMAs in 16 bits)
+  sage::bwd_preprocess_kernel<T, D>
+      <<<static_cast<int>(rows / kRowsPerCta), sage::kQuantThreads, 0, st>>>(
+          reinterpret_cast<const T*>(o), reinterpret_cast<const T*>(dout), dvec, nullptr,
+          nullptr, dqacc, N, p->q_block);
+  if (launch_status() != SAGE_OK) return SAGE_ERR_CUDA;
+  CUtensorMap tqc, tkc, tqs, tks, tdo, tv;
+  const uint64_t seq_rows = static_cast<uint64_t>(BH) * D;
+  if (!make_map(&tqc, fb->q_fp4, 1, D / 2, rows, D / 2, sage::fp4::bwd::BQ) ||
+      !make_map(&tkc, fb->k_fp4, 1, D / 2, rows, D / 2, sage::fp4::bwd::BKT) ||
+      !make_map(&tqs, fb->q_fp4_t, 1, N / 2, seq_rows, 64, D) ||
+      !make_map(&tks, fb->k_fp4_t, 1, N / 2, seq_rows, 64, D) ||
+      !make_map(&tdo, dout, 2, D, rows, 64, sage::fp4::bwd::BQ) ||
+      !make_map(&tv, v, 2, D, rows, 64, sage::fp4::bwd::BKT))
+    return SAGE_ERR_CUDA;
+  sage::fp4::bwd::Args a;
+  a.q_sf = fb->q_sf;
+  a.k_sf = fb->k_sf;
+  a.q_sf_t = fb->q_sf_t;
+  a.k_sf_t = fb->k_sf_t;
+  a.q_genc = fb->q_genc;
+  a.k_genc = fb->k_genc;
+  a.lse = lse;
+  a.dvec = dvec;
+  a.k_raw = k;
+  a.k_inv_rms = fb->k_inv_rms;
+  a.dq_acc = dqacc;
+  a.dk = dk;
+  a.dv = dv;
+  a.N = N;
+  a.causal = p->causal;
+  a.qknorm = p->qknorm;
+  a.tau = tau_of(p);
+  a.scale_log2 = a.tau * 1.4426950408889634f;
+  const size_t smem = sage::fp4::bwd::smem_bytes<T, D>();
+  auto kern = sage::fp4::bwd::attn_bwd_kernel<T, D>;
+  if (set_smem(kern, smem) != SAGE_OK) return SAGE_ERR_CUDA;
+  // register split between warpgroups (setmaxnreg) assumes exactly kLaunchRegs at launch
+  if (launch_regs(kern) != sage::fp4::bwd::kLaunchRegs) return SAGE_ERR_UNSUPPORTED;
+  kern<<<BH * (N / sage::fp4::bwd::BKT), sage::fp4::bwd::kThreads, smem, st>>>(tqc, tkc, tqs,
+                                                                             tks, tdo, tv, a);
+  if (launch_status() != SAGE_OK) return SAGE_ERR_CUDA;
+  sage::dq_finalize_kernel<T, D><<<static_cast<int>(rows / kRowsPerCta), kRowThreads, 0, st>>>(
+      dqacc, reinterpret_cast<const T*>(q), fb->q_inv_rms, reinterpret_cast<T*>(dq), p->qknorm);
+  return launch_status();
+}
+
 // ---- end-to-end pipeline over host buffers -------------------------------------------------
 // One chunk slot of sage_fwd_bwd_host's device workspace: the chunk's 16-bit inputs and
 // outputs, its quantized views, LSE and the prologue / backward scratch; offsets from the
@@ -685,7 +756,7 @@ int sage_fwd_bwd_host(const sage_params* p, const void* q, const void* k, const 
 
 size_t sage_fp4_workspace_bytes(const sage_params* p, int which) {
   if (check_fp4(p) != SAGE_OK) return 0;
-  return which == 0 ? fp4_ws(p).total : 0;
+  return which == 0 ? fp4_ws(p).total : which == 2 ? fp4_bwd_ws(p).total : 0;
 }
 
 int sage_fp4_quant_prologue(const sage_params* p, const void* q, const void* k,
@@ -721,6 +792,32 @@ int sage_fp4_attn_fwd(const sage_params* p, const sage_fp4_bufs* fb, const void*
               : run_fp4_fwd<__half, 128>(p, fb, v, o, lse, st);
   return bf ? run_fp4_fwd<__nv_bfloat16, 64>(p, fb, v, o, lse, st)
             : run_fp4_fwd<__half, 64>(p, fb, v, o, lse, st);
+}
+
+int sage_fp4_attn_bwd(const sage_params* p, const void* q, const void* k, const void* v,
+                      const sage_fp4_bufs* fb, const void* o, const float* lse, const void* dout,
+                      void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  int s = check_fp4(p);
+  if (s != SAGE_OK) return s;
+  if ((s = check_fp4bufs(p, fb)) != SAGE_OK) return s;
+  if (!fb->q_fp4_t || !fb->k_fp4_t) return SAGE_ERR_INVALID_ARG;
+  if (p->qknorm && (!fb->q_inv_rms || !fb->k_inv_rms)) return SAGE_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return SAGE_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return SAGE_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < fp4_bwd_ws(p).total) return SAGE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_fp4_bwd<__nv_bfloat16, 128>(p, q, k, v, fb, o, lse, dout, dq, dk, dv,
+                                                 workspace, st)
+              : run_fp4_bwd<__half, 128>(p, q, k, v, fb, o, lse, dout, dq, dk, dv, workspace,
+                                         st);
+  return bf ? run_fp4_bwd<__nv_bfloat16, 64>(p, q, k, v, fb, o, lse, dout, dq, dk, dv,
+                                              workspace, st)
+            : run_fp4_bwd<__half, 64>(p, q, k, v, fb, o, lse, dout, dq, dk, dv, workspace, st);
 }
 
 int sage_last_device_status(void* stream) {

@@ -91,3 +91,26 @@ def attn_fwd(fb: Fp4Bufs, v: torch.Tensor, cfg: Config, o=None, lse=None):
         ctypes.byref(prm), ctypes.byref(st), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
         _stream(v.device)))
     return o, lse
+
+
+def bwd_workspace_bytes(cfg: Config, like: torch.Tensor) -> int:
+    return int(lib().sage_fp4_workspace_bytes(ctypes.byref(cfg.params(like)), 2))
+
+
+def attn_bwd(q, k, v, fb: Fp4Bufs, o, lse, do, cfg: Config, dq=None, dk=None, dv=None,
+             workspace: Optional[torch.Tensor] = None):
+    """Backward with dS in NVFP4, P^T dO and dO V^T in 16 bits (sage_fp4_attn_bwd): returns
+    (dq, dk, dv).  ``fb`` must hold the sequence views (``quant_prologue(..., seq=True)``)."""
+    _check_inputs(q, k, v, o, do)
+    prm = cfg.params(q)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_bytes(cfg, q), dtype=torch.uint8, device=q.device)
+    st = fb.c_struct()
+    check("sage_fp4_attn_bwd", lib().sage_fp4_attn_bwd(
+        ctypes.byref(prm), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(st),
+        o.data_ptr(), lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+        workspace.data_ptr(), workspace.numel(), _stream(q.device)))
+    return dq, dk, dv

@@ -52,7 +52,8 @@ typedef struct {
 } sage_fp4_bufs;
 
 /* Workspace bytes: which = 0 prologue (K-mean partials when ksmooth, plus 2*B*H words for the
- * global maxima), 1 forward (0).  Returns 0 for invalid parameters. */
+ * global maxima), 1 forward (0), 2 backward (D = rowsum(dO o O) [B,H,N] float32, then the
+ * float32 dQ accumulator [B,H,N,d]).  Returns 0 for invalid parameters. */
 size_t sage_fp4_workspace_bytes(const sage_params* p, int which);
 
 /* QK-norm -> K-smoothing -> NVFP4 views of q and k (an absolute-maximum pass, then the
@@ -67,6 +68,29 @@ int sage_fp4_quant_prologue(const sage_params* p, const void* q, const void* k,
  * lse: [B,H,N] float32, natural log of sum_j exp(z_ij). */
 int sage_fp4_attn_fwd(const sage_params* p, const sage_fp4_bufs* fb, const void* v, void* o,
                       float* lse, void* stream);
+
+/* Backward ("Full-Stack FP4" section 2.4: dS in NVFP4; P^T dO and dO V^T in 16 bits):
+ *   S = Q K^T from the forward's NVFP4 views (block-scaled MMA), P = exp(tau S - lse) (causal
+ *   mask); dP = dO V^T (16-bit operands, FP32 accumulation); D = rowsum(dO o O);
+ *   dS = P o (dP - D) in float32;
+ *   dV = P^T dO with P rounded to the 16-bit type of v;
+ *   per 128 x 128 (query, key) tile, dS is quantized twice with the tile's own global scale
+ *   genc = 2688 / max|dS_tile| and the steps listed above: in 16-key blocks (dS_k) and in
+ *   16-query blocks (dS_q);
+ *   dQ = tau dS_k K_seq and dK = tau dS_q^T Q_seq (block-scaled MMA), K_seq / Q_seq the
+ *   sequence views of fb (16-token blocks), which must be present;
+ *   with qknorm, the RMSNorm backward dx = inv (dxhat - xhat (dxhat . xhat) / d) of each row.
+ * q, k, v, o, dout: [B,H,N,d] in p->dtype (the raw inputs, the forward's output and the
+ * output gradient); lse: the forward's [B,H,N]; dq, dk, dv: [B,H,N,d] in p->dtype.
+ * Workspace: sage_fp4_workspace_bytes(p, 2) bytes, 16-byte aligned.
+ * Errors: SAGE_ERR_INVALID_ARG (a null pointer, missing sequence views, or missing inverse RMS
+ * with qknorm), SAGE_ERR_ALIGNMENT, SAGE_ERR_WORKSPACE, SAGE_ERR_UNSUPPORTED (qsmooth, or a
+ * launch the register split cannot take), SAGE_ERR_CUDA (launch failure); a bounded wait that
+ * gives up is reported by sage_last_device_status. */
+int sage_fp4_attn_bwd(const sage_params* p, const void* q, const void* k, const void* v,
+                      const sage_fp4_bufs* fb, const void* o, const float* lse, const void* dout,
+                      void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                      void* stream);
 
 #ifdef __cplusplus
 }

@@ -270,12 +270,15 @@ def qattn_bwd_head(qd, kd, q_seq, k_seq, v, o, lse, do, *, causal: bool, tau: fl
 
 def qattn_attention(q, k, v, do, *, causal: bool, qknorm: bool, ksmooth: bool,
                     tau: float | None = None, eps: float = 1e-6,
-                    quant: bool = True) -> Dict[str, np.ndarray]:
+                    quant: bool = True, dtype: str | None = None) -> Dict[str, np.ndarray]:
     """NVFP4 Q-Attn forward and backward over every (batch, head).
 
     Inputs float32 ``[BH, N, d]`` (exact 16-bit values).  Returns the forward's results
     (``qattn_forward``) plus ``dq, dk, dv`` with respect to the raw q, k, v (RMSNorm backward
     applied when ``qknorm``).  ``quant=False``: full precision (float64, no quantizer).
+    ``dtype`` ("bf16" / "fp16"): the outputs are stored in that 16-bit type, as the INT8
+    path's ``sage_attention`` does -- ``o`` is rounded before the backward reads it (so
+    ``D = rowsum(dO o O)`` takes the stored output) and ``dq, dk, dv`` at the end.
     """
     q, k, v, do = (np.asarray(t, F32) for t in (q, k, v, do))
     BH, N, d = q.shape
@@ -301,6 +304,8 @@ def qattn_attention(q, k, v, do, *, causal: bool, qknorm: bool, ksmooth: bool,
         for h in range(BH):
             o[h], lse[h], _ = qattn_fwd_head(qd[h], kd[h], v[h], causal=causal, tau=tau)
         res.update(o=o, lse=lse)
+    if dtype is not None:
+        res["o"] = S8.round_to_storage(res["o"], dtype).astype(F64)
     dq = np.zeros((BH, N, d))
     dk = np.zeros((BH, N, d))
     dv = np.zeros((BH, N, d))
@@ -312,5 +317,7 @@ def qattn_attention(q, k, v, do, *, causal: bool, qknorm: bool, ksmooth: bool,
             dqh = S8.rms_norm_bwd(dqh, res["q_hat"][h], res["q_inv_rms"][h])
             dkh = S8.rms_norm_bwd(dkh, res["k_hat"][h], res["k_inv_rms"][h])
         dq[h], dk[h] = dqh, dkh
+    if dtype is not None:
+        dq, dk, dv = (S8.round_to_storage(t, dtype).astype(F64) for t in (dq, dk, dv))
     res.update(dq=dq, dk=dk, dv=dv, tau=tau)
     return res

@@ -31,7 +31,8 @@ def test_exports_every_declared_symbol(L):
     names = _declared()
     assert len(names) == 14
     fp4 = _declared("sage_nvfp4.h")
-    assert fp4 == ["sage_fp4_attn_fwd", "sage_fp4_quant_prologue", "sage_fp4_workspace_bytes"]
+    assert fp4 == ["sage_fp4_attn_bwd", "sage_fp4_attn_fwd", "sage_fp4_quant_prologue",
+                   "sage_fp4_workspace_bytes"]
     for n in names + fp4:
         assert hasattr(L, n), n
 
@@ -115,6 +116,36 @@ def test_fp4_workspace_and_argument_checks(L):
                                None) == _lib.SAGE_ERR_INVALID_ARG
     assert L.sage_fp4_attn_fwd(ctypes.byref(p), ctypes.byref(fb), fake, fake + 4, fake,
                                None) == _lib.SAGE_ERR_ALIGNMENT
+
+
+def test_fp4_backward_workspace_and_argument_checks(L):
+    from fwd_bwd_b200._lib import SageFp4Bufs
+
+    BH, N, d = 8, 1024, 128
+    p = _params()
+    wsb = L.sage_fp4_workspace_bytes(ctypes.byref(p), 2)
+    assert wsb == BH * N * 4 + BH * N * d * 4  # D, then the float32 dQ accumulator
+    assert L.sage_fp4_workspace_bytes(ctypes.byref(_params(qsmooth=1)), 2) == 0
+    fake = 1 << 20  # never dereferenced: every call below fails its host-side checks
+    full = SageFp4Bufs(*([fake] * 13))
+    noseq = SageFp4Bufs(*([fake] * 9 + [None] * 4))
+    noinv = SageFp4Bufs(*([fake] * 6 + [None, None] + [fake] * 5))
+    f = L.sage_fp4_attn_bwd
+
+    def call(prm=p, fb=full, ptrs=None, ws=wsb, wsp=fake):
+        t = ptrs if ptrs is not None else [fake] * 3
+        return f(ctypes.byref(prm), *t, ctypes.byref(fb), fake, fake, fake, fake, fake, fake,
+                 wsp, ws, None)
+
+    assert call(fb=noseq) == _lib.SAGE_ERR_INVALID_ARG  # the sequence views are operands
+    assert call(fb=noinv) == _lib.SAGE_ERR_INVALID_ARG  # qknorm needs the inverse RMS
+    assert call(ptrs=[None, fake, fake]) == _lib.SAGE_ERR_INVALID_ARG
+    assert call(ptrs=[fake, fake + 8, fake]) == _lib.SAGE_ERR_ALIGNMENT
+    assert call(ws=wsb - 1) == _lib.SAGE_ERR_WORKSPACE
+    assert call(wsp=None) == _lib.SAGE_ERR_WORKSPACE
+    assert call(prm=_params(qsmooth=1)) == _lib.SAGE_ERR_UNSUPPORTED
+    assert call(prm=_params(d=96)) == _lib.SAGE_ERR_UNSUPPORTED
+    assert call(prm=_params(N=1000)) == _lib.SAGE_ERR_UNSUPPORTED
 
 
 def _params(**kw):

@@ -1,0 +1,121 @@
+"""NVFP4 Q-Attn backward parity: the CUDA path (sage_fp4_attn_bwd) against the NVFP4 oracle
+(qattn_attention, outputs stored in the 16-bit type) on the same seeded inputs.
+
+Both sides quantize dS per 128 x 128 tile with the tile's own global scale, in 16-key blocks
+for dQ and 16-query blocks for dK, and multiply the same NVFP4 sequence views (the prologue is
+bit-exact), so dQ and dK share the oracle's quantization error.  What separates them:
+  * dS itself: the kernel's P = exp2(S c - lse log2 e) (FP32 arguments, the exp2
+    approximation) and dP (FP32 accumulation) move dS by a few float32 ulps.  That changes an
+    E2M1 code only where dS sits on a rounding boundary -- rare, but the element then moves by
+    a whole code step;
+  * dV: the kernel rounds P to the 16-bit type of dO before P^T dO (the tensor-core operand
+    precision), the oracle keeps P exact: a relative error of at most u16 per product
+    (u16 = 2^-8 for bf16, 2^-11 for fp16), partly cancelling over the queries;
+  * the outputs' rounding to the 16-bit type, shared: one ulp where the two sit on either
+    side of a rounding boundary.
+
+test_nvfp4_backward_matches_oracle feeds the kernel the oracle's own forward results (O as
+stored, LSE in float32), which isolates the backward: gates rel-L2 <= TOL_DQK for dQ, dK
+(code flips are rare here: 1e-4 and below on every case) and <= TOL_DV[dtype] for dV (the P
+rounding alone gives about u16 / 1.5).
+
+test_nvfp4_fwd_bwd_chain runs the CUDA forward into the CUDA backward.  The forward's O
+differs from the oracle's by the P V operand rounding (u16-sized, see test_gpu_nvfp4.py);
+through D = rowsum(dO o O) that moves dS by about u16 |D| P, which flips E2M1 codes of dS
+far more often.  Gate: the chain's distance to the oracle is at most CHAIN_FRAC of the
+oracle's own distance to full-precision (float64, no quantizer) gradients, and its cosine
+similarity to those gradients is within COS_SLACK of the oracle's.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.nvfp4_oracle as F
+from fwd_bwd_b200 import nvfp4, ops
+from fwd_bwd_b200.inputs import WORKLOADS, make_inputs
+
+from gpu_helpers import TORCH_DT, cosine, rel_l2, to_device
+
+pytestmark = pytest.mark.gpu
+
+TOL_DQK = 1e-3
+TOL_DV = {"bf16": 4e-3, "fp16": 1e-3}
+CHAIN_FRAC = 0.25
+COS_SLACK = 2e-3
+
+BASE = WORKLOADS["sweep8192"]
+CASES = {
+    "d128_bf16_causal": BASE.replace(B=1, H=2, N=384),
+    "d128_bf16_full": BASE.replace(B=1, H=2, N=256, causal=False),
+    "d128_fp16_causal": BASE.replace(B=2, H=1, N=512, dtype="fp16"),
+    "d64_bf16_causal": WORKLOADS["llama325m"].replace(B=1, H=2, N=384),
+    "d64_fp16_full": WORKLOADS["llama325m"].replace(B=1, H=2, N=256, dtype="fp16",
+                                                   causal=False),
+    "koutlier_norm_off": WORKLOADS["koutlier"].replace(B=1, H=2, N=256, qknorm=False),
+    "koutlier_all_off": WORKLOADS["koutlier"].replace(B=1, H=2, N=384, qknorm=False,
+                                                     ksmooth=False),
+    "small_ds_regime": WORKLOADS["long16k"].replace(H=1, N=512),
+    "single_tile": BASE.replace(B=1, H=1, N=128),
+}
+
+
+def _cfg(w):
+    return ops.Config(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth, q_block=w.q_block,
+                      k_block=w.k_block)
+
+
+def _oracle(w, x, quant=True):
+    BH = w.B * w.H
+    args = [x[n + "_f32"].reshape(BH, w.N, w.d) for n in ("q", "k", "v", "do")]
+    return F.qattn_attention(*args, causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth,
+                             quant=quant, dtype=w.dtype if quant else None)
+
+
+def _gpu(w, x, o_lse=None):
+    """Prologue (with the sequence views), forward unless ``o_lse`` is given, backward."""
+    q, k, v, do = (to_device(x[n], w.dtype) for n in ("q", "k", "v", "do"))
+    cfg = _cfg(w)
+    fb = nvfp4.quant_prologue(q, k, cfg, seq=True)
+    if o_lse is None:
+        o, lse = nvfp4.attn_fwd(fb, v, cfg)
+    else:
+        o, lse = o_lse
+    dq, dk, dv = nvfp4.attn_bwd(q, k, v, fb, o, lse, do, cfg)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    BH = w.B * w.H
+    return {n: t.float().cpu().numpy().astype(np.float64).reshape(BH, w.N, w.d)
+            for n, t in (("dq", dq), ("dk", dk), ("dv", dv))}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_nvfp4_backward_matches_oracle(name):
+    w = CASES[name]
+    x = make_inputs(w)
+    ref = _oracle(w, x)
+    shape = (w.B, w.H, w.N, w.d)
+    o = torch.from_numpy(ref["o"].astype(np.float32).reshape(shape)).to(TORCH_DT[w.dtype])
+    lse = torch.from_numpy(ref["lse"].astype(np.float32).reshape(shape[:3]))
+    g = _gpu(w, x, (o.cuda(), lse.cuda()))
+    for n in ("dq", "dk", "dv"):
+        err = rel_l2(g[n], ref[n])
+        print(f"{name} {n}: rel_l2 {err:.3e}")
+        tol = TOL_DV[w.dtype] if n == "dv" else TOL_DQK
+        assert np.isfinite(g[n]).all()
+        assert err <= tol, (n, err)
+
+
+@pytest.mark.parametrize("name", ["d128_bf16_causal", "d64_fp16_full", "koutlier_all_off"])
+def test_nvfp4_fwd_bwd_chain(name):
+    w = CASES[name]
+    x = make_inputs(w)
+    ref = _oracle(w, x)
+    exact = _oracle(w, x, quant=False)
+    g = _gpu(w, x)
+    for n in ("dq", "dk", "dv"):
+        d_chain, d_quant = rel_l2(g[n], ref[n]), rel_l2(ref[n], exact[n])
+        c_chain, c_ref = cosine(g[n], exact[n]), cosine(ref[n], exact[n])
+        print(f"{name} {n}: chain-oracle {d_chain:.3e}  oracle-exact {d_quant:.3e}  "
+              f"cos chain {c_chain:.5f} oracle {c_ref:.5f}")
+        assert d_chain <= CHAIN_FRAC * d_quant, (n, d_chain, d_quant)
+        assert c_chain >= c_ref - COS_SLACK, (n, c_chain, c_ref)

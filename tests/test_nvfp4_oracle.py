@@ -16,6 +16,7 @@ import pytest
 import torch
 
 import oracle.nvfp4_oracle as F
+import oracle.sage_oracle as S8
 
 # ------------------------------------------------------------------------------------------
 # E2M1
@@ -405,3 +406,22 @@ def test_qattn_bwd_planted_mistakes_are_caught(monkeypatch):
         with monkeypatch.context() as m:
             m.setattr(F, "qattn_bwd_head", fake)
             assert _fails(test_qattn_bwd_full_precision_vs_torch_autograd, True, True, True)
+
+
+def test_qattn_attention_storage_rounding():
+    """dtype="bf16": O is stored (rounded) before the backward reads it, and the gradients are
+    rounded at the end; the stored O changes D = rowsum(dO o O) and so the gradients."""
+    rng = np.random.default_rng(5)
+    q, k, v, do = (rng.standard_normal((1, 128, 64)).astype(np.float32) for _ in range(4))
+    kw = dict(causal=True, qknorm=False, ksmooth=False)
+    plain = F.qattn_attention(q, k, v, do, **kw)
+    st = F.qattn_attention(q, k, v, do, dtype="bf16", **kw)
+    bf = lambda a: np.asarray(a, np.float32).view(np.uint32) & 0xFFFF  # noqa: E731
+    for n in ("o", "dq", "dk", "dv"):
+        assert (bf(st[n]) == 0).all(), n  # bf16 values
+    np.testing.assert_array_equal(st["o"], S8.round_to_storage(plain["o"], "bf16"))
+    np.testing.assert_array_equal(st["dv"], S8.round_to_storage(plain["dv"], "bf16"))  # no D
+    D_plain = (do[0] * plain["o"][0]).sum(1)
+    D_st = (do[0] * st["o"][0]).sum(1)
+    assert np.abs(D_plain - D_st).max() > 0
+    assert not np.array_equal(st["dq"], S8.round_to_storage(plain["dq"], "bf16"))
