@@ -34,7 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd+bwd effective TOPS at 1 B200 and % of INT8/FP16 TC roofline"
-METRIC_FP4 = "NVFP4 Q-Attn forward effective TOPS at 1 B200 and % of FP4/16-bit TC roofline"
+METRIC_FP4 = "NVFP4 Q-Attn fwd+bwd effective TOPS at 1 B200 and % of FP4/16-bit TC roofline"
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--no-peaks", action="store_true",
                     help="skip the tensor-core peak loop (profiling runs; no roofline fraction)")
     ap.add_argument("--variant", default="int8", choices=["int8", "nvfp4"],
-                    help="int8: the SageBwd step (default); nvfp4: the NVFP4 Q-Attn forward")
+                    help="int8: the SageBwd step (default); nvfp4: the NVFP4 Q-Attn fwd+bwd step")
     return ap.parse_args()
 
 
@@ -227,7 +227,8 @@ def run_reference(args, w):
 
 
 def cpu_baseline_fp4(w, n_heads: int):
-    """Time the NVFP4 oracle (as it stands) on the first n_heads heads: prologue + forward."""
+    """Time the NVFP4 oracle (as it stands) on the first n_heads heads: prologue + forward +
+    backward."""
     from threadpoolctl import threadpool_info
 
     import oracle.nvfp4_oracle as F
@@ -235,14 +236,14 @@ def cpu_baseline_fp4(w, n_heads: int):
 
     x = make_inputs(w, heads=range(n_heads))
     t0 = time.perf_counter()
-    F.qattn_forward(x["q_f32"], x["k_f32"], x["v_f32"], causal=w.causal, qknorm=w.qknorm,
-                    ksmooth=w.ksmooth)
+    F.qattn_attention(x["q_f32"], x["k_f32"], x["v_f32"], x["do_f32"], causal=w.causal,
+                      qknorm=w.qknorm, ksmooth=w.ksmooth, dtype=w.dtype)
     dt = time.perf_counter() - t0
-    ops = w.ops("fwd") / (w.B * w.H) * n_heads
+    ops = w.ops() / (w.B * w.H) * n_heads
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
             "sample": f"{n_heads} of {w.B * w.H} heads (flattened b*H+h = 0..{n_heads - 1}) of "
-                      f"the workload, NVFP4 prologue+forward, numpy oracle"}
+                      f"the workload, NVFP4 prologue+forward+backward, numpy oracle"}
 
 
 def l2_policy(w) -> tuple:
@@ -278,7 +279,8 @@ def timed_steps(step, nev: int, steps: int, dev, flush_buf=None):
 
 
 def run_nvfp4(args, w):
-    """The NVFP4 Q-Attn forward: step = NVFP4 prologue (amax + quantization) + forward."""
+    """The NVFP4 Q-Attn step: NVFP4 prologue (with the sequence views) + forward + backward
+    (preprocess, main kernel, dQ finalize)."""
     import torch
 
     from fwd_bwd_b200 import nvfp4, ops
@@ -290,13 +292,16 @@ def run_nvfp4(args, w):
     torch.cuda.set_device(dev)
     cfg = ops.Config(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth)
     x = make_inputs_fast(w, device=str(dev))
-    q, k, v = x["q"], x["k"], x["v"]
-    fb = nvfp4.Fp4Bufs.empty(tuple(q.shape), cfg, dev)
+    q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+    fb = nvfp4.Fp4Bufs.empty(tuple(q.shape), cfg, dev, seq=True)
     ws = torch.empty(nvfp4.workspace_bytes(cfg, q), dtype=torch.uint8, device=dev)
+    wsb = torch.empty(nvfp4.bwd_workspace_bytes(cfg, q), dtype=torch.uint8, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 2 * int(w.ksmooth) + 2 + 1
+    # prologue: (K statistics: 2 when ksmooth) + amax + quantization; forward 1; backward 3
+    launches_per_step = 2 * int(w.ksmooth) + 2 + 1 + 3
     flush, _ = l2_policy(w)
     flush_buf = torch.empty(2 ** 27, dtype=torch.float32, device=dev) if flush else None
 
@@ -305,49 +310,68 @@ def run_nvfp4(args, w):
         ev[1].record(stream)
         nvfp4.attn_fwd(fb, v, cfg, o=o, lse=lse)
         ev[2].record(stream)
+        for stage in range(3):  # preprocess, main kernel, dQ finalize
+            nvfp4.attn_bwd(q, k, v, fb, o, lse, do, cfg, dq=dq, dk=dk, dv=dv, workspace=wsb,
+                           stage=stage)
+            ev[3 + stage].record(stream)
 
     for _ in range(args.warmup):
-        step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+        step([torch.cuda.Event(enable_timing=True) for _ in range(6)])
     torch.cuda.synchronize(dev)
     tc = None if args.no_peaks else measure_tc_peaks(dev, w.dtype)
     torch.cuda.synchronize(dev)
     sampler = ClockSampler(uuid_of(dev))
     time.sleep(0.3)
-    evs = timed_steps(step, 3, args.steps, dev, flush_buf)
+    evs = timed_steps(step, 6, args.steps, dev, flush_buf)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     if ops.device_status(dev) != 0:
         raise RuntimeError("device status reports a kernel timeout in the timed region")
-    ms = statistics.mean(e[0].elapsed_time(e[2]) for e in evs)
-    fwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    fwd_ops = w.ops("fwd")
-    value = fwd_ops / (ms * 1e-3) / 1e12
-    achieved = fwd_ops / (fwd_ms * 1e-3) / 1e12
-    traffic = (traffic_per_launch("fp4::attn_fwd_kernel", "fwd_bwd_b200/csrc/nvfp4.cuh")
-               if w.name == "sweep8192" and w.B == 32 else None)
-    roofline = {"bound": "tensor", "kernel": "fp4::attn_fwd_kernel", "achieved": achieved,
+    mean = lambda a, b: statistics.mean(e[a].elapsed_time(e[b]) for e in evs)  # noqa: E731
+    ms = mean(0, 5)
+    stages = {"prologue": mean(0, 1), "fwd": mean(1, 2), "bwd_preprocess": mean(2, 3),
+              "bwd": mean(3, 4), "dq_finalize": mean(4, 5)}
+    value = w.ops() / (ms * 1e-3) / 1e12
+    kern = {"fp4::attn_fwd_kernel": (stages["fwd"], w.ops("fwd"), 1, 1),
+            "fp4::bwd::attn_bwd_kernel": (stages["bwd"], w.ops("bwd"), 3, 2)}
+    kernels = {}
+    for name, (kms, kops, n4, n16) in kern.items():
+        ach = kops / (kms * 1e-3) / 1e12
+        kernels[name] = {"ms": round(kms, 4), "tops": round(ach, 2)}
+        if tc is not None:
+            # NVFP4 GEMMs at 4x the measured 16-bit rate (the nominal dense ratio 9 : 2.25
+            # POPS), 16-bit GEMMs at the measured rate; equal op counts per GEMM
+            pk = mixed_peak(4.0 * tc["f16"]["tops"], tc["f16"]["tops"], n4, n16)
+            kernels[name].update(peak=round(pk, 1), frac=round(ach / pk, 4))
+    top = max(kernels, key=lambda n: kernels[n]["ms"])
+    src = {"fp4::attn_fwd_kernel": "fwd_bwd_b200/csrc/nvfp4.cuh",
+           "fp4::bwd::attn_bwd_kernel": "fwd_bwd_b200/csrc/nvfp4_bwd.cuh"}[top]
+    traffic = (traffic_per_launch(top, src) if w.name == "sweep8192" and w.B == 32 else None)
+    roofline = {"bound": "tensor", "kernel": top, "achieved": kernels[top]["tops"],
                 "unit": "TFLOP/s", "traffic": traffic}
     if tc is not None:
-        # Q K^T at the FP4 rate (4x the measured 16-bit rate: the nominal dense ratio 9 : 2.25
-        # POPS), P V at the measured 16-bit rate; equal op counts
         p16 = tc["f16"]["tops"]
-        p_fwd = mixed_peak(4.0 * p16, p16, 1, 1)
-        roofline.update(peak=p_fwd, frac=achieved / p_fwd,
+        roofline.update(peak=kernels[top]["peak"], frac=kernels[top]["frac"],
                         peak_note=f"measured in this run: own tcgen05 kind::f16 loop "
                                   f"{p16:.0f} TOPS; NVFP4 = 4x that (nominal ratio), weighted "
-                                  f"1:1 with the 16-bit P V")
+                                  f"by the kernel's GEMM mix (fwd 1 NVFP4 : 1 16-bit, bwd "
+                                  f"3 : 2)")
     e2e = None
     if not args.no_e2e:
-        hin = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t) for t in (q, k, v)]
-        hout = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        qd, kd, vd = (torch.empty_like(t) for t in (q, k, v))
+        hin = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
+               for t in (q, k, v, do)]
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (dq, dk, dv)]
+        qd, kd, vd, dod = (torch.empty_like(t) for t in (q, k, v, do))
 
         def host_step():
-            for h, d_ in zip(hin, (qd, kd, vd)):
+            for h, d_ in zip(hin, (qd, kd, vd, dod)):
                 d_.copy_(h, non_blocking=True)
             nvfp4.quant_prologue(qd, kd, cfg, out=fb, workspace=ws)
             nvfp4.attn_fwd(fb, vd, cfg, o=o, lse=lse)
-            hout.copy_(o, non_blocking=True)
+            nvfp4.attn_bwd(qd, kd, vd, fb, o, lse, dod, cfg, dq=dq, dk=dk, dv=dv,
+                           workspace=wsb)
+            for h, d_ in zip(hout, (dq, dk, dv)):
+                h.copy_(d_, non_blocking=True)
             torch.cuda.synchronize(dev)
 
         host_step()
@@ -355,20 +379,20 @@ def run_nvfp4(args, w):
         for _ in range(args.steps):
             host_step()
         e_ms = (time.perf_counter() - w0) * 1e3 / args.steps
-        e2e = {"value": fwd_ops / (e_ms * 1e-3) / 1e12, "unit": "TOPS",
+        e2e = {"value": w.ops() / (e_ms * 1e-3) / 1e12, "unit": "TOPS",
                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hin),
-               "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout),
+               "note": "one stream, copies not overlapped with the kernels"}
     line = {"metric": METRIC_FP4, "value": value, "unit": "TOPS", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "nvfp4+bf16", "data": "synthetic",
-            "config": dict(config_of(w), variant="nvfp4 forward"),
-            "kernels": {"fp4::attn_fwd_kernel": {"ms": round(fwd_ms, 4),
-                                                 "tops": round(achieved, 2)}},
-            "tensor_peaks": tc, "roofline": roofline, "clocks": clocks, "e2e": e2e,
-            "gpu_launches": launches_per_step * args.steps}
+            "config": dict(config_of(w), variant="nvfp4 fwd+bwd"),
+            "stages_ms": {kk: round(vv, 4) for kk, vv in stages.items()},
+            "kernels": kernels, "tensor_peaks": tc, "roofline": roofline, "clocks": clocks,
+            "e2e": e2e, "gpu_launches": launches_per_step * args.steps}
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_fp4(w, 4)
+        line["cpu_baseline"] = cpu_baseline_fp4(w, 2)
     print(json.dumps(line), flush=True)
 
 

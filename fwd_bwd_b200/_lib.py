@@ -84,6 +84,9 @@ def lib() -> ctypes.CDLL:
         L.sage_fp4_attn_bwd.argtypes = [P(SageParams), vp, vp, vp, P(SageFp4Bufs), vp, vp, vp,
                                         vp, vp, vp, vp, sz, vp]
         L.sage_fp4_attn_bwd.restype = i
+        L.sage_fp4_attn_bwd_stage.argtypes = [i, P(SageParams), vp, vp, vp, P(SageFp4Bufs), vp,
+                                              vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sage_fp4_attn_bwd_stage.restype = i
         L.sage_fwd_bwd_host_workspace_bytes.argtypes = [P(SageParams), i]
         L.sage_fwd_bwd_host_workspace_bytes.restype = sz
         L.sage_fwd_bwd_host.argtypes = [P(SageParams), vp, vp, vp, vp, vp, vp, vp, vp, i, vp, sz,

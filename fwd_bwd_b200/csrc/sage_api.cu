@@ -449,8 +449,9 @@ Fp4BwdWs fp4_bwd_ws(const sage_params* p) {
   return w;
 }
 
+// stage 0: preprocess (D, the dQ accumulator cleared); 1: main kernel; 2: dq finalize.
 template <typename T, int D>
-int run_fp4_bwd(const sage_params* p, const void* q, const void* k, const void* v,
+int run_fp4_bwd(int stage, const sage_params* p, const void* q, const void* k, const void* v,
                 const sage_fp4_bufs* fb, const void* o, const float* lse, const void* dout,
                 void* dq, void* dk, void* dv, void* ws, cudaStream_t st) {
   const int BH = p->B * p->H, N = p->N;
@@ -459,12 +460,20 @@ int run_fp4_bwd(const sage_params* p, const void* q, const void* k, const void* 
   uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
   float* dvec = reinterpret_cast<float*>(wsb + w.dvec);
   float* dqacc = reinterpret_cast<float*>(wsb + w.dq);
-  // D and the cleared dQ accumulator (no INT8 dO codes: dO enters the MMAs in 16 bits)
-  sage::bwd_preprocess_kernel<T, D>
-      <<<static_cast<int>(rows / kRowsPerCta), sage::kQuantThreads, 0, st>>>(
-          reinterpret_cast<const T*>(o), reinterpret_cast<const T*>(dout), dvec, nullptr,
-          nullptr, dqacc, N, p->q_block);
-  if (launch_status() != SAGE_OK) return SAGE_ERR_CUDA;
+  if (stage == 0) {
+    // D and the cleared dQ accumulator (no INT8 dO codes: dO enters the MMAs in 16 bits)
+    sage::bwd_preprocess_kernel<T, D>
+        <<<static_cast<int>(rows / kRowsPerCta), sage::kQuantThreads, 0, st>>>(
+            reinterpret_cast<const T*>(o), reinterpret_cast<const T*>(dout), dvec, nullptr,
+            nullptr, dqacc, N, p->q_block);
+    return launch_status();
+  }
+  if (stage == 2) {
+    sage::dq_finalize_kernel<T, D><<<static_cast<int>(rows / kRowsPerCta), kRowThreads, 0, st>>>(
+        dqacc, reinterpret_cast<const T*>(q), fb->q_inv_rms, reinterpret_cast<T*>(dq),
+        p->qknorm);
+    return launch_status();
+  }
   CUtensorMap tqc, tkc, tqs, tks, tdo, tv;
   const uint64_t seq_rows = static_cast<uint64_t>(BH) * D;
   if (!make_map(&tqc, fb->q_fp4, 1, D / 2, rows, D / 2, sage::fp4::bwd::BQ) ||
@@ -500,10 +509,35 @@ int run_fp4_bwd(const sage_params* p, const void* q, const void* k, const void* 
   if (launch_regs(kern) != sage::fp4::bwd::kLaunchRegs) return SAGE_ERR_UNSUPPORTED;
   kern<<<BH * (N / sage::fp4::bwd::BKT), sage::fp4::bwd::kThreads, smem, st>>>(tqc, tkc, tqs,
                                                                              tks, tdo, tv, a);
-  if (launch_status() != SAGE_OK) return SAGE_ERR_CUDA;
-  sage::dq_finalize_kernel<T, D><<<static_cast<int>(rows / kRowsPerCta), kRowThreads, 0, st>>>(
-      dqacc, reinterpret_cast<const T*>(q), fb->q_inv_rms, reinterpret_cast<T*>(dq), p->qknorm);
   return launch_status();
+}
+
+int fp4_bwd_stage(int stage, const sage_params* p, const void* q, const void* k, const void* v,
+                  const sage_fp4_bufs* fb, const void* o, const float* lse, const void* dout,
+                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  int s = check_fp4(p);
+  if (s != SAGE_OK) return s;
+  if (stage < 0 || stage > 2) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_fp4bufs(p, fb)) != SAGE_OK) return s;
+  if (!fb->q_fp4_t || !fb->k_fp4_t) return SAGE_ERR_INVALID_ARG;
+  if (p->qknorm && (!fb->q_inv_rms || !fb->k_inv_rms)) return SAGE_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return SAGE_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return SAGE_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < fp4_bwd_ws(p).total) return SAGE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_fp4_bwd<__nv_bfloat16, 128>(stage, p, q, k, v, fb, o, lse, dout, dq, dk, dv,
+                                                 workspace, st)
+              : run_fp4_bwd<__half, 128>(stage, p, q, k, v, fb, o, lse, dout, dq, dk, dv,
+                                         workspace, st);
+  return bf ? run_fp4_bwd<__nv_bfloat16, 64>(stage, p, q, k, v, fb, o, lse, dout, dq, dk, dv,
+                                              workspace, st)
+            : run_fp4_bwd<__half, 64>(stage, p, q, k, v, fb, o, lse, dout, dq, dk, dv, workspace,
+                                      st);
 }
 
 // ---- end-to-end pipeline over host buffers -------------------------------------------------
@@ -798,26 +832,20 @@ int sage_fp4_attn_bwd(const sage_params* p, const void* q, const void* k, const 
                       const sage_fp4_bufs* fb, const void* o, const float* lse, const void* dout,
                       void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
                       void* stream) {
-  int s = check_fp4(p);
-  if (s != SAGE_OK) return s;
-  if ((s = check_fp4bufs(p, fb)) != SAGE_OK) return s;
-  if (!fb->q_fp4_t || !fb->k_fp4_t) return SAGE_ERR_INVALID_ARG;
-  if (p->qknorm && (!fb->q_inv_rms || !fb->k_inv_rms)) return SAGE_ERR_INVALID_ARG;
-  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return SAGE_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
-  for (const void* ptr : ptrs)
-    if (ptr && !aligned16(ptr)) return SAGE_ERR_ALIGNMENT;
-  if (!workspace || workspace_bytes < fp4_bwd_ws(p).total) return SAGE_ERR_WORKSPACE;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const bool bf = p->dtype == SAGE_BF16;
-  if (p->d == 128)
-    return bf ? run_fp4_bwd<__nv_bfloat16, 128>(p, q, k, v, fb, o, lse, dout, dq, dk, dv,
-                                                 workspace, st)
-              : run_fp4_bwd<__half, 128>(p, q, k, v, fb, o, lse, dout, dq, dk, dv, workspace,
-                                         st);
-  return bf ? run_fp4_bwd<__nv_bfloat16, 64>(p, q, k, v, fb, o, lse, dout, dq, dk, dv,
-                                              workspace, st)
-            : run_fp4_bwd<__half, 64>(p, q, k, v, fb, o, lse, dout, dq, dk, dv, workspace, st);
+  for (int stage = 0; stage < 3; ++stage) {
+    const int s = fp4_bwd_stage(stage, p, q, k, v, fb, o, lse, dout, dq, dk, dv, workspace,
+                                workspace_bytes, stream);
+    if (s != SAGE_OK) return s;
+  }
+  return SAGE_OK;
+}
+
+int sage_fp4_attn_bwd_stage(int stage, const sage_params* p, const void* q, const void* k,
+                            const void* v, const sage_fp4_bufs* fb, const void* o,
+                            const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  return fp4_bwd_stage(stage, p, q, k, v, fb, o, lse, dout, dq, dk, dv, workspace,
+                       workspace_bytes, stream);
 }
 
 int sage_last_device_status(void* stream) {

@@ -98,9 +98,11 @@ def bwd_workspace_bytes(cfg: Config, like: torch.Tensor) -> int:
 
 
 def attn_bwd(q, k, v, fb: Fp4Bufs, o, lse, do, cfg: Config, dq=None, dk=None, dv=None,
-             workspace: Optional[torch.Tensor] = None):
+             workspace: Optional[torch.Tensor] = None, stage: Optional[int] = None):
     """Backward with dS in NVFP4, P^T dO and dO V^T in 16 bits (sage_fp4_attn_bwd): returns
-    (dq, dk, dv).  ``fb`` must hold the sequence views (``quant_prologue(..., seq=True)``)."""
+    (dq, dk, dv).  ``fb`` must hold the sequence views (``quant_prologue(..., seq=True)``).
+    ``stage`` in {0, 1, 2} runs only that stage (sage_fp4_attn_bwd_stage); the caller then owns
+    ``workspace`` across the three calls."""
     _check_inputs(q, k, v, o, do)
     prm = cfg.params(q)
     dq = torch.empty_like(q) if dq is None else dq
@@ -109,8 +111,11 @@ def attn_bwd(q, k, v, fb: Fp4Bufs, o, lse, do, cfg: Config, dq=None, dk=None, dv
     if workspace is None:
         workspace = torch.empty(bwd_workspace_bytes(cfg, q), dtype=torch.uint8, device=q.device)
     st = fb.c_struct()
-    check("sage_fp4_attn_bwd", lib().sage_fp4_attn_bwd(
-        ctypes.byref(prm), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(st),
-        o.data_ptr(), lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-        workspace.data_ptr(), workspace.numel(), _stream(q.device)))
+    args = (ctypes.byref(prm), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(st),
+            o.data_ptr(), lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+            dv.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream(q.device))
+    if stage is None:
+        check("sage_fp4_attn_bwd", lib().sage_fp4_attn_bwd(*args))
+    else:
+        check("sage_fp4_attn_bwd_stage", lib().sage_fp4_attn_bwd_stage(stage, *args))
     return dq, dk, dv

@@ -92,6 +92,18 @@ int sage_fp4_attn_bwd(const sage_params* p, const void* q, const void* k, const 
                       void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
                       void* stream);
 
+/* The three stages sage_fp4_attn_bwd runs, for callers that schedule or time them separately;
+ * same arguments and checks as sage_fp4_attn_bwd, and they must run in order on the same
+ * workspace:
+ *   stage 0  D = rowsum(dO o O) into the workspace, the float32 dQ accumulator cleared;
+ *   stage 1  the tensor-core kernel: dk and dv written, dQ accumulated in the workspace;
+ *   stage 2  dq from the accumulator (with the RMSNorm backward when qknorm).
+ * Returns SAGE_ERR_INVALID_ARG for any other stage. */
+int sage_fp4_attn_bwd_stage(int stage, const sage_params* p, const void* q, const void* k,
+                            const void* v, const sage_fp4_bufs* fb, const void* o,
+                            const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

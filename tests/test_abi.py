@@ -31,8 +31,8 @@ def test_exports_every_declared_symbol(L):
     names = _declared()
     assert len(names) == 14
     fp4 = _declared("sage_nvfp4.h")
-    assert fp4 == ["sage_fp4_attn_bwd", "sage_fp4_attn_fwd", "sage_fp4_quant_prologue",
-                   "sage_fp4_workspace_bytes"]
+    assert fp4 == ["sage_fp4_attn_bwd", "sage_fp4_attn_bwd_stage", "sage_fp4_attn_fwd",
+                   "sage_fp4_quant_prologue", "sage_fp4_workspace_bytes"]
     for n in names + fp4:
         assert hasattr(L, n), n
 
@@ -146,6 +146,12 @@ def test_fp4_backward_workspace_and_argument_checks(L):
     assert call(prm=_params(qsmooth=1)) == _lib.SAGE_ERR_UNSUPPORTED
     assert call(prm=_params(d=96)) == _lib.SAGE_ERR_UNSUPPORTED
     assert call(prm=_params(N=1000)) == _lib.SAGE_ERR_UNSUPPORTED
+    g = L.sage_fp4_attn_bwd_stage
+    for stage in (-1, 3):
+        assert g(stage, ctypes.byref(p), fake, fake, fake, ctypes.byref(full), fake, fake, fake,
+                 fake, fake, fake, fake, wsb, None) == _lib.SAGE_ERR_INVALID_ARG
+    assert g(1, ctypes.byref(p), fake, fake, fake, ctypes.byref(noseq), fake, fake, fake, fake,
+             fake, fake, fake, wsb, None) == _lib.SAGE_ERR_INVALID_ARG
 
 
 def _params(**kw):
