@@ -18,8 +18,9 @@
 //      block scales in the tensor core's scale-factor order;
 //   5. dQ_t = dS_k K_seq and dK_t = dS_q^T Q_seq (kind::mxf4nvf4; K_seq / Q_seq are the
 //      prologue's sequence views, 16-token blocks) into TMEM; dQ_t * tau / (genc genc_K) is
-//      added to the float32 dQ accumulator in global memory, dK_t * tau / (genc genc_Q) to
-//      float32 registers.
+//      staged in shared memory and added to the float32 dQ accumulator in global memory by
+//      TMA reductions (asynchronous: the next tile's work overlaps them), dK_t * tau /
+//      (genc genc_Q) to float32 registers.
 // After the last tile: dV from TMEM, dK (with the RMSNorm backward when qknorm) to global memory.
 //
 // Warps 0-7 compute, warp 8 is the TMA producer, warp 9 the MMA issuer, warps 10-11 idle (they
@@ -73,11 +74,16 @@ struct Smem {
   alignas(128) uint8_t qssf[2 * 512];
   alignas(128) uint8_t dsksf[2 * 512];
   alignas(128) uint8_t dsqsf[2 * 512];
-  float dst[BKT][BQ + 1];  // dS transposed, [key][query] (padded: conflict-free columns)
+  // dS transposed, [key][query]; rows padded to 132 floats: the column writes of pass A and
+  // the 16-byte row reads of pass B are both conflict-free.  After pass B the same bytes stage
+  // the tile's dQ for the TMA reductions: per compute warp D/64 boxes of 32 query rows x 32
+  // channels (4 KB, 128-byte swizzle)
+  alignas(1024) float dst[BKT][BQ + 4];
   alignas(16) float red[2][8];  // per-warp max |dS|, [tile parity][warp]
   float dot[BKT];               // RMSNorm-backward row dot products (warpgroup 1 -> 0)
   uint64_t kv_full, st_full, st_free, sdp_full, p_ready, ds_ready, dkdq_full, tmem_free;
   uint64_t red_full[2];
+  uint64_t stage_free;  // the previous tile's dQ reductions have read the staging boxes
   uint32_t tmem_base;
   int abort;
 };
@@ -105,7 +111,7 @@ struct Args {
   const float* dvec;      // [BH, N]
   const void* k_raw;      // [BH, N, D] (RMSNorm backward of dk)
   const float* k_inv_rms; // [BH, N]
-  float* dq_acc;          // [BH, N, D] float32
+  float* dq_acc;          // [BH, N, D] float32 (the kernel adds into it through tm_dq)
   void* dk;
   void* dv;
   int N, causal, qknorm;
@@ -113,24 +119,37 @@ struct Args {
   float tau;         // softmax_scale
 };
 
+// Eight E2M1 codes of values already multiplied by their block's encode factor: element 2i
+// in the low nibble of byte i (hardware conversion: nearest, ties to even, saturating at 6).
+__device__ __forceinline__ uint32_t e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+  return r;
+}
+
 // Quantizes one 16-element block to NVFP4 with global encode scale genc (the prologue's
 // float32 steps): returns the 8 code bytes (element 2i in the low nibble of byte i) and the
 // E4M3 scale byte.
 __device__ __forceinline__ uint2 quant_block16(const float (&x)[16], float genc, uint32_t& sc) {
   float am = 0.0f;
 #pragma unroll
-  for (int e = 0; e < 16; ++e) am = fmaxf(am, fabsf(x[e]));
+  for (int e = 0; e < 16; e += 2) am = fmax3(am, fabsf(x[e]), fabsf(x[e + 1]));
   const float u = __fdiv_rn(__fmul_rn(am, genc), 6.0f);
   sc = e4m3_code(u);
   const float sd = e4m3_value(sc);
   const float mult = sd > 0.0f ? __fdiv_rn(genc, sd) : 0.0f;
-  uint32_t w0 = 0, w1 = 0;
+  const float2 m2 = make_float2(mult, mult);
+  float2 y[8];
 #pragma unroll
-  for (int e = 0; e < 8; e += 2) {
-    w0 |= e2m1x2(__fmul_rn(x[e], mult), __fmul_rn(x[e + 1], mult)) << (4 * e);
-    w1 |= e2m1x2(__fmul_rn(x[8 + e], mult), __fmul_rn(x[9 + e], mult)) << (4 * e);
-  }
-  return make_uint2(w0, w1);
+  for (int e = 0; e < 8; ++e) y[e] = __fmul2_rn(make_float2(x[2 * e], x[2 * e + 1]), m2);
+  return make_uint2(e2m1x8(y[0], y[1], y[2], y[3]), e2m1x8(y[4], y[5], y[6], y[7]));
 }
 
 template <typename T, int D>
@@ -140,8 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_qs,
                     const __grid_constant__ CUtensorMap tm_ks,
                     const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_v, Args args) {
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_dq, Args args) {
   static_assert(D == 64 || D == 128, "head dimension");
+  static_assert(sizeof(float) * BKT * (BQ + 4) >= 8 * (D / 64) * 4096, "dQ staging space");
   constexpr int DH = D / 2;
   constexpr uint32_t kSfBytes = D / 64 * 512;
   constexpr uint32_t kSwC = (D == 128) ? kSwizzle64B : kSwizzle32B;  // Q / K code tiles
@@ -170,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.tmem_free, kCompute);
     mbar_init(&sm.red_full[0], 8);
     mbar_init(&sm.red_full[1], 8);
+    mbar_init(&sm.stage_free, 8);
     fence_barrier_init();
   }
   __syncthreads();
@@ -196,6 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_ks);
       tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_dq);
       // resident: K codes and scales, V, the K sequence view and its scales
       mbar_arrive_expect_tx(&sm.kv_full, BKT * D / 2 + kSfBytes + BKT * D * 2 + D * 64 + 1024);
       tma_load_2d(sm.kc, &tm_kc, 0, row_base + t * BKT, &sm.kv_full);
@@ -306,38 +329,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool diag = args.causal && qt == t;
       mbar_wait(&sm.sdp_full, it & 1, 410);
       tc_fence_after();
-      // pass A: this row's 64 keys of warpgroup h, 16 columns at a time
+      if (it >= 1) {  // pass A rewrites the bytes the previous tile's dQ was staged in
+        if (lane == 0) {
+          bulk_wait_read_0();
+          mbar_arrive(&sm.stage_free);
+        }
+        mbar_wait(&sm.stage_free, (it - 1) & 1, 413);
+      }
+      // pass A: this row's 64 keys of warpgroup h, 32 columns at a time
       float ds[64];
       float dsmax = 0.0f;
       uint8_t* patom = reinterpret_cast<uint8_t*>(sm.p) + h * (BQ * 128);
+      const float2 c2 = make_float2(c, c), nlse2 = make_float2(-lse2, -lse2);
+      const float2 ndvr2 = make_float2(-dvr, -dvr);
 #pragma unroll
-      for (int c16 = 0; c16 < 4; ++c16) {
-        const int col = h * 64 + c16 * 16;
-        uint32_t sx[16], px[16];
-        tmem_ld16(lane_base + kColS + col, sx);
-        tmem_ld16(lane_base + kColDP + col, px);
-        tmem_ld_wait_regs(sx, px);
-        uint32_t w[8];
+      for (int c32 = 0; c32 < 2; ++c32) {
+        const int col = h * 64 + c32 * 32;
+        uint32_t s0[16], s1[16], q0[16], q1[16];
+        tmem_ld32x(lane_base + kColS + col, s0, s1);
+        tmem_ld32x(lane_base + kColDP + col, q0, q1);
+        tmem_ld_wait_regs4(s0, s1, q0, q1);
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float p0 = ex2_approx(fmaf(__uint_as_float(sx[e]), c, -lse2));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sx[e + 1]), c, -lse2));
-          if (diag && col + e > r) p0 = 0.0f;  // key index - query index = col - r
-          if (diag && col + e + 1 > r) p1 = 0.0f;
-          const float d0 = p0 * (__uint_as_float(px[e]) - dvr);
-          const float d1 = p1 * (__uint_as_float(px[e + 1]) - dvr);
-          ds[c16 * 16 + e] = d0;
-          ds[c16 * 16 + e + 1] = d1;
-          dsmax = fmax3(dsmax, fabsf(d0), fabsf(d1));
-          w[e / 2] = Cvt<T>::pack2(p0, p1);
-          sm.dst[col + e][r] = d0;
-          sm.dst[col + e + 1][r] = d1;
+        for (int half = 0; half < 2; ++half) {
+          const uint32_t(&sx)[16] = half ? s1 : s0;
+          const uint32_t(&px)[16] = half ? q1 : q0;
+          const int cc = col + half * 16;  // first key of these 16 columns
+          uint32_t w[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            const float2 z = __ffma2_rn(make_float2(__uint_as_float(sx[e]), __uint_as_float(sx[e + 1])),
+                                        c2, nlse2);
+            float p0 = ex2_approx(z.x), p1 = ex2_approx(z.y);
+            if (diag && cc + e > r) p0 = 0.0f;  // key index - query index = cc + e - r
+            if (diag && cc + e + 1 > r) p1 = 0.0f;
+            const float2 d = __fmul2_rn(
+                make_float2(p0, p1),
+                __fadd2_rn(make_float2(__uint_as_float(px[e]), __uint_as_float(px[e + 1])), ndvr2));
+            const int j = c32 * 32 + half * 16 + e;
+            ds[j] = d.x;
+            ds[j + 1] = d.y;
+            dsmax = fmax3(dsmax, fabsf(d.x), fabsf(d.y));
+            w[e / 2] = Cvt<T>::pack2(p0, p1);
+            sm.dst[cc + e][r] = d.x;
+            sm.dst[cc + e + 1][r] = d.y;
+          }
+          // keys cc .. cc+15 are 16-byte chunks 2 c16 and 2 c16 + 1 of this row's atom
+          const int c16 = c32 * 2 + half;
+          *reinterpret_cast<uint4*>(patom + swz_offset(r, 2 * c16, 128)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(patom + swz_offset(r, 2 * c16 + 1, 128)) =
+              make_uint4(w[4], w[5], w[6], w[7]);
         }
-        // keys col .. col+15 are 16-byte chunks 2 c16 and 2 c16 + 1 of this row's atom
-        *reinterpret_cast<uint4*>(patom + swz_offset(r, 2 * c16, 128)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(patom + swz_offset(r, 2 * c16 + 1, 128)) =
-            make_uint4(w[4], w[5], w[6], w[7]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -378,10 +420,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int qb = 0; qb < 4; qb += 2) {
           uint32_t sc0, sc1;
           float xa[16], xb[16];
+          const float4* row = reinterpret_cast<const float4*>(&sm.dst[k][qh * 64 + qb * 16]);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            xa[e] = sm.dst[k][qh * 64 + qb * 16 + e];
-            xb[e] = sm.dst[k][qh * 64 + qb * 16 + 16 + e];
+          for (int e = 0; e < 4; ++e) {
+            const float4 fa = row[e], fb = row[4 + e];
+            xa[4 * e] = fa.x;
+            xa[4 * e + 1] = fa.y;
+            xa[4 * e + 2] = fa.z;
+            xa[4 * e + 3] = fa.w;
+            xb[4 * e] = fb.x;
+            xb[4 * e + 1] = fb.y;
+            xb[4 * e + 2] = fb.z;
+            xb[4 * e + 3] = fb.w;
           }
           const uint2 ca = quant_block16(xa, genc, sc0);
           const uint2 cb = quant_block16(xb, genc, sc1);
@@ -400,26 +450,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float sk = __fdiv_rn(args.tau, __fmul_rn(genc, qg));
       mbar_wait(&sm.dkdq_full, it & 1, 412);
       tc_fence_after();
-      float* dqrow = args.dq_acc + grow * D + h * DH;
+      // dQ_t scaled into this warp's staging boxes and dK_t into the accumulators; then the TMEM
+      // columns are released (the next tile's S / dP MMAs start) and one lane hands the boxes
+      // to the TMA unit, which adds them into the float32 dQ accumulator
+      uint8_t* stage = reinterpret_cast<uint8_t*>(&sm.dst[0][0]) + warp * (D / 64) * 4096;
 #pragma unroll
-      for (int c0 = 0; c0 < DH; c0 += 16) {
-        uint32_t a[16], kx[16];
-        tmem_ld16(lane_base + kColS + h * DH + c0, a);
-        tmem_ld16(lane_base + kColDP + h * DH + c0, kx);
-        tmem_ld_wait_regs(a, kx);
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        uint32_t a0[16], a1[16], k0[16], k1[16];
+        tmem_ld32x(lane_base + kColS + h * DH + c0, a0, a1);
+        tmem_ld32x(lane_base + kColDP + h * DH + c0, k0, k1);
+        tmem_ld_wait_regs4(a0, a1, k0, k1);
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          const float4 v4 = make_float4(__uint_as_float(a[e]) * sq, __uint_as_float(a[e + 1]) * sq,
-                                        __uint_as_float(a[e + 2]) * sq,
-                                        __uint_as_float(a[e + 3]) * sq);
-          atomicAdd(reinterpret_cast<float4*>(dqrow + c0 + e), v4);
+        for (int e = 0; e < 16; ++e) {
+          acck[c0 + e] = fmaf(__uint_as_float(k0[e]), sk, acck[c0 + e]);
+          acck[c0 + 16 + e] = fmaf(__uint_as_float(k1[e]), sk, acck[c0 + 16 + e]);
         }
+        uint8_t* box = stage + (c0 / 32) * 4096;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acck[c0 + e] = fmaf(__uint_as_float(kx[e]), sk, acck[c0 + e]);
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t(&a)[16] = ch < 4 ? a0 : a1;
+          const int e = (ch & 3) * 4;
+          *reinterpret_cast<float4*>(box + swz_offset(lane, ch, 128)) =
+              make_float4(__uint_as_float(a[e]) * sq, __uint_as_float(a[e + 1]) * sq,
+                          __uint_as_float(a[e + 2]) * sq, __uint_as_float(a[e + 3]) * sq);
+        }
       }
       tc_fence_before();
       mbar_arrive(&sm.tmem_free);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < D / 64; ++j)
+          tma_reduce_add_2d(&tm_dq, stage + j * 4096, h * DH + 32 * j,
+                            row_base + qt * BQ + quarter * 32);
+        bulk_commit();
+      }
     }
+    if (lane == 0) bulk_wait_all();  // this warp's dQ reductions have completed
     // epilogue: dV from TMEM, dK from the registers (thread = key row r, channels h*D/2 ..);
     // every dV MMA has completed: the last tile's dK/dQ commit follows them
     {

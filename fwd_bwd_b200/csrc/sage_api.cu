@@ -474,14 +474,15 @@ int run_fp4_bwd(int stage, const sage_params* p, const void* q, const void* k, c
         p->qknorm);
     return launch_status();
   }
-  CUtensorMap tqc, tkc, tqs, tks, tdo, tv;
+  CUtensorMap tqc, tkc, tqs, tks, tdo, tv, tdq;
   const uint64_t seq_rows = static_cast<uint64_t>(BH) * D;
   if (!make_map(&tqc, fb->q_fp4, 1, D / 2, rows, D / 2, sage::fp4::bwd::BQ) ||
       !make_map(&tkc, fb->k_fp4, 1, D / 2, rows, D / 2, sage::fp4::bwd::BKT) ||
       !make_map(&tqs, fb->q_fp4_t, 1, N / 2, seq_rows, 64, D) ||
       !make_map(&tks, fb->k_fp4_t, 1, N / 2, seq_rows, 64, D) ||
       !make_map(&tdo, dout, 2, D, rows, 64, sage::fp4::bwd::BQ) ||
-      !make_map(&tv, v, 2, D, rows, 64, sage::fp4::bwd::BKT))
+      !make_map(&tv, v, 2, D, rows, 64, sage::fp4::bwd::BKT) ||
+      !make_map(&tdq, dqacc, 4, D, rows, 32, 32))  // 32 x 32 float32 boxes, 128-byte swizzle
     return SAGE_ERR_CUDA;
   sage::fp4::bwd::Args a;
   a.q_sf = fb->q_sf;
@@ -508,7 +509,8 @@ int run_fp4_bwd(int stage, const sage_params* p, const void* q, const void* k, c
   // register split between warpgroups (setmaxnreg) assumes exactly kLaunchRegs at launch
   if (launch_regs(kern) != sage::fp4::bwd::kLaunchRegs) return SAGE_ERR_UNSUPPORTED;
   kern<<<BH * (N / sage::fp4::bwd::BKT), sage::fp4::bwd::kThreads, smem, st>>>(tqc, tkc, tqs,
-                                                                             tks, tdo, tv, a);
+                                                                             tks, tdo, tv, tdq,
+                                                                             a);
   return launch_status();
 }
 
