@@ -55,24 +55,26 @@ namespace fp4 {
 // ---------------------------------------------------------------------------------------------
 // Number formats
 // ---------------------------------------------------------------------------------------------
-// Unsigned E4M3 code of u >= 0: nearest, ties to even, 448 and above -> 448 (0x7E).
+// Unsigned E4M3 code of u >= 0: nearest, ties to even, 448 and above -> 448 (0x7E).  Both the
+// subnormal and the normal candidate are computed and one is selected (no branches).
 __device__ __forceinline__ uint32_t e4m3_code(float u) {
-  if (u >= 448.0f) return 0x7Eu;
-  if (u < 0.015625f) return static_cast<uint32_t>(__float2int_rn(u * 512.0f));  // m * 2^-9
+  // subnormal codes: m * 2^-9, m = rint(u * 512) in [0, 8] (8 is the smallest normal, 2^-6)
+  const uint32_t cs = static_cast<uint32_t>(__float2int_rn(u * 512.0f));
+  // normal codes: with e = floor(log2 u), u * 2^(3-e) lies in [8, 16) and is exact (a
+  // power-of-two scaling); its rounding q in [8, 16] gives code ((e + 7) << 3) + (q - 8), where
+  // q = 16 carries into the exponent field.  (Meaningless for u < 2^-6, where cs is taken.)
   const int e = static_cast<int>((__float_as_uint(u) >> 23) & 0xFFu) - 127;
-  // u * 2^(3-e) lies in [8, 16) and is exact (a power-of-two scaling)
-  int q = __float2int_rn(u * __uint_as_float(static_cast<uint32_t>(130 - e) << 23));
-  int ee = e;
-  if (q == 16) {
-    q = 8;
-    ee = e + 1;
-  }
-  return static_cast<uint32_t>(((ee + 7) << 3) | (q - 8));
+  const int q = __float2int_rn(u * __uint_as_float(static_cast<uint32_t>(130 - e) << 23));
+  const uint32_t cn = static_cast<uint32_t>(((e + 7) << 3) + (q - 8));
+  const uint32_t c = u < 0.015625f ? cs : cn;
+  return u >= 448.0f ? 0x7Eu : c;
 }
 
 __device__ __forceinline__ float e4m3_value(uint32_t c) {
   const uint32_t e = c >> 3, m = c & 7u;
-  return e == 0 ? static_cast<float>(m) * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  const float sub = static_cast<float>(m) * 0.001953125f;
+  const float nrm = __uint_as_float(((e + 120u) << 23) | (m << 20));
+  return e == 0 ? sub : nrm;
 }
 
 // Two E2M1 codes in one byte (lo in bits 0-3, hi in bits 4-7) by the hardware conversion:

@@ -320,22 +320,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int e = 0; e < DH; ++e) acck[e] = 0.0f;
 
+    // this row's LSE and D, loaded one tile ahead
+    size_t grow_n = static_cast<size_t>(row_base) + i_first * BQ + r;
+    float lse_n = args.lse[grow_n], dvr_n = args.dvec[grow_n];
     for (int it = 0; it < nq; ++it) {
       const int qt = i_first + it;
       const int b = it & 1;
-      const size_t grow = static_cast<size_t>(row_base) + qt * BQ + r;
-      const float lse2 = args.lse[grow] * 1.4426950408889634f;
-      const float dvr = args.dvec[grow];
+      const size_t grow = grow_n;
+      const float lse2 = lse_n * 1.4426950408889634f;
+      const float dvr = dvr_n;
+      if (it + 1 < nq) {
+        grow_n += BQ;
+        lse_n = args.lse[grow_n];
+        dvr_n = args.dvec[grow_n];
+      }
       const bool diag = args.causal && qt == t;
       mbar_wait(&sm.sdp_full, it & 1, 410);
       tc_fence_after();
-      if (it >= 1) {  // pass A rewrites the bytes the previous tile's dQ was staged in
-        if (lane == 0) {
-          bulk_wait_read_0();
-          mbar_arrive(&sm.stage_free);
-        }
-        mbar_wait(&sm.stage_free, (it - 1) & 1, 413);
-      }
       // pass A: this row's 64 keys of warpgroup h, 32 columns at a time
       float ds[64];
       float dsmax = 0.0f;
@@ -370,8 +371,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ds[j + 1] = d.y;
             dsmax = fmax3(dsmax, fabsf(d.x), fabsf(d.y));
             w[e / 2] = Cvt<T>::pack2(p0, p1);
-            sm.dst[cc + e][r] = d.x;
-            sm.dst[cc + e + 1][r] = d.y;
           }
           // keys cc .. cc+15 are 16-byte chunks 2 c16 and 2 c16 + 1 of this row's atom
           const int c16 = c32 * 2 + half;
@@ -384,6 +383,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sm.p_ready);
+      // dS transposed into shared memory, once the previous tile's dQ reductions have read
+      // the same bytes
+      if (it >= 1) {
+        if (lane == 0) {
+          bulk_wait_read_0();
+          mbar_arrive(&sm.stage_free);
+        }
+        mbar_wait(&sm.stage_free, (it - 1) & 1, 413);
+      }
+#pragma unroll
+      for (int j = 0; j < 64; ++j) sm.dst[h * 64 + j][r] = ds[j];
       dsmax = warp_max(dsmax);
       __syncwarp();  // this warp's transposed dS writes precede lane 0's arrival
       if (lane == 0) {
@@ -395,51 +405,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int w8 = 0; w8 < 8; ++w8) tmax = fmaxf(tmax, sm.red[b][w8]);
       const float genc = tmax > 0.0f ? __fdiv_rn(kGlobalRange, tmax) : 1.0f;
-      // pass B (1): dS in 16-key blocks along this query row -> A of dQ
+      // pass B, two 32-element halves, each quantizing a pair of blocks in both orientations:
+      // (1) dS in 16-key blocks along this query row -> A of dQ;
+      // (2) dS^T in 16-query blocks along key row k = threadIdx % 128 (queries 64 qh .. +63,
+      //     read back from the transposed tile) -> A of dK
+      const int k = threadIdx.x & 127, qh = threadIdx.x >> 7;
 #pragma unroll
-      for (int kb = 0; kb < 4; kb += 2) {
-        uint32_t sc0, sc1;
-        float xa[16], xb[16];
+      for (int pb = 0; pb < 4; pb += 2) {
+        uint32_t s0, s1, s2, s3;
+        float xa[16], xb[16], ya[16], yb[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          xa[e] = ds[kb * 16 + e];
-          xb[e] = ds[kb * 16 + 16 + e];
+          xa[e] = ds[pb * 16 + e];
+          xb[e] = ds[pb * 16 + 16 + e];
         }
-        const uint2 ca = quant_block16(xa, genc, sc0);
-        const uint2 cb = quant_block16(xb, genc, sc1);
-        *reinterpret_cast<uint4*>(sm.dsk + swz_offset(r, 2 * h + kb / 2, 64)) =
+        const float4* row = reinterpret_cast<const float4*>(&sm.dst[k][qh * 64 + pb * 16]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 fa = row[e], fb = row[4 + e];
+          ya[4 * e] = fa.x;
+          ya[4 * e + 1] = fa.y;
+          ya[4 * e + 2] = fa.z;
+          ya[4 * e + 3] = fa.w;
+          yb[4 * e] = fb.x;
+          yb[4 * e + 1] = fb.y;
+          yb[4 * e + 2] = fb.z;
+          yb[4 * e + 3] = fb.w;
+        }
+        const uint2 ca = quant_block16(xa, genc, s0);
+        const uint2 cb = quant_block16(xb, genc, s1);
+        const uint2 da = quant_block16(ya, genc, s2);
+        const uint2 db = quant_block16(yb, genc, s3);
+        *reinterpret_cast<uint4*>(sm.dsk + swz_offset(r, 2 * h + pb / 2, 64)) =
             make_uint4(ca.x, ca.y, cb.x, cb.y);
-        sm.dsksf[h * 512 + (r & 31) * 16 + (r >> 5) * 4 + kb] = static_cast<uint8_t>(sc0);
-        sm.dsksf[h * 512 + (r & 31) * 16 + (r >> 5) * 4 + kb + 1] = static_cast<uint8_t>(sc1);
-      }
-      // pass B (2): dS^T in 16-query blocks along each key row -> A of dK; thread -> key
-      // k = threadIdx % 128, queries 64 qh .. 64 qh + 63
-      {
-        const int k = threadIdx.x & 127, qh = threadIdx.x >> 7;
-#pragma unroll
-        for (int qb = 0; qb < 4; qb += 2) {
-          uint32_t sc0, sc1;
-          float xa[16], xb[16];
-          const float4* row = reinterpret_cast<const float4*>(&sm.dst[k][qh * 64 + qb * 16]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float4 fa = row[e], fb = row[4 + e];
-            xa[4 * e] = fa.x;
-            xa[4 * e + 1] = fa.y;
-            xa[4 * e + 2] = fa.z;
-            xa[4 * e + 3] = fa.w;
-            xb[4 * e] = fb.x;
-            xb[4 * e + 1] = fb.y;
-            xb[4 * e + 2] = fb.z;
-            xb[4 * e + 3] = fb.w;
-          }
-          const uint2 ca = quant_block16(xa, genc, sc0);
-          const uint2 cb = quant_block16(xb, genc, sc1);
-          *reinterpret_cast<uint4*>(sm.dsq + swz_offset(k, 2 * qh + qb / 2, 64)) =
-              make_uint4(ca.x, ca.y, cb.x, cb.y);
-          sm.dsqsf[qh * 512 + (k & 31) * 16 + (k >> 5) * 4 + qb] = static_cast<uint8_t>(sc0);
-          sm.dsqsf[qh * 512 + (k & 31) * 16 + (k >> 5) * 4 + qb + 1] = static_cast<uint8_t>(sc1);
-        }
+        sm.dsksf[h * 512 + (r & 31) * 16 + (r >> 5) * 4 + pb] = static_cast<uint8_t>(s0);
+        sm.dsksf[h * 512 + (r & 31) * 16 + (r >> 5) * 4 + pb + 1] = static_cast<uint8_t>(s1);
+        *reinterpret_cast<uint4*>(sm.dsq + swz_offset(k, 2 * qh + pb / 2, 64)) =
+            make_uint4(da.x, da.y, db.x, db.y);
+        sm.dsqsf[qh * 512 + (k & 31) * 16 + (k >> 5) * 4 + pb] = static_cast<uint8_t>(s2);
+        sm.dsqsf[qh * 512 + (k & 31) * 16 + (k >> 5) * 4 + pb + 1] = static_cast<uint8_t>(s3);
       }
       fence_proxy_async_smem();
       tc_fence_before();
