@@ -80,8 +80,15 @@ struct Smem {
   // channels (4 KB, 128-byte swizzle)
   alignas(1024) float dst[BKT][BQ + 4];
   alignas(16) float red[2][8];  // per-warp max |dS|, [tile parity][warp]
+  float mult[128];              // the tile's genc / E4M3 value, by scale code
   float dot[BKT];               // RMSNorm-backward row dot products (warpgroup 1 -> 0)
-  uint64_t kv_full, st_full, st_free, sdp_full, p_ready, ds_ready, dkdq_full, tmem_free;
+  uint64_t kv_full;
+  // S and dP landed; P written; dS codes written (16-key blocks, 16-query blocks); dQ_t and
+  // dK_t landed; the S / dQ_t and the dP / dK_t columns read out
+  uint64_t s_full, dp_full, p_ready, dsk_ready, dsq_ready, dq_full, dk_full, s_free, dp_free;
+  // the query tile's operands, each loaded as soon as its last reader of the previous tile
+  // has completed: Q codes and scales (S), dO (dP, dV), the Q sequence view (dK)
+  uint64_t q_full, q_free, do_full, do_free, qs_full, qs_free;
   uint64_t red_full[2];
   uint64_t stage_free;  // the previous tile's dQ reductions have read the staging boxes
   uint32_t tmem_base;
@@ -134,17 +141,29 @@ __device__ __forceinline__ uint32_t e2m1x8(float2 a, float2 b, float2 c, float2 
   return r;
 }
 
+// x / 6 without a division: q = x * r with r = RN(1/6), the exact residual e = x - 6 q by one
+// FMA, then q + e r by a second FMA (the correction step of Markstein's division algorithm).
+// The result is the correctly rounded quotient whenever that quotient is a normal float32
+// (one binade decides it: power-of-two scaling is exact); for x < 6 * 2^-126 it may differ,
+// but both lie far below 2^-10, so the E4M3 code taken from it is 0 either way.  Checked
+// against __fdiv_rn for every non-negative float32: no E4M3 code differs.
+__device__ __forceinline__ float div6_rn(float x) {
+  const float r = 0.16666667f;  // RN(1/6)
+  const float q = __fmul_rn(x, r);
+  const float e = __fmaf_rn(-q, 6.0f, x);
+  return __fmaf_rn(e, r, q);
+}
+
 // Quantizes one 16-element block to NVFP4 with global encode scale genc (the prologue's
 // float32 steps): returns the 8 code bytes (element 2i in the low nibble of byte i) and the
-// E4M3 scale byte.
-__device__ __forceinline__ uint2 quant_block16(const float (&x)[16], float genc, uint32_t& sc) {
+// E4M3 scale byte.  mult_tab[c] = genc / e4m3_value(c) (0 for c = 0), made once per tile.
+__device__ __forceinline__ uint2 quant_block16(const float (&x)[16], float genc,
+                                               const float* mult_tab, uint32_t& sc) {
   float am = 0.0f;
 #pragma unroll
   for (int e = 0; e < 16; e += 2) am = fmax3(am, fabsf(x[e]), fabsf(x[e + 1]));
-  const float u = __fdiv_rn(__fmul_rn(am, genc), 6.0f);
-  sc = e4m3_code(u);
-  const float sd = e4m3_value(sc);
-  const float mult = sd > 0.0f ? __fdiv_rn(genc, sd) : 0.0f;
+  sc = e4m3_code(div6_rn(__fmul_rn(am, genc)));
+  const float mult = mult_tab[sc];
   const float2 m2 = make_float2(mult, mult);
   float2 y[8];
 #pragma unroll
@@ -182,13 +201,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     sm.abort = device_aborted() ? 1 : 0;
     mbar_init(&sm.kv_full, 1);
-    mbar_init(&sm.st_full, 1);
-    mbar_init(&sm.st_free, 1);
-    mbar_init(&sm.sdp_full, 1);
+    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_free, 1);
+    mbar_init(&sm.do_full, 1);
+    mbar_init(&sm.do_free, 1);
+    mbar_init(&sm.qs_full, 1);
+    mbar_init(&sm.qs_free, 1);
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.dp_full, 1);
     mbar_init(&sm.p_ready, kCompute);
-    mbar_init(&sm.ds_ready, kCompute);
-    mbar_init(&sm.dkdq_full, 1);
-    mbar_init(&sm.tmem_free, kCompute);
+    mbar_init(&sm.dsk_ready, kCompute);
+    mbar_init(&sm.dsq_ready, kCompute);
+    mbar_init(&sm.dq_full, 1);
+    mbar_init(&sm.dk_full, 1);
+    mbar_init(&sm.s_free, kCompute);
+    mbar_init(&sm.dp_free, kCompute);
     mbar_init(&sm.red_full[0], 8);
     mbar_init(&sm.red_full[1], 8);
     mbar_init(&sm.stage_free, 8);
@@ -230,15 +257,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       bulk_load(sm.kssf, args.k_sf_t + (seq_atoms + 2 * t) * 512, 1024, &sm.kv_full);
       for (int it = 0; it < nq; ++it) {
         const int qt = i_first + it;
-        if (it >= 1) mbar_wait(&sm.st_free, (it - 1) & 1, 400);
-        mbar_arrive_expect_tx(&sm.st_full, BQ * D / 2 + kSfBytes + BQ * D * 2 + D * 64 + 1024);
-        tma_load_2d(sm.qc, &tm_qc, 0, row_base + qt * BQ, &sm.st_full);
+        if (it >= 1) mbar_wait(&sm.q_free, (it - 1) & 1, 400);
+        mbar_arrive_expect_tx(&sm.q_full, BQ * D / 2 + kSfBytes);
+        tma_load_2d(sm.qc, &tm_qc, 0, row_base + qt * BQ, &sm.q_full);
         bulk_load(sm.qsf, args.q_sf + (static_cast<size_t>(bh) * nqt + qt) * kSfBytes, kSfBytes,
-                  &sm.st_full);
+                  &sm.q_full);
+        if (it >= 1) mbar_wait(&sm.do_free, (it - 1) & 1, 406);
+        mbar_arrive_expect_tx(&sm.do_full, BQ * D * 2);
         for (int a = 0; a < D / 64; ++a)
-          tma_load_2d(sm.dor + a * BQ * 64, &tm_do, a * 64, row_base + qt * BQ, &sm.st_full);
-        tma_load_2d(sm.qs, &tm_qs, qt * 64, bh * D, &sm.st_full);
-        bulk_load(sm.qssf, args.q_sf_t + (seq_atoms + 2 * qt) * 512, 1024, &sm.st_full);
+          tma_load_2d(sm.dor + a * BQ * 64, &tm_do, a * 64, row_base + qt * BQ, &sm.do_full);
+        if (it >= 1) mbar_wait(&sm.qs_free, (it - 1) & 1, 407);
+        mbar_arrive_expect_tx(&sm.qs_full, D * 64 + 1024);
+        tma_load_2d(sm.qs, &tm_qs, qt * 64, bh * D, &sm.qs_full);
+        bulk_load(sm.qssf, args.q_sf_t + (seq_atoms + 2 * qt) * 512, 1024, &sm.qs_full);
       }
     } else if (warp == kMmaWarp && lane == 0) {
       constexpr uint32_t kFmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
@@ -258,24 +289,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       cp_atoms(sf_k, sm.ksf, D / 64);
       cp_atoms(sf_kseq, sm.kssf, 2);
       for (int it = 0; it < nq; ++it) {
-        mbar_wait(&sm.st_full, it & 1, 402);
-        if (it >= 1) mbar_wait(&sm.tmem_free, (it - 1) & 1, 403);
+        // 1. S = Q K^T (NVFP4) into columns the previous tile's dQ_t has been read out of
+        mbar_wait(&sm.q_full, it & 1, 402);
+        if (it >= 1) mbar_wait(&sm.s_free, (it - 1) & 1, 403);
         tc_fence_after();
-        // 1. S = Q K^T (NVFP4) and dP = dO V^T (16-bit)
         cp_atoms(sf_q, sm.qsf, D / 64);
 #pragma unroll
         for (int kk = 0; kk < D / 64; ++kk)
           mma_nvf4(tmem + kColS, smem_desc(qca + 32 * kk, 16, kSboC, kSwC),
                    smem_desc(kca + 32 * kk, 16, kSboC, kSwC), id_s, sf_q + 4 * kk,
                    sf_k + 4 * kk, kk > 0 ? 1u : 0u);
+        mma_commit(&sm.s_full);
+        mma_commit(&sm.q_free);  // the Q codes and scales have been read
+        // 2. dP = dO V^T (16-bit) into columns the previous tile's dK_t has been read out of
+        mbar_wait(&sm.do_full, it & 1, 408);
+        if (it >= 1) mbar_wait(&sm.dp_free, (it - 1) & 1, 414);
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk * 16 / 64) * (BQ * 128) + (kk * 16 % 64) * 2;
           mma_f16(tmem + kColDP, smem_desc(dora + off, 16, 1024, kSwizzle128B),
                   smem_desc(va + off, 16, 1024, kSwizzle128B), id_dp, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sm.sdp_full);
-        // 2. dV += P^T dO: A = P read MN-major (M = keys), B = dO read MN-major (N = channels)
+        mma_commit(&sm.dp_full);
+        // 3. dV += P^T dO: A = P read MN-major (M = keys), B = dO read MN-major (N = channels)
         mbar_wait(&sm.p_ready, it & 1, 404);
         tc_fence_after();
 #pragma unroll
@@ -283,24 +320,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_f16(tmem + kColDV, smem_desc(pa + kk * 16 * 128, BQ * 128, 1024, kSwizzle128B),
                   smem_desc(dora + kk * 16 * 128, BQ * 128, 1024, kSwizzle128B), id_dv,
                   (it > 0 || kk > 0) ? 1u : 0u);
-        // 5. dQ_t = dS_k K_seq into S's columns, dK_t = dS_q^T Q_seq into dP's
-        mbar_wait(&sm.ds_ready, it & 1, 405);
+        mma_commit(&sm.do_free);  // dP and dV have read dO
+        // 4. dQ_t = dS_k K_seq into S's columns (S has been read: pass A precedes pass B)
+        mbar_wait(&sm.dsk_ready, it & 1, 405);
         tc_fence_after();
         cp_atoms(sf_dsk, sm.dsksf, 2);
-        cp_atoms(sf_dsq, sm.dsqsf, 2);
-        cp_atoms(sf_qseq, sm.qssf, 2);
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk)
           mma_nvf4(tmem + kColS, smem_desc(dska + 32 * kk, 16, 512, kSwizzle64B),
                    smem_desc(ksa + 32 * kk, 16, 512, kSwizzle64B), id_g, sf_dsk + 4 * kk,
                    sf_kseq + 4 * kk, kk > 0 ? 1u : 0u);
+        mma_commit(&sm.dq_full);
+        // 5. dK_t = dS_q^T Q_seq into dP's columns
+        mbar_wait(&sm.qs_full, it & 1, 409);
+        tc_fence_after();
+        cp_atoms(sf_qseq, sm.qssf, 2);
+        mbar_wait(&sm.dsq_ready, it & 1, 415);
+        tc_fence_after();
+        cp_atoms(sf_dsq, sm.dsqsf, 2);
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk)
           mma_nvf4(tmem + kColDP, smem_desc(dsqa + 32 * kk, 16, 512, kSwizzle64B),
                    smem_desc(qsa + 32 * kk, 16, 512, kSwizzle64B), id_g, sf_dsq + 4 * kk,
                    sf_qseq + 4 * kk, kk > 0 ? 1u : 0u);
-        mma_commit(&sm.dkdq_full);
-        mma_commit(&sm.st_free);  // every reader of the query tile's stage has completed
+        mma_commit(&sm.dk_full);
+        mma_commit(&sm.qs_free);  // dK has read the Q sequence view
       }
     }
     __syncwarp();
@@ -326,7 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int it = 0; it < nq; ++it) {
       const int qt = i_first + it;
       const int b = it & 1;
-      const size_t grow = grow_n;
       const float lse2 = lse_n * 1.4426950408889634f;
       const float dvr = dvr_n;
       if (it + 1 < nq) {
@@ -335,25 +378,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         dvr_n = args.dvec[grow_n];
       }
       const bool diag = args.causal && qt == t;
-      mbar_wait(&sm.sdp_full, it & 1, 410);
-      tc_fence_after();
-      // pass A: this row's 64 keys of warpgroup h, 32 columns at a time
+      // pass A (thread = query row r, warpgroup h = keys 64h .. 64h + 63), first P from S (the
+      // dP MMA runs meanwhile), then dS from dP
       float ds[64];
       float dsmax = 0.0f;
       uint8_t* patom = reinterpret_cast<uint8_t*>(sm.p) + h * (BQ * 128);
       const float2 c2 = make_float2(c, c), nlse2 = make_float2(-lse2, -lse2);
       const float2 ndvr2 = make_float2(-dvr, -dvr);
+      mbar_wait(&sm.s_full, it & 1, 410);
+      tc_fence_after();
 #pragma unroll
       for (int c32 = 0; c32 < 2; ++c32) {
         const int col = h * 64 + c32 * 32;
-        uint32_t s0[16], s1[16], q0[16], q1[16];
+        uint32_t s0[16], s1[16];
         tmem_ld32x(lane_base + kColS + col, s0, s1);
-        tmem_ld32x(lane_base + kColDP + col, q0, q1);
-        tmem_ld_wait_regs4(s0, s1, q0, q1);
+        tmem_ld_wait_regs(s0, s1);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           const uint32_t(&sx)[16] = half ? s1 : s0;
-          const uint32_t(&px)[16] = half ? q1 : q0;
           const int cc = col + half * 16;  // first key of these 16 columns
           uint32_t w[8];
 #pragma unroll
@@ -363,13 +405,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             float p0 = ex2_approx(z.x), p1 = ex2_approx(z.y);
             if (diag && cc + e > r) p0 = 0.0f;  // key index - query index = cc + e - r
             if (diag && cc + e + 1 > r) p1 = 0.0f;
-            const float2 d = __fmul2_rn(
-                make_float2(p0, p1),
-                __fadd2_rn(make_float2(__uint_as_float(px[e]), __uint_as_float(px[e + 1])), ndvr2));
             const int j = c32 * 32 + half * 16 + e;
-            ds[j] = d.x;
-            ds[j + 1] = d.y;
-            dsmax = fmax3(dsmax, fabsf(d.x), fabsf(d.y));
+            ds[j] = p0;
+            ds[j + 1] = p1;
             w[e / 2] = Cvt<T>::pack2(p0, p1);
           }
           // keys cc .. cc+15 are 16-byte chunks 2 c16 and 2 c16 + 1 of this row's atom
@@ -383,6 +421,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&sm.p_ready);
+      mbar_wait(&sm.dp_full, it & 1, 416);
+      tc_fence_after();
+#pragma unroll
+      for (int c32 = 0; c32 < 2; ++c32) {
+        uint32_t q0[16], q1[16];
+        tmem_ld32x(lane_base + kColDP + h * 64 + c32 * 32, q0, q1);
+        tmem_ld_wait_regs(q0, q1);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const uint32_t(&px)[16] = e < 16 ? q0 : q1;
+          const int j = c32 * 32 + e;
+          const float2 d = __fmul2_rn(
+              make_float2(ds[j], ds[j + 1]),
+              __fadd2_rn(make_float2(__uint_as_float(px[e & 15]), __uint_as_float(px[(e & 15) + 1])),
+                         ndvr2));
+          ds[j] = d.x;
+          ds[j + 1] = d.y;
+          dsmax = fmax3(dsmax, fabsf(d.x), fabsf(d.y));
+        }
+      }
       // dS transposed into shared memory, once the previous tile's dQ reductions have read
       // the same bytes
       if (it >= 1) {
@@ -405,70 +463,79 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int w8 = 0; w8 < 8; ++w8) tmax = fmaxf(tmax, sm.red[b][w8]);
       const float genc = tmax > 0.0f ? __fdiv_rn(kGlobalRange, tmax) : 1.0f;
-      // pass B, two 32-element halves, each quantizing a pair of blocks in both orientations:
-      // (1) dS in 16-key blocks along this query row -> A of dQ;
-      // (2) dS^T in 16-query blocks along key row k = threadIdx % 128 (queries 64 qh .. +63,
-      //     read back from the transposed tile) -> A of dK
-      const int k = threadIdx.x & 127, qh = threadIdx.x >> 7;
+      if (threadIdx.x < 128) {
+        const uint32_t code = threadIdx.x;
+        sm.mult[code] = code == 0 ? 0.0f : __fdiv_rn(genc, e4m3_value(code));
+      }
+      named_barrier_sync(2, kCompute);
+      // pass B (1): dS in 16-key blocks along this query row -> A of dQ (the dQ MMA then runs
+      // during pass B (2))
 #pragma unroll
       for (int pb = 0; pb < 4; pb += 2) {
-        uint32_t s0, s1, s2, s3;
-        float xa[16], xb[16], ya[16], yb[16];
+        uint32_t s0, s1;
+        float xa[16], xb[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           xa[e] = ds[pb * 16 + e];
           xb[e] = ds[pb * 16 + 16 + e];
         }
-        const float4* row = reinterpret_cast<const float4*>(&sm.dst[k][qh * 64 + pb * 16]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float4 fa = row[e], fb = row[4 + e];
-          ya[4 * e] = fa.x;
-          ya[4 * e + 1] = fa.y;
-          ya[4 * e + 2] = fa.z;
-          ya[4 * e + 3] = fa.w;
-          yb[4 * e] = fb.x;
-          yb[4 * e + 1] = fb.y;
-          yb[4 * e + 2] = fb.z;
-          yb[4 * e + 3] = fb.w;
-        }
-        const uint2 ca = quant_block16(xa, genc, s0);
-        const uint2 cb = quant_block16(xb, genc, s1);
-        const uint2 da = quant_block16(ya, genc, s2);
-        const uint2 db = quant_block16(yb, genc, s3);
+        const uint2 ca = quant_block16(xa, genc, sm.mult, s0);
+        const uint2 cb = quant_block16(xb, genc, sm.mult, s1);
         *reinterpret_cast<uint4*>(sm.dsk + swz_offset(r, 2 * h + pb / 2, 64)) =
             make_uint4(ca.x, ca.y, cb.x, cb.y);
         sm.dsksf[h * 512 + (r & 31) * 16 + (r >> 5) * 4 + pb] = static_cast<uint8_t>(s0);
         sm.dsksf[h * 512 + (r & 31) * 16 + (r >> 5) * 4 + pb + 1] = static_cast<uint8_t>(s1);
-        *reinterpret_cast<uint4*>(sm.dsq + swz_offset(k, 2 * qh + pb / 2, 64)) =
-            make_uint4(da.x, da.y, db.x, db.y);
-        sm.dsqsf[qh * 512 + (k & 31) * 16 + (k >> 5) * 4 + pb] = static_cast<uint8_t>(s2);
-        sm.dsqsf[qh * 512 + (k & 31) * 16 + (k >> 5) * 4 + pb + 1] = static_cast<uint8_t>(s3);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&sm.ds_ready);
-      // 5. read-outs: dQ_t (lane = query row) to the global accumulator, dK_t (lane = key row)
-      // into registers; thread (h) takes channels h*D/2 ..
+      mbar_arrive(&sm.dsk_ready);
+      // pass B (2): dS^T in 16-query blocks along key row k = threadIdx % 128 (queries
+      // 64 qh .. 64 qh + 63, read back from the transposed tile) -> A of dK
+      {
+        const int k = threadIdx.x & 127, qh = threadIdx.x >> 7;
+#pragma unroll
+        for (int pb = 0; pb < 4; pb += 2) {
+          uint32_t s0, s1;
+          float ya[16], yb[16];
+          const float4* row = reinterpret_cast<const float4*>(&sm.dst[k][qh * 64 + pb * 16]);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float4 fa = row[e], fb = row[4 + e];
+            ya[4 * e] = fa.x;
+            ya[4 * e + 1] = fa.y;
+            ya[4 * e + 2] = fa.z;
+            ya[4 * e + 3] = fa.w;
+            yb[4 * e] = fb.x;
+            yb[4 * e + 1] = fb.y;
+            yb[4 * e + 2] = fb.z;
+            yb[4 * e + 3] = fb.w;
+          }
+          const uint2 da = quant_block16(ya, genc, sm.mult, s0);
+          const uint2 db = quant_block16(yb, genc, sm.mult, s1);
+          *reinterpret_cast<uint4*>(sm.dsq + swz_offset(k, 2 * qh + pb / 2, 64)) =
+              make_uint4(da.x, da.y, db.x, db.y);
+          sm.dsqsf[qh * 512 + (k & 31) * 16 + (k >> 5) * 4 + pb] = static_cast<uint8_t>(s0);
+          sm.dsqsf[qh * 512 + (k & 31) * 16 + (k >> 5) * 4 + pb + 1] = static_cast<uint8_t>(s1);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&sm.dsq_ready);
+      // read-outs.  dQ_t (lane = query row): scaled into this warp's staging boxes; the S / dQ_t
+      // columns are then released (the next tile's S MMA starts) and one lane hands the boxes
+      // to the TMA unit, which adds them into the float32 dQ accumulator
       const float sq = __fdiv_rn(args.tau, __fmul_rn(genc, kg));
       const float sk = __fdiv_rn(args.tau, __fmul_rn(genc, qg));
-      mbar_wait(&sm.dkdq_full, it & 1, 412);
-      tc_fence_after();
-      // dQ_t scaled into this warp's staging boxes and dK_t into the accumulators; then the TMEM
-      // columns are released (the next tile's S / dP MMAs start) and one lane hands the boxes
-      // to the TMA unit, which adds them into the float32 dQ accumulator
       uint8_t* stage = reinterpret_cast<uint8_t*>(&sm.dst[0][0]) + warp * (D / 64) * 4096;
+      // the staging boxes overlay the transposed tile: every thread's pass B (2) has read it
+      mbar_wait(&sm.dsq_ready, it & 1, 418);
+      mbar_wait(&sm.dq_full, it & 1, 412);
+      tc_fence_after();
 #pragma unroll
       for (int c0 = 0; c0 < DH; c0 += 32) {
-        uint32_t a0[16], a1[16], k0[16], k1[16];
+        uint32_t a0[16], a1[16];
         tmem_ld32x(lane_base + kColS + h * DH + c0, a0, a1);
-        tmem_ld32x(lane_base + kColDP + h * DH + c0, k0, k1);
-        tmem_ld_wait_regs4(a0, a1, k0, k1);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          acck[c0 + e] = fmaf(__uint_as_float(k0[e]), sk, acck[c0 + e]);
-          acck[c0 + 16 + e] = fmaf(__uint_as_float(k1[e]), sk, acck[c0 + 16 + e]);
-        }
+        tmem_ld_wait_regs(a0, a1);
         uint8_t* box = stage + (c0 / 32) * 4096;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
@@ -480,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&sm.tmem_free);
+      mbar_arrive(&sm.s_free);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
@@ -490,6 +557,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                             row_base + qt * BQ + quarter * 32);
         bulk_commit();
       }
+      // dK_t (lane = key row) into the accumulators; then the dP / dK_t columns are released
+      mbar_wait(&sm.dk_full, it & 1, 417);
+      tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < DH; c0 += 32) {
+        uint32_t k0[16], k1[16];
+        tmem_ld32x(lane_base + kColDP + h * DH + c0, k0, k1);
+        tmem_ld_wait_regs(k0, k1);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          acck[c0 + e] = fmaf(__uint_as_float(k0[e]), sk, acck[c0 + e]);
+          acck[c0 + 16 + e] = fmaf(__uint_as_float(k1[e]), sk, acck[c0 + 16 + e]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.dp_free);
     }
     if (lane == 0) bulk_wait_all();  // this warp's dQ reductions have completed
     // epilogue: dV from TMEM, dK from the registers (thread = key row r, channels h*D/2 ..);
