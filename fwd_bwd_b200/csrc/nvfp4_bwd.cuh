@@ -402,7 +402,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 16; e += 2) {
             const float2 z = __ffma2_rn(make_float2(__uint_as_float(sx[e]), __uint_as_float(sx[e + 1])),
                                         c2, nlse2);
-            float p0 = ex2_approx(z.x), p1 = ex2_approx(z.y);
+            // one pair in four on the FMA pipe (exp2_poly2), the rest on the MUFU unit
+            float p0, p1;
+            if ((e & 6) == 6) {
+              const float2 p = exp2_poly2(z);
+              p0 = p.x;
+              p1 = p.y;
+            } else {
+              p0 = ex2_approx(z.x);
+              p1 = ex2_approx(z.y);
+            }
             if (diag && cc + e > r) p0 = 0.0f;  // key index - query index = cc + e - r
             if (diag && cc + e + 1 > r) p1 = 0.0f;
             const int j = c32 * 32 + half * 16 + e;

@@ -527,4 +527,32 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^z for a pair, on the FMA pipe instead of the special-function unit (the kernels route a
+// share of their exponentials here so that both units work).  z = j + f with j = rint(z) (the
+// 1.5 * 2^23 rounding trick) and f in [-1/2, 1/2] exact; p(f) ~ 2^f is the degree-5 polynomial
+// of minimax relative error (Remez exchange, coefficients from fwd_bwd_b200/exp2_fit.py),
+// evaluated by packed FMAs; j is added to the exponent field.  Maximum relative error
+// 2.2e-7 (float32 evaluation included).  z < -125 gives 0, as the flushing ex2.approx does
+// below -126; z must stay below 128.
+__device__ __forceinline__ float2 exp2_poly2(float2 z) {
+  constexpr float kC0 = 1.0000001192092896f, kC1 = 0.6931469440460205f,
+                  kC2 = 0.24022120237350464f, kC3 = 0.05550713092088699f,
+                  kC4 = 0.009675540961325169f, kC5 = 0.0013276472454890609f;
+  const float2 lo = make_float2(-125.0f, -125.0f);
+  const float2 zc = make_float2(fmaxf(z.x, lo.x), fmaxf(z.y, lo.y));
+  const float2 t = __fadd2_rn(zc, make_float2(kMagic, kMagic));       // rint(z) + 1.5 * 2^23
+  const float2 j = __fadd2_rn(t, make_float2(-kMagic, -kMagic));      // rint(z), exact
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), zc);      // z - rint(z), exact
+  float2 q = __ffma2_rn(make_float2(kC5, kC5), f, make_float2(kC4, kC4));
+  q = __ffma2_rn(q, f, make_float2(kC3, kC3));
+  q = __ffma2_rn(q, f, make_float2(kC2, kC2));
+  q = __ffma2_rn(q, f, make_float2(kC1, kC1));
+  q = __ffma2_rn(q, f, make_float2(kC0, kC0));
+  const int jx = static_cast<int>(__float_as_uint(t.x) - kMagicBits);
+  const int jy = static_cast<int>(__float_as_uint(t.y) - kMagicBits);
+  const float rx = __int_as_float(__float_as_int(q.x) + (jx << 23));
+  const float ry = __int_as_float(__float_as_int(q.y) + (jy << 23));
+  return make_float2(z.x < lo.x ? 0.0f : rx, z.y < lo.y ? 0.0f : ry);
+}
+
 }  // namespace sage
