@@ -119,3 +119,47 @@ def test_nvfp4_fwd_bwd_chain(name):
               f"cos chain {c_chain:.5f} oracle {c_ref:.5f}")
         assert d_chain <= CHAIN_FRAC * d_quant, (n, d_chain, d_quant)
         assert c_chain >= c_ref - COS_SLACK, (n, c_chain, c_ref)
+
+
+FULL_HEADS = [0, 511]  # flattened b*H+h of B32 H16 N8192 d128 (the bench workload)
+
+
+def test_nvfp4_backward_full_size_sampled_heads():
+    """The whole batch in the launch configuration bench.py --variant nvfp4 times (512 heads);
+    the sampled heads carry the seeded per-head inputs and, as in the isolated test, the
+    oracle's O (stored) and LSE, and are checked one head at a time (heads are independent)."""
+    w = WORKLOADS["sweep8192"]
+    dev = torch.device("cuda")
+    dt = TORCH_DT[w.dtype]
+    g = torch.Generator(device=dev).manual_seed(3)
+    shape = (w.B * w.H, w.N, w.d)
+    sig = {"q": w.sigma_qkv, "k": w.sigma_qkv, "v": w.sigma_qkv, "do": w.sigma_do}
+    t = {n: (torch.randn(shape, generator=g, device=dev) * s).to(dt) for n, s in sig.items()}
+    x = make_inputs(w, heads=FULL_HEADS)
+    for n in t:
+        for i, bh in enumerate(FULL_HEADS):
+            t[n][bh] = torch.from_numpy(x[n][i].view(np.int16)).view(dt).to(dev)
+    q, k, v, do = (t[n].view(w.B, w.H, w.N, w.d) for n in ("q", "k", "v", "do"))
+    cfg = _cfg(w)
+    fb = nvfp4.quant_prologue(q, k, cfg, seq=True)
+    o, lse = nvfp4.attn_fwd(fb, v, cfg)
+    refs = []
+    for i, bh in enumerate(FULL_HEADS):
+        one = [x[n + "_f32"][i:i + 1] for n in ("q", "k", "v", "do")]
+        ref = F.qattn_attention(*one, causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth,
+                                dtype=w.dtype)
+        b_, h_ = divmod(bh, w.H)
+        o[b_, h_] = torch.from_numpy(ref["o"][0].astype(np.float32)).to(dt).to(dev)
+        lse[b_, h_] = torch.from_numpy(ref["lse"][0].astype(np.float32)).to(dev)
+        refs.append(ref)
+    dq, dk, dv = nvfp4.attn_bwd(q, k, v, fb, o, lse, do, cfg)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    for i, bh in enumerate(FULL_HEADS):
+        b_, h_ = divmod(bh, w.H)
+        for n, tg in (("dq", dq), ("dk", dk), ("dv", dv)):
+            got = tg[b_, h_].float().cpu().numpy().astype(np.float64)
+            err = rel_l2(got, refs[i][n][0])
+            print(f"head {bh} {n}: rel_l2 {err:.3e}")
+            tol = TOL_DV[w.dtype] if n == "dv" else TOL_DQK
+            assert np.isfinite(got).all() and err <= tol, (bh, n, err)
