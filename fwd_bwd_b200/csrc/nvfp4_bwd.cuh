@@ -154,21 +154,33 @@ __device__ __forceinline__ float div6_rn(float x) {
   return __fmaf_rn(e, r, q);
 }
 
-// Quantizes one 16-element block to NVFP4 with global encode scale genc (the prologue's
-// float32 steps): returns the 8 code bytes (element 2i in the low nibble of byte i) and the
-// E4M3 scale byte.  mult_tab[c] = genc / e4m3_value(c) (0 for c = 0), made once per tile.
-__device__ __forceinline__ uint2 quant_block16(const float (&x)[16], float genc,
-                                               const float* mult_tab, uint32_t& sc) {
-  float am = 0.0f;
+// Four consecutive 16-element blocks of x quantized to NVFP4 with the global encode scale genc
+// (the prologue's float32 steps: u = (max|x| genc) / 6, sd = e4m3(u), code = e2m1(x genc / sd)),
+// in four independent chains (the scale codes first, then the multipliers, then the codes).
+// mult_tab[c] = genc / e4m3_value(c) (0 for c = 0), made once per tile.  codes[b] holds block
+// b's 8 code bytes (element 2i in the low nibble of byte i); the return value holds the four
+// E4M3 scale bytes (block b in byte b).
+__device__ __forceinline__ uint32_t quant_blocks4(const float (&x)[64], float genc,
+                                                  const float* mult_tab, uint2 (&codes)[4]) {
+  uint32_t sc[4];
 #pragma unroll
-  for (int e = 0; e < 16; e += 2) am = fmax3(am, fabsf(x[e]), fabsf(x[e + 1]));
-  sc = e4m3_code(div6_rn(__fmul_rn(am, genc)));
-  const float mult = mult_tab[sc];
-  const float2 m2 = make_float2(mult, mult);
-  float2 y[8];
+  for (int b = 0; b < 4; ++b) {
+    float am = 0.0f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) y[e] = __fmul2_rn(make_float2(x[2 * e], x[2 * e + 1]), m2);
-  return make_uint2(e2m1x8(y[0], y[1], y[2], y[3]), e2m1x8(y[4], y[5], y[6], y[7]));
+    for (int e = 0; e < 16; e += 2) am = fmax3(am, fabsf(x[16 * b + e]), fabsf(x[16 * b + e + 1]));
+    sc[b] = e4m3_code(div6_rn(__fmul_rn(am, genc)));
+  }
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const float mult = mult_tab[sc[b]];
+    const float2 m2 = make_float2(mult, mult);
+    float2 y[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      y[e] = __fmul2_rn(make_float2(x[16 * b + 2 * e], x[16 * b + 2 * e + 1]), m2);
+    codes[b] = make_uint2(e2m1x8(y[0], y[1], y[2], y[3]), e2m1x8(y[4], y[5], y[6], y[7]));
+  }
+  return sc[0] | (sc[1] << 8) | (sc[2] << 16) | (sc[3] << 24);
 }
 
 template <typename T, int D>
@@ -478,22 +490,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       named_barrier_sync(2, kCompute);
       // pass B (1): dS in 16-key blocks along this query row -> A of dQ (the dQ MMA then runs
-      // during pass B (2))
-#pragma unroll
-      for (int pb = 0; pb < 4; pb += 2) {
-        uint32_t s0, s1;
-        float xa[16], xb[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          xa[e] = ds[pb * 16 + e];
-          xb[e] = ds[pb * 16 + 16 + e];
-        }
-        const uint2 ca = quant_block16(xa, genc, sm.mult, s0);
-        const uint2 cb = quant_block16(xb, genc, sm.mult, s1);
-        *reinterpret_cast<uint4*>(sm.dsk + swz_offset(r, 2 * h + pb / 2, 64)) =
-            make_uint4(ca.x, ca.y, cb.x, cb.y);
-        sm.dsksf[h * 512 + (r & 31) * 16 + (r >> 5) * 4 + pb] = static_cast<uint8_t>(s0);
-        sm.dsksf[h * 512 + (r & 31) * 16 + (r >> 5) * 4 + pb + 1] = static_cast<uint8_t>(s1);
+      // during pass B (2)); the row's four scales of this key half are one 32-bit word
+      {
+        uint2 cd[4];
+        const uint32_t scw = quant_blocks4(ds, genc, sm.mult, cd);
+        *reinterpret_cast<uint4*>(sm.dsk + swz_offset(r, 2 * h, 64)) =
+            make_uint4(cd[0].x, cd[0].y, cd[1].x, cd[1].y);
+        *reinterpret_cast<uint4*>(sm.dsk + swz_offset(r, 2 * h + 1, 64)) =
+            make_uint4(cd[2].x, cd[2].y, cd[3].x, cd[3].y);
+        *reinterpret_cast<uint32_t*>(sm.dsksf + h * 512 + (r & 31) * 16 + (r >> 5) * 4) = scw;
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -502,30 +507,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // 64 qh .. 64 qh + 63, read back from the transposed tile) -> A of dK
       {
         const int k = threadIdx.x & 127, qh = threadIdx.x >> 7;
+        float y[64];
+        const float4* row = reinterpret_cast<const float4*>(&sm.dst[k][qh * 64]);
 #pragma unroll
-        for (int pb = 0; pb < 4; pb += 2) {
-          uint32_t s0, s1;
-          float ya[16], yb[16];
-          const float4* row = reinterpret_cast<const float4*>(&sm.dst[k][qh * 64 + pb * 16]);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float4 fa = row[e], fb = row[4 + e];
-            ya[4 * e] = fa.x;
-            ya[4 * e + 1] = fa.y;
-            ya[4 * e + 2] = fa.z;
-            ya[4 * e + 3] = fa.w;
-            yb[4 * e] = fb.x;
-            yb[4 * e + 1] = fb.y;
-            yb[4 * e + 2] = fb.z;
-            yb[4 * e + 3] = fb.w;
-          }
-          const uint2 da = quant_block16(ya, genc, sm.mult, s0);
-          const uint2 db = quant_block16(yb, genc, sm.mult, s1);
-          *reinterpret_cast<uint4*>(sm.dsq + swz_offset(k, 2 * qh + pb / 2, 64)) =
-              make_uint4(da.x, da.y, db.x, db.y);
-          sm.dsqsf[qh * 512 + (k & 31) * 16 + (k >> 5) * 4 + pb] = static_cast<uint8_t>(s0);
-          sm.dsqsf[qh * 512 + (k & 31) * 16 + (k >> 5) * 4 + pb + 1] = static_cast<uint8_t>(s1);
+        for (int e = 0; e < 16; ++e) {
+          const float4 f4 = row[e];
+          y[4 * e] = f4.x;
+          y[4 * e + 1] = f4.y;
+          y[4 * e + 2] = f4.z;
+          y[4 * e + 3] = f4.w;
         }
+        uint2 cd[4];
+        const uint32_t scw = quant_blocks4(y, genc, sm.mult, cd);
+        *reinterpret_cast<uint4*>(sm.dsq + swz_offset(k, 2 * qh, 64)) =
+            make_uint4(cd[0].x, cd[0].y, cd[1].x, cd[1].y);
+        *reinterpret_cast<uint4*>(sm.dsq + swz_offset(k, 2 * qh + 1, 64)) =
+            make_uint4(cd[2].x, cd[2].y, cd[3].x, cd[3].y);
+        *reinterpret_cast<uint32_t*>(sm.dsqsf + qh * 512 + (k & 31) * 16 + (k >> 5) * 4) = scw;
       }
       fence_proxy_async_smem();
       tc_fence_before();
