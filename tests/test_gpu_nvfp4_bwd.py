@@ -163,3 +163,45 @@ def test_nvfp4_backward_full_size_sampled_heads():
             print(f"head {bh} {n}: rel_l2 {err:.3e}")
             tol = TOL_DV[w.dtype] if n == "dv" else TOL_DQK
             assert np.isfinite(got).all() and err <= tol, (bh, n, err)
+
+
+def _degenerate(kind, BH=2, N=256, d=128):
+    rng = np.random.default_rng(17)
+    q, k, v, do = (rng.standard_normal((BH, N, d)).astype(np.float32) for _ in range(4))
+    if kind == "zero_do_head":     # dS = 0 on head 0: every tile's maximum is 0 (genc = 1)
+        do[0] = 0.0
+    elif kind == "tiny_do":        # dS ~ 2^-100: tiny (still normal) tile maxima and genc ~ 2^100
+        do *= np.float32(2.0 ** -100)
+    elif kind == "zero_qk_head":   # S = 0 on head 0: uniform attention, G = 0 for Q and K
+        q[0] = 0.0
+        k[0] = 0.0
+    return q, k, v, do
+
+
+@pytest.mark.parametrize("kind", ["zero_do_head", "tiny_do", "zero_qk_head"])
+def test_nvfp4_backward_degenerate(kind):
+    q, k, v, do = _degenerate(kind)
+    BH, N, d = q.shape
+    dt = torch.bfloat16
+    tq, tk, tv, tdo = (torch.from_numpy(a).to(dt) for a in (q, k, v, do))
+    qf, kf, vf, dof = (t.float().numpy() for t in (tq, tk, tv, tdo))  # exact bf16 values
+    ref = F.qattn_attention(qf, kf, vf, dof, causal=True, qknorm=False, ksmooth=True,
+                            dtype="bf16")
+    cfg = ops.Config(causal=True, qknorm=False, ksmooth=True)
+    dev = torch.device("cuda")
+    shape = (1, BH, N, d)
+    q_, k_, v_ = (t.reshape(shape).to(dev) for t in (tq, tk, tv))
+    fb = nvfp4.quant_prologue(q_, k_, cfg, seq=True)
+    o = torch.from_numpy(ref["o"].astype(np.float32).reshape(shape)).to(dt).to(dev)
+    lse = torch.from_numpy(ref["lse"].astype(np.float32).reshape(shape[:3])).to(dev)
+    dq_, dk_, dv_ = nvfp4.attn_bwd(q_, k_, v_, fb, o, lse, tdo.reshape(shape).to(dev), cfg)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    for n, t in (("dq", dq_), ("dk", dk_), ("dv", dv_)):
+        got = t.float().cpu().numpy().astype(np.float64).reshape(BH, N, d)
+        assert np.isfinite(got).all(), n
+        if kind == "zero_do_head":
+            assert (got[0] == 0).all(), n  # no gradient flows from a zero output gradient
+        err = rel_l2(got, ref[n])
+        print(f"{kind} {n}: rel_l2 {err:.3e}")
+        assert err <= (TOL_DV["bf16"] if n == "dv" else TOL_DQK), (n, err)
