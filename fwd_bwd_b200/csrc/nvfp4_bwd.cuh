@@ -3,25 +3,29 @@
 // quantized views of Q and K made by the prologue are reused).
 //
 // Per CTA: one tile of 128 keys of one (batch, head), walking the tiles of 128 queries that can
-// see it.  Per query tile:
+// see it (from the diagonal on when causal).  Per query tile:
 //   1. S = Q K^T (kind::mxf4nvf4 from the forward's NVFP4 views: Q / K codes and block scales)
-//      and dP = dO V^T (kind::f16 on the raw 16-bit dO and V) into TMEM;
-//   2. pass A (thread = query row, warpgroup h = keys 64h .. 64h+63): P = exp2(S c - LSE log2 e),
-//      dS = P (dP - D); P in the 16-bit type of dO / V goes to shared memory as the A operand of
-//      dV += P^T dO (kind::f16, accumulated in TMEM over every query tile); dS stays in
-//      registers and is also written, transposed, to a float32 shared-memory tile;
+//      and dP = dO V^T (kind::f16 on the raw 16-bit dO and V) into TMEM, committed separately;
+//   2. pass A (thread = query row, warpgroup h = keys 64h .. 64h+63): as soon as S lands,
+//      P = exp2(S c - LSE log2 e) in the 16-bit type of dO / V into shared memory (the A operand
+//      of dV += P^T dO, kind::f16, accumulated in TMEM over every query tile); once dP lands,
+//      dS = P (dP - D) in registers, also written transposed to a float32 shared-memory tile;
 //   3. the tile's absolute maximum of dS (every warp's maximum through shared memory) gives the
-//      tile's global encode scale genc = 2688 / max;
+//      tile's global encode scale genc = 2688 / max, and a table of genc / e4m3(c) per scale
+//      code c;
 //   4. pass B: dS quantized twice with that global scale -- per query row in 16-key blocks
-//      (the A operand of dQ = dS K) and, from the transposed tile, per key row in 16-query
-//      blocks (the A operand of dK = dS^T Q): E2M1 codes in 64-byte swizzled rows and E4M3
-//      block scales in the tensor core's scale-factor order;
-//   5. dQ_t = dS_k K_seq and dK_t = dS_q^T Q_seq (kind::mxf4nvf4; K_seq / Q_seq are the
-//      prologue's sequence views, 16-token blocks) into TMEM; dQ_t * tau / (genc genc_K) is
-//      staged in shared memory and added to the float32 dQ accumulator in global memory by
-//      TMA reductions (asynchronous: the next tile's work overlaps them), dK_t * tau /
-//      (genc genc_Q) to float32 registers.
+//      (the A operand of dQ_t = dS_k K_seq; its MMA starts while the second quantization runs)
+//      and, from the transposed tile, per key row in 16-query blocks (the A operand of
+//      dK_t = dS_q^T Q_seq): E2M1 codes in 64-byte swizzled rows and E4M3 block scales in the
+//      tensor core's scale-factor order.  K_seq / Q_seq are the prologue's sequence views
+//      (16-token blocks), multiplied by kind::mxf4nvf4;
+//   5. read-outs: dQ_t * tau / (genc genc_K) is staged in shared memory (over the transposed
+//      tile) and added to the float32 dQ accumulator in global memory by TMA reductions, which
+//      run while the next tile starts; dK_t * tau / (genc genc_Q) goes to float32 registers.
+//      The S / dQ_t and the dP / dK_t columns are released separately.
 // After the last tile: dV from TMEM, dK (with the RMSNorm backward when qknorm) to global memory.
+// The query tile's operands (Q codes and scales, dO, the Q sequence view) each have their own
+// full / free barrier pair, so each is reloaded as soon as its last reader is done.
 //
 // Warps 0-7 compute, warp 8 is the TMA producer, warp 9 the MMA issuer, warps 10-11 idle (they
 // complete the producer warpgroup, which gives registers to the compute warpgroups).
@@ -118,7 +122,6 @@ struct Args {
   const float* dvec;      // [BH, N]
   const void* k_raw;      // [BH, N, D] (RMSNorm backward of dk)
   const float* k_inv_rms; // [BH, N]
-  float* dq_acc;          // [BH, N, D] float32 (the kernel adds into it through tm_dq)
   void* dk;
   void* dv;
   int N, causal, qknorm;

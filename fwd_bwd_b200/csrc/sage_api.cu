@@ -495,7 +495,6 @@ int run_fp4_bwd(int stage, const sage_params* p, const void* q, const void* k, c
   a.dvec = dvec;
   a.k_raw = k;
   a.k_inv_rms = fb->k_inv_rms;
-  a.dq_acc = dqacc;
   a.dk = dk;
   a.dv = dv;
   a.N = N;
