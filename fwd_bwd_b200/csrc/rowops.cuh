@@ -107,11 +107,38 @@ __device__ __forceinline__ float quant_magic(float x, float s) {
   return s > 0.0f ? __fadd_rn(__fdiv_rn(x, s), kMagic) : kMagic;
 }
 
-__device__ __forceinline__ uint2 quant8(const float (&x)[8], float s) {
+// The same code without a division per element: q = x * r with r = RN(1/s) is within
+// 1.5 * 2^-16 of RN(x / s) for every element of the block (|x / s| < 128: both carry a relative
+// error below 2^-23 and 2^-24), so rint(q) = rint(RN(x / s)) unless a half-integer lies within
+// that distance of q -- then |q - rint(q)| >= 0.5 - 2^-15 and the IEEE quotient decides (ties
+// included).  r_ok is false when r is not finite (s below 2^-128): every element takes the IEEE
+// quotient.  Returns kMagic + code, as quant_magic.
+__device__ __forceinline__ float quant_magic_r(float x, float s, float r, bool r_ok) {
+  const float q = __fmul_rn(x, r);
+  const float t = __fadd_rn(q, kMagic);                  // kMagic + rint(q)
+  const float f = __fsub_rn(q, __fsub_rn(t, kMagic));    // q - rint(q), exact
+  if (!r_ok || fabsf(f) >= 0.5f - 0x1p-15f) return quant_magic(x, s);
+  return t;
+}
+
+// Eight codes by the IEEE quotient (the backward preprocess's dO codes: there the division-free
+// path measured slower).
+__device__ __forceinline__ uint2 quant8_div(const float (&x)[8], float s) {
   return make_uint2(pack_magic4(quant_magic(x[0], s), quant_magic(x[1], s),
                                 quant_magic(x[2], s), quant_magic(x[3], s)),
                     pack_magic4(quant_magic(x[4], s), quant_magic(x[5], s),
                                 quant_magic(x[6], s), quant_magic(x[7], s)));
+}
+
+// Eight codes by the division-free path (the prologue's Q, K and V codes).
+__device__ __forceinline__ uint2 quant8(const float (&x)[8], float s) {
+  if (!(s > 0.0f)) return make_uint2(0u, 0u);  // all-zero block: codes 0
+  const float r = __frcp_rn(s);
+  const bool r_ok = r < INFINITY;
+  return make_uint2(pack_magic4(quant_magic_r(x[0], s, r, r_ok), quant_magic_r(x[1], s, r, r_ok),
+                                quant_magic_r(x[2], s, r, r_ok), quant_magic_r(x[3], s, r, r_ok)),
+                    pack_magic4(quant_magic_r(x[4], s, r, r_ok), quant_magic_r(x[5], s, r, r_ok),
+                                quant_magic_r(x[6], s, r, r_ok), quant_magic_r(x[7], s, r, r_ok)));
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -381,7 +408,7 @@ __global__ void __launch_bounds__(kQuantThreads, 2) bwd_preprocess_kernel(
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
     const int r = warp * RPW + s * GPW + grp;
-    *reinterpret_cast<uint2*>(do_codes + (row0 + r) * D + sub * 8) = quant8(x[s], sc);
+    *reinterpret_cast<uint2*>(do_codes + (row0 + r) * D + sub * 8) = quant8_div(x[s], sc);
   }
 }
 

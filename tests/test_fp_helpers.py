@@ -65,3 +65,60 @@ def test_div6_correction_step_is_needed():
     e_bad = _rn32(x.astype(F64) - 5.0 * q.astype(F64))
     bad = _rn32(q.astype(F64) + e_bad.astype(F64) * F64(r))
     assert not np.array_equal(bad.view(np.uint32), want.view(np.uint32))
+
+
+def _quant_fast(x, s):
+    """The INT8 prologue quantizer's division-free path (rowops.cuh quant_magic_r), in float32
+    numpy operations (each IEEE-rounded, as the kernel's): rint(x * RN(1/s)) unless that product
+    lies within 2^-15 of a half-integer, where the correctly rounded quotient decides."""
+    x = np.asarray(x, F32)
+    s = F32(s)
+    r = F32(1.0) / s
+    q = x * r
+    magic = F32(12582912.0)
+    t = q + magic
+    f = q - (t - magic)
+    amb = ~np.isfinite(r) | (np.abs(f) >= F32(0.5) - F32(2.0 ** -15))
+    exact = np.rint(x / s)
+    return np.where(amb, exact, (t - magic)), amb
+
+
+def _blocks(rng, n):
+    """Blocks of 8 values with their scale s = RN(absmax / 127), including values planted on
+    (and one ulp either side of) half-integer multiples of s, and tiny / huge magnitudes."""
+    out = []
+    for i in range(n):
+        mag = F32(2.0) ** F32(rng.integers(-120, 120))
+        x = (rng.standard_normal(8) * mag).astype(F32)
+        am = np.abs(x).max()
+        s = F32(am) / F32(127.0)
+        if i % 3 == 0:  # plant half-integer quotients
+            k = rng.integers(-126, 126, 4).astype(F32) + F32(0.5)
+            p = (k * s).astype(F32)
+            p = np.clip(p, -am, am)
+            x[:4] = p
+            x[4] = np.nextafter(p[0], F32(np.inf))
+            x[5] = np.nextafter(p[1], F32(-np.inf))
+        out.append((x, s))
+    return out
+
+
+def test_int8_quantizer_fast_path_is_exact():
+    rng = np.random.default_rng(7)
+    n_amb = 0
+    for x, s in _blocks(rng, 20000):
+        got, amb = _quant_fast(x, s)
+        want = np.rint(x / s)  # the IEEE quotient, rounded half to even
+        assert np.array_equal(got, want), (x, s)
+        n_amb += int(amb.sum())
+    assert n_amb > 0  # the planted half-integers reach the exact path
+
+
+def test_int8_quantizer_bound_is_needed():
+    """Without the fallback (rint of x * RN(1/s) alone) some planted ties round differently."""
+    rng = np.random.default_rng(8)
+    bad = 0
+    for x, s in _blocks(rng, 20000):
+        r = F32(1.0) / s
+        bad += int((np.rint(x * r) != np.rint(x / s)).sum())
+    assert bad > 0
