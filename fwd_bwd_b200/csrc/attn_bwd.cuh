@@ -85,9 +85,10 @@ struct Smem {
   uint8_t v[BKT * D * 2];  // raw 16-bit V, [D/64 atoms][128 rows][128 B]
   int8_t pc[BQ * BKT];     // P codes  [128 q][128 keys], 128-byte swizzle
   int8_t dsc[BQ * BKT];    // dS codes [128 q][128 keys], 128-byte swizzle
-  // d = 128: dQ staging for the asynchronous bulk reduction,
-  // [compute warp][buffer][query row][channel of the warp]
-  float dqs[D == 128 ? 8 : 1][2][D == 128 ? kDqRows * kDqCols : 4];
+  // dQ staging for the asynchronous bulk reduction, per compute warp 4 KB:
+  // d = 128: [buffer][query row][channel of the warp], 2 x 16 x 32 floats;
+  // d = 64: one box of 32 query rows x 32 channels (128-byte swizzle)
+  float dqs[8][2][kDqRows * kDqCols];
   alignas(256) uint8_t fill[kFillBytes];  // operands of the preload MMA (mma_fill_magic)
   alignas(16) float red_p[2][8];  // per-warp tile maxima of P, [tile parity][warp]
   alignas(16) float red_ds[2][8];  // and of |dS|
@@ -130,7 +131,6 @@ struct Args {
   const float* dvec;      // [BH, N]
   const void* k_raw;      // [BH, N, D] (RMSNorm backward of dk)
   const float* k_inv_rms; // [BH, N]
-  float* dq_acc;          // [BH, N, D] float32
   void* dk;
   void* dv;
   int BH, N, q_block, causal, qknorm;
@@ -487,7 +487,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = it & 1;
       const uint32_t lane_base = tmem + lane_off + b * 256;
       const int qt = i_first + it;
-      const size_t grow = static_cast<size_t>(row_base) + qt * BQ + r;
       if (it + 1 < nq) row_inputs(it + 1, c_n, lse2_n, dvr_n);  // loads in flight during pass B
       // pass B: INT8 codes into shared memory.  The TMEM loads of chunk ch+1 are in flight while
       // chunk ch is converted (two keys per FMA).
@@ -674,14 +673,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (rr + 1 < 64 / kDqRows) tmem_ld_wait_regs(a0, a1);
         }
       } else {
-        // thread = query row r, d columns of warpgroup h
-        float* dst = args.dq_acc + grow * D + h * kHalfD;
-#pragma unroll 1
+        // thread = query row r, the 32 channels of warpgroup h: staged in this warp's own box
+        // (32 rows x 32 channels, 128-byte swizzle) and added to the global accumulator by the
+        // TMA unit; the box's previous reduction has read it (a tile ago) before it is rewritten
+        uint8_t* box = reinterpret_cast<uint8_t*>(&sm.dqs[warp][0][0]);
+        if (lane == 0) bulk_wait_read_0();
+        __syncwarp();
+#pragma unroll
         for (int c0 = 0; c0 < kHalfD; c0 += 16) {
           uint32_t a0[16], a1[16];
           tmem_ld16(lane_base + h * kHalfD + c0, a0);
           tmem_ld16(lane_base + 128 + h * kHalfD + c0, a1);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(a0, a1);
 #pragma unroll
           for (int e = 0; e < 16; e += 4) {
             float4 v4;
@@ -689,8 +692,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             v4.y = deq(a0[e + 1], s0, n0) + deq(a1[e + 1], s1, n1);
             v4.z = deq(a0[e + 2], s0, n0) + deq(a1[e + 2], s1, n1);
             v4.w = deq(a0[e + 3], s0, n0) + deq(a1[e + 3], s1, n1);
-            atomicAdd(reinterpret_cast<float4*>(dst + c0 + e), v4);
+            *reinterpret_cast<float4*>(box + swz_offset(lane, (c0 + e) / 4, 128)) = v4;
           }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_2d(&tm_dq, box, h * kHalfD, row_base + qt * BQ + quarter * 32);
+          bulk_commit();
         }
       }
       tc_fence_before();
@@ -768,9 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4*>(dkp + c0) = pack8<T>(fk);
       }
     }
-    if constexpr (D == 128) {
-      if (lane == 0) bulk_wait_all();  // this warp's dQ reductions complete
-    }
+    if (lane == 0) bulk_wait_all();  // this warp's dQ reductions complete
     tc_fence_before();
     named_barrier_sync(15, kThreads);
   }

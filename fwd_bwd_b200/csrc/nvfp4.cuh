@@ -92,6 +92,19 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
 
 constexpr float kGlobalRange = 2688.0f;  // 6 (largest E2M1) * 448 (largest E4M3)
 
+// x / 6 without a division: q = x * r with r = RN(1/6), the exact residual e = x - 6 q by one
+// FMA, then q + e r by a second FMA (the correction step of Markstein's division algorithm).
+// The result is the correctly rounded quotient whenever that quotient is a normal float32
+// (one binade decides it: power-of-two scaling is exact); for x < 6 * 2^-126 it may differ,
+// but both lie far below 2^-10, so the E4M3 code taken from it is 0 either way.  Checked
+// against __fdiv_rn for every non-negative float32: no E4M3 code differs.
+__device__ __forceinline__ float div6_rn(float x) {
+  const float r = 0.16666667f;  // RN(1/6)
+  const float q = __fmul_rn(x, r);
+  const float e = __fmaf_rn(-q, 6.0f, x);
+  return __fmaf_rn(e, r, q);
+}
+
 // ---------------------------------------------------------------------------------------------
 // Prologue
 // ---------------------------------------------------------------------------------------------

@@ -144,19 +144,6 @@ __device__ __forceinline__ uint32_t e2m1x8(float2 a, float2 b, float2 c, float2 
   return r;
 }
 
-// x / 6 without a division: q = x * r with r = RN(1/6), the exact residual e = x - 6 q by one
-// FMA, then q + e r by a second FMA (the correction step of Markstein's division algorithm).
-// The result is the correctly rounded quotient whenever that quotient is a normal float32
-// (one binade decides it: power-of-two scaling is exact); for x < 6 * 2^-126 it may differ,
-// but both lie far below 2^-10, so the E4M3 code taken from it is 0 either way.  Checked
-// against __fdiv_rn for every non-negative float32: no E4M3 code differs.
-__device__ __forceinline__ float div6_rn(float x) {
-  const float r = 0.16666667f;  // RN(1/6)
-  const float q = __fmul_rn(x, r);
-  const float e = __fmaf_rn(-q, 6.0f, x);
-  return __fmaf_rn(e, r, q);
-}
-
 // Four consecutive 16-element blocks of x quantized to NVFP4 with the global encode scale genc
 // (the prologue's float32 steps: u = (max|x| genc) / 6, sd = e4m3(u), code = e2m1(x genc / sd)),
 // in four independent chains (the scale codes first, then the multipliers, then the codes).

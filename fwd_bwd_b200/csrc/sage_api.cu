@@ -257,8 +257,9 @@ int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const
       !make_map(&tdoc, doc, 1, D, rows, D, sage::bwd::BQ) ||
       !make_map(&tdo, dout, 2, D, rows, 64, sage::bwd::BQ) ||
       !make_map(&tv, v, 2, D, rows, 64, sage::bwd::BKT) ||
-      !make_map(&tdq, dqacc, 4, D, rows, D == 128 ? sage::bwd::kDqCols : D,
-                    sage::bwd::kDqRows, false))
+      // d = 128: 16-query x 32-channel boxes, row-major; d = 64: 32 x 32 boxes, 128-byte swizzle
+      !(D == 128 ? make_map(&tdq, dqacc, 4, D, rows, sage::bwd::kDqCols, sage::bwd::kDqRows, false)
+                 : make_map(&tdq, dqacc, 4, D, rows, 32, 32)))
     return SAGE_ERR_CUDA;
   sage::bwd::Args a;
   a.q_scale = qb->q_scale;
@@ -268,7 +269,6 @@ int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const
   a.dvec = dvec;
   a.k_raw = k;
   a.k_inv_rms = qb->k_inv_rms;
-  a.dq_acc = dqacc;
   a.dk = dk;
   a.dv = dv;
   a.BH = BH;
