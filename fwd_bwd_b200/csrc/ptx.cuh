@@ -338,16 +338,6 @@ __device__ __forceinline__ void tmem_ld_wait_regs8(uint32_t (&a)[8], uint32_t (&
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
-
 // Fills 16 consecutive 32-bit columns of the thread's TMEM lane with the same word.
 __device__ __forceinline__ void tmem_fill16(uint32_t taddr, uint32_t v) {
   asm volatile(
@@ -379,11 +369,6 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// TMEM address of (lane, column) relative to an allocation base.
-__device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint32_t col) {
-  return base + (lane << 16) + col;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -499,22 +484,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
-// Exact int32 -> float for |v| < 2^22: the integer is placed in the mantissa of 1.5 * 2^23.
-__device__ __forceinline__ float i2f_exact(uint32_t v) {
-  return __int_as_float(static_cast<int>(v) + 0x4B400000) - 12582912.0f;
-}
-
-// round-half-to-even(x) for |x| <= 2^22, returned as the low byte of the integer (an int8
-// two's-complement code).  x + 1.5 * 2^23 rounds to an integer in float32 RNE; its mantissa
-// then holds the integer plus 2^22.
-__device__ __forceinline__ uint32_t rne_byte(float x) {
-  return static_cast<uint32_t>(__float_as_int(__fadd_rn(x, 12582912.0f))) & 0xFFu;
-}
-
-__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
-  return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-}
-
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

@@ -228,26 +228,9 @@ __global__ void prologue_kmean_kernel(const float* __restrict__ partials,
   }
 }
 
-// Block absmax over the CTA's 128 rows: rows 0-63 are warps 0-3, rows 64-127 warps 4-7.
-// Returns the absmax of the block this thread's row belongs to (blocks of `blk` rows).
-__device__ __forceinline__ float block_absmax(float local, int blk, float* red) {
-  const int warp = threadIdx.x >> 5;
-  const float wm = warp_max(local);
-  if ((threadIdx.x & 31) == 0) red[warp] = wm;
-  __syncthreads();
-  float a = 0.0f;
-  if (blk == 128) {
-#pragma unroll
-    for (int w = 0; w < 8; ++w) a = fmaxf(a, red[w]);
-  } else {
-    const int w0 = (warp >> 2) << 2;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) a = fmaxf(a, red[w0 + w]);
-  }
-  return a;
-}
-
-// The same over NW warps (rows 0-63 in the first half of the warps, 64-127 in the second).
+// Block absmax over the CTA's 128 rows held by NW warps (rows 0-63 in the first half of the
+// warps, 64-127 in the second); returns the absmax of the block (of `blk` rows) this thread's
+// row belongs to.
 template <int NW>
 __device__ __forceinline__ float block_absmax_n(float local, int blk, float* red) {
   const int warp = threadIdx.x >> 5;
