@@ -119,3 +119,29 @@ def attn_bwd(q, k, v, fb: Fp4Bufs, o, lse, do, cfg: Config, dq=None, dk=None, dv
     else:
         check("sage_fp4_attn_bwd_stage", lib().sage_fp4_attn_bwd_stage(stage, *args))
     return dq, dk, dv
+
+
+class _QAttn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, cfg: Config):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        fb = quant_prologue(q, k, cfg, seq=True)
+        o, lse = attn_fwd(fb, v, cfg)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.fb, ctx.cfg = fb, cfg
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = attn_bwd(q, k, v, ctx.fb, o, lse, do.contiguous(), ctx.cfg)
+        return dq, dk, dv, None
+
+
+def qattn_attention(q, k, v, causal: bool = True, qknorm: bool = True, ksmooth: bool = True,
+                    softmax_scale: float = 0.0, rms_eps: float = 1e-6):
+    """NVFP4 Q-Attn attention with autograd (Q K^T and dS in NVFP4, P V, P^T dO and dO V^T in
+    16 bits): q, k, v are CUDA [B, H, N, d] fp16 / bf16 tensors.  The forward keeps the NVFP4
+    views (with the sequence views the backward multiplies) for the backward."""
+    cfg = Config(causal, qknorm, ksmooth, 128, 64, softmax_scale, rms_eps, False)
+    return _QAttn.apply(q, k, v, cfg)

@@ -205,3 +205,34 @@ def test_nvfp4_backward_degenerate(kind):
         err = rel_l2(got, ref[n])
         print(f"{kind} {n}: rel_l2 {err:.3e}")
         assert err <= (TOL_DV["bf16"] if n == "dv" else TOL_DQK), (n, err)
+
+
+def test_nvfp4_autograd_and_stages_match_direct_calls():
+    """nvfp4.qattn_attention (autograd) and the three staged backward calls give the direct
+    calls' results: O, dK, dV bit for bit (deterministic kernels), dQ within float32 summation
+    order (its tiles are added by asynchronous reductions in no fixed order)."""
+    w = CASES["d128_bf16_causal"]
+    x = make_inputs(w)
+    q, k, v, do = (to_device(x[n], w.dtype) for n in ("q", "k", "v", "do"))
+    cfg = _cfg(w)
+    fb = nvfp4.quant_prologue(q, k, cfg, seq=True)
+    o, lse = nvfp4.attn_fwd(fb, v, cfg)
+    dq, dk, dv = nvfp4.attn_bwd(q, k, v, fb, o, lse, do, cfg)
+    ws = torch.empty(nvfp4.bwd_workspace_bytes(cfg, q), dtype=torch.uint8, device=q.device)
+    sq, sk, sv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    for stage in range(3):
+        nvfp4.attn_bwd(q, k, v, fb, o, lse, do, cfg, dq=sq, dk=sk, dv=sv, workspace=ws,
+                       stage=stage)
+    qa, ka, va = (t.clone().requires_grad_(True) for t in (q, k, v))
+    oa = nvfp4.qattn_attention(qa, ka, va, causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth)
+    oa.backward(do)
+    torch.cuda.synchronize()
+    assert ops.device_status() == 0
+    assert torch.equal(oa.detach(), o)
+    for a, b in ((sk, dk), (sv, dv), (ka.grad, dk), (va.grad, dv)):
+        assert torch.equal(a, b)
+    for a in (sq, qa.grad):
+        err = rel_l2(a.float().cpu().numpy(), dq.float().cpu().numpy())
+        # one bf16 ulp (2^-8 relative) in the rare elements whose float32 sum moves across a
+        # rounding boundary: far below 1e-3 over the tensor
+        assert err <= 1e-3, err
