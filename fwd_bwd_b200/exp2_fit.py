@@ -1,6 +1,6 @@
-"""Coefficients of the kernels' polynomial exp2 (ptx.cuh, exp2_poly).
+"""Coefficients of the kernels' polynomial exp2 (ptx.cuh, exp2_poly2).
 
-exp2_poly(z) splits z = j + f with j = rint(z) and f in [-1/2, 1/2], evaluates p(f) ~ 2^f with a
+exp2_poly2(z) splits z = j + f with j = rint(z) and f in [-1/2, 1/2], evaluates p(f) ~ 2^f with a
 degree-5 polynomial in Horner form (float32 FMAs) and adds j to the exponent field.  The
 coefficients minimise the maximum relative error max |p(f) / 2^f - 1| over [-1/2, 1/2]: the Remez
 exchange algorithm (E. Ya. Remez, 1934) on the error function p(f) 2^-f - 1, run here in

@@ -1,4 +1,5 @@
-"""Parity at the full BASELINE sizes, in the launch configuration bench.py times.
+"""Parity at the workloads' full sizes (listed in CASES below), in the launch configuration
+bench.py times.
 
 The whole batch runs on the GPU; a few sampled (batch, head) pairs carry inputs from the seeded
 per-head numpy streams (the rest are filled on the device) and are checked against the oracle
