@@ -351,17 +351,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m = fmax3(m, f0, f1);
               }
             } else if (diag) {
+              float mo = -INFINITY;  // second chain (odd columns)
 #pragma unroll
               for (int cc = 0; cc < 16; ++cc) {
                 const int k0 = key0 + h * 32 + cc;
                 const float f0 = k0 <= i ? __uint_as_float(x0[cc]) : -INFINITY;
                 const float f1 = k0 + 16 <= i ? __uint_as_float(x1[cc]) : -INFINITY;
-                m = fmax3(m, f0, f1);
+                if (cc & 1)
+                  mo = fmax3(mo, f0, f1);
+                else
+                  m = fmax3(m, f0, f1);
               }
+              m = fmaxf(m, mo);
             } else {
+              float mo = -INFINITY;
 #pragma unroll
-              for (int cc = 0; cc < 16; ++cc)
+              for (int cc = 0; cc < 16; cc += 2) {
                 m = fmax3(m, __uint_as_float(x0[cc]), __uint_as_float(x1[cc]));
+                mo = fmax3(mo, __uint_as_float(x0[cc + 1]), __uint_as_float(x1[cc + 1]));
+              }
+              m = fmaxf(m, mo);
             }
           };
           maxh(a0, a1, 0, m0);

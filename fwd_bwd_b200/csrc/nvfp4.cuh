@@ -213,8 +213,9 @@ __global__ void __launch_bounds__(kQuantThreads, 2) prologue_quant_kernel(Prolog
   // this lane's 8 channels are half of the 16-channel block (sub / 2)
   const int kb = sub >> 1;
   uint8_t* codes = which == 0 ? a.codes[0] : a.codes[1];
-  uint8_t* sf_tile = (which == 0 ? a.sf[0] : a.sf[1]) + (static_cast<size_t>(bh) * nchunk + ch) * (D / 64) * 512 +
-                     (kb >> 2) * 512 + (kb & 3);
+  uint8_t* sf_tile = (which == 0 ? a.sf[0] : a.sf[1]) +
+                     (static_cast<size_t>(bh) * nchunk + ch) * (D / 64) * 512 + (kb >> 2) * 512 +
+                     (kb & 3);
 #pragma unroll
   for (int s = 0; s < STEPS; ++s) {
     float am = 0.0f;
@@ -528,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait_regs(x0, x1);
       tmem_ld_wait_regs(x2, x3);
       tmem_ld_wait_regs(y0, y1);
-      float m0 = -INFINITY, m1 = -INFINITY;
+      float m0 = -INFINITY, m1 = -INFINITY, m0b = -INFINITY, m1b = -INFINITY;  // four chains
       auto maxh = [&](const uint32_t (&xa)[16], const uint32_t (&xb)[16], int k0, float& mm) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -542,13 +543,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld16(so + 32, y0);
       tmem_ld16(so + 48, y1);
       maxh(x0, x1, key0, m0);
-      maxh(x2, x3, key0 + 32, m0);
+      maxh(x2, x3, key0 + 32, m0b);
       tmem_ld_wait_regs(y0, y1);
       tc_fence_before();
       mbar_arrive(&sm.s_free);
-      maxh(y0, y1, okey0 + 32, m1);
+      maxh(y0, y1, okey0 + 32, m1b);
       // block maximum of the raw scores over visible keys (c > 0 keeps the order)
-      const float mn = fmaxf(m, fmaxf(m0, m1) * c);
+      const float mn = fmaxf(m, fmaxf(fmaxf(m0, m0b), fmaxf(m1, m1b)) * c);
       const float alpha = ex2_approx(m - mn);
       // p = exp2(S c - mn) in V's type into this half's swizzle atom (64 keys), row sum
       float rs0 = 0.0f, rs1 = 0.0f;
