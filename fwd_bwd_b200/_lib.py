@@ -92,6 +92,18 @@ def lib() -> ctypes.CDLL:
         L.sage_fwd_bwd_host.argtypes = [P(SageParams), vp, vp, vp, vp, vp, vp, vp, vp, i, vp, sz,
                                         vp, vp, vp]
         L.sage_fwd_bwd_host.restype = i
+        L.sage_quant_prologue_part.argtypes = [P(SageParams), vp, vp, vp, P(SageQBufs), vp, sz, i,
+                                               vp]
+        L.sage_quant_prologue_part.restype = i
+        L.sage_attn_fwd_partial.argtypes = [P(SageParams), P(SageQBufs), vp, vp, vp]
+        L.sage_attn_fwd_partial.restype = i
+        L.sage_attn_merge.argtypes = [P(SageParams), vp, vp, vp, vp, vp, vp]
+        L.sage_attn_merge.restype = i
+        L.sage_attn_bwd_partial.argtypes = [P(SageParams), vp, P(SageQBufs), vp, vp, vp, vp, i,
+                                            vp, sz, vp]
+        L.sage_attn_bwd_partial.restype = i
+        L.sage_kv_finalize.argtypes = [P(SageParams), vp, P(SageQBufs), vp, vp, vp, vp, vp]
+        L.sage_kv_finalize.restype = i
         L.sage_last_device_status.argtypes = [vp]
         L.sage_last_device_status.restype = i
         L.sage_status_string.argtypes = [i]

@@ -138,6 +138,12 @@ struct Args {
   float tau;         // softmax_scale
   const float* k_bias;  // [BH, N] (Q-smoothing)
   const float* q_mean;  // [BH, D] (Q-smoothing)
+  // context-parallel partial (both set, Q-smoothing off): the CTA's raw dK_hat / dV rows go to
+  // these float32 [BH, N, D] accumulators instead of being finished and stored; acc_add = 0
+  // stores them (the first chunk of queries), 1 adds them
+  float* dk_acc;
+  float* dv_acc;
+  int acc_add;
 };
 
 template <int D>
@@ -709,7 +715,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       sdsc = sdsc_n;
     }
     // epilogue: dv, dk from the register accumulators (thread = key row r, d half h)
-    {
+    if (args.dk_acc != nullptr) {
+      // partial over one query chunk: accumulate; the keys' owner applies the RMSNorm
+      // backward once every chunk's contribution is in
+      const size_t off = (static_cast<size_t>(row_base) + key_base + r) * D + h * kHalfD;
+      float4* ka = reinterpret_cast<float4*>(args.dk_acc + off);
+      float4* va = reinterpret_cast<float4*>(args.dv_acc + off);
+#pragma unroll
+      for (int c4 = 0; c4 < kHalfD / 4; ++c4) {
+        float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f), b = a;
+        if (args.acc_add) {
+          a = ka[c4];
+          b = va[c4];
+        }
+        a.x += acck[2 * c4].x;
+        a.y += acck[2 * c4].y;
+        a.z += acck[2 * c4 + 1].x;
+        a.w += acck[2 * c4 + 1].y;
+        b.x += accv[2 * c4].x;
+        b.y += accv[2 * c4].y;
+        b.z += accv[2 * c4 + 1].x;
+        b.w += accv[2 * c4 + 1].y;
+        ka[c4] = a;
+        va[c4] = b;
+      }
+    } else {
       const size_t krow = static_cast<size_t>(row_base) + key_base + r;
       T* dvp = reinterpret_cast<T*>(args.dv) + krow * D + h * kHalfD;
       T* dkp = reinterpret_cast<T*>(args.dk) + krow * D + h * kHalfD;

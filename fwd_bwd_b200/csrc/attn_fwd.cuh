@@ -94,6 +94,7 @@ struct Args {
   float scale_log2;  // softmax_scale * log2(e)
   int nsup;          // CTAs per head: ceil(N / 256)
   const float* k_bias;  // [BH, N] (Q-smoothing)
+  float* o_f32;  // when set, O is written here in float32 [BH, N, D] instead of to `o`
 };
 
 template <int D>
@@ -455,16 +456,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       fold_pv(nb[g] - 1);
       // epilogue: O / l in the output type, LSE = (m2 + log2 l) ln 2
       const float inv_l = 1.0f / l;
-      T* orow = reinterpret_cast<T*>(args.o) + (static_cast<size_t>(bh) * N + i) * D;
+      if (args.o_f32 != nullptr) {
+        // float32 partial result (context parallelism merges several of them)
+        float4* of = reinterpret_cast<float4*>(args.o_f32 + (static_cast<size_t>(bh) * N + i) * D);
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 8) {
-        float f[8];
+        for (int c0 = 0; c0 < D; c0 += 4)
+          of[c0 / 4] = make_float4(O[c0 / 2].x * inv_l, O[c0 / 2].y * inv_l,
+                                   O[c0 / 2 + 1].x * inv_l, O[c0 / 2 + 1].y * inv_l);
+      } else {
+        T* orow = reinterpret_cast<T*>(args.o) + (static_cast<size_t>(bh) * N + i) * D;
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          f[e] = O[(c0 + e) / 2].x * inv_l;
-          f[e + 1] = O[(c0 + e) / 2].y * inv_l;
+        for (int c0 = 0; c0 < D; c0 += 8) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            f[e] = O[(c0 + e) / 2].x * inv_l;
+            f[e + 1] = O[(c0 + e) / 2].y * inv_l;
+          }
+          *reinterpret_cast<uint4*>(orow + c0) = pack8<T>(f);
         }
-        *reinterpret_cast<uint4*>(orow + c0) = pack8<T>(f);
       }
       args.lse[static_cast<size_t>(bh) * N + i] = (m2 + log2f(l)) * 0.69314718055994531f;
     }

@@ -433,4 +433,55 @@ __global__ void __launch_bounds__(kRowThreads) dq_finalize_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Merge of two attention results over disjoint key sets (context parallelism).  With
+// L = ln(e^La + e^Lb), the softmax over the union of the keys gives
+// O = e^(La - L) O_a + e^(Lb - L) O_b.  o_acc / lse_acc (float32, natural-log LSE; -inf marks
+// an empty result) are updated in place with the partial o_part / lse_part; when `out` is
+// set, the merged O is also written there in the 16-bit type.  Without a partial (o_part and
+// lse_part null) the accumulator is only converted to `out`.  One thread per 8 channels of a
+// row; the grid covers rows * D / 8 threads exactly (rows a multiple of 128).
+// ---------------------------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(256) attn_merge_kernel(float* __restrict__ o_acc,
+                                                         float* __restrict__ lse_acc,
+                                                         const float* __restrict__ o_part,
+                                                         const float* __restrict__ lse_part,
+                                                         T* __restrict__ out) {
+  constexpr int TPR = D / 8;  // threads per row (a row never straddles a warp)
+  const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t row = tid / TPR;
+  const int c = static_cast<int>(tid % TPR) * 8;
+  const float la = lse_acc[row];
+  const float lb = lse_part != nullptr ? lse_part[row] : -INFINITY;
+  const float4* pa = reinterpret_cast<const float4*>(o_acc + row * D + c);
+  const float4 a0 = pa[0], a1 = pa[1];
+  float f[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};  // empty partial: keep acc
+  float lnew = la;
+  if (lb != -INFINITY) {
+    const float4* pb = reinterpret_cast<const float4*>(o_part + row * D + c);
+    const float4 b0 = pb[0], b1 = pb[1];
+    const float g[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    if (la == -INFINITY) {  // empty accumulator: take the partial
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = g[e];
+      lnew = lb;
+    } else {
+      const float m = fmaxf(la, lb);
+      const float ea = expf(la - m), eb = expf(lb - m);
+      const float sum = ea + eb;
+      lnew = m + logf(sum);
+      const float wa = ea / sum, wb = eb / sum;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = fmaf(f[e], wa, g[e] * wb);
+    }
+  }
+  float4* po = reinterpret_cast<float4*>(o_acc + row * D + c);
+  po[0] = make_float4(f[0], f[1], f[2], f[3]);
+  po[1] = make_float4(f[4], f[5], f[6], f[7]);
+  if (out != nullptr) *reinterpret_cast<uint4*>(out + row * D + c) = pack8<T>(f);
+  __syncwarp();  // every thread of the row has read lse_acc[row]
+  if (c == 0) lse_acc[row] = lnew;
+}
+
 }  // namespace sage

@@ -147,14 +147,16 @@ int launch_regs(K kernel) {
 
 // ---- prologue ---------------------------------------------------------------------------
 template <typename T, int D>
+// part -1: statistics and quantization; 0: statistics only (the smoothing means); 1:
+// quantization only, with the means already in `out`.
 int run_prologue(const sage_params* p, const void* q, const void* k, const void* v,
-                 const sage_qbufs* out, void* ws, cudaStream_t st) {
+                 const sage_qbufs* out, void* ws, cudaStream_t st, int part = -1) {
   const int BH = p->B * p->H, N = p->N;
   float* partials = reinterpret_cast<float*>(ws);
   const int total = BH * (N / 64);
   const int per_cta = (kRowThreads / 32) * (32 / (D / 8));
   // smoothing means: K's (ksmooth), then Q's (qsmooth), each from its own partials
-  for (int which = 1; which >= 0; --which) {
+  for (int which = 1; which >= 0 && part != 1; --which) {
     if (which == 1 ? !p->ksmooth : !p->qsmooth) continue;
     sage::prologue_kstats_kernel<T, D><<<(total + per_cta - 1) / per_cta, kRowThreads, 0, st>>>(
         reinterpret_cast<const T*>(which == 1 ? k : q), partials, total, p->qknorm,
@@ -163,6 +165,7 @@ int run_prologue(const sage_params* p, const void* q, const void* k, const void*
         partials, which == 1 ? out->k_mean : out->q_mean, N / 64, N);
     partials += prologue_partials(p);
   }
+  if (part == 0) return launch_status();
   sage::PrologueArgs a;
   a.src[0] = q;
   a.src[1] = k;
@@ -192,7 +195,8 @@ int run_prologue(const sage_params* p, const void* q, const void* k, const void*
 
 // ---- forward ----------------------------------------------------------------------------
 template <typename T, int D>
-int run_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse, cudaStream_t st) {
+int run_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse, cudaStream_t st,
+            float* o_f32 = nullptr) {
   const int BH = p->B * p->H, N = p->N;
   const uint64_t rows = static_cast<uint64_t>(BH) * N;
   CUtensorMap tq, tk, tv;
@@ -213,6 +217,7 @@ int run_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse, cud
   a.scale_log2 = tau_of(p) * 1.4426950408889634f;
   a.nsup = (N + sage::fwd::NT * sage::fwd::BM - 1) / (sage::fwd::NT * sage::fwd::BM);
   a.k_bias = qb->k_bias;
+  a.o_f32 = o_f32;
   const size_t smem = sage::fwd::smem_bytes<D>();
   auto kern = p->qsmooth ? sage::fwd::attn_fwd_kernel<T, D, true>
                          : sage::fwd::attn_fwd_kernel<T, D, false>;
@@ -229,7 +234,8 @@ int run_fwd(const sage_params* p, const sage_qbufs* qb, void* o, float* lse, cud
 template <typename T, int D>
 int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const void* v,
             const sage_qbufs* qb, const void* o, const float* lse, const void* dout, void* dq,
-            void* dk, void* dv, void* ws, cudaStream_t st) {
+            void* dk, void* dv, void* ws, cudaStream_t st, float* dk_acc = nullptr,
+            float* dv_acc = nullptr, int acc_add = 0) {
   const int BH = p->B * p->H, N = p->N;
   const uint64_t rows = static_cast<uint64_t>(BH) * N;
   const BwdWs w = bwd_ws(p);
@@ -280,6 +286,9 @@ int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const
   a.scale_log2 = a.tau * 1.4426950408889634f;
   a.k_bias = qb->k_bias;
   a.q_mean = qb->q_mean;
+  a.dk_acc = dk_acc;
+  a.dv_acc = dv_acc;
+  a.acc_add = acc_add;
   const size_t smem = sage::bwd::smem_bytes<D>();
   auto kern = p->qsmooth ? sage::bwd::attn_bwd_kernel<T, D, true>
                          : sage::bwd::attn_bwd_kernel<T, D, false>;
@@ -290,6 +299,31 @@ int run_bwd(int stage, const sage_params* p, const void* q, const void* k, const
   if (launch_regs(kern) != sage::bwd::kLaunchRegs) return SAGE_ERR_UNSUPPORTED;
   kern<<<BH * (N / sage::bwd::BKT), sage::bwd::kThreads, smem, st>>>(tqc, tkc, tdoc, tdo, tv, tdq,
                                                                      a);
+  return launch_status();
+}
+
+// ---- context parallelism: merge of partial results, key-side finalize ---------------------
+template <typename T, int D>
+int run_merge(const sage_params* p, float* o_acc, float* lse_acc, const float* o_part,
+              const float* lse_part, void* out, cudaStream_t st) {
+  // N is a multiple of 128, so rows * D / 8 threads fill whole 256-thread blocks
+  const size_t rows = static_cast<size_t>(p->B) * p->H * p->N;
+  const size_t blocks = rows * (D / 8) / 256;
+  sage::attn_merge_kernel<T, D><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      o_acc, lse_acc, o_part, lse_part, reinterpret_cast<T*>(out));
+  return launch_status();
+}
+
+template <typename T, int D>
+int run_kv_finalize(const sage_params* p, const void* k, const sage_qbufs* qb,
+                    const float* dk_acc, const float* dv_acc, void* dk, void* dv, cudaStream_t st) {
+  const size_t rows = static_cast<size_t>(p->B) * p->H * p->N;
+  const int grid = static_cast<int>(rows / kRowsPerCta);
+  sage::dq_finalize_kernel<T, D><<<grid, kRowThreads, 0, st>>>(
+      dk_acc, reinterpret_cast<const T*>(k), qb ? qb->k_inv_rms : nullptr,
+      reinterpret_cast<T*>(dk), p->qknorm);
+  sage::dq_finalize_kernel<T, D><<<grid, kRowThreads, 0, st>>>(
+      dv_acc, nullptr, nullptr, reinterpret_cast<T*>(dv), 0);
   return launch_status();
 }
 
@@ -940,6 +974,110 @@ int sage_mma_peak(int kind, int n_ctas, int groups, const void* fill, size_t fil
   sage::dbg::mma_peak_kernel<<<n_ctas, 128, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const uint4*>(fill), kind, groups);
   return launch_status();
+}
+
+// ---- context parallelism ------------------------------------------------------------------
+int sage_quant_prologue_part(const sage_params* p, const void* q, const void* k, const void* v,
+                             const sage_qbufs* out, void* workspace, size_t workspace_bytes,
+                             int part, void* stream) {
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if (part != 0 && part != 1) return SAGE_ERR_INVALID_ARG;
+  if (p->qsmooth) return SAGE_ERR_UNSUPPORTED;
+  if (!q || !k || !v) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_qbufs(p, out)) != SAGE_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SAGE_ERR_ALIGNMENT;
+  const size_t need = part == 0 ? prologue_ws(p) : 0;
+  if (need > 0 && (!workspace || workspace_bytes < need)) return SAGE_ERR_WORKSPACE;
+  if (workspace && !aligned16(workspace)) return SAGE_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_prologue<__nv_bfloat16, 128>(p, q, k, v, out, workspace, st, part)
+              : run_prologue<__half, 128>(p, q, k, v, out, workspace, st, part);
+  return bf ? run_prologue<__nv_bfloat16, 64>(p, q, k, v, out, workspace, st, part)
+            : run_prologue<__half, 64>(p, q, k, v, out, workspace, st, part);
+}
+
+int sage_attn_fwd_partial(const sage_params* p, const sage_qbufs* qb, float* o_part,
+                          float* lse_part, void* stream) {
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if (p->qsmooth) return SAGE_ERR_UNSUPPORTED;
+  if ((s = check_qbufs(p, qb)) != SAGE_OK) return s;
+  if (!o_part || !lse_part) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(o_part) || !aligned16(lse_part)) return SAGE_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_fwd<__nv_bfloat16, 128>(p, qb, nullptr, lse_part, st, o_part)
+              : run_fwd<__half, 128>(p, qb, nullptr, lse_part, st, o_part);
+  return bf ? run_fwd<__nv_bfloat16, 64>(p, qb, nullptr, lse_part, st, o_part)
+            : run_fwd<__half, 64>(p, qb, nullptr, lse_part, st, o_part);
+}
+
+int sage_attn_merge(const sage_params* p, float* o_acc, float* lse_acc, const float* o_part,
+                    const float* lse_part, void* out, void* stream) {
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if (!o_acc || !lse_acc || (o_part == nullptr) != (lse_part == nullptr))
+    return SAGE_ERR_INVALID_ARG;
+  const void* ptrs[] = {o_acc, lse_acc, o_part, lse_part, out};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return SAGE_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_merge<__nv_bfloat16, 128>(p, o_acc, lse_acc, o_part, lse_part, out, st)
+              : run_merge<__half, 128>(p, o_acc, lse_acc, o_part, lse_part, out, st);
+  return bf ? run_merge<__nv_bfloat16, 64>(p, o_acc, lse_acc, o_part, lse_part, out, st)
+            : run_merge<__half, 64>(p, o_acc, lse_acc, o_part, lse_part, out, st);
+}
+
+int sage_attn_bwd_partial(const sage_params* p, const void* v, const sage_qbufs* qb,
+                          const float* lse, const void* dout, float* dk_acc, float* dv_acc,
+                          int accumulate, void* workspace, size_t workspace_bytes, void* stream) {
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if (accumulate != 0 && accumulate != 1) return SAGE_ERR_INVALID_ARG;
+  if (p->qsmooth) return SAGE_ERR_UNSUPPORTED;
+  if ((s = check_qbufs(p, qb)) != SAGE_OK) return s;
+  if (!v || !lse || !dout || !dk_acc || !dv_acc) return SAGE_ERR_INVALID_ARG;
+  const void* ptrs[] = {v, lse, dout, dk_acc, dv_acc, workspace};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return SAGE_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < bwd_ws(p).total) return SAGE_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_bwd<__nv_bfloat16, 128>(1, p, nullptr, nullptr, v, qb, nullptr, lse, dout,
+                                             nullptr, nullptr, nullptr, workspace, st, dk_acc,
+                                             dv_acc, accumulate)
+              : run_bwd<__half, 128>(1, p, nullptr, nullptr, v, qb, nullptr, lse, dout, nullptr,
+                                     nullptr, nullptr, workspace, st, dk_acc, dv_acc, accumulate);
+  return bf ? run_bwd<__nv_bfloat16, 64>(1, p, nullptr, nullptr, v, qb, nullptr, lse, dout,
+                                          nullptr, nullptr, nullptr, workspace, st, dk_acc, dv_acc,
+                                          accumulate)
+            : run_bwd<__half, 64>(1, p, nullptr, nullptr, v, qb, nullptr, lse, dout, nullptr,
+                                  nullptr, nullptr, workspace, st, dk_acc, dv_acc, accumulate);
+}
+
+int sage_kv_finalize(const sage_params* p, const void* k, const sage_qbufs* qb,
+                     const float* dk_acc, const float* dv_acc, void* dk, void* dv, void* stream) {
+  int s = check_params(p);
+  if (s != SAGE_OK) return s;
+  if (!dk_acc || !dv_acc || !dk || !dv) return SAGE_ERR_INVALID_ARG;
+  if (p->qknorm && (!k || !qb || !qb->k_inv_rms)) return SAGE_ERR_INVALID_ARG;
+  const void* ptrs[] = {k, dk_acc, dv_acc, dk, dv};
+  for (const void* ptr : ptrs)
+    if (ptr && !aligned16(ptr)) return SAGE_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf = p->dtype == SAGE_BF16;
+  if (p->d == 128)
+    return bf ? run_kv_finalize<__nv_bfloat16, 128>(p, k, qb, dk_acc, dv_acc, dk, dv, st)
+              : run_kv_finalize<__half, 128>(p, k, qb, dk_acc, dv_acc, dk, dv, st);
+  return bf ? run_kv_finalize<__nv_bfloat16, 64>(p, k, qb, dk_acc, dv_acc, dk, dv, st)
+            : run_kv_finalize<__half, 64>(p, k, qb, dk_acc, dv_acc, dk, dv, st);
 }
 
 }  // extern "C"

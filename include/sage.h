@@ -177,6 +177,61 @@ int sage_fwd_bwd_host(const sage_params* p, const void* q, const void* k, const 
                       void* workspace, size_t workspace_bytes, void* stream_in,
                       void* stream_compute, void* stream_out);
 
+/* ---- context parallelism: one long sequence split into chunks held by different ranks ----
+ * The sequence of N_total tokens is cut into W contiguous chunks of N tokens (p->N is the
+ * chunk length; N_total = W * N); rank r holds tokens [r*N, (r+1)*N) of every (batch, head).
+ * The blocks of every quantization (Q, K, V per block of tokens; P, dS, dO per tile) never
+ * straddle a chunk boundary, so the pieces below give the single-sequence result of
+ * sage_quant_prologue / sage_attn_fwd / sage_attn_bwd up to float32 rounding order.  The
+ * ranks exchange data between the calls (ring order; fwd_bwd_b200/cp.py).  Q-smoothing
+ * (qsmooth) is not supported here (SAGE_ERR_UNSUPPORTED).
+ *
+ * sage_quant_prologue_part: the prologue in two parts.  part 0: the K-smoothing statistics of
+ *   this chunk only: out->k_mean = per-channel mean over the chunk's tokens of the normalized
+ *   k (needs the prologue workspace; nothing else is written).  The ranks then average their
+ *   means (all equal-sized chunks, so the average is the mean over all N_total tokens, the
+ *   K-smoothing paragraph's mean over the sequence).  part 1: QK-norm, smoothing with the
+ *   caller's out->k_mean, and the per-block codes and scales of the chunk (no workspace).
+ *   Without ksmooth, part 0 does nothing and part 1 equals sage_quant_prologue. */
+int sage_quant_prologue_part(const sage_params* p, const void* q, const void* k, const void* v,
+                             const sage_qbufs* out, void* workspace, size_t workspace_bytes,
+                             int part, void* stream);
+
+/* sage_attn_fwd_partial: attention of this chunk's queries over ONE chunk of keys, whose codes
+ *   and scales qb->k_* / qb->v_* point at (the local chunk or one received from another
+ *   rank; qb->q_* are the local queries').  p->causal: 1 for the diagonal chunk (the same
+ *   token range as the queries), 0 for a chunk of earlier keys; chunks of later keys are not
+ *   computed under a causal mask.  o_part: float32 [B,H,N,d], normalized over this chunk's
+ *   keys; lse_part: float32 [B,H,N], natural-log sum of exponentials of the scaled scores. */
+int sage_attn_fwd_partial(const sage_params* p, const sage_qbufs* qb, float* o_part,
+                          float* lse_part, void* stream);
+
+/* sage_attn_merge: softmax over the union of two disjoint key sets from their partial results:
+ *   L = ln(e^La + e^Lb), O = e^(La-L) O_a + e^(Lb-L) O_b, written back into (o_acc, lse_acc)
+ *   (float32 [B,H,N,d] / [B,H,N]; lse = -inf marks an empty result).  When `out` is not NULL
+ *   the merged O is also stored there in dtype ([B,H,N,d]).  With o_part and lse_part both
+ *   NULL the accumulator is only converted to `out`. */
+int sage_attn_merge(const sage_params* p, float* o_acc, float* lse_acc, const float* o_part,
+                    const float* lse_part, void* out, void* stream);
+
+/* sage_attn_bwd_partial: the backward tensor-core kernel for this chunk's queries against one
+ *   chunk of keys (qb->k_*: its codes and scales, v: its raw 16-bit values for dP; p->causal
+ *   as in sage_attn_fwd_partial).  Needs stage 0 of sage_attn_bwd_stage run first on the same
+ *   workspace with this chunk's o, dout and the merged lse; dQ accumulates in the workspace
+ *   across calls (stage 2 then finishes dq).  The keys' raw gradients (before the RMSNorm
+ *   backward) go to dk_acc / dv_acc (float32 [B,H,N,d]): stored when accumulate = 0 (the first
+ *   chunk of queries to see these keys), added when accumulate = 1.  They travel back to the
+ *   keys' owner, which finishes them with sage_kv_finalize. */
+int sage_attn_bwd_partial(const sage_params* p, const void* v, const sage_qbufs* qb,
+                          const float* lse, const void* dout, float* dk_acc, float* dv_acc,
+                          int accumulate, void* workspace, size_t workspace_bytes, void* stream);
+
+/* sage_kv_finalize: dk = RMSNorm backward of dk_acc (with qknorm; k the raw keys and
+ *   qb->k_inv_rms their inverse RMS from the prologue; otherwise dk = dk_acc), dv = dv_acc,
+ *   both stored in dtype ([B,H,N,d]). */
+int sage_kv_finalize(const sage_params* p, const void* k, const sage_qbufs* qb,
+                     const float* dk_acc, const float* dv_acc, void* dk, void* dv, void* stream);
+
 /* Synchronizes `stream`, returns the device status word of the current device (SAGE_OK or
  * SAGE_ERR_TIMEOUT) and clears it.  Returns SAGE_ERR_CUDA if the synchronization fails. */
 int sage_last_device_status(void* stream);

@@ -29,7 +29,7 @@ def _declared(header="sage.h"):
 
 def test_exports_every_declared_symbol(L):
     names = _declared()
-    assert len(names) == 14
+    assert len(names) == 19
     fp4 = _declared("sage_nvfp4.h")
     assert fp4 == ["sage_fp4_attn_bwd", "sage_fp4_attn_bwd_stage", "sage_fp4_attn_fwd",
                    "sage_fp4_quant_prologue", "sage_fp4_workspace_bytes"]
@@ -239,3 +239,37 @@ def test_debug_entry_validation(L):
         _lib.SAGE_ERR_UNSUPPORTED
     assert L.sage_debug_umma_gemm(0, 0, 0, 64, 64, None, 16, 16, None) == \
         _lib.SAGE_ERR_INVALID_ARG
+
+
+def test_context_parallel_entry_argument_checks(L):
+    """The context-parallel entry points refuse bad arguments before any launch."""
+    from ctypes import byref
+    E = _lib
+    p, pq = _params(), _params(qsmooth=1)
+    qb = SageQBufs(*([16] * 9))
+    f = 1 << 20  # never dereferenced
+    part = L.sage_quant_prologue_part
+    assert part(byref(p), f, f, f, byref(qb), f, 1 << 40, 2, None) == E.SAGE_ERR_INVALID_ARG
+    assert part(byref(pq), f, f, f, byref(qb), f, 1 << 40, 0, None) == E.SAGE_ERR_UNSUPPORTED
+    assert part(byref(p), None, f, f, byref(qb), f, 1 << 40, 1, None) == E.SAGE_ERR_INVALID_ARG
+    assert part(byref(p), f, f, f + 2, byref(qb), f, 1 << 40, 1, None) == E.SAGE_ERR_ALIGNMENT
+    assert part(byref(p), f, f, f, byref(qb), f, 100, 0, None) == E.SAGE_ERR_WORKSPACE
+    fwd = L.sage_attn_fwd_partial
+    assert fwd(byref(pq), byref(qb), f, f, None) == E.SAGE_ERR_UNSUPPORTED
+    assert fwd(byref(p), byref(qb), None, f, None) == E.SAGE_ERR_INVALID_ARG
+    assert fwd(byref(p), byref(qb), f + 4, f, None) == E.SAGE_ERR_ALIGNMENT
+    merge = L.sage_attn_merge
+    assert merge(byref(p), None, f, f, f, None, None) == E.SAGE_ERR_INVALID_ARG
+    assert merge(byref(p), f, f, None, f, None, None) == E.SAGE_ERR_INVALID_ARG  # o without lse
+    assert merge(byref(p), f, f, f, f, f + 8, None) == E.SAGE_ERR_ALIGNMENT
+    bwd = L.sage_attn_bwd_partial
+    assert bwd(byref(p), f, byref(qb), f, f, f, f, 2, f, 1 << 40, None) == E.SAGE_ERR_INVALID_ARG
+    assert bwd(byref(pq), f, byref(qb), f, f, f, f, 0, f, 1 << 40, None) == \
+        E.SAGE_ERR_UNSUPPORTED
+    assert bwd(byref(p), f, byref(qb), f, f, None, f, 1, f, 1 << 40, None) == \
+        E.SAGE_ERR_INVALID_ARG
+    assert bwd(byref(p), f, byref(qb), f, f, f, f, 1, f, 100, None) == E.SAGE_ERR_WORKSPACE
+    fin = L.sage_kv_finalize
+    assert fin(byref(p), None, byref(qb), f, f, f, f, None) == E.SAGE_ERR_INVALID_ARG  # qknorm
+    assert fin(byref(p), f, byref(qb), f, f, None, f, None) == E.SAGE_ERR_INVALID_ARG
+    assert fin(byref(p), f, byref(qb), f, f, f + 2, f, None) == E.SAGE_ERR_ALIGNMENT
