@@ -29,6 +29,9 @@
 // thread holds 168, afterwards 256 x 216 + 128 x 72 = 64512 = 384 x 168.  The MMA thread keeps
 // 72: with 56 it spilled and its reloads delayed the tensor-core issue; the compute warps' 216
 // leave them fewer spills than 208 (-0.9% time).
+// Context parallelism (Args::dk_acc set): the epilogue stores or adds the raw dK_hat / dV rows
+// into float32 accumulators instead of finishing them, since other chunks of queries add
+// theirs; the keys' owner applies the RMSNorm backward afterwards.
 // Q-smoothing (template flag QS): pass A adds the per-key bias to the recomputed scores, and
 // pass B also sums each key's dS codes over the tile's rows (one warp reduction per key), so
 // the epilogue can add dK_bias = tau * (sum over tiles of sdS * column sum) * mu_Q.

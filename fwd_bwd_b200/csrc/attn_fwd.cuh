@@ -18,7 +18,8 @@
 // each MMA (see kMagicBits), so results read back as floats that one FMA dequantizes; the MMA
 // thread writes the preload with one bf16 MMA (mma_fill_magic), so the softmax warps only read
 // TMEM.
-// O (float32) lives in registers.
+// O (float32) lives in registers; it is stored in the 16-bit type, or in float32 when
+// Args::o_f32 is set (a partial result of context parallelism, merged by log-sum-exp later).
 //
 // Q-smoothing (template flag QS): every score of key j gains the per-key bias k_bias_j, copied
 // with the K block into shared memory; the block maximum is then taken over the biased scores
