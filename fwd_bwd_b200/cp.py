@@ -19,7 +19,8 @@ Backward (``backward``): the K codes and scales, the raw 16-bit V (for the 16-bi
 and two float32 accumulators for the keys' raw dK and dV travel around the ring; each rank adds
 its queries' contribution (``sage_attn_bwd_partial``; dQ accumulates locally), and after W
 shifts the accumulators are back with the keys' owner, which applies the RMSNorm backward
-(``sage_kv_finalize``).
+(``sage_kv_finalize``).  The keys' transfer overlaps the step's kernels; the accumulators' can
+only follow them.
 
 Two transports run the same per-rank code:
   * ``RingComm``: one process per GPU, torch.distributed point-to-point (NCCL on GPUs);
@@ -302,22 +303,27 @@ def backward(state: ForwardState, dout: torch.Tensor,
         0, ctypes.byref(prm), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(st),
         state.o.data_ptr(), state.lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
         dv.data_ptr(), ws.data_ptr(), n, stream))
-    dk_acc = torch.empty(q.shape, dtype=torch.float32, device=dev)
-    dv_acc = torch.empty_like(dk_acc)
-    payload = [qb.k_codes, qb.k_scale, v, dk_acc, dv_acc]
+    keys = [qb.k_codes, qb.k_scale, v]  # read-only on the way
+    acc = [torch.empty(q.shape, dtype=torch.float32, device=dev) for _ in range(2)]  # dK, dV
     for s, _, mode in schedule(comm.rank, comm.world, cfg.causal):
+        # the next chunk's keys are on their way while this one is computed; the accumulators
+        # follow once this rank has added to them, and after the last step only they travel,
+        # back to their owner
+        more = s + 1 < comm.world
+        pending = comm.shift_start(keys) if more else None
         if mode is not None:
             pp = _pair_params(cfg, q, mode)
-            pq = _pair_qbufs(qb, payload[0], payload[1])
+            pq = _pair_qbufs(qb, keys[0], keys[1])
             # the keys' owner computes first (step 0) and stores; later ranks add
             check("sage_attn_bwd_partial", lib().sage_attn_bwd_partial(
-                ctypes.byref(pp), payload[2].data_ptr(), ctypes.byref(pq),
-                state.lse.data_ptr(), dout.data_ptr(), payload[3].data_ptr(),
-                payload[4].data_ptr(), int(s > 0), ws.data_ptr(), n, stream))
-        # the accumulators move on; after the last step only they travel, back to their owner
+                ctypes.byref(pp), keys[2].data_ptr(), ctypes.byref(pq), state.lse.data_ptr(),
+                dout.data_ptr(), acc[0].data_ptr(), acc[1].data_ptr(), int(s > 0),
+                ws.data_ptr(), n, stream))
         if comm.world > 1:
-            payload = comm.shift(payload if s + 1 < comm.world else payload[3:])
-    dk_acc, dv_acc = payload[-2], payload[-1]
+            acc = comm.shift(acc)
+        if pending is not None:
+            keys = pending.wait()
+    dk_acc, dv_acc = acc
     check("sage_attn_bwd_stage", lib().sage_attn_bwd_stage(
         2, ctypes.byref(prm), q.data_ptr(), k.data_ptr(), v.data_ptr(), ctypes.byref(st),
         state.o.data_ptr(), state.lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),

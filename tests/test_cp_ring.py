@@ -106,21 +106,26 @@ def _worker(rank, world, port, causal, out_q):
     # backward: dQ local, dK / dV accumulators travel with the keys
     Dv = (do * o_acc).sum(axis=1)
     dq = np.zeros_like(q)
-    payload = [torch.from_numpy(k.copy()), torch.from_numpy(v.copy()),
-               torch.zeros(N, d, dtype=torch.float64), torch.zeros(N, d, dtype=torch.float64)]
+    # as fwd_bwd_b200/cp.py: the keys travel ahead (overlapping the step), the accumulators
+    # after the step, and after the last step only they travel, back to their owner
+    keys = [torch.from_numpy(k.copy()), torch.from_numpy(v.copy())]
+    acc = [torch.zeros(N, d, dtype=torch.float64), torch.zeros(N, d, dtype=torch.float64)]
     for s, j, mode in schedule(rank, world, causal):
+        pend = comm.shift_start(keys) if s + 1 < world else None
         if mode is not None:
-            kj, vj = payload[0].numpy(), payload[1].numpy()
+            kj, vj = keys[0].numpy(), keys[1].numpy()
             z = tau * q @ kj.T
             p = np.where(visible(mode), np.exp(z - lse_acc[:, None]), 0.0)
             dp = do @ vj.T
             ds = p * (dp - Dv[:, None])
             dq += tau * ds @ kj
-            payload[2] += torch.from_numpy(tau * ds.T @ q)
-            payload[3] += torch.from_numpy(p.T @ do)
+            acc[0] += torch.from_numpy(tau * ds.T @ q)
+            acc[1] += torch.from_numpy(p.T @ do)
         if world > 1:
-            payload = comm.shift(payload if s + 1 < world else payload[2:])
-    dk, dv = payload[-2].numpy(), payload[-1].numpy()
+            acc = comm.shift(acc)
+        if pend is not None:
+            keys = pend.wait()
+    dk, dv = acc[0].numpy(), acc[1].numpy()
 
     shards = [None] * world
     dist.all_gather_object(shards, dict(o=o_acc, lse=lse_acc, dq=dq, dk=dk, dv=dv))
