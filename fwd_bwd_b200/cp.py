@@ -155,7 +155,9 @@ class LocalRing:
         for t in threads:
             t.join()
         if errors:
-            raise errors[0]
+            # the rank that failed first breaks the barrier; the others then see only that
+            root = [e for e in errors if not isinstance(e, threading.BrokenBarrierError)]
+            raise (root or errors)[0]
         return results
 
 
