@@ -54,6 +54,10 @@ def parse():
                     help="skip the tensor-core peak loop (profiling runs; no roofline fraction)")
     ap.add_argument("--variant", default="int8", choices=["int8", "nvfp4"],
                     help="int8: the SageBwd step (default); nvfp4: the NVFP4 Q-Attn fwd+bwd step")
+    ap.add_argument("--cp", type=int, default=0,
+                    help="context parallelism: the workload's sequence in this many chunks, the "
+                         "ranks as threads on one GPU (cp.LocalRing), beside the single-sequence "
+                         "step")
     return ap.parse_args()
 
 
@@ -278,6 +282,77 @@ def timed_steps(step, nev: int, steps: int, dev, flush_buf=None):
     return evs
 
 
+def run_cp(args, w):
+    """Context parallelism on one GPU: the workload's sequence cut into `args.cp` chunks whose
+    ranks run as threads (cp.LocalRing; device-to-device copies stand in for the NVLink
+    transfers), timed beside the single-sequence step of the same workload in the same run.
+    Each step is bracketed by CUDA events on the launching thread's stream, recorded after every
+    rank's stream has drained, so the ranks' host-side launch overhead is inside the time."""
+    import statistics
+
+    import torch
+
+    from fwd_bwd_b200 import cp, ops
+    from fwd_bwd_b200.inputs import make_inputs_fast
+
+    W = args.cp
+    if w.N % (128 * W) != 0 or w.qsmooth:
+        raise SystemExit(f"--cp {W}: N must split into chunks of a multiple of 128 tokens, "
+                         "without Q-smoothing")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = ops.Config(causal=w.causal, qknorm=w.qknorm, ksmooth=w.ksmooth, q_block=w.q_block,
+                     k_block=w.k_block)
+    x = make_inputs_fast(w, device=str(dev))
+    q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+    n = w.N // W
+    per_rank = [tuple(t[:, :, r * n:(r + 1) * n].contiguous() for t in (q, k, v, do)) + (cfg,)
+                for r in range(W)]
+    ring = cp.LocalRing(W, dev)
+
+    def ring_step():
+        ring.run(lambda comm, *a: cp.forward_backward(*a, comm=comm), per_rank)
+
+    def single_step():
+        qb = ops.quant_prologue(q, k, v, cfg)
+        o, lse = ops.attn_fwd(qb, q, cfg)
+        ops.attn_bwd(q, k, v, qb, o, lse, do, cfg)
+
+    def median_ms(step):
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(args.steps):
+            e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+            e0.record()
+            step()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    single_ms = median_ms(single_step)
+    ring_ms = median_ms(ring_step)
+    assert ops.device_status() == 0
+    tops = w.ops() / (ring_ms * 1e-3) / 1e12
+    elems = w.B * w.H * n * w.d
+    line = {
+        "metric": "attention fwd+bwd effective TOPS through the context-parallel ring "
+                  "(ranks emulated on 1 B200)",
+        "value": tops, "unit": "TOPS", "n_gpus": 1, "cp_ranks": W, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ring_ms,
+        "single_sequence_ms": single_ms, "ring_over_single_sequence": ring_ms / single_ms,
+        "higher_is_better": True, "dtype": "int8+bf16", "data": "synthetic",
+        # bytes each rank sends per ring step: INT8 K and V codes (forward); K codes, raw
+        # 16-bit V and the float32 dK / dV accumulators (backward); block scales excluded
+        "ring_bytes_per_rank_step": {"forward": 2 * elems, "backward": 11 * elems},
+        "config": dict(config_of(w), transport="cp.LocalRing: the ranks as threads on one GPU, "
+                       "device-to-device copies in place of NVLink"),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_nvfp4(args, w):
     """The NVFP4 Q-Attn step: NVFP4 prologue (with the sequence views) + forward + backward
     (preprocess, main kernel, dQ finalize)."""
@@ -408,6 +483,9 @@ def main():
         return
     if args.variant == "nvfp4":
         run_nvfp4(args, w)
+        return
+    if args.cp > 0:
+        run_cp(args, w)
         return
 
     import torch

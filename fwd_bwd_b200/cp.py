@@ -26,7 +26,7 @@ Two transports run the same per-rank code:
   * ``RingComm``: one process per GPU, torch.distributed point-to-point (NCCL on GPUs);
   * ``LocalRing``: W ranks as threads of one process sharing one GPU, for tests and debugging.
     Each thread has its own CUDA stream; hand-offs are device-to-device copies ordered by CUDA
-    events, so no kernel ever waits on a kernel of another rank.
+    events (stream dependencies: no kernel spins on another rank's progress).
 
 Every step of the computation runs in libsage's kernels; this module only schedules calls and
 moves buffers.  Q-smoothing is not supported here.
@@ -165,11 +165,13 @@ class _LocalComm:
     def __init__(self, ring: LocalRing, rank: int):
         self.ring, self.rank, self.world = ring, rank, ring.world
 
-    def _exchange(self, item):
-        """Posts `item` with an event of this rank's stream; returns every rank's post."""
+    def _exchange(self, item, ev=None):
+        """Posts `item` with an event of this rank's stream (recorded now unless given); returns
+        every rank's post."""
         ring = self.ring
-        ev = torch.cuda.Event()
-        ev.record(torch.cuda.current_stream())
+        if ev is None:
+            ev = torch.cuda.Event()
+            ev.record(torch.cuda.current_stream())
         ring._box[self.rank] = (item, ev)
         ring._barrier.wait()
         posts = list(ring._box)
@@ -177,21 +179,27 @@ class _LocalComm:
         return posts
 
     def shift_start(self, tensors: Sequence[torch.Tensor]) -> _Pending:
-        return _Pending(None, [], lambda: self.shift(tensors))
+        # the tensors are ready now: the next rank's copy must not wait for the kernels this
+        # rank enqueues before wait() (as a transfer issued before them would not)
+        ev = torch.cuda.Event()
+        ev.record(torch.cuda.current_stream())
+        tensors = list(tensors)
+        return _Pending(None, [], lambda: self._shift(tensors, ev))
 
     def shift(self, tensors: Sequence[torch.Tensor]) -> List[torch.Tensor]:
-        ring, st = self.ring, torch.cuda.current_stream()
-        posts = self._exchange(list(tensors))
+        return self._shift(list(tensors), None)
+
+    def _shift(self, tensors, ev) -> List[torch.Tensor]:
+        st = torch.cuda.current_stream()
+        posts = self._exchange(tensors, ev)
         src, src_ev = posts[(self.rank - 1) % self.world]
         st.wait_event(src_ev)
         recv = [t.clone() for t in src]  # device-to-device copies on this rank's stream
-        done = torch.cuda.Event()
-        done.record(st)
-        ring._done[self.rank] = done
-        ring._barrier.wait()
-        # this rank's sent tensors may change only after the next rank has copied them
-        st.wait_event(ring._done[(self.rank + 1) % self.world])
-        ring._barrier.wait()
+        for t in src:
+            # the previous rank may drop these tensors once it returns: the caching allocator
+            # then reuses their memory only after this stream's copies have run
+            t.record_stream(st)
+        self.ring._barrier.wait()  # every copy is recorded before any rank returns
         return recv
 
     def average_(self, t: torch.Tensor) -> None:
