@@ -355,6 +355,34 @@ def test_qmode_k_outlier_trend():
     assert errs[True] < errs[False]
 
 
+def test_qmode_k_outlier_ablation():
+    """The K-outlier workload's four runs (K-smoothing on/off x QK-norm on/off; two heads at
+    N = 1024): the recipe's accuracy against full precision.  K-smoothing is what keeps dQ
+    accurate (the error-propagation paragraph: dQ = dS K inherits K's quantization error), and
+    with both on every output keeps cosine >= 0.995."""
+    w = WORKLOADS["koutlier"].replace(B=1, H=2, N=1024)
+    x = make_inputs(w)
+    args = [_heads(x[n + "_f32"], w) for n in ("q", "k", "v", "do")]
+    err, cos = {}, {}
+    for qn in (True, False):
+        for ks in (True, False):
+            kw = dict(causal=True, qknorm=qn, ksmooth=ks, q_block=128, k_block=64,
+                      dtype="bf16")
+            rq = O.sage_attention(*args, **kw)
+            rx = O.sage_attention(*args, quant=False, round_outputs=False, **kw)
+            for n in ("o", "dq", "dk", "dv"):
+                a, b = rq[n].ravel(), rx[n].ravel()
+                err[qn, ks, n] = _rel(rq[n], rx[n])
+                cos[qn, ks, n] = float(a @ b / np.sqrt((a @ a) * (b @ b)))
+    for qn in (True, False):
+        assert err[qn, False, "dq"] > 3 * err[qn, True, "dq"]  # smoothing matters most for dQ
+        assert err[qn, False, "o"] > err[qn, True, "o"]
+    for ks in (True, False):
+        assert err[False, ks, "o"] > err[True, ks, "o"]  # QK-norm helps too
+    for n in ("o", "dq", "dk", "dv"):
+        assert cos[True, True, n] >= 0.995, n
+
+
 # ------------------------------------------------------------------------------------------
 # Q-smoothing
 # ------------------------------------------------------------------------------------------
