@@ -1,4 +1,4 @@
-"""Pins for the quantized products of the oracle's Q-mode backward pass.
+"""Pins for the quantized products of the oracle's Q-mode backward (and forward) pass.
 
 The SageBwd page ("SageBwd: trainable low-bit attention", error-propagation paragraph) puts
 the recipe's risk in ``dQ = dS K`` and ``dK = dS^T Q``: the quantization error of dS flows
@@ -10,6 +10,11 @@ rounding.  The inputs have strongly different magnitudes per block (QK-norm off)
 taken from the wrong block, a per-row instead of per-tile dS scale, dO quantized on the wrong
 token blocks, or a dropped dS scale all change the result; ``test_planted_mistakes`` applies
 each of these mistakes to the oracle's source and checks that the pin fails.
+
+The forward pass gets the same treatment: O and LSE recomputed row by row (the softmax over
+the visible keys, P quantized with one scale per query row and K block, the integer P V product
+of each block dequantized by that scale and the V block's), against ``attn_fwd_head``, with
+planted mistakes of the same kind.
 
 Also pinned here: the oracle's bf16 output rounding against torch's bf16 conversion (a library
 routine) on ties, large values and subnormals.
@@ -202,6 +207,87 @@ def test_unmutated_source_passes():
     """The mutation harness itself is sound: the source recompiled unchanged passes."""
     src_fn = _mutated("qz = _Quant(quant)", "qz = _Quant(quant)")
     assert all(_products_agree(c, src_fn) for c in CASES)
+
+
+# ------------------------------------------------------------------------------------------
+# forward products
+# ------------------------------------------------------------------------------------------
+def _brute_forward(p):
+    """O and LSE of the recipe row by row (float64 continuous arithmetic)."""
+    N, d, BQ, BK, tau = p["N"], p["d"], p["q_block"], p["k_block"], p["tau"]
+    qc, kc = p["qc"].astype(np.int64), p["kc"].astype(np.int64)
+    vc = p["vc"].astype(np.int64)
+    O_ = np.zeros((N, d))
+    lse = np.zeros(N)
+    for i in range(N):
+        z = [None] * N
+        for j in range(N):
+            if p["causal"] and j > i:
+                continue
+            a = int(np.dot(qc[i], kc[j]))
+            z[j] = a * (float(p["sq"][i // BQ]) * float(p["sk"][j // BK])) * tau
+        m = max(v for v in z if v is not None)
+        e = [0.0 if v is None else math.exp(v - m) for v in z]
+        l = math.fsum(e)
+        acc = np.zeros(d)
+        for b in range(N // BK):
+            # one scale per (query row, K block), the block's maximum / 127
+            codes, s = _tile_quant_brute(np.array(e[b * BK:(b + 1) * BK])[None, :])
+            iv = codes[0] @ vc[b * BK:(b + 1) * BK]
+            acc += iv * (float(s) * float(p["sv"][b]))
+        O_[i] = acc / l
+        lse[i] = m + math.log(l)
+    return O_, lse
+
+
+def _oracle_forward(p, fwd=None):
+    fwd = fwd or O.attn_fwd_head
+    return fwd(p["qc"], p["sq"], p["kc"], p["sk"], p["vc"], p["sv"], q_block=p["q_block"],
+               k_block=p["k_block"], causal=p["causal"], tau=p["tau"])
+
+
+_BRUTE_FWD = {}
+
+
+def _forward_agrees(case, fwd=None):
+    if case not in _BRUTE_FWD:
+        p = _problem(*case)
+        _BRUTE_FWD[case] = (p, _brute_forward(p))
+    p, ref = _BRUTE_FWD[case]
+    got = _oracle_forward(p, fwd)
+    return all(np.allclose(g, r, rtol=1e-12, atol=1e-12 * np.abs(r).max())
+               for g, r in zip(got, ref))
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_qmode_fwd_products_brute_force(case):
+    assert _forward_agrees(case)
+
+
+FWD_MUTATIONS = {
+    "V scale of the wrong block": (
+        "(sp * F64(v_scale[j]))", "(sp * F64(v_scale[(j + 1) % (N // k_block)]))"),
+    "one P scale per tile instead of per row": (
+        "pc, sp = qz.rows_per_block(e[:, cols])", "pc, sp = qz.tile(e[:, cols])"),
+    "Q scale of the wrong block": (
+        "_scores(qc[rows], sq_row[rows],", "_scores(qc[rows], sq_row[::-1][rows],"),
+    "LSE in base 2": ("LSE[rows] = m + np.log(l)", "LSE[rows] = m + np.log2(l)"),
+}
+
+
+def _mutated_fwd(old, new):
+    src = textwrap.dedent(inspect.getsource(O.attn_fwd_head))
+    assert src.count(old) == 1, old
+    ns = dict(vars(O))
+    exec(compile(src.replace(old, new), "<mutated attn_fwd_head>", "exec"), ns)
+    return ns["attn_fwd_head"]
+
+
+@pytest.mark.parametrize("name", sorted(FWD_MUTATIONS))
+def test_planted_forward_mistakes(name):
+    fwd = _mutated_fwd(*FWD_MUTATIONS[name])
+    with np.errstate(invalid="ignore", divide="ignore"):
+        assert not all(_forward_agrees(c, fwd) for c in CASES), name
 
 
 # ------------------------------------------------------------------------------------------
